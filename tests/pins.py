@@ -1,0 +1,560 @@
+"""Pins of the CPU oracle: checks against what the pages and the mathematics
+fix, each independent of the oracle's own code path.
+
+Every pin is a plain function that raises AssertionError on failure, so that
+test_oracle_pins.py runs them one by one and test_oracle_mutations.py can
+run them all against an oracle with a mistake planted in it (see
+qo_set_fault) and require that some pin catches each mistake.
+
+Sources:
+* eq. (1) and its decay / delta / write-gate choices: "LinQuant: Functional
+  Invariances for Low-Precision Linear Recurrences", Theoretical Foundation;
+* invariances used as properties: same page, The Seven Functional
+  Invariances, key-side rotation (1/7), key-side rescaling (2/7),
+  value-side rescaling (4/7);
+* policies: "When Dynamic Scaling Fails" project page (per-token dynamic,
+  static/persistent, yoked to a full-precision reference);
+* BDR: "Preserving Updates in Low-Bit Recurrent State Quantization",
+  abstract.
+"""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+
+from oracle import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+F32 = np.float32
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _unit(g):
+    return g / np.linalg.norm(g, axis=-1, keepdims=True)
+
+
+def _inputs(rng, T, dk, dv, decay, unit_k=True, alpha=None, beta=None):
+    q = rng.standard_normal((T, dk))
+    k = rng.standard_normal((T, dk))
+    if unit_k:
+        k = _unit(k)
+    v = rng.standard_normal((T, dv))
+    if alpha is None:
+        alpha = rng.uniform(0.8, 1.0, size=(T, dk) if decay == "diagonal" else (T,))
+    if beta is None:
+        beta = rng.uniform(0.1, 1.0, size=(T,))
+    f = lambda a: np.ascontiguousarray(a, dtype=F32)
+    return f(q), f(k), f(v), f(np.broadcast_to(alpha, (T, dk) if decay == "diagonal" else (T,))), \
+        f(np.broadcast_to(beta, (T,)))
+
+
+def _decay64(alpha, decay, dk):
+    a = alpha.astype(np.float64)
+    return a if decay == "diagonal" else np.repeat(a[:, None], dk, axis=1)
+
+
+# --------------------------------------------------------------------------
+# The FP32 recurrence (the oracle's unquantized step)
+# --------------------------------------------------------------------------
+
+def pin_linear_write_sum_of_outer_products():
+    """delta = 0, Lambda = I, beta = 1, S0 = 0  =>  S_H = sum_t v_t k_t^T."""
+    rng = _rng(10)
+    for decay in ("scalar", "diagonal"):
+        T, dk, dv, H = 3, 16, 5, 12
+        cfg = O.OracleConfig(T, dk, dv, 8, 16, 0, decay)
+        S = np.zeros((T, dv, dk), F32)
+        acc = np.zeros((T, dv, dk))
+        for _ in range(H):
+            q, k, v, a, b = _inputs(rng, T, dk, dv, decay, unit_k=False,
+                                    alpha=1.0, beta=1.0)
+            O.fp32_step(cfg, S, q, k, v, a, b, want_o=False)
+            acc += np.einsum("ti,tj->tij", v.astype(np.float64), k.astype(np.float64))
+        err = np.abs(S - acc).max() / np.abs(acc).max()
+        assert err < 1e-6, err
+
+
+def pin_decay_closed_form():
+    """delta = 0, S0 = 0:  S_H = sum_t beta_t v_t (k_t * prod_{s>t} a_s)^T
+    for scalar and diagonal decay (the decay multiplies the key side)."""
+    rng = _rng(11)
+    for decay in ("scalar", "diagonal"):
+        T, dk, dv, H = 2, 32, 3, 10
+        cfg = O.OracleConfig(T, dk, dv, 8, 16, 0, decay)
+        S = np.zeros((T, dv, dk), F32)
+        steps = [_inputs(rng, T, dk, dv, decay, unit_k=False) for _ in range(H)]
+        for q, k, v, a, b in steps:
+            O.fp32_step(cfg, S, q, k, v, a, b, want_o=False)
+        ref = np.zeros((T, dv, dk))
+        for t, (q, k, v, a, b) in enumerate(steps):
+            later = np.ones((T, dk))
+            for s in range(t + 1, H):
+                later *= _decay64(steps[s][3], decay, dk)
+            ref += b.astype(np.float64)[:, None, None] * np.einsum(
+                "ti,tj->tij", v.astype(np.float64), k.astype(np.float64) * later)
+        err = np.abs(S - ref).max() / np.abs(ref).max()
+        assert err < 1e-5, (decay, err)
+
+
+def pin_delta_rule_key_recall():
+    """delta = 1, ||k|| = 1:  S_t k_t = (1 - beta_t) S_{t-1} Lambda_t k_t + beta_t v_t,
+    for any decay; with beta = 1 the key recalls its value exactly."""
+    rng = _rng(12)
+    for decay in ("scalar", "diagonal"):
+        for beta_one in (False, True):
+            T, dk, dv = 3, 32, 6
+            cfg = O.OracleConfig(T, dk, dv, 8, 16, 1, decay)
+            S = (rng.standard_normal((T, dv, dk)) * 0.3).astype(F32)
+            for _ in range(8):
+                q, k, v, a, b = _inputs(rng, T, dk, dv, decay,
+                                        beta=1.0 if beta_one else None)
+                prev = S.astype(np.float64).copy()
+                O.fp32_step(cfg, S, q, k, v, a, b, want_o=False)
+                k64 = k.astype(np.float64)
+                lhs = np.einsum("tij,tj->ti", S.astype(np.float64), k64)
+                Sd = prev * _decay64(a, decay, dk)[:, None, :]
+                rhs = (1 - b.astype(np.float64))[:, None] * np.einsum("tij,tj->ti", Sd, k64) \
+                    + b.astype(np.float64)[:, None] * v.astype(np.float64)
+                scale = 1.0 + np.abs(rhs).max()
+                assert np.abs(lhs - rhs).max() < 2e-5 * scale, (decay, beta_one)
+
+
+def pin_readout_is_state_times_q():
+    """o_t = S_t q_t with S_t the updated state (FP32 recurrence)."""
+    rng = _rng(13)
+    for delta in (0, 1):
+        T, dk, dv = 2, 64, 4
+        cfg = O.OracleConfig(T, dk, dv, 8, 16, delta, "scalar")
+        S = (rng.standard_normal((T, dv, dk)) * 0.2).astype(F32)
+        for _ in range(4):
+            q, k, v, a, b = _inputs(rng, T, dk, dv, "scalar")
+            o = O.fp32_step(cfg, S, q, k, v, a, b)
+            ref = np.einsum("tij,tj->ti", S.astype(np.float64), q.astype(np.float64))
+            assert np.abs(o - ref).max() < 1e-5 * (1 + np.abs(ref).max())
+
+
+def pin_value_rescaling_exact():
+    """v -> D_V v with D_V a positive diagonal of powers of two: the FP32
+    state becomes D_V S bit for bit, and the quantized state keeps its codes
+    while its scales take the factor (LinQuant 4/7, exact for powers of two)."""
+    rng = _rng(14)
+    T, dk, dv = 2, 32, 8
+    d = (2.0 ** rng.integers(-3, 4, size=dv)).astype(F32)
+    for delta in (0, 1):
+        for decay in ("scalar", "diagonal"):
+            cfg = O.OracleConfig(T, dk, dv, 8, 16, delta, decay)
+            S = (rng.standard_normal((T, dv, dk)) * 0.2).astype(F32)
+            S2 = (S * d[None, :, None]).astype(F32)
+            for _ in range(5):
+                q, k, v, a, b = _inputs(rng, T, dk, dv, decay)
+                O.fp32_step(cfg, S, q, k, v, a, b, want_o=False)
+                O.fp32_step(cfg, S2, q, k, (v * d[None, :]).astype(F32), a, b, want_o=False)
+            assert np.array_equal(S2, (S * d[None, :, None]).astype(F32))
+            for policy in ("dynamic", "persistent", "yoked"):
+                for rounding in ("nearest", "bdr"):
+                    qc = O.OracleConfig(T, dk, dv, 4, 16, delta, decay, policy, rounding)
+                    S0 = (rng.standard_normal((T, dv, dk)) * 0.2).astype(F32)
+                    A = O.init(qc, S0)
+                    B = O.init(qc, (S0 * d[None, :, None]).astype(F32))
+                    for _ in range(5):
+                        q, k, v, a, b = _inputs(rng, T, dk, dv, decay)
+                        O.step(A, q, k, v, a, b, want_o=False)
+                        O.step(B, q, k, (v * d[None, :]).astype(F32), a, b, want_o=False)
+                    assert np.array_equal(A.codes, B.codes), (policy, rounding)
+                    assert np.array_equal(B.scales, (A.scales * d[None, :, None]).astype(F32))
+
+
+def _rotation(rng, n):
+    Q, R = np.linalg.qr(rng.standard_normal((n, n)))
+    return Q * np.sign(np.diag(R))[None, :]
+
+
+def pin_key_rotation():
+    """(q, k) -> (R q, R k) with R orthogonal leaves the readout unchanged
+    when R commutes with Lambda (no or scalar decay), also for the delta rule
+    (LinQuant 1/7); diagonal decay breaks it."""
+    rng = _rng(15)
+    T, dk, dv, H = 2, 32, 4, 6
+    R = _rotation(rng, dk)
+    for decay, delta, should_hold in (("scalar", 0, True), ("scalar", 1, True),
+                                      ("diagonal", 0, False)):
+        cfg = O.OracleConfig(T, dk, dv, 8, 16, delta, decay)
+        S = np.zeros((T, dv, dk), F32)
+        Sr = np.zeros((T, dv, dk), F32)
+        worst = 0.0
+        for _ in range(H):
+            q, k, v, a, b = _inputs(rng, T, dk, dv, decay)
+            o = O.fp32_step(cfg, S, q, k, v, a, b)
+            orot = O.fp32_step(cfg, Sr, (q @ R.T).astype(F32), (k @ R.T).astype(F32), v, a, b)
+            worst = max(worst, np.abs(o - orot).max() / (1 + np.abs(o).max()))
+        assert (worst < 1e-5) == should_hold, (decay, delta, worst)
+
+
+def pin_key_rescaling():
+    """(q, k) -> (D q, D^-1 k), D positive diagonal (powers of two): the
+    readout is unchanged bit for bit for linear writes under scalar or
+    diagonal decay; the delta rule does not preserve it (LinQuant 2/7)."""
+    rng = _rng(16)
+    T, dk, dv, H = 2, 32, 4, 6
+    d = (2.0 ** rng.integers(-2, 3, size=dk)).astype(F32)
+    for decay, delta, should_hold in (("scalar", 0, True), ("diagonal", 0, True),
+                                      ("scalar", 1, False)):
+        cfg = O.OracleConfig(T, dk, dv, 8, 16, delta, decay)
+        S = np.zeros((T, dv, dk), F32)
+        Sd = np.zeros((T, dv, dk), F32)
+        same = True
+        for _ in range(H):
+            q, k, v, a, b = _inputs(rng, T, dk, dv, decay)
+            o = O.fp32_step(cfg, S, q, k, v, a, b)
+            od = O.fp32_step(cfg, Sd, (q * d).astype(F32), (k / d).astype(F32), v, a, b)
+            same = same and np.array_equal(o, od)
+        assert same == should_hold, (decay, delta)
+
+
+# --------------------------------------------------------------------------
+# Quantizer, policies, BDR
+# --------------------------------------------------------------------------
+
+def _x64(prev: "O.State", q, k, v, a, b, cfg):
+    """Updated state x in float64 from the previous quantized state, written
+    from eq. (1) with numpy (independent of the oracle's loops)."""
+    d = prev.codes.astype(np.float64) * np.repeat(prev.scales.astype(np.float64), cfg.group, axis=-1)
+    Sd = d * _decay64(a, cfg.decay, cfg.dk)[:, None, :]
+    k64 = k.astype(np.float64)
+    if cfg.delta:
+        w = b.astype(np.float64)[:, None] * (v.astype(np.float64) - np.einsum("tij,tj->ti", Sd, k64))
+    else:
+        w = b.astype(np.float64)[:, None] * v.astype(np.float64)
+    return Sd + w[:, :, None] * k64[:, None, :], Sd, w
+
+
+def pin_quantizer_error_bound():
+    """Quantize -> dequantize error is at most half a grid step per element,
+    except where the persistent (or yoked) scale clips."""
+    rng = _rng(17)
+    T, dk, dv = 3, 64, 8
+    for bits in (4, 8):
+        for policy in ("dynamic", "persistent", "yoked"):
+            cfg = O.OracleConfig(T, dk, dv, bits, 32, 1, "scalar", policy)
+            S0 = (rng.standard_normal((T, dv, dk)) * 0.3).astype(F32)
+            st = O.init(cfg, S0)
+            # init itself: |S0 - n s| <= s/2 (init uses the dynamic rule)
+            deq = st.codes * np.repeat(st.scales, cfg.group, axis=-1).astype(np.float64)
+            s_el = np.repeat(st.scales, cfg.group, axis=-1).astype(np.float64)
+            assert np.all(np.abs(S0 - deq) <= 0.5 * s_el * (1 + 1e-6))
+            for _ in range(6):
+                q, k, v, a, b = _inputs(rng, T, dk, dv, "scalar")
+                prev = st.copy()
+                x64, _, _ = _x64(prev, q, k, v, a, b, cfg)
+                O.step(st, q, k, v, a, b, want_o=False)
+                s_el = np.repeat(st.scales, cfg.group, axis=-1).astype(np.float64)
+                err = np.abs(x64 - st.codes * s_el)
+                clipped = np.abs(st.codes) == cfg.qmax
+                ok = err <= 0.5 * s_el * (1 + 1e-5) + 1e-6 * np.abs(x64)
+                assert np.all(ok | (clipped & (policy != "dynamic"))), (bits, policy)
+
+
+def pin_dynamic_scale_reaches_qmax():
+    """Dynamic scale = group max|x| / qmax: every group with a nonzero entry
+    has an element at code magnitude qmax, and the scale equals the group
+    maximum of the float64 update over qmax to FP32 precision."""
+    rng = _rng(18)
+    T, dk, dv = 3, 64, 8
+    for bits in (4, 8):
+        cfg = O.OracleConfig(T, dk, dv, bits, 32, 1, "scalar", "dynamic")
+        st = O.init(cfg, (rng.standard_normal((T, dv, dk)) * 0.3).astype(F32))
+        for _ in range(5):
+            q, k, v, a, b = _inputs(rng, T, dk, dv, "scalar")
+            x64, _, _ = _x64(st.copy(), q, k, v, a, b, cfg)
+            O.step(st, q, k, v, a, b, want_o=False)
+            m = np.abs(st.codes).reshape(T, dv, dk // 32, 32).max(axis=-1)
+            assert np.all(m == cfg.qmax)
+            gmax = np.abs(x64).reshape(T, dv, dk // 32, 32).max(axis=-1)
+            assert np.allclose(st.scales, gmax / cfg.qmax, rtol=2e-6, atol=0)
+
+
+def pin_persistent_zero_update():
+    """A zero update (k = 0, alpha = 1) leaves persistent codes and scales
+    bit-identical, for both write kinds."""
+    rng = _rng(19)
+    T, dk, dv = 3, 64, 8
+    for bits in (4, 8):
+        for delta in (0, 1):
+            for rounding in ("nearest", "bdr"):
+                cfg = O.OracleConfig(T, dk, dv, bits, 32, delta, "scalar", "persistent", rounding)
+                st = O.init(cfg, (rng.standard_normal((T, dv, dk)) * 0.3).astype(F32))
+                before = st.copy()
+                q, _, v, _, b = _inputs(rng, T, dk, dv, "scalar")
+                O.step(st, q, np.zeros((T, dk), F32), v, np.ones(T, F32), b, want_o=False)
+                assert np.array_equal(st.codes, before.codes)
+                assert np.array_equal(st.scales, before.scales)
+
+
+def pin_persistent_scales_fixed():
+    """Persistent scales are those of the quantization start, forever."""
+    rng = _rng(20)
+    T, dk, dv = 2, 64, 8
+    cfg = O.OracleConfig(T, dk, dv, 4, 32, 1, "scalar", "persistent")
+    S0 = (rng.standard_normal((T, dv, dk)) * 0.3).astype(F32)
+    st = O.init(cfg, S0)
+    s0 = st.scales.copy()
+    for _ in range(10):
+        O.step(st, *_inputs(rng, T, dk, dv, "scalar"), want_o=False)
+    assert np.array_equal(st.scales, s0)
+    # and they are max|S0| / qmax of each group
+    gmax = np.abs(S0.astype(np.float64)).reshape(T, dv, 2, 32).max(axis=-1)
+    assert np.allclose(s0, gmax / cfg.qmax, rtol=1e-6, atol=0)
+
+
+def pin_zero_scale_group():
+    """A group that is all zero at the quantization start has scale 0 and
+    codes 0; under the persistent scale it stays 0."""
+    rng = _rng(21)
+    T, dk, dv = 1, 64, 4
+    S0 = (rng.standard_normal((T, dv, dk)) * 0.3).astype(F32)
+    S0[0, 1, 32:64] = 0.0
+    cfg = O.OracleConfig(T, dk, dv, 8, 32, 1, "scalar", "persistent")
+    st = O.init(cfg, S0)
+    assert st.scales[0, 1, 1] == 0.0 and np.all(st.codes[0, 1, 32:] == 0)
+    for _ in range(3):
+        O.step(st, *_inputs(rng, T, dk, dv, "scalar"), want_o=False)
+    assert st.scales[0, 1, 1] == 0.0 and np.all(st.codes[0, 1, 32:] == 0)
+
+
+def pin_bdr_bruteforce():
+    """BDR against brute force over every code: with sigma = sign(w) sign(k_j),
+    the chosen code is nearest or nearest + sigma; its dequantized value never
+    lies on the far side of the pre-update value S' from the update unless
+    clamped; it equals nearest when sigma = 0 or nearest does not reverse; and
+    otherwise it is the non-reversing code closest to the nearest one."""
+    rng = _rng(22)
+    T, dk, dv = 8, 16, 4
+    for bits in (4, 8):
+        for policy in ("persistent", "dynamic"):
+            qmax = (1 << (bits - 1)) - 1
+            cN = O.OracleConfig(T, dk, dv, bits, 16, 0, "diagonal", policy, "nearest")
+            cB = O.OracleConfig(T, dk, dv, bits, 16, 0, "diagonal", policy, "bdr")
+            S0 = (rng.standard_normal((T, dv, dk)) * 0.5).astype(F32)
+            B = O.init(cB, S0)
+            for _ in range(8):
+                q, k, v, a, b = _inputs(rng, T, dk, dv, "diagonal")
+                k[:, ::5] = 0.0          # some columns with no update
+                v[:, 0] = 0.0            # a row with no update
+                v = (v * 0.05).astype(F32)   # small updates: reversals are common
+                prev = B.copy()
+                # nearest rounding from the same state and inputs
+                Nst = O.State(cN, prev.codes.copy(), prev.scales.copy())
+                O.step(Nst, q, k, v, a, b, want_o=False)
+                O.step(B, q, k, v, a, b, want_o=False)
+                d = (prev.codes.astype(F32) * np.repeat(prev.scales, 16, axis=-1)).astype(F32)
+                Sp = (d * a[:, None, :]).astype(F32)
+                w = (b[:, None] * v).astype(F32)
+                sigma = np.sign(w)[:, :, None] * np.sign(k)[:, None, :]
+                s_el = np.repeat(B.scales, 16, axis=-1)
+                n_near, n = Nst.codes, B.codes
+                assert np.array_equal(Nst.scales, B.scales)
+                step = n - n_near
+                assert np.all((step == 0) | (step == sigma))
+                dq = (n.astype(F32) * s_el).astype(F32)
+                reverse = ((sigma > 0) & (dq < Sp)) | ((sigma < 0) & (dq > Sp))
+                clamped = np.abs(n) == qmax
+                assert not np.any(reverse & ~clamped)
+                dqn = (n_near.astype(F32) * s_el).astype(F32)
+                near_rev = ((sigma > 0) & (dqn < Sp)) | ((sigma < 0) & (dqn > Sp))
+                assert np.all(n[~near_rev] == n_near[~near_rev])
+                # brute force: the smallest move in the update direction
+                live = near_rev & ~clamped & (s_el > 0)
+                for idx in zip(*np.nonzero(live)):
+                    sg = sigma[idx]
+                    cands = [c for c in range(-qmax, qmax + 1)
+                             if (F32(c) * s_el[idx] - Sp[idx]) * sg >= 0]
+                    best = min(cands, key=lambda c: abs(c - n_near[idx]))
+                    assert n[idx] == best
+
+
+def pin_yoked_shadow_is_fp32_run():
+    """The yoked shadow follows the unquantized FP32 recurrence bit for bit
+    (the full-precision reference run alongside)."""
+    rng = _rng(23)
+    T, dk, dv = 2, 64, 8
+    for decay in ("scalar", "diagonal"):
+        cfg = O.OracleConfig(T, dk, dv, 4, 32, 1, decay, "yoked")
+        S0 = (rng.standard_normal((T, dv, dk)) * 0.3).astype(F32)
+        st = O.init(cfg, S0)
+        S = S0.copy()
+        for _ in range(6):
+            inp = _inputs(rng, T, dk, dv, decay)
+            O.step(st, *inp, want_o=False)
+            O.fp32_step(cfg, S, *inp, want_o=False)
+        assert np.array_equal(st.shadow, S)
+
+
+def pin_yoked_scale_from_shadow_only():
+    """Yoked scales are a function of the shadow trajectory alone: two runs
+    that share the shadow but start from different codes get the same scales
+    (the feedback loop from the quantized state to the scale is cut)."""
+    rng = _rng(24)
+    T, dk, dv = 2, 64, 8
+    cfg = O.OracleConfig(T, dk, dv, 4, 32, 1, "scalar", "yoked")
+    S0 = (rng.standard_normal((T, dv, dk)) * 0.3).astype(F32)
+    A = O.init(cfg, S0)
+    B = A.copy()
+    B.codes = np.clip(B.codes + rng.integers(-2, 3, size=B.codes.shape), -7, 7).astype(np.int32)
+    for _ in range(4):
+        inp = _inputs(rng, T, dk, dv, "scalar")
+        O.step(A, *inp, want_o=False)
+        O.step(B, *inp, want_o=False)
+        assert np.array_equal(A.scales, B.scales)
+    assert not np.array_equal(A.codes, B.codes)
+    gmax = np.abs(A.shadow.astype(np.float64)).reshape(T, dv, 2, 32).max(axis=-1)
+    assert np.allclose(A.scales, gmax / cfg.qmax, rtol=1e-6, atol=0)
+
+
+def pin_high_bit_tracks_fp32():
+    """With a 16-bit grid the quantized trajectory stays within ~1e-4 of the
+    unquantized FP32 one: the quantized path is the same recurrence."""
+    rng = _rng(25)
+    T, dk, dv, H = 2, 64, 8, 20
+    for decay in ("scalar", "diagonal"):
+        for delta in (0, 1):
+            for policy in ("dynamic", "yoked"):
+                cfg = O.OracleConfig(T, dk, dv, 16, 32, delta, decay, policy)
+                S0 = (rng.standard_normal((T, dv, dk)) * 0.3).astype(F32)
+                st = O.init(cfg, S0)
+                S = S0.copy()
+                for _ in range(H):
+                    inp = _inputs(rng, T, dk, dv, decay)
+                    oq = O.step(st, *inp)
+                    o = O.fp32_step(cfg, S, *inp)
+                    assert np.abs(oq - o).max() < 1e-3 * (1 + np.abs(o).max()), (decay, delta, policy)
+                err = np.abs(st.dequantized() - S).max() / np.abs(S).max()
+                assert err < 2e-4, (decay, delta, policy, err)
+
+
+def pin_error_accumulation_bound():
+    """Persistent scale, non-expansive steps (||k|| = 1, alpha <= 1,
+    beta in (0, 1]): ||S^q_t - S_t||_F <= ||S^q_0 - S_0||_F + sum_tau ||eps_tau||_F
+    where eps_tau is the rounding error of step tau (float64 closed-form
+    check)."""
+    rng = _rng(26)
+    T, dk, dv, H = 2, 64, 8, 40
+    for bits in (4, 8):
+        for rounding in ("nearest", "bdr"):
+            cfg = O.OracleConfig(T, dk, dv, bits, 32, 1, "scalar", "persistent", rounding)
+            S0 = (rng.standard_normal((T, dv, dk)) * 0.3).astype(F32)
+            st = O.init(cfg, S0)
+            S = S0.astype(np.float64)
+            bound = np.linalg.norm((st.dequantized() - S).reshape(T, -1), axis=1)
+            for _ in range(H):
+                q, k, v, a, b = _inputs(rng, T, dk, dv, "scalar")
+                x64, _, _ = _x64(st.copy(), q, k, v, a, b, cfg)
+                O.step(st, q, k, v, a, b, want_o=False)
+                eps = st.dequantized().astype(np.float64) - x64
+                bound = bound + np.linalg.norm(eps.reshape(T, -1), axis=1)
+                Sd = S * a.astype(np.float64)[:, None, None]
+                k64 = k.astype(np.float64)
+                w = b.astype(np.float64)[:, None] * (v - np.einsum("tij,tj->ti", Sd, k64))
+                S = Sd + w[:, :, None] * k64[:, None, :]
+                gap = np.linalg.norm((st.dequantized() - S).reshape(T, -1), axis=1)
+                assert np.all(gap <= bound * (1 + 1e-4) + 1e-5), (bits, rounding)
+
+
+# --------------------------------------------------------------------------
+# Worked examples and layout / order fixtures
+# --------------------------------------------------------------------------
+
+def _dense(spec, n):
+    out = np.zeros(n, F32)
+    for key, val in spec.items():
+        out[int(key)] = val
+    return out
+
+
+def pin_worked_steps():
+    """The hand-worked steps of tests/golden/worked_steps.json."""
+    with open(os.path.join(GOLDEN, "worked_steps.json")) as f:
+        data = json.load(f)
+    for case in data["cases"]:
+        dk, dv = case["dk"], case["dv"]
+        cfg = O.OracleConfig(1, dk, dv, case["bits"], case["group"], case["delta"],
+                             case["decay"], case["policy"], case["rounding"])
+        S0 = _dense(case["S0"], dk).reshape(1, 1, dk).repeat(dv, axis=1)
+        st = O.init(cfg, S0)
+        assert np.array_equal(st.codes[0, 0], _dense(case["init_codes"], dk).astype(np.int32)), case["name"]
+        assert st.scales[0, 0, 0] == F32(case["init_scale"]), case["name"]
+        alpha = np.full((1,), case["alpha"], F32) if case["decay"] == "scalar" else \
+            np.full((1, dk), case["alpha"], F32)
+        o = O.step(st, _dense(case["q"], dk)[None], _dense(case["k"], dk)[None],
+                   np.array([case["v"]], F32), alpha, np.array([case["beta"]], F32))
+        assert np.array_equal(st.codes[0, 0], _dense(case["codes"], dk).astype(np.int32)), case["name"]
+        assert st.scales[0, 0, 0] == F32(case["scale"]), case["name"]
+        assert np.array_equal(o[0], np.array(case["o"], F32)), case["name"]
+        if "codes_nearest" in case:
+            from dataclasses import replace
+            c2 = replace(cfg, rounding="nearest")
+            st2 = O.init(c2, S0)
+            O.step(st2, _dense(case["q"], dk)[None], _dense(case["k"], dk)[None],
+                   np.array([case["v"]], F32), alpha, np.array([case["beta"]], F32))
+            assert np.array_equal(st2.codes[0, 0], _dense(case["codes_nearest"], dk).astype(np.int32))
+
+
+def pin_pack_layout():
+    with open(os.path.join(GOLDEN, "layout_and_order.json")) as f:
+        data = json.load(f)
+    for bits, key in ((4, "int4_pack"), (8, "int8_pack")):
+        codes = np.array(data[key]["codes"], np.int32)
+        packed = O.pack(bits, codes[None])[0]
+        assert list(packed) == data[key]["bytes"]
+        assert np.array_equal(O.unpack(bits, packed[None], codes.size)[0], codes)
+
+
+def pin_dot_order():
+    """The fixed dot-product order: pairwise tree over 16-column segments."""
+    with open(os.path.join(GOLDEN, "layout_and_order.json")) as f:
+        d = json.load(f)["dot_order"]
+    n = d["n"]
+    a = np.zeros(n, F32)
+    b = np.zeros(n, F32)
+    for s, val in enumerate(d["segment_values"]):
+        a[16 * s + 3] = val
+        b[16 * s + 3] = 1.0
+    assert O.dot(a, b) == F32(d["expected"])
+    # and within the error bound of the exact value on random data
+    rng = _rng(27)
+    for n in (16, 32, 64, 128, 256):
+        for _ in range(20):
+            a = rng.standard_normal(n).astype(F32)
+            b = rng.standard_normal(n).astype(F32)
+            exact = float(np.dot(a.astype(np.float64), b.astype(np.float64)))
+            bound = (16 + np.log2(n // 16) + 2) * 2.0 ** -24 * float(np.abs(a.astype(np.float64) * b).sum())
+            assert abs(float(O.dot(a, b)) - exact) <= bound
+
+
+ALL_PINS = [
+    pin_linear_write_sum_of_outer_products,
+    pin_decay_closed_form,
+    pin_delta_rule_key_recall,
+    pin_readout_is_state_times_q,
+    pin_value_rescaling_exact,
+    pin_key_rotation,
+    pin_key_rescaling,
+    pin_quantizer_error_bound,
+    pin_dynamic_scale_reaches_qmax,
+    pin_persistent_zero_update,
+    pin_persistent_scales_fixed,
+    pin_zero_scale_group,
+    pin_bdr_bruteforce,
+    pin_yoked_shadow_is_fp32_run,
+    pin_yoked_scale_from_shadow_only,
+    pin_high_bit_tracks_fp32,
+    pin_error_accumulation_bound,
+    pin_worked_steps,
+    pin_pack_layout,
+    pin_dot_order,
+]
