@@ -1,0 +1,561 @@
+#!/usr/bin/env python
+"""Benchmark of the quantized-state decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload gdn|mamba2|gla|stack24|tiny-gdn]
+
+One "step" advances the workload's batch by one token under each of its
+arms (for the default Gated DeltaNet-shaped workload: INT4 G32 with dynamic,
+persistent and yoked scales, one kernel launch each, readout on).  The
+metric is decode steps/s (whole job; N GPUs run independent shards, so
+scaling is weak) and the algorithmic state traffic in GB/s as a fraction of
+the measured HBM peak.
+
+L2 residency: the workload's state is smaller than B200's L2, so steps rotate
+over G independent request groups whose states together exceed 2x the L2
+size; step t uses group t mod G and pool slot t mod P of the inputs.  No
+state or input is therefore warm in L2 when its step runs.
+
+Timing: W untimed warm-up steps per arm (eager and graph), then the states
+are re-initialized and each arm's K steps are replayed from CUDA graphs,
+bracketed by CUDA events on the launching stream, with a barrier and a
+device synchronize on both sides; the max over ranks is reported.  SM clocks
+and throttle reasons are sampled through NVML during the timed region.
+
+The `e2e` figure runs the same steps through the public API with host
+buffers: each step copies its inputs from pinned host memory, launches the
+arms and copies the readouts back, all inside the timed region.
+
+`--impl reference` times the CPU oracle (the plain C implementation used
+as the correctness reference) on the host cores on a bounded sample of
+tiles per step, reported in the same unit.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from ssm_decode_step_b200 import workloads as W  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------------------
+# bytes per launch (algorithmic)
+# ---------------------------------------------------------------------------
+
+def arm_bytes(w: W.Workload, arm: W.Arm, readout: bool = True) -> int:
+    """Algorithmic bytes one decode-step launch must move: codes read and
+    written, scales read (and written unless persistent), q, k, v, alpha,
+    beta read, o written, and the FP32 shadow read and written (yoked)."""
+    T, dk, dv = w.tiles, w.dk, w.dv
+    codes = T * dv * dk * arm.bits // 8
+    scales = T * dv * (dk // arm.group) * 4
+    alpha = T * (dk if w.decay == "diagonal" else 1) * 4
+    inputs = T * ((dk if readout else 0) + dk + dv) * 4 + alpha + T * 4
+    out = T * dv * 4 if readout else 0
+    b = 2 * codes + scales * (1 if arm.policy == "persistent" else 2) + inputs + out
+    if arm.policy == "yoked":
+        b += 2 * T * dv * dk * 4
+    return b
+
+
+def state_bytes(w: W.Workload, arm: W.Arm) -> int:
+    T, dk, dv = w.tiles, w.dk, w.dv
+    b = T * dv * dk * arm.bits // 8 + T * dv * (dk // arm.group) * 4
+    if arm.policy == "yoked":
+        b += T * dv * dk * 4
+    return b
+
+
+def source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "ssm_decode_step_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def load_traffic(kernel_key: str):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel
+    sources have not changed since it was taken."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            data = json.load(f)
+        ent = data.get(kernel_key)
+        if ent and ent.get("source_sha") == source_sha():
+            return ent["dram_bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML on a thread."""
+
+    def __init__(self, torch_device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.max_mhz = None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thr = None
+        self.h = None
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            self.N = N
+            import torch
+            props = torch.cuda.get_device_properties(torch_device_index)
+            bus = getattr(props, "pci_bus_id", None)
+            dom = getattr(props, "pci_domain_id", 0)
+            dev = getattr(props, "pci_device_id", 0)
+            if bus is not None:
+                busid = "%08x:%02x:%02x.0" % (dom, bus, dev)
+                self.h = N.nvmlDeviceGetHandleByPciBusId(busid.encode())
+            else:
+                self.h = N.nvmlDeviceGetHandleByIndex(torch_device_index)
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM)
+        except Exception:
+            self.h = None
+
+    def _reasons(self):
+        N = self.N
+        for fn in ("nvmlDeviceGetCurrentClocksEventReasons", "nvmlDeviceGetCurrentClocksThrottleReasons"):
+            if hasattr(N, fn):
+                return getattr(N, fn)(self.h)
+        return 0
+
+    def _run(self):
+        N = self.N
+        while not self._stop.is_set():
+            try:
+                self.samples.append((N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM), self._reasons()))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.h is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thr is not None:
+            self._thr.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [m for m, _ in self.samples]
+        mask = 0
+        for _, r in self.samples:
+            mask |= int(r)
+        reasons = [name for bit, name in REASON_BITS.items() if mask & bit and name != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (barrier and max over ranks only; no data-path collective)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def dist_init(ws, backend):
+    if ws <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(dist, values, device):
+    if dist is None:
+        return values
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle as it stands, on a bounded sample of tiles
+# ---------------------------------------------------------------------------
+
+def oracle_sample_rate(w: W.Workload, steps: int, budget_s: float, max_tiles: int = 256):
+    """Oracle steps/s on the host, estimated from `steps` steps of a tile
+    sample sized so the whole measurement takes about budget_s seconds."""
+    from oracle import oracle as O
+    rng = np.random.default_rng(12345)
+    # calibrate on one tile per arm
+    calib_tiles = np.array([0])
+    S0 = W.initial_state(w, calib_tiles)
+    slot0 = W.slot(w, 0, calib_tiles)
+    t0 = time.perf_counter()
+    for arm in w.arms:
+        cfg = O.OracleConfig(1, w.dk, w.dv, arm.bits, arm.group, w.delta, w.decay, arm.policy,
+                             arm.rounding)
+        st = O.init(cfg, S0)
+        O.step(st, *slot0, want_o=w.readout)
+    per_tile_step = max(time.perf_counter() - t0, 1e-6)
+    threads = O.num_threads()
+    n = int(budget_s * threads / (per_tile_step * max(steps, 1)))
+    n = max(threads, min(n, max_tiles, w.tiles))
+    tiles = np.sort(rng.choice(w.tiles, size=n, replace=False))
+    S0 = W.initial_state(w, tiles)
+    states = []
+    for arm in w.arms:
+        cfg = O.OracleConfig(n, w.dk, w.dv, arm.bits, arm.group, w.delta, w.decay, arm.policy,
+                             arm.rounding)
+        states.append(O.init(cfg, S0))
+    P = min(steps, 16)
+    pool = [W.slot(w, t, tiles) for t in range(P)]
+    t0 = time.perf_counter()
+    for t in range(steps):
+        inp = pool[t % P]
+        for st in states:
+            O.step(st, *inp, want_o=w.readout)
+    dt = time.perf_counter() - t0
+    rate = (n / w.tiles) * steps / dt
+    sample = f"{n} of {w.tiles} tiles (seeded random), {steps} steps, all {len(w.arms)} arms"
+    return rate, threads, sample, dt
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = dist_init(ws, "nccl")
+
+    from ssm_decode_step_b200 import Config, QState, qstate as Q
+    Q.lib()
+    w = W.get(args.workload)
+    arms = list(w.arms)
+    K, Wm = args.steps, args.warmup
+    readout = w.readout
+
+    # input pool on the device: P slots of (q, k, v, alpha, beta)
+    P = args.pool
+    host = W.pool(w, P)
+    pool = [torch.from_numpy(a).to(dev) for a in host]
+
+    # request groups so that all groups' states exceed 2x L2
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    per_group = sum(state_bytes(w, a) for a in arms)
+    G = args.groups or max(1, -(-2 * l2 // per_group))
+    while P % G:
+        G += 1
+    S0 = torch.from_numpy(W.initial_state(w)).to(dev)
+
+    cfgs = [Config(w.tiles, w.dk, w.dv, a.bits, a.group, w.delta, w.decay, a.policy, a.rounding)
+            for a in arms]
+    states = [[QState(c, dev) for _ in range(G)] for c in cfgs]
+    outs = [torch.empty((w.tiles, w.dv), dtype=torch.float32, device=dev) if readout else None
+            for _ in arms]
+
+    def reinit():
+        for ai, c in enumerate(cfgs):
+            for g in range(G):
+                states[ai][g].init(S0)
+
+    def launch(ai, t):
+        s = t % P
+        st = states[ai][t % G]
+        st.step(pool[0][s], pool[1][s], pool[2][s], pool[3][s], pool[4][s], outs[ai])
+
+    stream = torch.cuda.Stream(device=dev)
+    reinit()
+    torch.cuda.synchronize()
+    # warm-up, eager
+    with torch.cuda.stream(stream):
+        for t in range(Wm):
+            for ai in range(len(arms)):
+                launch(ai, t)
+    stream.synchronize()
+
+    # graphs of P steps per arm (one full cycle of groups and slots), and a tail
+    n_main, tail = divmod(K, P)
+
+    def capture(ai, nsteps):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for t in range(nsteps):
+                launch(ai, t)
+        return g
+
+    graphs = [capture(ai, P) for ai in range(len(arms))]
+    tails = [capture(ai, tail) if tail else None for ai in range(len(arms))]
+    # warm the graph path, then restart every state from S0
+    with torch.cuda.stream(stream):
+        for ai in range(len(arms)):
+            graphs[ai].replay()
+    stream.synchronize()
+    reinit()
+    torch.cuda.synchronize()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in arms]
+    sampler = ClockSampler(local)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        with torch.cuda.stream(stream):
+            for ai in range(len(arms)):
+                ev[ai][0].record(stream)
+                for _ in range(n_main):
+                    graphs[ai].replay()
+                if tails[ai] is not None:
+                    tails[ai].replay()
+                ev[ai][1].record(stream)
+        stream.synchronize()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    arm_ms = [a.elapsed_time(b) for a, b in ev]
+    arm_ms = max_over_ranks(dist, arm_ms, dev)
+    total_ms = sum(arm_ms)
+    clocks = sampler.summary()
+
+    # ---- end to end through the public API with host buffers
+    e2e = run_e2e(args, w, arms, cfgs, states, dev, stream, dist, host, reinit)
+
+    peak, peak_src = load_peak()
+    bytes_step = sum(arm_bytes(w, a, readout) for a in arms)
+    value = ws * K / (total_ms / 1e3)
+    gbs = bytes_step * K / (total_ms / 1e3) / 1e9
+    dom = int(np.argmax(arm_ms))
+    dom_bytes = arm_bytes(w, arms[dom], readout)
+    dom_s = arm_ms[dom] / 1e3 / K
+    achieved = dom_bytes / dom_s / 1e9
+    kernel_key = f"{w.name}:{arms[dom].name}"
+    traffic = load_traffic(kernel_key)
+    per_arm = {}
+    for ai, a in enumerate(arms):
+        s = arm_ms[ai] / 1e3 / K
+        b = arm_bytes(w, a, readout)
+        per_arm[a.name] = {"us_per_launch": round(s * 1e6, 3), "bytes_per_launch": b,
+                           "gbs": round(b / s / 1e9, 1), "frac": round(b / s / 1e9 / peak, 4),
+                           "traffic": load_traffic(f"{w.name}:{a.name}")}
+
+    line = {
+        "metric": "quantized-state decode steps/sec; state GB/s as fraction of B200 HBM peak",
+        "value": round(value, 2),
+        "unit": "steps/s",
+        "n_gpus": ws,
+        "steps": K,
+        "warmup": Wm,
+        "ms_per_step": round(total_ms / K, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded; shapes and value laws of the workload)",
+        "config": {
+            "workload": w.description,
+            "tiles": w.tiles,
+            "step": f"one token for all {w.tiles} tiles under each arm ({len(arms)} launches)",
+            "arms": [a.name for a in arms],
+            "readout": readout,
+            "l2": f"inputs larger than L2: {G} request groups x {per_group / 1e6:.1f} MB state "
+                  f"+ {P} input slots rotated (L2 {l2 / 1e6:.0f} MB)",
+            "parallelism": f"independent tile shards, {ws} GPU(s), no collective on the step",
+        },
+        "state_gbs": round(gbs, 1),
+        "state_frac": round(gbs / peak, 4),
+        "arms": per_arm,
+        "roofline": {
+            "bound": "hbm",
+            "kernel": f"step_kernel ({kernel_key})",
+            "achieved": round(achieved, 1),
+            "peak": peak,
+            "peak_source": peak_src,
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": traffic,
+            "algorithmic_bytes_per_launch": dom_bytes,
+        },
+        "e2e": e2e,
+        "gpu_launches": K * len(arms),
+        "clocks": clocks,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        rate, threads, sample, dt = oracle_sample_rate(w, steps=4, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(rate, 4), "unit": "steps/s", "cores": threads,
+                                "kind": "oracle", "sample": sample, "seconds": round(dt, 2)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for g in graphs + [t for t in tails if t is not None]:
+        del g
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def run_e2e(args, w, arms, cfgs, states, dev, stream, dist, host, reinit):
+    """Same steps through the public API with host buffers: per step, copy
+    the inputs from pinned host memory, launch every arm, copy the readouts
+    back; all inside the timed region."""
+    import torch
+
+    K = min(args.steps, args.e2e_steps)
+    P = args.pool
+    G = len(states[0])
+    T = w.tiles
+    # one packed pinned buffer per slot: q | k | v | alpha | beta
+    parts = [np.ascontiguousarray(a) for a in host]
+    sizes = [a[0].size for a in parts]
+    packed = torch.empty((P, sum(sizes)), dtype=torch.float32).pin_memory()
+    for s in range(P):
+        packed[s] = torch.from_numpy(np.concatenate([a[s].reshape(-1) for a in parts]))
+    dbuf = torch.empty(sum(sizes), dtype=torch.float32, device=dev)
+    views, off = [], 0
+    for a, n in zip(parts, sizes):
+        views.append(dbuf[off:off + n].view(a.shape[1:]))
+        off += n
+    readout = w.readout
+    o_dev = torch.empty((len(arms), T, w.dv), dtype=torch.float32, device=dev)
+    o_host = torch.empty((len(arms), T, w.dv), dtype=torch.float32).pin_memory()
+
+    def one(t):
+        dbuf.copy_(packed[t % P], non_blocking=True)
+        for ai in range(len(arms)):
+            states[ai][t % G].step(views[0] if readout else None, views[1], views[2], views[3],
+                                   views[4], o_dev[ai] if readout else None)
+        if readout:
+            o_host.copy_(o_dev, non_blocking=True)
+
+    reinit()
+    with torch.cuda.stream(stream):
+        for t in range(max(3, args.warmup)):
+            one(t)
+    stream.synchronize()
+    reinit()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for t in range(K):
+            one(t)
+        e1.record(stream)
+    stream.synchronize()
+    ms = max_over_ranks(dist, [e0.elapsed_time(e1)], dev)[0]
+    ws = dist.get_world_size() if dist is not None else 1
+    return {"value": round(ws * K / (ms / 1e3), 2), "unit": "steps/s",
+            "h2d_bytes_per_step": int(sum(sizes) * 4),
+            "d2h_bytes_per_step": int(len(arms) * T * w.dv * 4) if readout else 0,
+            "steps": K}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    w = W.get(args.workload)
+    from oracle import oracle as O
+    # warm-up on a single tile (untimed), then the timed steps on a sample
+    rate, threads, sample, dt = oracle_sample_rate(w, steps=args.steps, budget_s=args.ref_budget)
+    peak, _ = load_peak()
+    bytes_step = sum(arm_bytes(w, a, w.readout) for a in w.arms)
+    line = {
+        "impl": "reference",
+        "metric": "quantized-state decode steps/sec; state GB/s as fraction of B200 HBM peak",
+        "value": round(rate, 4),
+        "unit": "steps/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(1e3 / rate, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded; shapes and value laws of the workload)",
+        "config": {"workload": w.description, "tiles": w.tiles,
+                   "step": f"one token for all {w.tiles} tiles under each arm ({len(w.arms)} arms)",
+                   "arms": [a.name for a in w.arms]},
+        "state_gbs": round(bytes_step * rate / 1e9, 3),
+        "cpu_baseline": {"value": round(rate, 4), "unit": "steps/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(rate, 4), "unit": "steps/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=8192,
+                    help="timed steps (default: 4 request groups x the 2048-token horizon)")
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="gdn", choices=list(W.WORKLOADS))
+    ap.add_argument("--pool", type=int, default=64, help="input slots on the device")
+    ap.add_argument("--groups", type=int, default=0, help="request groups (0: enough to exceed 2x L2)")
+    ap.add_argument("--e2e-steps", type=int, default=1024)
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
+    ap.add_argument("--ref-budget", type=float, default=90.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

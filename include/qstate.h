@@ -1,0 +1,168 @@
+/*
+ * qstate — quantized recurrent-state decode step for NVIDIA B200 (sm_100a).
+ *
+ * One decode step of the linear recurrence of "LinQuant: Functional
+ * Invariances for Low-Precision Linear Recurrences" (Theoretical
+ * Foundation, eq. (1)):
+ *
+ *     S_t = S_{t-1} Lambda_t (I - delta beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *
+ * with readout o_t = S_t q_t (same page, Low-Precision Chunkwise
+ * Realization, "state read").  S is a Dv x Dk matrix per tile, one tile
+ * per (layer, batch, head); tiles are independent.  The state lives in
+ * device memory as group-wise INT4 or INT8 codes plus one FP32 scale per
+ * group of `group` consecutive columns of a row, and every step
+ * dequantizes, decays, writes, reads out and requantizes it in one pass
+ * (a quantizer applied inside the recurrence: "When Dynamic Scaling
+ * Fails", abstract).
+ *
+ * Element-level definition (FP32, IEEE round to nearest even; "fused"
+ * means one rounding), for tile t, row i, column j, group g = j / group:
+ *   d_ij  = c_ij * s_ig                      dequantized previous state
+ *   S'_ij = d_ij * a_j                       a_j = alpha_t (QS_DECAY_SCALAR)
+ *                                            or alpha_tj (QS_DECAY_DIAGONAL)
+ *   w_i   = beta_t * (v_i - u_i), u_i = S'_i . k   (delta = 1)
+ *   w_i   = beta_t * v_i                           (delta = 0)
+ *   x_ij  = fused(w_i * k_j + S'_ij)         updated state
+ *   o_i   = x_i . q                          readout, before requantization
+ *   s'_ig = max_{j in g} |x_ij| / qmax       QS_SCALE_DYNAMIC
+ *         = s_ig                             QS_SCALE_PERSISTENT
+ *         = max_{j in g} |R_ij| / qmax       QS_SCALE_YOKED, R = FP32 shadow
+ *                                            updated by the same steps
+ *   if s'_ig > 0: n_ij = clamp(round_half_even(x_ij * (1/s'_ig)), +-qmax),
+ *                 the product taken exactly; else n_ij = 0 for the group
+ *   BDR: with sigma = sign(w_i) sign(k_j), if sigma > 0 and n s' < S'_ij
+ *        then n += 1; if sigma < 0 and n s' > S'_ij then n -= 1; clamp.
+ *        ("Preserving Updates in Low-Bit Recurrent State Quantization",
+ *        abstract: elements whose rounding moves against their update are
+ *        rounded one step toward it.)
+ * qmax = 2^(bits-1) - 1.  Dot products "." are evaluated in one fixed
+ * order: Dk/16 segments of 16 consecutive columns, each a fused
+ * multiply-add chain from +0 in column order, summed by a balanced
+ * pairwise tree.  Codes, scales and the shadow are therefore reproducible
+ * bit for bit on any conforming implementation.
+ *
+ * Scale policies ("When Dynamic Scaling Fails", project page): per-token
+ * dynamic reads its scale from the state it is about to quantize;
+ * persistent fixes the scale at the quantization start (qstate_init) and
+ * clips; yoked takes it from a full-precision reference run alongside.
+ *
+ * Memory layout (all row-major, tile-major, no padding):
+ *   codes   [T][Dv][Dk*bits/8] bytes, two's complement; INT4 packs the even
+ *           column in the low nibble of each byte
+ *   scales  [T][Dv][Dk/group]  float
+ *   shadow  [T][Dv][Dk]        float   (QS_SCALE_YOKED only)
+ *   q, k    [T][Dk]            float
+ *   v       [T][Dv]            float
+ *   alpha   [T] (scalar decay) or [T][Dk] (diagonal decay)  float
+ *   beta    [T]                float
+ *   o       [T][Dv]            float
+ *
+ * Conventions for every entry point:
+ *   - All array pointers are DEVICE pointers owned by the caller; the
+ *     library allocates no memory and keeps no state between calls.
+ *   - codes, scales, shadow are updated in place; other inputs are read.
+ *   - Work is enqueued on `stream` and returns immediately; QS_OK means
+ *     "validated and launched".  Execution errors surface at the caller's
+ *     next synchronization on that stream.
+ *   - Arguments are validated before anything is launched.  A NULL
+ *     required pointer, a misaligned pointer (codes, shadow: 32 bytes;
+ *     S0, scales, q, k, v, alpha when diagonal: 16 bytes; alpha when
+ *     scalar, beta, o: 4 bytes), overlapping buffers, or an out-of-range field
+ *     returns QS_ERR_INVALID_ARG; a valid configuration this build has no
+ *     kernel for returns QS_ERR_UNSUPPORTED; a failed launch returns
+ *     QS_ERR_CUDA.  Nothing aborts or throws across this boundary.
+ *   - Values: beta > 0 and |Lambda| <= 1 are the caller's contract and are
+ *     not checked.  Non-finite inputs give unspecified codes but every
+ *     access stays in bounds.
+ *   - Calls that overlap on the GPU must not share state buffers.
+ *
+ * Supported by this build: dk in {64, 128}; dv a multiple of 16 with
+ * 16 <= dv <= 128 (dk = 128) or <= 256 (dk = 64); bits in {4, 8};
+ * group in {32, 64, 128} with group <= dk; any num_tiles >= 0.
+ */
+#ifndef QSTATE_H
+#define QSTATE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define QS_API __attribute__((visibility("default")))
+#else
+#define QS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QS_OK = 0,
+  QS_ERR_INVALID_ARG = 1,
+  QS_ERR_UNSUPPORTED = 2,
+  QS_ERR_CUDA = 3
+} qs_status;
+
+typedef enum { QS_DECAY_SCALAR = 0, QS_DECAY_DIAGONAL = 1 } qs_decay;
+typedef enum {
+  QS_SCALE_DYNAMIC = 0,
+  QS_SCALE_PERSISTENT = 1,
+  QS_SCALE_YOKED = 2
+} qs_policy;
+typedef enum { QS_ROUND_NEAREST = 0, QS_ROUND_BDR = 1 } qs_rounding;
+
+/* Configuration of one family of states (eq. (1) choices + storage).
+ * Fixed-width fields so the layout is the same from any language. */
+typedef struct {
+  int32_t num_tiles; /* layers * batch * heads; tiles are independent      */
+  int32_t dk;        /* key dimension (columns of S)                      */
+  int32_t dv;        /* value dimension (rows of S)                       */
+  int32_t bits;      /* 4 or 8                                            */
+  int32_t group;     /* quantization group length along dk                */
+  int32_t delta;     /* 0: linear write; 1: delta-rule correction         */
+  int32_t decay;     /* qs_decay: Lambda = alpha I or diag(alpha)          */
+  int32_t policy;    /* qs_policy                                          */
+  int32_t rounding;  /* qs_rounding                                        */
+} qs_config;
+
+/* Bytes of each state buffer for `cfg` (shadow_bytes is 0 unless yoked).
+ * Any of the output pointers may be NULL.  Host-only; launches nothing. */
+QS_API qs_status qstate_query_sizes(const qs_config* cfg, size_t* codes_bytes,
+                             size_t* scales_bytes, size_t* shadow_bytes);
+
+/* Quantization start: from the FP32 state S0 [T][Dv][Dk] (device), write
+ * codes and scales with the dynamic rule (scale = group max|S0| / qmax,
+ * nearest rounding) — under QS_SCALE_PERSISTENT these scales stay fixed
+ * from here on — and, for QS_SCALE_YOKED, copy S0 into the shadow.
+ * shadow is ignored (may be NULL) for the other policies. */
+QS_API qs_status qstate_init(const qs_config* cfg, const float* S0, void* codes,
+                      float* scales, float* shadow, cudaStream_t stream);
+
+/* One decode step, in place on (codes, scales, shadow), as defined above.
+ * q may be NULL only when o is NULL; o == NULL skips the readout.
+ * alpha is [T] for QS_DECAY_SCALAR and [T][Dk] for QS_DECAY_DIAGONAL. */
+QS_API qs_status qstate_decode_step(const qs_config* cfg, void* codes, float* scales,
+                             float* shadow, const float* q, const float* k,
+                             const float* v, const float* alpha,
+                             const float* beta, float* o, cudaStream_t stream);
+
+/* Readout of the stored state without changing it: o_i = d_i . q with
+ * d_ij = c_ij * s_ig (the fixed dot order above). */
+QS_API qs_status qstate_readout(const qs_config* cfg, const void* codes,
+                         const float* scales, const float* q, float* o,
+                         cudaStream_t stream);
+
+/* Static, human-readable name of a status code. */
+QS_API const char* qstate_status_string(qs_status status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+QS_API int qstate_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QSTATE_H */

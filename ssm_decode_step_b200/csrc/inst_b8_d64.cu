@@ -1,0 +1,6 @@
+// Kernel instances for 8-bit codes and Dk = 64.
+#include "qstate_launch_impl.cuh"
+
+namespace qs {
+QS_INSTANTIATE_ALL(8, 64)
+}  // namespace qs

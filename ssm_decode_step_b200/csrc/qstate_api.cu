@@ -1,0 +1,238 @@
+// The C ABI of include/qstate.h: argument validation and dispatch to the
+// compile-time kernel instances.  No memory is allocated here; the only
+// process-wide state is the per-device SM count and the once-per-kernel
+// shared-memory attribute.
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/qstate.h"
+#include "qstate_launch.h"
+
+namespace qs {
+
+int device_sm_count() {
+  static std::mutex mu;
+  static int counts[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
+  std::lock_guard<std::mutex> lock(mu);
+  if (counts[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 1;
+    counts[dev] = n;
+  }
+  return counts[dev];
+}
+
+}  // namespace qs
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct Range {
+  uintptr_t lo, hi;  // [lo, hi)
+};
+
+Range range_of(const void* p, size_t bytes) {
+  const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+  return {lo, lo + bytes};
+}
+
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi && a.hi > a.lo && b.hi > b.lo; }
+
+// Field ranges of the configuration; 0 = fine, else the status to return.
+qs_status check_config(const qs_config* c) {
+  if (c == nullptr) return QS_ERR_INVALID_ARG;
+  if (c->num_tiles < 0) return QS_ERR_INVALID_ARG;
+  if (c->dk < 1 || c->dv < 1) return QS_ERR_INVALID_ARG;
+  if (c->bits != 4 && c->bits != 8) return QS_ERR_INVALID_ARG;
+  if (c->group < 1 || c->dk % c->group != 0) return QS_ERR_INVALID_ARG;
+  if (c->delta != 0 && c->delta != 1) return QS_ERR_INVALID_ARG;
+  if (c->decay != QS_DECAY_SCALAR && c->decay != QS_DECAY_DIAGONAL) return QS_ERR_INVALID_ARG;
+  if (c->policy != QS_SCALE_DYNAMIC && c->policy != QS_SCALE_PERSISTENT && c->policy != QS_SCALE_YOKED)
+    return QS_ERR_INVALID_ARG;
+  if (c->rounding != QS_ROUND_NEAREST && c->rounding != QS_ROUND_BDR) return QS_ERR_INVALID_ARG;
+  // what this build has kernels for
+  if (c->dk != 64 && c->dk != 128) return QS_ERR_UNSUPPORTED;
+  if (c->dv % 16 != 0 || c->dv * (c->dk / 32) > qs::kMaxThreads) return QS_ERR_UNSUPPORTED;
+  if (c->group != 32 && c->group != 64 && c->group != 128) return QS_ERR_UNSUPPORTED;
+  return QS_OK;
+}
+
+struct Sizes {
+  size_t codes, scales, shadow, vec_k, vec_v, alpha, tile_scalars;
+};
+
+Sizes sizes_of(const qs_config* c) {
+  const size_t T = static_cast<size_t>(c->num_tiles);
+  Sizes s;
+  s.codes = T * c->dv * c->dk * c->bits / 8;
+  s.scales = T * c->dv * (c->dk / c->group) * sizeof(float);
+  s.shadow = c->policy == QS_SCALE_YOKED ? T * c->dv * c->dk * sizeof(float) : 0;
+  s.vec_k = T * c->dk * sizeof(float);
+  s.vec_v = T * c->dv * sizeof(float);
+  s.alpha = c->decay == QS_DECAY_DIAGONAL ? s.vec_k : T * sizeof(float);
+  s.tile_scalars = T * sizeof(float);
+  return s;
+}
+
+qs_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QS_OK : QS_ERR_CUDA; }
+
+// Written buffers must not overlap each other or any input.
+bool any_overlap(const Range* written, int nw, const Range* read, int nr) {
+  for (int i = 0; i < nw; ++i) {
+    for (int j = i + 1; j < nw; ++j)
+      if (overlap(written[i], written[j])) return true;
+    for (int j = 0; j < nr; ++j)
+      if (overlap(written[i], read[j])) return true;
+  }
+  return false;
+}
+
+template <int BITS, int DK>
+cudaError_t dispatch_step(const qs_config* c, const qs::StepParams& p, cudaStream_t s) {
+  const bool bdr = c->rounding == QS_ROUND_BDR, delta = c->delta == 1, diag = c->decay == QS_DECAY_DIAGONAL;
+  const int sel = (c->policy * 8) + (bdr ? 4 : 0) + (delta ? 2 : 0) + (diag ? 1 : 0);
+  using namespace qs;
+  switch (sel) {
+#define QS_CASE(P, R, DE, DI) \
+  case (P * 8 + R * 4 + DE * 2 + DI): return launch_step<BITS, DK, P, R, DE, DI>(p, s);
+    QS_CASE(0, 0, 0, 0) QS_CASE(0, 0, 0, 1) QS_CASE(0, 0, 1, 0) QS_CASE(0, 0, 1, 1)
+    QS_CASE(0, 1, 0, 0) QS_CASE(0, 1, 0, 1) QS_CASE(0, 1, 1, 0) QS_CASE(0, 1, 1, 1)
+    QS_CASE(1, 0, 0, 0) QS_CASE(1, 0, 0, 1) QS_CASE(1, 0, 1, 0) QS_CASE(1, 0, 1, 1)
+    QS_CASE(1, 1, 0, 0) QS_CASE(1, 1, 0, 1) QS_CASE(1, 1, 1, 0) QS_CASE(1, 1, 1, 1)
+    QS_CASE(2, 0, 0, 0) QS_CASE(2, 0, 0, 1) QS_CASE(2, 0, 1, 0) QS_CASE(2, 0, 1, 1)
+    QS_CASE(2, 1, 0, 0) QS_CASE(2, 1, 0, 1) QS_CASE(2, 1, 1, 0) QS_CASE(2, 1, 1, 1)
+#undef QS_CASE
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int qstate_version(void) { return 100; }
+
+const char* qstate_status_string(qs_status s) {
+  switch (s) {
+    case QS_OK: return "ok";
+    case QS_ERR_INVALID_ARG: return "invalid argument";
+    case QS_ERR_UNSUPPORTED: return "configuration not supported by this build";
+    case QS_ERR_CUDA: return "CUDA launch error";
+  }
+  return "unknown status";
+}
+
+qs_status qstate_query_sizes(const qs_config* cfg, size_t* codes_bytes, size_t* scales_bytes,
+                             size_t* shadow_bytes) {
+  const qs_status st = check_config(cfg);
+  if (st != QS_OK) return st;
+  const Sizes s = sizes_of(cfg);
+  if (codes_bytes) *codes_bytes = s.codes;
+  if (scales_bytes) *scales_bytes = s.scales;
+  if (shadow_bytes) *shadow_bytes = s.shadow;
+  return QS_OK;
+}
+
+qs_status qstate_init(const qs_config* cfg, const float* S0, void* codes, float* scales,
+                      float* shadow, cudaStream_t stream) {
+  qs_status st = check_config(cfg);
+  if (st != QS_OK) return st;
+  const bool yoked = cfg->policy == QS_SCALE_YOKED;
+  if (cfg->num_tiles == 0) return QS_OK;
+  if (!S0 || !codes || !scales || (yoked && !shadow)) return QS_ERR_INVALID_ARG;
+  if (!aligned(S0, 16) || !aligned(codes, 32) || !aligned(scales, 16) || (yoked && !aligned(shadow, 32)))
+    return QS_ERR_INVALID_ARG;
+  const Sizes s = sizes_of(cfg);
+  const Range w[3] = {range_of(codes, s.codes), range_of(scales, s.scales),
+                      range_of(yoked ? shadow : nullptr, s.shadow)};
+  const Range r[1] = {range_of(S0, static_cast<size_t>(cfg->num_tiles) * cfg->dv * cfg->dk * 4)};
+  if (any_overlap(w, 3, r, 1)) return QS_ERR_INVALID_ARG;
+  const long long rows = static_cast<long long>(cfg->num_tiles) * cfg->dv;
+  uint8_t* c8 = static_cast<uint8_t*>(codes);
+  float* sh = yoked ? shadow : nullptr;
+  cudaError_t e;
+  if (cfg->bits == 4)
+    e = cfg->dk == 64 ? qs::launch_init<4, 64>(S0, c8, scales, sh, rows, cfg->group, stream)
+                      : qs::launch_init<4, 128>(S0, c8, scales, sh, rows, cfg->group, stream);
+  else
+    e = cfg->dk == 64 ? qs::launch_init<8, 64>(S0, c8, scales, sh, rows, cfg->group, stream)
+                      : qs::launch_init<8, 128>(S0, c8, scales, sh, rows, cfg->group, stream);
+  return from_cuda(e);
+}
+
+qs_status qstate_decode_step(const qs_config* cfg, void* codes, float* scales, float* shadow,
+                             const float* q, const float* k, const float* v, const float* alpha,
+                             const float* beta, float* o, cudaStream_t stream) {
+  qs_status st = check_config(cfg);
+  if (st != QS_OK) return st;
+  if (cfg->num_tiles == 0) return QS_OK;
+  const bool yoked = cfg->policy == QS_SCALE_YOKED;
+  const bool diag = cfg->decay == QS_DECAY_DIAGONAL;
+  if (!codes || !scales || !k || !v || !alpha || !beta || (yoked && !shadow) || (o && !q))
+    return QS_ERR_INVALID_ARG;
+  if (!aligned(codes, 32) || !aligned(scales, 16) || !aligned(k, 16) || !aligned(v, 16) ||
+      (q && !aligned(q, 16)) || (yoked && !aligned(shadow, 32)) || !aligned(alpha, diag ? 16 : 4) ||
+      !aligned(beta, 4) || (o && !aligned(o, 4)))
+    return QS_ERR_INVALID_ARG;
+  const Sizes s = sizes_of(cfg);
+  const Range w[4] = {range_of(codes, s.codes), range_of(scales, s.scales),
+                      range_of(yoked ? shadow : nullptr, s.shadow), range_of(o, o ? s.vec_v : 0)};
+  const Range r[5] = {range_of(q, q ? s.vec_k : 0), range_of(k, s.vec_k), range_of(v, s.vec_v),
+                      range_of(alpha, s.alpha), range_of(beta, s.tile_scalars)};
+  if (any_overlap(w, 4, r, 5)) return QS_ERR_INVALID_ARG;
+
+  qs::StepParams p;
+  p.codes = static_cast<uint8_t*>(codes);
+  p.scales = scales;
+  p.shadow = yoked ? shadow : nullptr;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.alpha = alpha;
+  p.beta = beta;
+  p.o = o;
+  p.tiles = cfg->num_tiles;
+  p.dv = cfg->dv;
+  p.group = cfg->group;
+  cudaError_t e;
+  if (cfg->bits == 4)
+    e = cfg->dk == 64 ? dispatch_step<4, 64>(cfg, p, stream) : dispatch_step<4, 128>(cfg, p, stream);
+  else
+    e = cfg->dk == 64 ? dispatch_step<8, 64>(cfg, p, stream) : dispatch_step<8, 128>(cfg, p, stream);
+  return from_cuda(e);
+}
+
+qs_status qstate_readout(const qs_config* cfg, const void* codes, const float* scales,
+                         const float* q, float* o, cudaStream_t stream) {
+  qs_status st = check_config(cfg);
+  if (st != QS_OK) return st;
+  if (cfg->num_tiles == 0) return QS_OK;
+  if (!codes || !scales || !q || !o) return QS_ERR_INVALID_ARG;
+  if (!aligned(codes, 32) || !aligned(scales, 16) || !aligned(q, 16) || !aligned(o, 4))
+    return QS_ERR_INVALID_ARG;
+  const Sizes s = sizes_of(cfg);
+  const Range w[1] = {range_of(o, s.vec_v)};
+  const Range r[3] = {range_of(codes, s.codes), range_of(scales, s.scales), range_of(q, s.vec_k)};
+  if (any_overlap(w, 1, r, 3)) return QS_ERR_INVALID_ARG;
+  qs::StepParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.codes = const_cast<uint8_t*>(static_cast<const uint8_t*>(codes));
+  p.scales = const_cast<float*>(scales);
+  p.q = q;
+  p.o = o;
+  p.tiles = cfg->num_tiles;
+  p.dv = cfg->dv;
+  p.group = cfg->group;
+  cudaError_t e;
+  if (cfg->bits == 4)
+    e = cfg->dk == 64 ? qs::launch_readout<4, 64>(p, stream) : qs::launch_readout<4, 128>(p, stream);
+  else
+    e = cfg->dk == 64 ? qs::launch_readout<8, 64>(p, stream) : qs::launch_readout<8, 128>(p, stream);
+  return from_cuda(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,96 @@
+// Definitions of the launchers declared in qstate_launch.h.
+#pragma once
+
+#include <mutex>
+
+#include "qstate_launch.h"
+
+namespace qs {
+
+// Stages of the cp.async ring: the yoked state carries a 64 KB FP32 shadow per
+// tile, so it keeps two stages; the others keep four.
+template <int POLICY>
+constexpr int step_stages() { return POLICY == 2 ? 2 : 4; }
+
+// Allow the kernel the device's full opt-in shared memory (once per kernel).
+template <typename K>
+static cudaError_t allow_smem(K kernel, std::once_flag& flag) {
+  cudaError_t err = cudaSuccess;
+  std::call_once(flag, [&] {
+    int dev = 0, optin = 0;
+    err = cudaGetDevice(&dev);
+    if (err == cudaSuccess) err = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (err == cudaSuccess)
+      err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  });
+  return err;
+}
+
+template <typename K>
+static cudaError_t launch_persistent(K kernel, int tiles, int threads, size_t smem,
+                                     const StepParams& p, cudaStream_t stream) {
+  int per_sm = 0;
+  cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem);
+  if (err != cudaSuccess) return err;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  long long grid = static_cast<long long>(per_sm) * device_sm_count();
+  if (grid > tiles) grid = tiles;
+  kernel<<<static_cast<int>(grid), threads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <int BITS, int DK, int POLICY, bool BDR, bool DELTA, bool DIAG>
+cudaError_t launch_step(const StepParams& p, cudaStream_t stream) {
+  constexpr int S = step_stages<POLICY>();
+  auto kernel = step_kernel<BITS, DK, POLICY, BDR, DELTA, DIAG, S>;
+  static std::once_flag flag;
+  cudaError_t err = allow_smem(kernel, flag);
+  if (err != cudaSuccess) return err;
+  const StageLayout L(BITS, DK, p.dv, p.group, DIAG, BDR, POLICY == 2);
+  return launch_persistent(kernel, p.tiles, p.dv * (DK / 32), static_cast<size_t>(S) * L.bytes, p,
+                           stream);
+}
+
+template <int BITS, int DK>
+cudaError_t launch_readout(const StepParams& p, cudaStream_t stream) {
+  constexpr int S = 4;
+  auto kernel = readout_kernel<BITS, DK, S>;
+  static std::once_flag flag;
+  cudaError_t err = allow_smem(kernel, flag);
+  if (err != cudaSuccess) return err;
+  const StageLayout L(BITS, DK, p.dv, p.group, false, false, false);
+  return launch_persistent(kernel, p.tiles, p.dv * (DK / 32), static_cast<size_t>(S) * L.bytes, p,
+                           stream);
+}
+
+template <int BITS, int DK>
+cudaError_t launch_init(const float* S0, uint8_t* codes, float* scales, float* shadow,
+                        long long rows, int group, cudaStream_t stream) {
+  const long long threads = rows * (DK / 32);
+  const long long blocks = (threads + 255) / 256;
+  init_kernel<BITS, DK><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(S0, codes, scales, shadow,
+                                                                         rows, group);
+  return cudaGetLastError();
+}
+
+#define QS_INSTANTIATE_STEP(B, D, P, R, DE, DI) \
+  template cudaError_t launch_step<B, D, P, R, DE, DI>(const StepParams&, cudaStream_t);
+
+#define QS_INSTANTIATE_ALL(B, D)                                                      \
+  QS_INSTANTIATE_STEP(B, D, 0, false, false, false) QS_INSTANTIATE_STEP(B, D, 0, false, false, true) \
+  QS_INSTANTIATE_STEP(B, D, 0, false, true, false)  QS_INSTANTIATE_STEP(B, D, 0, false, true, true)  \
+  QS_INSTANTIATE_STEP(B, D, 0, true, false, false)  QS_INSTANTIATE_STEP(B, D, 0, true, false, true)  \
+  QS_INSTANTIATE_STEP(B, D, 0, true, true, false)   QS_INSTANTIATE_STEP(B, D, 0, true, true, true)   \
+  QS_INSTANTIATE_STEP(B, D, 1, false, false, false) QS_INSTANTIATE_STEP(B, D, 1, false, false, true) \
+  QS_INSTANTIATE_STEP(B, D, 1, false, true, false)  QS_INSTANTIATE_STEP(B, D, 1, false, true, true)  \
+  QS_INSTANTIATE_STEP(B, D, 1, true, false, false)  QS_INSTANTIATE_STEP(B, D, 1, true, false, true)  \
+  QS_INSTANTIATE_STEP(B, D, 1, true, true, false)   QS_INSTANTIATE_STEP(B, D, 1, true, true, true)   \
+  QS_INSTANTIATE_STEP(B, D, 2, false, false, false) QS_INSTANTIATE_STEP(B, D, 2, false, false, true) \
+  QS_INSTANTIATE_STEP(B, D, 2, false, true, false)  QS_INSTANTIATE_STEP(B, D, 2, false, true, true)  \
+  QS_INSTANTIATE_STEP(B, D, 2, true, false, false)  QS_INSTANTIATE_STEP(B, D, 2, true, false, true)  \
+  QS_INSTANTIATE_STEP(B, D, 2, true, true, false)   QS_INSTANTIATE_STEP(B, D, 2, true, true, true)   \
+  template cudaError_t launch_readout<B, D>(const StepParams&, cudaStream_t);        \
+  template cudaError_t launch_init<B, D>(const float*, uint8_t*, float*, float*, long long, int, \
+                                         cudaStream_t);
+
+}  // namespace qs

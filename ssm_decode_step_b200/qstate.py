@@ -1,0 +1,176 @@
+"""Python binding of the qstate C ABI (include/qstate.h).
+
+Argument marshalling only: every step of the decode path runs in the CUDA
+kernels of libqstate.so.  Tensors are torch CUDA tensors (PyTorch supplies
+device memory and streams); their data pointers and the current CUDA stream
+are handed to the library.  There is no CPU fallback: if libqstate.so is
+missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqstate.so")
+
+DECAY = {"scalar": 0, "diagonal": 1}
+POLICY = {"dynamic": 0, "persistent": 1, "yoked": 2}
+ROUNDING = {"nearest": 0, "bdr": 1}
+
+QS_OK, QS_ERR_INVALID_ARG, QS_ERR_UNSUPPORTED, QS_ERR_CUDA = 0, 1, 2, 3
+
+# Every entry point that include/qstate.h declares.
+EXPORTS = ("qstate_query_sizes", "qstate_init", "qstate_decode_step", "qstate_readout",
+           "qstate_status_string", "qstate_version")
+
+
+class QStateError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+class qs_config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "num_tiles", "dk", "dv", "bits", "group", "delta", "decay", "policy", "rounding")]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libqstate.so (built by ssm_decode_step_b200/build.py)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: run `python -m ssm_decode_step_b200.build` "
+                              "(or __graft_entry__.build()) first")
+        L = ctypes.CDLL(LIB_PATH)
+        P, C = ctypes.c_void_p, ctypes.POINTER(qs_config)
+        sz = ctypes.POINTER(ctypes.c_size_t)
+        L.qstate_query_sizes.argtypes = [C, sz, sz, sz]
+        L.qstate_init.argtypes = [C, P, P, P, P, P]
+        L.qstate_decode_step.argtypes = [C, P, P, P, P, P, P, P, P, P, P]
+        L.qstate_readout.argtypes = [C, P, P, P, P, P]
+        for f in (L.qstate_query_sizes, L.qstate_init, L.qstate_decode_step, L.qstate_readout):
+            f.restype = ctypes.c_int
+        L.qstate_status_string.argtypes = [ctypes.c_int]
+        L.qstate_status_string.restype = ctypes.c_char_p
+        L.qstate_version.argtypes = []
+        L.qstate_version.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().qstate_status_string(status).decode()
+
+
+@dataclass(frozen=True)
+class Config:
+    """One family of quantized states (the fields of qs_config)."""
+    num_tiles: int
+    dk: int
+    dv: int
+    bits: int
+    group: int
+    delta: int
+    decay: str = "scalar"
+    policy: str = "persistent"
+    rounding: str = "nearest"
+
+    def c(self) -> qs_config:
+        return qs_config(self.num_tiles, self.dk, self.dv, self.bits, self.group, self.delta,
+                         DECAY[self.decay], POLICY[self.policy], ROUNDING[self.rounding])
+
+    @property
+    def groups(self) -> int:
+        return self.dk // self.group
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, what: str) -> None:
+    if status != QS_OK:
+        raise QStateError(status, what)
+
+
+def query_sizes(cfg: Config):
+    """(codes_bytes, scales_bytes, shadow_bytes) for cfg."""
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    cc = cfg.c()
+    _check(lib().qstate_query_sizes(ctypes.byref(cc), ctypes.byref(a), ctypes.byref(b),
+                                    ctypes.byref(c)), "qstate_query_sizes")
+    return a.value, b.value, c.value
+
+
+def init(cfg: Config, S0, codes, scales, shadow=None, stream=None) -> None:
+    cc = cfg.c()
+    _check(lib().qstate_init(ctypes.byref(cc), _ptr(S0), _ptr(codes), _ptr(scales), _ptr(shadow),
+                             _stream(stream)), "qstate_init")
+
+
+def decode_step(cfg: Config, codes, scales, shadow, q, k, v, alpha, beta, o=None,
+                stream=None) -> None:
+    cc = cfg.c()
+    _check(lib().qstate_decode_step(ctypes.byref(cc), _ptr(codes), _ptr(scales), _ptr(shadow),
+                                    _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(o),
+                                    _stream(stream)), "qstate_decode_step")
+
+
+def readout(cfg: Config, codes, scales, q, o, stream=None) -> None:
+    cc = cfg.c()
+    _check(lib().qstate_readout(ctypes.byref(cc), _ptr(codes), _ptr(scales), _ptr(q), _ptr(o),
+                                _stream(stream)), "qstate_readout")
+
+
+class QState:
+    """Device buffers of one quantized state family plus convenience calls.
+
+    Buffers are torch tensors on the current CUDA device:
+      codes  uint8 [T, dv, dk*bits/8], scales float32 [T, dv, dk/group],
+      shadow float32 [T, dv, dk] (yoked only).
+    """
+
+    def __init__(self, cfg: Config, device=None):
+        import torch
+        self.cfg = cfg
+        dev = torch.device("cuda") if device is None else torch.device(device)
+        T, dv, dk = cfg.num_tiles, cfg.dv, cfg.dk
+        self.codes = torch.empty((T, dv, dk * cfg.bits // 8), dtype=torch.uint8, device=dev)
+        self.scales = torch.empty((T, dv, cfg.groups), dtype=torch.float32, device=dev)
+        self.shadow = (torch.empty((T, dv, dk), dtype=torch.float32, device=dev)
+                       if cfg.policy == "yoked" else None)
+        cb, sb, hb = query_sizes(cfg)
+        assert cb == self.codes.numel() and sb == 4 * self.scales.numel()
+        assert hb == (0 if self.shadow is None else 4 * self.shadow.numel())
+
+    def init(self, S0, stream=None) -> "QState":
+        init(self.cfg, S0, self.codes, self.scales, self.shadow, stream)
+        return self
+
+    def step(self, q, k, v, alpha, beta, o=None, stream=None):
+        decode_step(self.cfg, self.codes, self.scales, self.shadow, q, k, v, alpha, beta, o, stream)
+        return o
+
+    def readout(self, q, o, stream=None):
+        readout(self.cfg, self.codes, self.scales, q, o, stream)
+        return o

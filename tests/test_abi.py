@@ -1,0 +1,128 @@
+"""The C ABI library: it loads, exports every entry point include/*.h
+declares, and rejects bad arguments before launching anything (so these
+run without a GPU)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from ssm_decode_step_b200 import qstate as Q
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        names += re.findall(r"QS_API\s+[\w\s\*]+?\b(qstate_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    declared = _declared()
+    assert declared, "no declarations found"
+    lib = Q.lib()
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(Q.EXPORTS) >= set(declared)
+
+
+def test_version_and_status_strings():
+    assert Q.lib().qstate_version() >= 100
+    for s in (0, 1, 2, 3):
+        assert Q.status_string(s)
+
+
+def _cfg(**kw):
+    base = dict(num_tiles=4, dk=128, dv=128, bits=4, group=32, delta=1, decay="scalar",
+                policy="persistent", rounding="nearest")
+    base.update(kw)
+    return Q.Config(**base)
+
+
+def _raw(cfg):
+    return cfg.c()
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("bits", 3, Q.QS_ERR_INVALID_ARG),
+    ("bits", 16, Q.QS_ERR_INVALID_ARG),
+    ("group", 48, Q.QS_ERR_INVALID_ARG),
+    ("group", 16, Q.QS_ERR_UNSUPPORTED),
+    ("dk", 96, Q.QS_ERR_UNSUPPORTED),
+    ("dk", 256, Q.QS_ERR_UNSUPPORTED),
+    ("dv", 24, Q.QS_ERR_UNSUPPORTED),
+    ("dv", 192, Q.QS_ERR_UNSUPPORTED),
+    ("dv", 0, Q.QS_ERR_INVALID_ARG),
+    ("num_tiles", -1, Q.QS_ERR_INVALID_ARG),
+    ("delta", 2, Q.QS_ERR_INVALID_ARG),
+    ("decay", 5, Q.QS_ERR_INVALID_ARG),
+    ("policy", 3, Q.QS_ERR_INVALID_ARG),
+    ("rounding", -1, Q.QS_ERR_INVALID_ARG),
+])
+def test_config_validation(field, value, status):
+    c = _raw(_cfg())
+    setattr(c, field, value)
+    lib = Q.lib()
+    assert lib.qstate_query_sizes(ctypes.byref(c), None, None, None) == status
+    assert lib.qstate_decode_step(ctypes.byref(c), 16, 16, None, 16, 16, 16, 16, 16, None, None) == status
+
+
+def test_null_config():
+    lib = Q.lib()
+    assert lib.qstate_query_sizes(None, None, None, None) == Q.QS_ERR_INVALID_ARG
+    assert lib.qstate_init(None, 16, 16, 16, None, None) == Q.QS_ERR_INVALID_ARG
+
+
+def test_sizes():
+    assert Q.query_sizes(_cfg(num_tiles=1024)) == (1024 * 128 * 64, 1024 * 128 * 4 * 4, 0)
+    assert Q.query_sizes(_cfg(num_tiles=3, bits=8, group=64, dv=64, policy="yoked")) == \
+        (3 * 64 * 128, 3 * 64 * 2 * 4, 3 * 64 * 128 * 4)
+
+
+# Fake device addresses: validation rejects these before any CUDA call.
+A = 1 << 20
+
+
+def _step(cfg, **ptrs):
+    p = dict(codes=A, scales=2 * A, shadow=None, q=3 * A, k=4 * A, v=5 * A, alpha=6 * A,
+             beta=7 * A, o=8 * A)
+    p.update(ptrs)
+    c = cfg.c()
+    return Q.lib().qstate_decode_step(ctypes.byref(c), p["codes"], p["scales"], p["shadow"],
+                                      p["q"], p["k"], p["v"], p["alpha"], p["beta"], p["o"], None)
+
+
+@pytest.mark.parametrize("ptrs", [
+    dict(codes=None), dict(scales=None), dict(k=None), dict(v=None), dict(alpha=None),
+    dict(beta=None), dict(q=None),                         # o given without q
+    dict(codes=A + 8), dict(codes=A + 16), dict(scales=2 * A + 4), dict(k=4 * A + 4), dict(q=3 * A + 8),
+    dict(v=5 * A + 12), dict(beta=7 * A + 2), dict(o=8 * A + 1),
+    dict(scales=A + 64),                                   # overlaps codes
+    dict(o=4 * A),                                         # output overlaps an input
+])
+def test_pointer_validation(ptrs):
+    assert _step(_cfg(), **ptrs) == Q.QS_ERR_INVALID_ARG
+
+
+def test_yoked_needs_shadow_and_diag_alpha_alignment():
+    assert _step(_cfg(policy="yoked")) == Q.QS_ERR_INVALID_ARG
+    assert _step(_cfg(policy="yoked"), shadow=9 * A + 4) == Q.QS_ERR_INVALID_ARG
+    assert _step(_cfg(policy="yoked"), shadow=9 * A + 16) == Q.QS_ERR_INVALID_ARG
+    assert _step(_cfg(decay="diagonal"), alpha=6 * A + 4) == Q.QS_ERR_INVALID_ARG
+
+
+def test_readout_validation():
+    c = _cfg().c()
+    lib = Q.lib()
+    assert lib.qstate_readout(ctypes.byref(c), None, 2 * A, 3 * A, 8 * A, None) == Q.QS_ERR_INVALID_ARG
+    assert lib.qstate_readout(ctypes.byref(c), A, 2 * A, 3 * A + 4, 8 * A, None) == Q.QS_ERR_INVALID_ARG
+    assert lib.qstate_readout(ctypes.byref(c), A, 2 * A, 3 * A, A + 16, None) == Q.QS_ERR_INVALID_ARG
+
+
+def test_binding_raises():
+    with pytest.raises(Q.QStateError):
+        Q.query_sizes(_cfg(bits=5))

@@ -1,0 +1,179 @@
+"""GPU parity: the CUDA decode step (through the C ABI) against the CPU
+oracle, element by element, on seeded inputs.
+
+Sizes span several tiles per CTA (persistent grid) and a ragged tail; the
+workloads' full sizes are covered on sampled tiles in the launch
+configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+from ssm_decode_step_b200 import Config, workloads as W
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+# (bits, dk, dv, group, delta, decay, policy, rounding, tiles)
+CASES = [
+    (4, 128, 128, 32, 1, "scalar", "persistent", "nearest", 333),
+    (4, 128, 128, 32, 1, "scalar", "dynamic", "nearest", 301),
+    (4, 128, 128, 32, 1, "scalar", "yoked", "nearest", 150),
+    (8, 128, 64, 64, 0, "scalar", "persistent", "nearest", 300),
+    (4, 128, 128, 32, 0, "diagonal", "persistent", "bdr", 151),
+    (4, 128, 128, 32, 0, "diagonal", "dynamic", "bdr", 40),
+    (4, 128, 128, 32, 1, "scalar", "persistent", "bdr", 40),
+    (8, 128, 128, 32, 1, "scalar", "dynamic", "nearest", 40),
+    (8, 64, 64, 64, 1, "scalar", "persistent", "nearest", 7),
+    (4, 64, 48, 32, 1, "diagonal", "yoked", "bdr", 9),
+    (8, 64, 16, 32, 0, "scalar", "dynamic", "bdr", 5),
+    (4, 128, 16, 128, 1, "diagonal", "dynamic", "nearest", 11),
+    (8, 128, 112, 128, 0, "diagonal", "yoked", "nearest", 13),
+    (4, 64, 256, 64, 1, "scalar", "persistent", "bdr", 6),
+    (8, 128, 32, 64, 1, "diagonal", "persistent", "nearest", 21),
+    (4, 128, 80, 64, 0, "scalar", "yoked", "bdr", 17),
+    (8, 64, 128, 32, 1, "diagonal", "dynamic", "bdr", 3),
+    (4, 64, 64, 32, 0, "scalar", "dynamic", "nearest", 1),
+]
+
+
+def _id(c):
+    b, dk, dv, g, de, dc, pol, r, T = c
+    return f"int{b}-dk{dk}-dv{dv}-g{g}-{'delta' if de else 'linear'}-{dc}-{pol}-{r}-T{T}"
+
+
+@pytest.mark.parametrize("case", CASES, ids=_id)
+def test_lockstep(case):
+    b, dk, dv, g, de, dc, pol, r, T = case
+    cfg = Config(T, dk, dv, b, g, de, dc, pol, r)
+    rng = np.random.default_rng(hash(_id(case)) % 2**32)
+    S0 = (rng.standard_normal((T, dv, dk)) * 0.3).astype(np.float32)
+    steps = P.random_steps(rng, T, dk, dv, dc, 6, scale=0.5)
+    rep = P.lockstep(cfg, S0, steps, label=_id(case))
+    assert rep.code_flips == 0, rep
+    # one more step without readout (o = NULL path)
+    gpu = P.GpuRun(cfg, S0)
+    ora = O.init(P.oracle_cfg(cfg), S0)
+    q, k, v, a, bb = steps[0]
+    gpu.step(None, k, v, a, bb, want_o=False)
+    O.step(ora, q, k, v, a, bb, want_o=False)
+    c, s, sh = gpu.state()
+    P.compare_state(cfg, c, s, ora, None, "no readout")
+
+
+def test_tiny_workload_full_horizon():
+    """The tiny gated delta-rule workload, all tiles, all 256 steps, free-run:
+    GPU and oracle never exchange state and must agree at every step."""
+    w = W.get(0)
+    arm = w.arms[0]
+    cfg = Config(w.tiles, w.dk, w.dv, arm.bits, arm.group, w.delta, w.decay, arm.policy, arm.rounding)
+    S0 = W.initial_state(w)
+    steps = [W.slot(w, t) for t in range(w.steps)]
+    rep = P.free_run(cfg, S0, steps, "tiny-gdn")
+    assert rep.code_flips == 0
+    assert rep.worst_o_rel <= P.READOUT_REL
+
+
+@pytest.mark.parametrize("policy,rounding,bits", [("persistent", "bdr", 4), ("dynamic", "nearest", 4),
+                                                  ("yoked", "nearest", 4), ("dynamic", "bdr", 8)])
+def test_long_free_run(policy, rounding, bits):
+    """A longer free run (512 steps) on a small gated delta-rule stack,
+    including the dynamic policy whose scale feeds back on the state."""
+    rng = np.random.default_rng(7)
+    T, dk, dv = 12, 128, 64
+    cfg = Config(T, dk, dv, bits, 32, 1, "scalar", policy, rounding)
+    S0 = (rng.standard_normal((T, dv, dk)) / np.sqrt(dk)).astype(np.float32)
+    steps = P.random_steps(rng, T, dk, dv, "scalar", 512)
+    rep = P.free_run(cfg, S0, steps, f"long-{policy}-{rounding}")
+    assert rep.code_flips == 0
+
+
+@pytest.mark.parametrize("bits,dk,dv,group", [(4, 128, 128, 32), (8, 128, 64, 64), (4, 64, 64, 64),
+                                              (8, 64, 32, 32)])
+def test_readout_entry(bits, dk, dv, group):
+    import torch
+    from ssm_decode_step_b200 import qstate as Q
+    rng = np.random.default_rng(bits * dk + dv)
+    T = 157
+    cfg = Config(T, dk, dv, bits, group, 1, "scalar", "persistent")
+    S0 = (rng.standard_normal((T, dv, dk)) * 0.4).astype(np.float32)
+    gpu = P.GpuRun(cfg, S0)
+    q = rng.standard_normal((T, dk)).astype(np.float32)
+    o = torch.empty((T, dv), dtype=torch.float32, device="cuda")
+    Q.readout(cfg, gpu.st.codes, gpu.st.scales, gpu.t(q), o)
+    ora = O.init(P.oracle_cfg(cfg), S0)
+    ref = O.readout(ora, q)
+    P.compare_readout(o.cpu().numpy(), ref, "readout")
+
+
+def test_zero_tiles_is_a_noop():
+    import torch
+    from ssm_decode_step_b200 import qstate as Q
+    cfg = Config(0, 128, 128, 4, 32, 1, "scalar", "persistent")
+    e = torch.empty(0, device="cuda")
+    Q.init(cfg, e, e, e)
+    Q.decode_step(cfg, e, e, None, e, e, e, e, e, e)
+    Q.readout(cfg, e, e, e, e)
+    torch.cuda.synchronize()
+
+
+def test_zero_state_and_zero_groups():
+    """S0 = 0: every scale is 0 and every code 0 (zero-scale rule); the
+    persistent state stays 0, the dynamic one picks up the first write."""
+    rng = np.random.default_rng(3)
+    T, dk, dv = 5, 128, 32
+    S0 = np.zeros((T, dv, dk), np.float32)
+    S0[1, :, 32:] = rng.standard_normal((dv, dk - 32)).astype(np.float32)   # one tile half zero
+    steps = P.random_steps(rng, T, dk, dv, "scalar", 3)
+    for pol in ("persistent", "dynamic", "yoked"):
+        cfg = Config(T, dk, dv, 4, 32, 1, "scalar", pol, "bdr")
+        P.lockstep(cfg, S0, steps, label=f"zero-{pol}")
+
+
+def test_zero_update_keeps_persistent_codes():
+    rng = np.random.default_rng(4)
+    T, dk, dv = 9, 128, 128
+    cfg = Config(T, dk, dv, 4, 32, 1, "scalar", "persistent")
+    S0 = (rng.standard_normal((T, dv, dk)) * 0.3).astype(np.float32)
+    gpu = P.GpuRun(cfg, S0)
+    c0, s0, _ = gpu.state()
+    q = rng.standard_normal((T, dk)).astype(np.float32)
+    v = rng.standard_normal((T, dv)).astype(np.float32)
+    gpu.step(q, np.zeros((T, dk), np.float32), v, np.ones(T, np.float32), np.full(T, 0.5, np.float32))
+    c1, s1, _ = gpu.state()
+    assert np.array_equal(c0, c1) and np.array_equal(s0, s1)
+
+
+def test_clipping_and_huge_updates():
+    """Persistent and yoked scales clip; updates of millions of grid steps
+    and overflowing values go through the clamping path."""
+    rng = np.random.default_rng(5)
+    T, dk, dv = 6, 128, 64
+    S0 = (rng.standard_normal((T, dv, dk)) * 1e-3).astype(np.float32)
+    steps = P.random_steps(rng, T, dk, dv, "scalar", 3, scale=1.0)
+    q, k, v, a, b = steps[1]
+    steps[1] = (q, k, (v * 1e4).astype(np.float32), a, b)
+    q, k, v, a, b = steps[2]
+    steps[2] = (q, k, np.full_like(v, 3e38), a, np.ones_like(b))
+    for pol in ("persistent", "yoked", "dynamic"):
+        for rnd in ("nearest", "bdr"):
+            cfg = Config(T, dk, dv, 8, 64, 0, "scalar", pol, rnd)
+            P.lockstep(cfg, S0, steps, label=f"clip-{pol}-{rnd}")
+
+
+# Full-size workloads at the benchmark's launch configuration, on sampled
+# tiles (tiles are independent, so a sampled tile is an exact check of that
+# tile).
+@pytest.mark.parametrize("wname", ["gdn", "mamba2", "gla", "stack24"])
+def test_workload_full_size_sampled(wname):
+    w = W.get(wname)
+    rng = np.random.default_rng(99)
+    tiles = np.sort(rng.choice(w.tiles, size=16, replace=False))
+    tiles[-1] = w.tiles - 1          # always include the ragged last tile
+    S0 = W.initial_state(w)
+    steps = [W.slot(w, t) for t in range(4)]
+    for arm in w.arms:
+        cfg = Config(w.tiles, w.dk, w.dv, arm.bits, arm.group, w.delta, w.decay, arm.policy,
+                     arm.rounding)
+        rep = P.lockstep(cfg, S0, steps, tiles=tiles, label=f"{wname}-{arm.name}")
+        assert rep.code_flips == 0, rep
