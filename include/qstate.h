@@ -18,8 +18,9 @@
  *
  * Element-level definition (FP32, IEEE round to nearest even; "fused"
  * means one rounding), for tile t, row i, column j, group g = j / group:
- *   d_ij  = c_ij * s_ig                      dequantized previous state
- *   S'_ij = d_ij * a_j                       a_j = alpha_t (QS_DECAY_SCALAR)
+ *   S'_ij = c_ij * (s_ig * a_j)              dequantized previous state with
+ *                                            the decay folded into the scale:
+ *                                            a_j = alpha_t (QS_DECAY_SCALAR)
  *                                            or alpha_tj (QS_DECAY_DIAGONAL)
  *   w_i   = beta_t * (v_i - u_i), u_i = S'_i . k   (delta = 1)
  *   w_i   = beta_t * v_i                           (delta = 0)
@@ -37,10 +38,11 @@
  *        abstract: elements whose rounding moves against their update are
  *        rounded one step toward it.)
  * qmax = 2^(bits-1) - 1.  Dot products "." are evaluated in one fixed
- * order: Dk/16 segments of 16 consecutive columns, each a fused
- * multiply-add chain from +0 in column order, summed by a balanced
- * pairwise tree.  Codes, scales and the shadow are therefore reproducible
- * bit for bit on any conforming implementation.
+ * order: each 32-column chunk is summed as two fused multiply-add chains
+ * from +0 in column order, one over its even and one over its odd columns,
+ * the chunk sum is even + odd, and the chunk sums are combined by a balanced
+ * pairwise tree in column order.  Codes, scales and the shadow are therefore
+ * reproducible bit for bit on any conforming implementation.
  *
  * Scale policies ("When Dynamic Scaling Fails", project page): per-token
  * dynamic reads its scale from the state it is about to quantize;
@@ -78,8 +80,8 @@
  *   - Calls that overlap on the GPU must not share state buffers.
  *
  * Supported by this build: dk in {64, 128}; dv a multiple of 16 with
- * 16 <= dv <= 128 (dk = 128) or <= 256 (dk = 64); bits in {4, 8};
- * group in {32, 64, 128} with group <= dk; any num_tiles >= 0.
+ * 16 <= dv <= 4096; bits in {4, 8}; group in {32, 64, 128} with
+ * group <= dk; num_tiles >= 0 with num_tiles * dv / 16 < 2^31.
  */
 #ifndef QSTATE_H
 #define QSTATE_H
@@ -150,10 +152,21 @@ QS_API qs_status qstate_decode_step(const qs_config* cfg, void* codes, float* sc
                              const float* beta, float* o, cudaStream_t stream);
 
 /* Readout of the stored state without changing it: o_i = d_i . q with
- * d_ij = c_ij * s_ig (the fixed dot order above). */
+ * d_ij = c_ij * s_ig (no decay; the fixed dot order above). */
 QS_API qs_status qstate_readout(const qs_config* cfg, const void* codes,
                          const float* scales, const float* q, float* o,
                          cudaStream_t stream);
+
+/* Self-check of the library's fast arithmetic on the current GPU.  The
+ * kernels compute the reciprocal of a scale and the division of a group
+ * maximum by qmax with short fused multiply-add sequences; this compares
+ * them bit for bit with the IEEE correctly rounded results on every input:
+ * the reciprocal on every float in [2^-126, 2^126), the divisions by 7 and
+ * by 127 on every finite non-negative float (about 6.4e9 evaluations).
+ * mismatches: device array of 3 unsigned 64-bit counters (reciprocal, /7,
+ * /127), 8-byte aligned, zeroed and filled on `stream`.  All three must be
+ * 0; the caller reads them after synchronizing. */
+QS_API qs_status qstate_selfcheck(unsigned long long* mismatches, cudaStream_t stream);
 
 /* Static, human-readable name of a status code. */
 QS_API const char* qstate_status_string(qs_status status);

@@ -8,7 +8,7 @@
  * where the operation order below says "fused".
  *
  * Element-level definition followed here, per tile and row i:
- *   1. dequantize and decay   d_j = c_ij * s_ig ;  S'_j = d_j * a_j
+ *   1. dequantize and decay   S'_j = c_ij * (s_ig * a_j)   (decayed scale)
  *        (a_j = alpha for scalar decay Lambda = alpha I, alpha_j for
  *         Lambda = diag(alpha): LinQuant, Key structural choices)
  *   2. write coefficient      w = beta * (v_i - u)   with u = S' . k  (delta 1)
@@ -28,7 +28,8 @@
  *                             n*s' < S'_j then n += 1; if sigma < 0 and
  *                             n*s' > S'_j then n -= 1; clamp again
  *   9. store                  codes, and s' for dynamic / yoked
- * Dot products "." use qo_dot's fixed order.
+ * Dot products "." use qo_dot's fixed order (even / odd chains per 32
+ * entries, pairwise tree over the chunks).
  */
 #include "qstate_oracle.h"
 
@@ -56,9 +57,9 @@ int qo_num_threads(void) {
 int qo_check(const qo_cfg* c) {
   if (!c) return -1;
   if (c->tiles < 0 || c->dv < 1) return -1;
-  if (c->dk < 16 || c->dk > QO_MAX_DK || c->dk % 16) return -1;
-  int segs = c->dk / 16;
-  if (segs & (segs - 1)) return -1;
+  if (c->dk < 32 || c->dk > QO_MAX_DK || c->dk % 32) return -1;
+  int chunks = c->dk / 32;
+  if (chunks & (chunks - 1)) return -1;
   if (c->qmax < 1 || c->qmax > (1 << 20)) return -1;
   if (c->group < 1 || c->dk % c->group) return -1;
   if (c->delta != 0 && c->delta != 1) return -1;
@@ -68,18 +69,23 @@ int qo_check(const qo_cfg* c) {
   return 0;
 }
 
-/* Fixed-order dot product: n/16 segments, each a fused multiply-add chain
- * over 16 consecutive entries starting from +0, then a balanced pairwise
- * tree over the segment sums in order: ((p0+p1)+(p2+p3))+... */
+/* Fixed-order dot product over n = 32 * 2^m entries: each 32-entry chunk is
+ * summed as two fused multiply-add chains from +0 in index order, one over
+ * its even entries and one over its odd entries; chunk sum = even + odd; the
+ * chunk sums are combined by a balanced pairwise tree in order:
+ * ((c0 + c1) + (c2 + c3)) + ... */
 float qo_dot(const float* a, const float* b, int n) {
-  float part[QO_MAX_DK / 16];
-  int segs = n / 16;
-  for (int s = 0; s < segs; ++s) {
-    float acc = 0.0f;
-    for (int j = 16 * s; j < 16 * s + 16; ++j) acc = fmaf(a[j], b[j], acc);
-    part[s] = acc;
+  float part[QO_MAX_DK / 32];
+  int chunks = n / 32;
+  for (int c = 0; c < chunks; ++c) {
+    float even = 0.0f, odd = 0.0f;
+    for (int i = 0; i < 16; ++i) {
+      even = fmaf(a[32 * c + 2 * i], b[32 * c + 2 * i], even);
+      odd = fmaf(a[32 * c + 2 * i + 1], b[32 * c + 2 * i + 1], odd);
+    }
+    part[c] = even + odd;
   }
-  for (int width = segs; width > 1; width /= 2)
+  for (int width = chunks; width > 1; width /= 2)
     for (int m = 0; m < width / 2; ++m) part[m] = part[2 * m] + part[2 * m + 1];
   return part[0];
 }
@@ -232,12 +238,12 @@ int qo_step(const qo_cfg* c, int32_t* codes, float* scales, float* shadow,
       size_t row = (size_t)t * dv + i;
       int32_t* crow = codes + row * dk;
       float* srow = scales + row * ng;
-      /* 1. dequantize and decay */
+      /* 1. dequantize with the decayed scale: S' = c * (s * a) */
       for (int j = 0; j < dk; ++j) {
         int g = j / G;
         if (g_fault == QO_FAULT_GROUP_INDEX) g = (g + 1) % ng;
         d[j] = (float)crow[j] * srow[g];
-        Sp[j] = d[j] * decay_at(c, alpha, t, i, j);
+        Sp[j] = (float)crow[j] * (srow[g] * decay_at(c, alpha, t, i, j));
       }
       /* 2-3. write */
       float w = row_write(c, Sp, kt, v[(size_t)t * dv + i], beta[t], x);

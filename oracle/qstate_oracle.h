@@ -22,10 +22,12 @@
  * Low-Bit Recurrent State Quantization", abstract).
  *
  * Arithmetic is IEEE FP32 in a fixed operation order (compiled with
- * -ffp-contract=off; fmaf only where written).  The order of the two dot
- * products is fixed as: Dk/16 segment sums, each a sequential fused
- * multiply-add chain over 16 consecutive columns starting from +0, combined
- * by a balanced pairwise tree in column order.
+ * -ffp-contract=off; fmaf only where written).  The dequantized, decayed
+ * state is c * (s * a) (the decay folded into the group scale first).  Dot
+ * products are fixed as: per 32-column chunk, one fused multiply-add chain
+ * over the even columns and one over the odd columns, each from +0 in column
+ * order, chunk sum = even + odd; chunk sums combined by a balanced pairwise
+ * tree in column order.
  *
  * Parity status: every function here is pinned by the CPU tests in
  * tests/test_oracle_pins.py (closed forms, invariants, brute force); the
@@ -46,7 +48,7 @@ enum { QO_ROUND_NEAREST = 0, QO_ROUND_BDR = 1 };
 
 typedef struct {
   int32_t tiles;    /* independent (layer, batch, head) states            */
-  int32_t dk, dv;   /* key and value dimensions; dk = 16 * 2^m            */
+  int32_t dk, dv;   /* key and value dimensions; dk = 32 * 2^m            */
   int32_t qmax;     /* largest code magnitude: 2^(bits-1) - 1             */
   int32_t group;    /* quantization group length along dk; divides dk     */
   int32_t delta;    /* 0 = linear write, 1 = delta-rule correction        */

@@ -23,6 +23,8 @@ HEADER = os.path.join(ROOT, "include", "qstate.h")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVFLAGS = ARCH + ["-O3", "-std=c++17", "-lineinfo", "-fmad=false", "-Xcompiler", "-fPIC",
                   "-Xcompiler", "-fvisibility=hidden", "-I", os.path.join(ROOT, "include")]
+# Extra nvcc flags (e.g. -DQS_MIN_BLOCKS=3) for tuning builds.
+NVFLAGS += os.environ.get("QSTATE_NVCC_FLAGS", "").split()
 
 
 def nvcc() -> str:

@@ -25,6 +25,27 @@ int device_sm_count() {
   return counts[dev];
 }
 
+// ---------------------------------------------------------------------------
+// self-check of the fast arithmetic against the IEEE routines
+// ---------------------------------------------------------------------------
+// Every float bit pattern in [lo, hi): recip_rn against __frcp_rn on its
+// fast range, and div_qmax_rn<7>, <127> against __fdiv_rn on all finite
+// non-negative values.  Mismatch counts are added to bad[0..2].
+__global__ void selfcheck_kernel(unsigned long long* bad, uint32_t lo, uint32_t hi) {
+  unsigned long long b0 = 0, b1 = 0, b2 = 0;
+  for (uint64_t i = lo + static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < hi;
+       i += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
+    const float x = __uint_as_float(static_cast<uint32_t>(i));
+    if (!(x >= 0.0f) || x > 3.40282347e38f) continue;
+    if (x >= 0x1p-126f && x < 0x1p126f) b0 += __float_as_uint(recip_rn(x)) != __float_as_uint(__frcp_rn(x));
+    b1 += __float_as_uint(div_qmax_rn<7>(x)) != __float_as_uint(__fdiv_rn(x, 7.0f));
+    b2 += __float_as_uint(div_qmax_rn<127>(x)) != __float_as_uint(__fdiv_rn(x, 127.0f));
+  }
+  if (b0) atomicAdd(&bad[0], b0);
+  if (b1) atomicAdd(&bad[1], b1);
+  if (b2) atomicAdd(&bad[2], b2);
+}
+
 }  // namespace qs
 
 namespace {
@@ -56,7 +77,8 @@ qs_status check_config(const qs_config* c) {
   if (c->rounding != QS_ROUND_NEAREST && c->rounding != QS_ROUND_BDR) return QS_ERR_INVALID_ARG;
   // what this build has kernels for
   if (c->dk != 64 && c->dk != 128) return QS_ERR_UNSUPPORTED;
-  if (c->dv % 16 != 0 || c->dv * (c->dk / 32) > qs::kMaxThreads) return QS_ERR_UNSUPPORTED;
+  if (c->dv % 16 != 0 || c->dv > 4096) return QS_ERR_UNSUPPORTED;
+  if (static_cast<long long>(c->num_tiles) * (c->dv / 16) > 0x7fffffffLL) return QS_ERR_UNSUPPORTED;
   if (c->group != 32 && c->group != 64 && c->group != 128) return QS_ERR_UNSUPPORTED;
   return QS_OK;
 }
@@ -115,6 +137,15 @@ cudaError_t dispatch_step(const qs_config* c, const qs::StepParams& p, cudaStrea
 extern "C" {
 
 int qstate_version(void) { return 100; }
+
+qs_status qstate_selfcheck(unsigned long long* mismatches, cudaStream_t stream) {
+  if (mismatches == nullptr || !aligned(mismatches, 8)) return QS_ERR_INVALID_ARG;
+  cudaError_t e = cudaMemsetAsync(mismatches, 0, 3 * sizeof(unsigned long long), stream);
+  if (e != cudaSuccess) return QS_ERR_CUDA;
+  // all non-negative finite float bit patterns
+  qs::selfcheck_kernel<<<qs::device_sm_count() * 16, 256, 0, stream>>>(mismatches, 0u, 0x7F800000u);
+  return from_cuda(cudaGetLastError());
+}
 
 const char* qstate_status_string(qs_status s) {
   switch (s) {

@@ -7,27 +7,29 @@
 //
 // Work decomposition.  Rows of a tile are independent: every reduction of
 // the step (u = S' k, o = x q, the group max) runs along one row.  A thread
-// owns a 32-column chunk of one row (LPR = Dk/32 lanes per row, consecutive
-// lanes), so the row's reductions are in-thread chains plus log2(LPR) xor
-// shuffles.  A CTA owns one tile at a time (blockDim = Dv * LPR threads) and
-// walks tiles with a stride of gridDim.x (persistent grid, sized to the SMs).
+// owns a 32-column chunk c of a row (LPR = Dk/32 consecutive lanes per row),
+// so a row's reductions are in-thread chains plus log2(LPR) xor shuffles.
+// A work unit is a block of rb rows of one tile; a CTA of kThreads threads
+// takes one unit per iteration (persistent grid sized to the SMs), and
+// thread (r0, c) handles rows r0, r0 + RP, ... of the unit, keeping the
+// unit's k (and q) chunk in registers across those rows.
 //
-// Memory path.  Each tile's codes, scales, v, k, q (and alpha, the FP32
-// shadow) are staged into shared memory with cp.async through an S-deep
-// ring, so S-1 tiles are in flight while one is computed.  k, q and a
-// diagonal alpha are scattered into a pair-interleaved layout (column m and
-// m+16 of a chunk side by side) so the packed FP32 instructions
-// (__ffma2_rn & co., sm_100) see their operands in register pairs.  New codes
-// leave as 16/32-byte coalesced stores straight from registers.
+// Memory path.  Each unit's codes, scales, v, k, q (alpha, the FP32 shadow)
+// are staged into shared memory with 16-byte cp.async through an S-deep
+// ring per CTA, so S-1 units are in flight while one is computed; new codes
+// and scales leave as coalesced 16/32-byte stores straight from registers.
 //
-// Order of FP32 operations.  Each thread evaluates its chunk's two 16-column
-// segments as two fused multiply-add chains in column order (the two lanes
-// of one packed instruction), adds the pair, then the lanes of the row add
-// their partials with xor shuffles 1, 2: exactly the balanced pairwise tree
-// over 16-column segments that the definition fixes.  Every other FP32
-// operation is element-wise, so packed and scalar forms give the same bits.
-// Explicit intrinsics (__fmul_rn, __fadd_rn, __ffma2_rn ...) keep the compiler
-// from contracting or reordering; the library is also built -fmad=false.
+// Arithmetic.  Each thread holds its chunk as 16 register pairs of adjacent
+// columns (2m, 2m+1) and works with the packed FP32 instructions of sm_100
+// (__ffma2_rn, __fmul2_rn, __fadd2_rn).  The two lanes of the packed dot
+// product chains are exactly the even-column and odd-column chains of the
+// fixed order; the lanes of a row then add their chunk sums with xor
+// shuffles 1, 2, which is the pairwise tree of the definition.  Every other
+// FP32 operation is element-wise, so packed and scalar forms give the same
+// bits; explicit rounding intrinsics keep the compiler from contracting or
+// reordering (and the library is built -fmad=false).  Codes are unpacked by
+// a byte permute into the mantissa of 2^23 (exact) and rounded by adding
+// 1.5 * 2^23 inside one fused multiply-add (exact product, ties to even).
 //
 // No kernel here spins on a flag or barrier: the only waits are
 // cp.async.wait_group and __syncthreads, so nothing can hang.
@@ -38,7 +40,26 @@
 
 namespace qs {
 
-constexpr int kMaxThreads = 512;
+constexpr int kThreads = 128;
+
+// Resident CTAs per SM the register allocation targets (kThreads each);
+// the yoked kernel is held to fewer by its shared memory and gets more
+// registers instead.
+#ifndef QS_MIN_BLOCKS
+#define QS_MIN_BLOCKS 4
+#endif
+#ifndef QS_MIN_BLOCKS_YOKED
+#define QS_MIN_BLOCKS_YOKED 3
+#endif
+// Keep the unit's q chunk in registers across rows (else re-read it from
+// shared memory for every row).
+#ifndef QS_Q_IN_REGS
+#define QS_Q_IN_REGS 0
+#endif
+// Rows a thread carries through the step together (1 or 2).
+#ifndef QS_ROWS_TOGETHER
+#define QS_ROWS_TOGETHER 1
+#endif
 
 // 1.5 * 2^23: adding it to a float of magnitude < 2^22 leaves the nearest
 // integer (ties to even) in the low mantissa bits.
@@ -57,6 +78,8 @@ struct StepParams {
   int tiles;
   int dv;
   int group;
+  int rb;              // rows per work unit (divides dv)
+  int units_per_tile;  // dv / rb
 };
 
 // ---------------------------------------------------------------------------
@@ -84,8 +107,6 @@ __device__ __forceinline__ void cp_async_wait() {
 
 __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
 
-__device__ __forceinline__ float2 abs2(float2 a) { return make_float2(fabsf(a.x), fabsf(a.y)); }
-
 template <int N>
 __device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[N]) {
   static_assert(N == 8, "256-bit store takes 8 words");
@@ -94,90 +115,137 @@ __device__ __forceinline__ void st_global_v8(void* p, const uint32_t (&w)[N]) {
                : "memory");
 }
 
-// Position of column r (0..31) of a chunk in the pair-interleaved layout:
-// columns m and m+16 sit side by side.
-__host__ __device__ __forceinline__ int pair_pos(int r) { return r < 16 ? 2 * r : 2 * (r - 16) + 1; }
+// ---------------------------------------------------------------------------
+// correctly rounded reciprocal and division by qmax
+// ---------------------------------------------------------------------------
+// Newton-Raphson with a fused correction (Markstein's method): from the
+// hardware approximation y of 1/s, e = 1 - s*y is exact in one fused
+// multiply-add and y + y*e rounds to 1/s.  Compared bit for bit with the
+// IEEE reciprocal on every float in [2^-126, 2^126) (qstate_selfcheck);
+// outside that range the IEEE routine is used.
+__device__ __forceinline__ float recip_rn(float s) {
+  if (s >= 0x1p-126f && s < 0x1p126f) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(s));
+    const float e = __fmaf_rn(-s, y, 1.0f);
+    return __fmaf_rn(y, e, y);
+  }
+  return __frcp_rn(s);
+}
 
-// Floats per interleaved chunk in shared memory (32 + 4 padding so that the
-// LPR chunks of a row start in different banks).
-constexpr int kChunkStride = 36;
+// m / Q for the constant Q = qmax: the product with RN(1/Q) corrected by the
+// exact remainder m - q*Q (division by a constant known in advance, after
+// Brisebarre, Muller and Raina).  Compared bit for bit with IEEE division on
+// every finite m >= 0 for Q = 7 and Q = 127 (qstate_selfcheck); infinities
+// and NaN take the IEEE routine.
+template <int Q>
+__device__ __forceinline__ float div_qmax_rn(float m) {
+  if (m <= 3.40282347e38f) {
+    constexpr float r = 1.0f / static_cast<float>(Q);
+    const float q0 = __fmul_rn(m, r);
+    const float rem = __fmaf_rn(-q0, static_cast<float>(Q), m);
+    return __fmaf_rn(rem, r, q0);
+  }
+  return __fdiv_rn(m, static_cast<float>(Q));
+}
 
 // ---------------------------------------------------------------------------
-// shared-memory stage layout (identical on host and device)
+// work units and the shared-memory stage layout (identical on host and device)
 // ---------------------------------------------------------------------------
 
 __host__ __device__ __forceinline__ int align_up(int x, int a) { return (x + a - 1) / a * a; }
 
+// Floats per 32-column chunk of a staged vector (32 + 4 padding so that the
+// LPR chunks of a row start in different banks).
+constexpr int kChunkStride = 36;
+
 struct StageLayout {
   int codes, scales, v, k, q, a, sk, misc, shadow, bytes;
 
-  __host__ __device__ StageLayout(int bits, int dk, int dv, int group, bool diag, bool bdr,
+  __host__ __device__ StageLayout(int bits, int dk, int rb, int group, bool diag, bool bdr,
                                   bool yoked) {
     const int vec = (dk / 32) * kChunkStride * 4;
     int off = 0;
-    codes = off;  off = align_up(off + dv * dk * bits / 8, 16);
-    scales = off; off = align_up(off + dv * (dk / group) * 4, 16);
-    v = off;      off = align_up(off + dv * 4, 16);
+    codes = off;  off = align_up(off + rb * dk * bits / 8, 16);
+    scales = off; off = align_up(off + rb * (dk / group) * 4, 16);
+    v = off;      off = align_up(off + rb * 4, 16);
     k = off;      off += vec;
     q = off;      off += vec;
     a = off;      off += diag ? vec : 0;
     sk = off;     off += bdr ? vec : 0;
     misc = off;   off += 16;
-    shadow = off; off += yoked ? dv * dk * 4 : 0;
+    shadow = off; off += yoked ? rb * dk * 4 : 0;
     bytes = align_up(off, 128);
   }
 };
 
-// Issue the cp.async copies of one tile into a stage.
+// 16-byte unit i of a staged Dk vector lands in chunk i/8 at the padded stride.
+__device__ __forceinline__ int vec_unit_offset(int i) { return (i >> 3) * (kChunkStride * 4) + (i & 7) * 16; }
+
+// Issue the cp.async copies of one work unit into a stage.
 template <int BITS, int DK, bool DIAG, bool YOKED, bool WITH_STATE_UPDATE>
 __device__ __forceinline__ void stage_load(unsigned char* st, const StageLayout& L,
-                                           const StepParams& p, int tile) {
-  const int tid = threadIdx.x, nt = blockDim.x;
-  const int dv = p.dv;
-  const size_t t = static_cast<size_t>(tile);
+                                           const StepParams& p, int unit) {
+  constexpr int VU = DK / 4;  // 16-byte units per Dk vector
+  const int tid = threadIdx.x;
+  const int rb = p.rb;
+  const size_t tile = static_cast<size_t>(unit / p.units_per_tile);
+  const size_t row0 = tile * p.dv + static_cast<size_t>(unit % p.units_per_tile) * rb;
+  const int ng = DK / p.group;
   {
-    const int n16 = dv * DK * BITS / 8 / 16;
-    const uint8_t* g = p.codes + t * (dv * DK * BITS / 8);
-    for (int i = tid; i < n16; i += nt) cp_async16(st + L.codes + 16 * i, g + 16 * i);
+    const int n16 = rb * DK * BITS / 128;
+    const uint8_t* g = p.codes + row0 * (DK * BITS / 8);
+    for (int i = tid; i < n16; i += kThreads) cp_async16(st + L.codes + 16 * i, g + 16 * i);
   }
   {
-    const int n16 = dv * (DK / p.group) * 4 / 16;
-    const float* g = p.scales + t * (dv * (DK / p.group));
-    for (int i = tid; i < n16; i += nt) cp_async16(st + L.scales + 16 * i, g + 4 * i);
+    const int n16 = rb * ng / 4;
+    const float* g = p.scales + row0 * ng;
+    for (int i = tid; i < n16; i += kThreads) cp_async16(st + L.scales + 16 * i, g + 4 * i);
   }
-  float* sk = reinterpret_cast<float*>(st + L.k);
-  float* sq = reinterpret_cast<float*>(st + L.q);
-  for (int j = tid; j < DK; j += nt) {
-    const int pos = (j / 32) * kChunkStride + pair_pos(j % 32);
-    if (p.o != nullptr) cp_async4(sq + pos, p.q + t * DK + j);
-    if constexpr (WITH_STATE_UPDATE) {
-      cp_async4(sk + pos, p.k + t * DK + j);
-      if constexpr (DIAG) cp_async4(reinterpret_cast<float*>(st + L.a) + pos, p.alpha + t * DK + j);
+  // the per-tile vectors k, q, alpha (diagonal): one 16-byte unit per thread
+  for (int i = tid; i < 3 * VU; i += kThreads) {
+    const int which = i / VU, u = i % VU;
+    if (which == 0) {
+      if (WITH_STATE_UPDATE) cp_async16(st + L.k + vec_unit_offset(u), p.k + tile * DK + 4 * u);
+    } else if (which == 1) {
+      if (p.o != nullptr) cp_async16(st + L.q + vec_unit_offset(u), p.q + tile * DK + 4 * u);
+    } else {
+      if (WITH_STATE_UPDATE && DIAG) cp_async16(st + L.a + vec_unit_offset(u), p.alpha + tile * DK + 4 * u);
     }
   }
   if constexpr (WITH_STATE_UPDATE) {
-    const int n16 = dv * 4 / 16;
-    for (int i = tid; i < n16; i += nt) cp_async16(st + L.v + 16 * i, p.v + t * dv + 4 * i);
-    if (tid == 0) {
+    for (int i = tid; i < rb / 4; i += kThreads) cp_async16(st + L.v + 16 * i, p.v + row0 + 4 * i);
+    if (tid == kThreads - 1) {
       float* misc = reinterpret_cast<float*>(st + L.misc);
-      if constexpr (!DIAG) cp_async4(misc + 0, p.alpha + t);
-      cp_async4(misc + 1, p.beta + t);
+      if constexpr (!DIAG) cp_async4(misc + 0, p.alpha + tile);
+      cp_async4(misc + 1, p.beta + tile);
     }
   }
   if constexpr (YOKED) {
-    // 16-byte unit u of row-chunk rc lands at unit position u ^ (rc & 7) so
-    // that the 8 lanes of a quarter-warp read 8 different bank groups.
-    const int n16 = dv * DK / 4;
-    const float* g = p.shadow + t * (dv * DK);
-    for (int i = tid; i < n16; i += nt) {
+    // 16-byte unit u of local row-chunk rc lands at unit position u ^ (rc & 7)
+    // so that the 8 lanes of a quarter-warp read 8 different bank groups.
+    const int n16 = rb * DK / 4;
+    const float* g = p.shadow + row0 * DK;
+    for (int i = tid; i < n16; i += kThreads) {
       const int rc = i >> 3, u = i & 7;
       cp_async16(st + L.shadow + rc * 128 + 16 * (u ^ (rc & 7)), g + 4 * i);
     }
   }
 }
 
+// Load a staged Dk vector's chunk c as 16 pairs (2m, 2m+1).
+__device__ __forceinline__ void load_pairs(const unsigned char* base, int c, float2 (&v)[16]) {
+  const float4* p4 = reinterpret_cast<const float4*>(base) + c * (kChunkStride / 4);
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const float4 t = p4[m];
+    v[2 * m] = make_float2(t.x, t.y);
+    v[2 * m + 1] = make_float2(t.z, t.w);
+  }
+}
+
 // ---------------------------------------------------------------------------
-// per-thread decode of a 32-column chunk into pairs e[m] = {c_m, c_{m+16}}
+// per-thread decode of a 32-column chunk into pairs e[m] = {c_2m, c_2m+1}
 // ---------------------------------------------------------------------------
 
 template <int BITS>
@@ -187,57 +255,47 @@ __device__ __forceinline__ void decode_chunk(const uint32_t (&w)[BITS], float2 (
   // 2^23 + field, and subtracting 2^23 + 2^(BITS-1) gives n exactly.
   constexpr float kBias = BITS == 4 ? 8388616.0f : 8388736.0f;
   if constexpr (BITS == 4) {
-    uint32_t lo[4], hi[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const uint32_t x = w[q] ^ 0x88888888u;
-      lo[q] = x & 0x0F0F0F0Fu;         // nibbles 0,2,4,6 of the word
-      hi[q] = (x >> 4) & 0x0F0F0F0Fu;  // nibbles 1,3,5,7
-    }
-    // element 8q + 2b -> byte b of lo[q]; element 8q + 2b + 1 -> byte b of hi[q]
+      const uint32_t lo = x & 0x0F0F0F0Fu;         // columns 8q, 8q+2, 8q+4, 8q+6
+      const uint32_t hi = (x >> 4) & 0x0F0F0F0Fu;  // columns 8q+1, 8q+3, 8q+5, 8q+7
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      const int qa = m / 8, qb = 2 + m / 8, nib = m % 8;
-      const uint32_t sa = (nib & 1) ? hi[qa] : lo[qa];
-      const uint32_t sb = (nib & 1) ? hi[qb] : lo[qb];
-      const uint32_t sel = 0x7540u | (nib >> 1);
-      const float fa = __uint_as_float(__byte_perm(sa, 0x4B000000u, sel));
-      const float fb = __uint_as_float(__byte_perm(sb, 0x4B000000u, sel));
-      e[m] = __fadd2_rn(make_float2(fa, fb), f2(-kBias));
+      for (int b = 0; b < 4; ++b) {
+        const uint32_t sel = 0x7540u | b;
+        e[4 * q + b] = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, sel)),
+                                              __uint_as_float(__byte_perm(hi, 0x4B000000u, sel))),
+                                  f2(-kBias));
+      }
     }
   } else {
-    uint32_t x[8];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) x[q] = w[q] ^ 0x80808080u;
+    for (int q = 0; q < 8; ++q) {
+      const uint32_t x = w[q] ^ 0x80808080u;        // columns 4q .. 4q+3
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      const int qa = m / 4, qb = 4 + m / 4, b = m % 4;
-      const uint32_t sel = 0x7540u | b;
-      const float fa = __uint_as_float(__byte_perm(x[qa], 0x4B000000u, sel));
-      const float fb = __uint_as_float(__byte_perm(x[qb], 0x4B000000u, sel));
-      e[m] = __fadd2_rn(make_float2(fa, fb), f2(-kBias));
+      for (int h = 0; h < 2; ++h) {
+        e[2 * q + h] = __fadd2_rn(
+            make_float2(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7540u | (2 * h))),
+                        __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7540u | (2 * h + 1)))),
+            f2(-kBias));
+      }
     }
   }
 }
 
-// Pack 32 rounded values (held as kMagic + bias + n floats in pairs) into
+// Pack 32 rounded values (floats kMagic + bias + n, as pairs (2m, 2m+1)) into
 // BITS words of two's complement codes.
 template <int BITS>
 __device__ __forceinline__ void pack_chunk(const float2 (&y)[16], uint32_t (&w)[BITS]) {
-  auto Y = [&](int e) -> uint32_t {
-    return __float_as_uint(e < 16 ? y[e].x : y[e - 16].y);
-  };
   if constexpr (BITS == 4) {
-    // Low 4 bits of each value are n + 8 in 1..15; (b << 4) + a has the byte
-    // (n_b + 8, n_a + 8) in its low 8 bits with no carry.
+    // Low 4 bits of each value are n + 8 in 1..15; (odd << 4) + even has the
+    // byte (n_odd + 8, n_even + 8) in its low 8 bits with no carry.
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       uint32_t by[4];
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const int e = 8 * q + 2 * b;
-        by[b] = (Y(e + 1) << 4) + Y(e);
-      }
+      for (int b = 0; b < 4; ++b)
+        by[b] = (__float_as_uint(y[4 * q + b].y) << 4) + __float_as_uint(y[4 * q + b].x);
       const uint32_t t0 = __byte_perm(by[0], by[1], 0x0040u);
       const uint32_t t1 = __byte_perm(by[2], by[3], 0x0040u);
       w[q] = __byte_perm(t0, t1, 0x5410u) ^ 0x88888888u;
@@ -245,15 +303,16 @@ __device__ __forceinline__ void pack_chunk(const float2 (&y)[16], uint32_t (&w)[
   } else {
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      const uint32_t t0 = __byte_perm(Y(4 * q), Y(4 * q + 1), 0x0040u);
-      const uint32_t t1 = __byte_perm(Y(4 * q + 2), Y(4 * q + 3), 0x0040u);
+      const uint32_t t0 = __byte_perm(__float_as_uint(y[2 * q].x), __float_as_uint(y[2 * q].y), 0x0040u);
+      const uint32_t t1 =
+          __byte_perm(__float_as_uint(y[2 * q + 1].x), __float_as_uint(y[2 * q + 1].y), 0x0040u);
       w[q] = __byte_perm(t0, t1, 0x5410u) ^ 0x80808080u;
     }
   }
 }
 
-// Sum of the chunk's two segment chains, then the pairwise tree across the
-// LPR lanes of the row (xor 1, then xor 2).
+// even + odd chains of the chunk, then the pairwise tree across the LPR
+// lanes of the row (xor 1, then xor 2)
 template <int LPR>
 __device__ __forceinline__ float row_tree(float2 acc) {
   float t = __fadd_rn(acc.x, acc.y);
@@ -304,18 +363,18 @@ __device__ __forceinline__ void round_chunk(const float2 (&x)[16], float inv, bo
 // lies on the wrong side of the pre-update value S'.
 template <int BITS>
 __device__ __forceinline__ void bdr_chunk(float2 (&y)[16], const float2 (&Sp)[16],
-                                          const float2* sk, float sw, float sp) {
+                                          const float2 (&sk)[16], float sw, float sp) {
   constexpr float kOff = kMagic + (BITS == 4 ? 8.0f : 128.0f);
   constexpr float kQ = BITS == 4 ? 7.0f : 127.0f;
 #pragma unroll
   for (int m = 0; m < 16; ++m) {
-    const float2 nf = __fadd2_rn(y[m], f2(-kOff));          // n, exact
-    const float2 dq = __fmul2_rn(nf, f2(sp));               // n * s'
+    const float2 nf = __fadd2_rn(y[m], f2(-kOff));                   // n, exact
+    const float2 dq = __fmul2_rn(nf, f2(sp));                        // n * s'
     const float2 e = __fadd2_rn(Sp[m], make_float2(-dq.x, -dq.y));  // sign of S' - n s'
-    const float2 sg = __fmul2_rn(sk[m], f2(sw));            // sigma in {-1, 0, 1}
-    const float2 t = __fmul2_rn(e, sg);                      // > 0 iff reversed
-    float yx = t.x > 0.0f ? __fadd_rn(y[m].x, sg.x) : y[m].x;
-    float yy = t.y > 0.0f ? __fadd_rn(y[m].y, sg.y) : y[m].y;
+    const float2 sg = __fmul2_rn(sk[m], f2(sw));                     // sigma in {-1, 0, 1}
+    const float2 t = __fmul2_rn(e, sg);                              // > 0 iff reversed
+    const float yx = t.x > 0.0f ? __fadd_rn(y[m].x, sg.x) : y[m].x;
+    const float yy = t.y > 0.0f ? __fadd_rn(y[m].y, sg.y) : y[m].y;
     y[m].x = fminf(fmaxf(yx, kOff - kQ), kOff + kQ);
     y[m].y = fminf(fmaxf(yy, kOff - kQ), kOff + kQ);
   }
@@ -326,34 +385,43 @@ __device__ __forceinline__ void bdr_chunk(float2 (&y)[16], const float2 (&Sp)[16
 // ---------------------------------------------------------------------------
 // POLICY: 0 dynamic, 1 persistent, 2 yoked.
 template <int BITS, int DK, int POLICY, bool BDR, bool DELTA, bool DIAG, int STAGES>
-__global__ void __launch_bounds__(kMaxThreads, 1) step_kernel(StepParams p) {
+__global__ void __launch_bounds__(kThreads, POLICY == 2 ? QS_MIN_BLOCKS_YOKED : QS_MIN_BLOCKS)
+    step_kernel(StepParams p) {
   constexpr int LPR = DK / 32;
+  constexpr int RP = kThreads / LPR;  // rows per pass of the CTA
   constexpr bool YOKED = POLICY == 2;
-  constexpr int CW = BITS;  // 32-bit words of codes per 32-column chunk
-  constexpr float kQf = BITS == 4 ? 7.0f : 127.0f;
+  constexpr int CW = BITS;            // 32-bit words of codes per 32-column chunk
+  constexpr int QMAX = BITS == 4 ? 7 : 127;
+  constexpr float kQf = static_cast<float>(QMAX);
   constexpr float kOff = kMagic + (BITS == 4 ? 8.0f : 128.0f);
+  // q stays in registers across the rows of a unit unless other per-column
+  // vectors need the registers
+  constexpr bool Q_REG = QS_Q_IN_REGS && !DIAG && !BDR && !YOKED;
+  // rows processed together by one thread (independent dependency chains)
+  constexpr int NR = (YOKED || BDR) ? 1 : QS_ROWS_TOGETHER;
 
   extern __shared__ __align__(128) unsigned char smem[];
-  const StageLayout L(BITS, DK, p.dv, p.group, DIAG, BDR, YOKED);
+  const StageLayout L(BITS, DK, p.rb, p.group, DIAG, BDR, YOKED);
   const int tid = threadIdx.x;
-  const int row = tid / LPR, c = tid % LPR;
+  const int c = tid % LPR, r0 = tid / LPR;
   const int ng = DK / p.group;
   const int g = (32 * c) / p.group;
   const bool readout = p.o != nullptr;
+  const bool writes_scale = (32 * c) % p.group == 0;
+  const int units = p.tiles * p.units_per_tile;
 
-  // prologue: STAGES-1 tiles in flight
 #pragma unroll
   for (int s = 0; s < STAGES - 1; ++s) {
-    const int tile = blockIdx.x + s * gridDim.x;
-    if (tile < p.tiles) stage_load<BITS, DK, DIAG, YOKED, true>(smem + s * L.bytes, L, p, tile);
+    const int unit = blockIdx.x + s * gridDim.x;
+    if (unit < units) stage_load<BITS, DK, DIAG, YOKED, true>(smem + s * L.bytes, L, p, unit);
     cp_async_commit();
   }
 
   int it = 0;
-  for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++it) {
+  for (int unit = blockIdx.x; unit < units; unit += gridDim.x, ++it) {
     {
-      const int pre = tile + (STAGES - 1) * gridDim.x;
-      if (pre < p.tiles)
+      const int pre = unit + (STAGES - 1) * gridDim.x;
+      if (pre < units)
         stage_load<BITS, DK, DIAG, YOKED, true>(smem + ((it + STAGES - 1) % STAGES) * L.bytes, L, p,
                                                 pre);
       cp_async_commit();
@@ -361,170 +429,226 @@ __global__ void __launch_bounds__(kMaxThreads, 1) step_kernel(StepParams p) {
     cp_async_wait<STAGES - 1>();
     __syncthreads();
     unsigned char* st = smem + (it % STAGES) * L.bytes;
+    const size_t tile = static_cast<size_t>(unit / p.units_per_tile);
+    const size_t grow0 = tile * p.dv + static_cast<size_t>(unit % p.units_per_tile) * p.rb;
 
     if constexpr (BDR) {
-      // sign(k_j) per column, same interleaved layout as k
+      // sign(k_j) per column, in the layout of k
       const float* kvals = reinterpret_cast<const float*>(st + L.k);
       float* ss = reinterpret_cast<float*>(st + L.sk);
-      for (int j = tid; j < DK; j += blockDim.x) {
-        const int pos = (j / 32) * kChunkStride + pair_pos(j % 32);
+      for (int j = tid; j < DK; j += kThreads) {
+        const int pos = (j / 32) * kChunkStride + (j % 32);
         const float kv = kvals[pos];
         ss[pos] = kv > 0.0f ? 1.0f : (kv < 0.0f ? -1.0f : 0.0f);
       }
       __syncthreads();
     }
 
-    // ---- a1: load and unpack this thread's 32 codes
-    uint32_t w[CW];
-    {
-      const uint4* src = reinterpret_cast<const uint4*>(st + L.codes + (row * LPR + c) * (4 * CW));
-#pragma unroll
-      for (int q = 0; q < CW / 4; ++q) {
-        const uint4 u = src[q];
-        w[4 * q + 0] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
-      }
+    // per-unit column vectors of this thread's chunk
+    float2 kk[16];
+    load_pairs(st + L.k, c, kk);
+    float2 qq[Q_REG ? 16 : 1];
+    if constexpr (Q_REG) {
+      if (readout) load_pairs(st + L.q, c, qq);
     }
-    const float s_old = reinterpret_cast<const float*>(st + L.scales)[row * ng + g];
     const float* miscf = reinterpret_cast<const float*>(st + L.misc);
     const float beta = miscf[1];
-    const float v_i = reinterpret_cast<const float*>(st + L.v)[row];
-    const float2* kp = reinterpret_cast<const float2*>(st + L.k) + c * (kChunkStride / 2);
-    float2 kk[16];
-#pragma unroll
-    for (int m = 0; m < 16; ++m) kk[m] = kp[m];
+    const float a_scalar = DIAG ? 1.0f : miscf[0];
 
-    // ---- a2: dequantize and decay
-    float2 Sp[16];
-    decode_chunk<BITS>(w, Sp);
-    if constexpr (DIAG) {
-      const float2* ap = reinterpret_cast<const float2*>(st + L.a) + c * (kChunkStride / 2);
+    // NR rows of the unit at a time (rows rb0, rb0 + RP, ...): their chains
+    // are independent, so the scheduler can overlap them.  A missing second
+    // row repeats the first and is not stored.
+#pragma unroll 1
+    for (int rb0 = r0; rb0 < p.rb; rb0 += NR * RP) {
+      int row[NR];
+      bool valid[NR];
 #pragma unroll
-      for (int m = 0; m < 16; ++m) Sp[m] = __fmul2_rn(__fmul2_rn(Sp[m], f2(s_old)), ap[m]);
-    } else {
-      const float a = miscf[0];
-#pragma unroll
-      for (int m = 0; m < 16; ++m) Sp[m] = __fmul2_rn(__fmul2_rn(Sp[m], f2(s_old)), f2(a));
-    }
-
-    // ---- a3/a4: key projection and rank-1 write
-    float wcoef;
-    if constexpr (DELTA) {
-      float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-      for (int m = 0; m < 16; ++m) acc = __ffma2_rn(Sp[m], kk[m], acc);
-      const float u = row_tree<LPR>(acc);
-      wcoef = __fmul_rn(beta, __fsub_rn(v_i, u));
-    } else {
-      wcoef = __fmul_rn(beta, v_i);
-    }
-    float2 x[16];
-#pragma unroll
-    for (int m = 0; m < 16; ++m) x[m] = __ffma2_rn(f2(wcoef), kk[m], Sp[m]);
-
-    // ---- a5: readout from the updated state
-    if (readout) {
-      const float2* qp = reinterpret_cast<const float2*>(st + L.q) + c * (kChunkStride / 2);
-      float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-      for (int m = 0; m < 16; ++m) acc = __ffma2_rn(x[m], qp[m], acc);
-      const float o = row_tree<LPR>(acc);
-      if (c == 0) p.o[static_cast<size_t>(tile) * p.dv + row] = o;
-    }
-
-    // ---- a6/a7: scale selection (yoked shadow update)
-    float sp;
-    if constexpr (POLICY == 0) {
-      const float m = row_max<LPR>(chunk_absmax(x), p.group);
-      sp = __fdiv_rn(m, kQf);
-    } else if constexpr (POLICY == 1) {
-      sp = s_old;
-    } else {
-      // shadow chunk from shared memory (swizzled 16-byte units)
-      const int rc = row * LPR + c;
-      const float4* rs = reinterpret_cast<const float4*>(st + L.shadow + rc * 128);
-      float r[32];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float4 t = rs[u ^ (rc & 7)];
-        r[4 * u] = t.x; r[4 * u + 1] = t.y; r[4 * u + 2] = t.z; r[4 * u + 3] = t.w;
+      for (int i = 0; i < NR; ++i) {
+        row[i] = rb0 + i * RP;
+        valid[i] = row[i] < p.rb;
+        if (!valid[i]) row[i] = rb0;
       }
-      // R' = R * a
-      if constexpr (DIAG) {
-        const float* ap = reinterpret_cast<const float*>(st + L.a) + c * kChunkStride;
+      // ---- a1: load and unpack this thread's 32 codes of each row
+      float2 Sp[NR][16];
+      float s_old[NR], v_i[NR];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) r[j] = __fmul_rn(r[j], ap[pair_pos(j)]);
-      } else {
-        const float a = miscf[0];
+      for (int i = 0; i < NR; ++i) {
+        uint32_t w[CW];
+        const uint4* src = reinterpret_cast<const uint4*>(st + L.codes + (row[i] * LPR + c) * (4 * CW));
 #pragma unroll
-        for (int j = 0; j < 32; ++j) r[j] = __fmul_rn(r[j], a);
-      }
-      float wr;
-      if constexpr (DELTA) {
-        float a0 = 0.0f, a1 = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          a0 = __fmaf_rn(r[j], kk[j].x, a0);
-          a1 = __fmaf_rn(r[16 + j], kk[j].y, a1);
+        for (int q = 0; q < CW / 4; ++q) {
+          const uint4 u = src[q];
+          w[4 * q + 0] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
         }
-        const float ur = row_tree<LPR>(make_float2(a0, a1));
-        wr = __fmul_rn(beta, __fsub_rn(v_i, ur));
-      } else {
-        wr = wcoef;
+        s_old[i] = reinterpret_cast<const float*>(st + L.scales)[row[i] * ng + g];
+        v_i[i] = reinterpret_cast<const float*>(st + L.v)[row[i]];
+        decode_chunk<BITS>(w, Sp[i]);
       }
-      float mr = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        r[j] = __fmaf_rn(wr, kk[j].x, r[j]);
-        r[16 + j] = __fmaf_rn(wr, kk[j].y, r[16 + j]);
-        mr = fmaxf(mr, fmaxf(fabsf(r[j]), fabsf(r[16 + j])));
-      }
-      float* rg = p.shadow + static_cast<size_t>(tile) * p.dv * DK + row * DK + 32 * c;
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        uint32_t ww[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ww[e] = __float_as_uint(r[8 * h + e]);
-        st_global_v8(rg + 8 * h, ww);
-      }
-      mr = row_max<LPR>(mr, p.group);
-      sp = __fdiv_rn(mr, kQf);
-    }
 
-    // ---- a8: round (and BDR)
-    uint32_t out[CW];
-    if (sp > 0.0f) {
-      const float inv = __frcp_rn(sp);
-      bool clamp;
+      // ---- a2: dequantize with the decayed scale, S' = c * (s * a)
+      if constexpr (DIAG) {
+        float2 aa[16];
+        load_pairs(st + L.a, c, aa);
+#pragma unroll
+        for (int i = 0; i < NR; ++i)
+#pragma unroll
+          for (int m = 0; m < 16; ++m) Sp[i][m] = __fmul2_rn(Sp[i][m], __fmul2_rn(f2(s_old[i]), aa[m]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+          const float sa = __fmul_rn(s_old[i], a_scalar);
+#pragma unroll
+          for (int m = 0; m < 16; ++m) Sp[i][m] = __fmul2_rn(Sp[i][m], f2(sa));
+        }
+      }
+
+      // ---- a3/a4: key projection and rank-1 write
+      float wcoef[NR];
+      if constexpr (DELTA) {
+        float2 acc[NR];
+#pragma unroll
+        for (int i = 0; i < NR; ++i) acc[i] = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int m = 0; m < 16; ++m)
+#pragma unroll
+          for (int i = 0; i < NR; ++i) acc[i] = __ffma2_rn(Sp[i][m], kk[m], acc[i]);
+#pragma unroll
+        for (int i = 0; i < NR; ++i) wcoef[i] = __fmul_rn(beta, __fsub_rn(v_i[i], row_tree<LPR>(acc[i])));
+      } else {
+#pragma unroll
+        for (int i = 0; i < NR; ++i) wcoef[i] = __fmul_rn(beta, v_i[i]);
+      }
+      float2 x[NR][16];
+#pragma unroll
+      for (int i = 0; i < NR; ++i)
+#pragma unroll
+        for (int m = 0; m < 16; ++m) x[i][m] = __ffma2_rn(f2(wcoef[i]), kk[m], Sp[i][m]);
+
+      // ---- a5: readout from the updated state
+      if (readout) {
+        float2 acc[NR];
+#pragma unroll
+        for (int i = 0; i < NR; ++i) acc[i] = make_float2(0.0f, 0.0f);
+        if constexpr (Q_REG) {
+#pragma unroll
+          for (int m = 0; m < 16; ++m)
+#pragma unroll
+            for (int i = 0; i < NR; ++i) acc[i] = __ffma2_rn(x[i][m], qq[m], acc[i]);
+        } else {
+          const float4* qp4 = reinterpret_cast<const float4*>(st + L.q) + c * (kChunkStride / 4);
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const float4 t = qp4[m];
+#pragma unroll
+            for (int i = 0; i < NR; ++i) {
+              acc[i] = __ffma2_rn(x[i][2 * m], make_float2(t.x, t.y), acc[i]);
+              acc[i] = __ffma2_rn(x[i][2 * m + 1], make_float2(t.z, t.w), acc[i]);
+            }
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+          const float o = row_tree<LPR>(acc[i]);
+          if (c == 0 && valid[i]) p.o[grow0 + row[i]] = o;
+        }
+      }
+
+      // ---- a6/a7: scale selection (yoked shadow update)
+      float sp[NR];
       if constexpr (POLICY == 0) {
-        // |x| <= group max, so |x * inv| <= qmax(1 + 2^-23) rounds inside the
-        // range unless the scale is not a normal finite float
-        clamp = !(sp >= 1.17549435e-38f && sp <= 3.40282347e38f);
-      } else {
-        const float xm = chunk_absmax(x);
-        clamp = !(__fmaf_rn(xm, inv, kOff) <= kOff + kQf);
-      }
-      float2 y[16];
-      round_chunk<BITS>(x, inv, clamp, y);
-      if constexpr (BDR) {
-        const float2* skp = reinterpret_cast<const float2*>(st + L.sk) + c * (kChunkStride / 2);
-        const float sw = wcoef > 0.0f ? 1.0f : (wcoef < 0.0f ? -1.0f : 0.0f);
-        bdr_chunk<BITS>(y, Sp, skp, sw, sp);
-      }
-      pack_chunk<BITS>(y, out);
-    } else {
 #pragma unroll
-      for (int q = 0; q < CW; ++q) out[q] = 0u;
-    }
+        for (int i = 0; i < NR; ++i) sp[i] = div_qmax_rn<QMAX>(row_max<LPR>(chunk_absmax(x[i]), p.group));
+      } else if constexpr (POLICY == 1) {
+#pragma unroll
+        for (int i = 0; i < NR; ++i) sp[i] = s_old[i];
+      } else {
+        static_assert(NR == 1, "the yoked path handles one row at a time");
+        // shadow chunk from shared memory (swizzled 16-byte units), as pairs
+        const int rc = row[0] * LPR + c;
+        const float4* rs = reinterpret_cast<const float4*>(st + L.shadow + rc * 128);
+        float2 rr[16];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float4 t = rs[u ^ (rc & 7)];
+          rr[2 * u] = make_float2(t.x, t.y);
+          rr[2 * u + 1] = make_float2(t.z, t.w);
+        }
+        // R' = R * a
+        if constexpr (DIAG) {
+          float2 aa[16];
+          load_pairs(st + L.a, c, aa);
+#pragma unroll
+          for (int m = 0; m < 16; ++m) rr[m] = __fmul2_rn(rr[m], aa[m]);
+        } else {
+#pragma unroll
+          for (int m = 0; m < 16; ++m) rr[m] = __fmul2_rn(rr[m], f2(a_scalar));
+        }
+        float wr;
+        if constexpr (DELTA) {
+          float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+          for (int m = 0; m < 16; ++m) acc = __ffma2_rn(rr[m], kk[m], acc);
+          wr = __fmul_rn(beta, __fsub_rn(v_i[0], row_tree<LPR>(acc)));
+        } else {
+          wr = wcoef[0];
+        }
+#pragma unroll
+        for (int m = 0; m < 16; ++m) rr[m] = __ffma2_rn(f2(wr), kk[m], rr[m]);
+        float* rg = p.shadow + (grow0 + row[0]) * DK + 32 * c;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          uint32_t ww[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            ww[2 * e] = __float_as_uint(rr[4 * h + e].x);
+            ww[2 * e + 1] = __float_as_uint(rr[4 * h + e].y);
+          }
+          st_global_v8(rg + 8 * h, ww);
+        }
+        sp[0] = div_qmax_rn<QMAX>(row_max<LPR>(chunk_absmax(rr), p.group));
+      }
 
-    // ---- a9: store codes (and scales)
-    uint8_t* cg = p.codes + static_cast<size_t>(tile) * p.dv * DK * BITS / 8 + (row * LPR + c) * (4 * CW);
-    if constexpr (CW == 4) {
-      *reinterpret_cast<uint4*>(cg) = make_uint4(out[0], out[1], out[2], out[3]);
-    } else {
-      st_global_v8(cg, out);
-    }
-    if constexpr (POLICY != 1) {
-      if ((32 * c) % p.group == 0) p.scales[(static_cast<size_t>(tile) * p.dv + row) * ng + g] = sp;
+      // ---- a8/a9: round (and BDR), pack, store codes (and scales)
+#pragma unroll
+      for (int i = 0; i < NR; ++i) {
+        uint32_t out[CW];
+        if (sp[i] > 0.0f) {
+          const float inv = recip_rn(sp[i]);
+          bool clamp;
+          if constexpr (POLICY == 0) {
+            // |x| <= group max, so |x * inv| <= qmax(1 + 2^-23) rounds inside
+            // the range whenever the scale is a normal float below 2^126
+            clamp = !(sp[i] >= 0x1p-126f && sp[i] < 0x1p126f);
+          } else {
+            const float xm = chunk_absmax(x[i]);
+            clamp = !(__fmaf_rn(xm, inv, kOff) <= kOff + kQf);
+          }
+          float2 y[16];
+          round_chunk<BITS>(x[i], inv, clamp, y);
+          if constexpr (BDR) {
+            float2 sk[16];
+            load_pairs(st + L.sk, c, sk);
+            const float sw = wcoef[i] > 0.0f ? 1.0f : (wcoef[i] < 0.0f ? -1.0f : 0.0f);
+            bdr_chunk<BITS>(y, Sp[i], sk, sw, sp[i]);
+          }
+          pack_chunk<BITS>(y, out);
+        } else {
+#pragma unroll
+          for (int q = 0; q < CW; ++q) out[q] = 0u;
+        }
+        if (valid[i]) {
+          const size_t grow = grow0 + row[i];
+          uint8_t* cg = p.codes + grow * (DK * BITS / 8) + c * (4 * CW);
+          if constexpr (CW == 4) {
+            *reinterpret_cast<uint4*>(cg) = make_uint4(out[0], out[1], out[2], out[3]);
+          } else {
+            st_global_v8(cg, out);
+          }
+          if constexpr (POLICY != 1) {
+            if (writes_scale) p.scales[grow * ng + g] = sp[i];
+          }
+        }
+      }
     }
     __syncthreads();
   }
@@ -532,30 +656,32 @@ __global__ void __launch_bounds__(kMaxThreads, 1) step_kernel(StepParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// readout of the stored state (no update)
+// readout of the stored state (no update): o = (c * s) . q
 // ---------------------------------------------------------------------------
 template <int BITS, int DK, int STAGES>
-__global__ void __launch_bounds__(kMaxThreads, 1) readout_kernel(StepParams p) {
+__global__ void __launch_bounds__(kThreads, QS_MIN_BLOCKS) readout_kernel(StepParams p) {
   constexpr int LPR = DK / 32;
+  constexpr int RP = kThreads / LPR;
   constexpr int CW = BITS;
   extern __shared__ __align__(128) unsigned char smem[];
-  const StageLayout L(BITS, DK, p.dv, p.group, false, false, false);
+  const StageLayout L(BITS, DK, p.rb, p.group, false, false, false);
   const int tid = threadIdx.x;
-  const int row = tid / LPR, c = tid % LPR;
+  const int c = tid % LPR, r0 = tid / LPR;
   const int ng = DK / p.group;
   const int g = (32 * c) / p.group;
+  const int units = p.tiles * p.units_per_tile;
 
 #pragma unroll
   for (int s = 0; s < STAGES - 1; ++s) {
-    const int tile = blockIdx.x + s * gridDim.x;
-    if (tile < p.tiles) stage_load<BITS, DK, false, false, false>(smem + s * L.bytes, L, p, tile);
+    const int unit = blockIdx.x + s * gridDim.x;
+    if (unit < units) stage_load<BITS, DK, false, false, false>(smem + s * L.bytes, L, p, unit);
     cp_async_commit();
   }
   int it = 0;
-  for (int tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++it) {
+  for (int unit = blockIdx.x; unit < units; unit += gridDim.x, ++it) {
     {
-      const int pre = tile + (STAGES - 1) * gridDim.x;
-      if (pre < p.tiles)
+      const int pre = unit + (STAGES - 1) * gridDim.x;
+      if (pre < units)
         stage_load<BITS, DK, false, false, false>(smem + ((it + STAGES - 1) % STAGES) * L.bytes, L,
                                                   p, pre);
       cp_async_commit();
@@ -563,22 +689,28 @@ __global__ void __launch_bounds__(kMaxThreads, 1) readout_kernel(StepParams p) {
     cp_async_wait<STAGES - 1>();
     __syncthreads();
     unsigned char* st = smem + (it % STAGES) * L.bytes;
-    uint32_t w[CW];
-    const uint4* src = reinterpret_cast<const uint4*>(st + L.codes + (row * LPR + c) * (4 * CW));
+    const size_t tile = static_cast<size_t>(unit / p.units_per_tile);
+    const size_t grow0 = tile * p.dv + static_cast<size_t>(unit % p.units_per_tile) * p.rb;
+    float2 qq[16];
+    load_pairs(st + L.q, c, qq);
+#pragma unroll 1
+    for (int r = r0; r < p.rb; r += RP) {
+      uint32_t w[CW];
+      const uint4* src = reinterpret_cast<const uint4*>(st + L.codes + (r * LPR + c) * (4 * CW));
 #pragma unroll
-    for (int q = 0; q < CW / 4; ++q) {
-      const uint4 u = src[q];
-      w[4 * q + 0] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
+      for (int q = 0; q < CW / 4; ++q) {
+        const uint4 u = src[q];
+        w[4 * q + 0] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
+      }
+      const float s = reinterpret_cast<const float*>(st + L.scales)[r * ng + g];
+      float2 d[16];
+      decode_chunk<BITS>(w, d);
+      float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int m = 0; m < 16; ++m) acc = __ffma2_rn(__fmul2_rn(d[m], f2(s)), qq[m], acc);
+      const float o = row_tree<LPR>(acc);
+      if (c == 0) p.o[grow0 + r] = o;
     }
-    const float s = reinterpret_cast<const float*>(st + L.scales)[row * ng + g];
-    float2 d[16];
-    decode_chunk<BITS>(w, d);
-    const float2* qp = reinterpret_cast<const float2*>(st + L.q) + c * (kChunkStride / 2);
-    float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-    for (int m = 0; m < 16; ++m) acc = __ffma2_rn(__fmul2_rn(d[m], f2(s)), qp[m], acc);
-    const float o = row_tree<LPR>(acc);
-    if (c == 0) p.o[static_cast<size_t>(tile) * p.dv + row] = o;
     __syncthreads();
   }
   cp_async_wait<0>();
@@ -593,27 +725,24 @@ __global__ void __launch_bounds__(256) init_kernel(const float* __restrict__ S0,
                                                    int group) {
   constexpr int LPR = DK / 32;
   constexpr int CW = BITS;
-  constexpr float kQf = BITS == 4 ? 7.0f : 127.0f;
+  constexpr int QMAX = BITS == 4 ? 7 : 127;
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long rowg = gid / LPR;
   const int c = static_cast<int>(gid % LPR);
   const bool active = rowg < rows;  // whole warps stay for the shuffles
-  float r[32];
-  const float* src = S0 + (active ? rowg : 0) * DK + 32 * c;
+  float2 x[16];
+  const float4* src = reinterpret_cast<const float4*>(S0 + (active ? rowg : 0) * DK + 32 * c);
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
-    const float4 t = reinterpret_cast<const float4*>(src)[u];
-    r[4 * u] = t.x; r[4 * u + 1] = t.y; r[4 * u + 2] = t.z; r[4 * u + 3] = t.w;
+    const float4 t = src[u];
+    x[2 * u] = make_float2(t.x, t.y);
+    x[2 * u + 1] = make_float2(t.z, t.w);
   }
-  float2 x[16];
-#pragma unroll
-  for (int m = 0; m < 16; ++m) x[m] = make_float2(r[m], r[16 + m]);
-  const float m = row_max<LPR>(chunk_absmax(x), group);
-  const float s = __fdiv_rn(m, kQf);
+  const float s = div_qmax_rn<QMAX>(row_max<LPR>(chunk_absmax(x), group));
   uint32_t out[CW];
   if (s > 0.0f) {
-    const float inv = __frcp_rn(s);
-    const bool clamp = !(s >= 1.17549435e-38f && s <= 3.40282347e38f);
+    const float inv = recip_rn(s);
+    const bool clamp = !(s >= 0x1p-126f && s < 0x1p126f);
     float2 y[16];
     round_chunk<BITS>(x, inv, clamp, y);
     pack_chunk<BITS>(y, out);
@@ -631,10 +760,9 @@ __global__ void __launch_bounds__(256) init_kernel(const float* __restrict__ S0,
   const int ng = DK / group, g = (32 * c) / group;
   if ((32 * c) % group == 0) scales[rowg * ng + g] = s;
   if (shadow != nullptr) {
-    float* dst = shadow + rowg * DK + 32 * c;
+    float4* dst = reinterpret_cast<float4*>(shadow + rowg * DK + 32 * c);
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
-      reinterpret_cast<float4*>(dst)[u] = make_float4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
+    for (int u = 0; u < 8; ++u) dst[u] = make_float4(x[2 * u].x, x[2 * u].y, x[2 * u + 1].x, x[2 * u + 1].y);
   }
 }
 

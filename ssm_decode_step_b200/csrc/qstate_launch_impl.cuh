@@ -7,10 +7,22 @@
 
 namespace qs {
 
-// Stages of the cp.async ring: the yoked state carries a 64 KB FP32 shadow per
-// tile, so it keeps two stages; the others keep four.
+// Stages of the cp.async ring per CTA.
 template <int POLICY>
-constexpr int step_stages() { return POLICY == 2 ? 2 : 4; }
+constexpr int step_stages() { return POLICY == 2 ? 3 : 4; }
+
+// Rows per work unit: the largest of 128, 64, 32, 16 that divides dv and keeps
+// one stage within `budget` bytes (so that three or four CTAs fit per SM).
+inline int choose_rb(int bits, int dk, int dv, int group, bool diag, bool bdr, bool yoked) {
+  const int budget = yoked ? 21 * 1024 : 13 * 1024;
+  int best = 16;
+  for (int rb = 128; rb >= 16; rb /= 2) {
+    if (dv % rb != 0) continue;
+    if (StageLayout(bits, dk, rb, group, diag, bdr, yoked).bytes <= budget) return rb;
+    best = rb;
+  }
+  return best;
+}
 
 // Allow the kernel the device's full opt-in shared memory (once per kernel).
 template <typename K>
@@ -27,40 +39,45 @@ static cudaError_t allow_smem(K kernel, std::once_flag& flag) {
 }
 
 template <typename K>
-static cudaError_t launch_persistent(K kernel, int tiles, int threads, size_t smem,
-                                     const StepParams& p, cudaStream_t stream) {
+static cudaError_t launch_persistent(K kernel, size_t smem, const StepParams& p,
+                                     cudaStream_t stream) {
   int per_sm = 0;
-  cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem);
+  cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, smem);
   if (err != cudaSuccess) return err;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  const long long units = static_cast<long long>(p.tiles) * p.units_per_tile;
   long long grid = static_cast<long long>(per_sm) * device_sm_count();
-  if (grid > tiles) grid = tiles;
-  kernel<<<static_cast<int>(grid), threads, smem, stream>>>(p);
+  if (grid > units) grid = units;
+  kernel<<<static_cast<int>(grid), kThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
 template <int BITS, int DK, int POLICY, bool BDR, bool DELTA, bool DIAG>
-cudaError_t launch_step(const StepParams& p, cudaStream_t stream) {
+cudaError_t launch_step(const StepParams& p0, cudaStream_t stream) {
   constexpr int S = step_stages<POLICY>();
   auto kernel = step_kernel<BITS, DK, POLICY, BDR, DELTA, DIAG, S>;
   static std::once_flag flag;
   cudaError_t err = allow_smem(kernel, flag);
   if (err != cudaSuccess) return err;
-  const StageLayout L(BITS, DK, p.dv, p.group, DIAG, BDR, POLICY == 2);
-  return launch_persistent(kernel, p.tiles, p.dv * (DK / 32), static_cast<size_t>(S) * L.bytes, p,
-                           stream);
+  StepParams p = p0;
+  p.rb = choose_rb(BITS, DK, p.dv, p.group, DIAG, BDR, POLICY == 2);
+  p.units_per_tile = p.dv / p.rb;
+  const StageLayout L(BITS, DK, p.rb, p.group, DIAG, BDR, POLICY == 2);
+  return launch_persistent(kernel, static_cast<size_t>(S) * L.bytes, p, stream);
 }
 
 template <int BITS, int DK>
-cudaError_t launch_readout(const StepParams& p, cudaStream_t stream) {
+cudaError_t launch_readout(const StepParams& p0, cudaStream_t stream) {
   constexpr int S = 4;
   auto kernel = readout_kernel<BITS, DK, S>;
   static std::once_flag flag;
   cudaError_t err = allow_smem(kernel, flag);
   if (err != cudaSuccess) return err;
-  const StageLayout L(BITS, DK, p.dv, p.group, false, false, false);
-  return launch_persistent(kernel, p.tiles, p.dv * (DK / 32), static_cast<size_t>(S) * L.bytes, p,
-                           stream);
+  StepParams p = p0;
+  p.rb = choose_rb(BITS, DK, p.dv, p.group, false, false, false);
+  p.units_per_tile = p.dv / p.rb;
+  const StageLayout L(BITS, DK, p.rb, p.group, false, false, false);
+  return launch_persistent(kernel, static_cast<size_t>(S) * L.bytes, p, stream);
 }
 
 template <int BITS, int DK>

@@ -24,7 +24,7 @@ QS_OK, QS_ERR_INVALID_ARG, QS_ERR_UNSUPPORTED, QS_ERR_CUDA = 0, 1, 2, 3
 
 # Every entry point that include/qstate.h declares.
 EXPORTS = ("qstate_query_sizes", "qstate_init", "qstate_decode_step", "qstate_readout",
-           "qstate_status_string", "qstate_version")
+           "qstate_selfcheck", "qstate_status_string", "qstate_version")
 
 
 class QStateError(RuntimeError):
@@ -55,7 +55,9 @@ def lib() -> ctypes.CDLL:
         L.qstate_init.argtypes = [C, P, P, P, P, P]
         L.qstate_decode_step.argtypes = [C, P, P, P, P, P, P, P, P, P, P]
         L.qstate_readout.argtypes = [C, P, P, P, P, P]
-        for f in (L.qstate_query_sizes, L.qstate_init, L.qstate_decode_step, L.qstate_readout):
+        L.qstate_selfcheck.argtypes = [P, P]
+        for f in (L.qstate_query_sizes, L.qstate_init, L.qstate_decode_step, L.qstate_readout,
+                  L.qstate_selfcheck):
             f.restype = ctypes.c_int
         L.qstate_status_string.argtypes = [ctypes.c_int]
         L.qstate_status_string.restype = ctypes.c_char_p
@@ -140,6 +142,16 @@ def readout(cfg: Config, codes, scales, q, o, stream=None) -> None:
     cc = cfg.c()
     _check(lib().qstate_readout(ctypes.byref(cc), _ptr(codes), _ptr(scales), _ptr(q), _ptr(o),
                                 _stream(stream)), "qstate_readout")
+
+
+def selfcheck(stream=None):
+    """Run qstate_selfcheck on the current GPU; returns the three mismatch
+    counts (reciprocal, division by 7, division by 127), all expected 0."""
+    import torch
+    bad = torch.zeros(3, dtype=torch.int64, device="cuda")
+    _check(lib().qstate_selfcheck(bad.data_ptr(), _stream(stream)), "qstate_selfcheck")
+    torch.cuda.synchronize()
+    return [int(x) for x in bad.cpu()]
 
 
 class QState:

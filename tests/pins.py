@@ -67,7 +67,7 @@ def pin_linear_write_sum_of_outer_products():
     """delta = 0, Lambda = I, beta = 1, S0 = 0  =>  S_H = sum_t v_t k_t^T."""
     rng = _rng(10)
     for decay in ("scalar", "diagonal"):
-        T, dk, dv, H = 3, 16, 5, 12
+        T, dk, dv, H = 3, 32, 5, 12
         cfg = O.OracleConfig(T, dk, dv, 8, 16, 0, decay)
         S = np.zeros((T, dv, dk), F32)
         acc = np.zeros((T, dv, dk))
@@ -334,7 +334,7 @@ def pin_bdr_bruteforce():
     clamped; it equals nearest when sigma = 0 or nearest does not reverse; and
     otherwise it is the non-reversing code closest to the nearest one."""
     rng = _rng(22)
-    T, dk, dv = 8, 16, 4
+    T, dk, dv = 8, 32, 4
     for bits in (4, 8):
         for policy in ("persistent", "dynamic"):
             qmax = (1 << (bits - 1)) - 1
@@ -352,8 +352,9 @@ def pin_bdr_bruteforce():
                 Nst = O.State(cN, prev.codes.copy(), prev.scales.copy())
                 O.step(Nst, q, k, v, a, b, want_o=False)
                 O.step(B, q, k, v, a, b, want_o=False)
-                d = (prev.codes.astype(F32) * np.repeat(prev.scales, 16, axis=-1)).astype(F32)
-                Sp = (d * a[:, None, :]).astype(F32)
+                # S' = c * (s * a), the decayed scale first (as the step defines it)
+                sa = (np.repeat(prev.scales, 16, axis=-1) * a[:, None, :]).astype(F32)
+                Sp = (prev.codes.astype(F32) * sa).astype(F32)
                 w = (b[:, None] * v).astype(F32)
                 sigma = np.sign(w)[:, :, None] * np.sign(k)[:, None, :]
                 s_el = np.repeat(B.scales, 16, axis=-1)
@@ -515,24 +516,32 @@ def pin_pack_layout():
 
 
 def pin_dot_order():
-    """The fixed dot-product order: pairwise tree over 16-column segments."""
+    """The fixed dot-product order: even / odd chains within each 32-column
+    chunk, pairwise tree over the chunks (worked examples in
+    tests/golden/layout_and_order.json)."""
     with open(os.path.join(GOLDEN, "layout_and_order.json")) as f:
-        d = json.load(f)["dot_order"]
-    n = d["n"]
-    a = np.zeros(n, F32)
-    b = np.zeros(n, F32)
-    for s, val in enumerate(d["segment_values"]):
-        a[16 * s + 3] = val
-        b[16 * s + 3] = 1.0
-    assert O.dot(a, b) == F32(d["expected"])
+        data = json.load(f)
+    for key in ("dot_order_chunks", "dot_order_even_odd"):
+        d = data[key]
+        a = np.zeros(d["n"], F32)
+        b = np.zeros(d["n"], F32)
+        for idx, val in d["products"].items():
+            a[int(idx)] = val
+            b[int(idx)] = 1.0
+        assert O.dot(a, b) == F32(d["expected"]), key
+        # the order matters: a left-to-right sum gives another value
+        acc = F32(0.0)
+        for j in range(d["n"]):
+            acc = F32(acc + F32(a[j] * b[j]))
+        assert acc == F32(d["left_to_right"]), key
     # and within the error bound of the exact value on random data
     rng = _rng(27)
-    for n in (16, 32, 64, 128, 256):
+    for n in (32, 64, 128, 256):
         for _ in range(20):
             a = rng.standard_normal(n).astype(F32)
             b = rng.standard_normal(n).astype(F32)
             exact = float(np.dot(a.astype(np.float64), b.astype(np.float64)))
-            bound = (16 + np.log2(n // 16) + 2) * 2.0 ** -24 * float(np.abs(a.astype(np.float64) * b).sum())
+            bound = (16 + np.log2(n // 32) + 3) * 2.0 ** -24 * float(np.abs(a.astype(np.float64) * b).sum())
             assert abs(float(O.dot(a, b)) - exact) <= bound
 
 

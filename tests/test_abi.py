@@ -55,7 +55,7 @@ def _raw(cfg):
     ("dk", 96, Q.QS_ERR_UNSUPPORTED),
     ("dk", 256, Q.QS_ERR_UNSUPPORTED),
     ("dv", 24, Q.QS_ERR_UNSUPPORTED),
-    ("dv", 192, Q.QS_ERR_UNSUPPORTED),
+    ("dv", 4112, Q.QS_ERR_UNSUPPORTED),
     ("dv", 0, Q.QS_ERR_INVALID_ARG),
     ("num_tiles", -1, Q.QS_ERR_INVALID_ARG),
     ("delta", 2, Q.QS_ERR_INVALID_ARG),
