@@ -11,9 +11,10 @@ metric is decode steps/s (whole job; N GPUs run independent shards, so
 scaling is weak) and the algorithmic state traffic in GB/s as a fraction of
 the measured HBM peak.
 
-L2 residency: the workload's state is smaller than B200's L2, so steps rotate
-over G independent request groups whose states together exceed 2x the L2
-size; step t uses group t mod G and pool slot t mod P of the inputs.  No
+L2 residency: an arm's state can be smaller than B200's L2, so each arm's
+steps rotate over G independent request groups whose states together exceed
+2x the L2 size (G chosen per arm, since the arms are timed one after the
+other); step t uses group t mod G and pool slot t mod P of the inputs.  No
 state or input is therefore warm in L2 when its step runs.
 
 Timing: W untimed warm-up steps per arm (eager and graph), then the states
@@ -223,42 +224,53 @@ def max_over_ranks(dist, values, device):
 # CPU baseline: the oracle as it stands, on a bounded sample of tiles
 # ---------------------------------------------------------------------------
 
-def oracle_sample_rate(w: W.Workload, steps: int, budget_s: float, max_tiles: int = 256):
-    """Oracle steps/s on the host, estimated from `steps` steps of a tile
-    sample sized so the whole measurement takes about budget_s seconds."""
+def oracle_sample_rate(w: W.Workload, budget_s: float, steps: int = 0, max_tiles: int = 256):
+    """Oracle steps/s on the host cores, measured on a seeded sample of tiles
+    and scaled to whole steps (tiles are independent, so time is linear in
+    the number of tiles).  With `steps` given, exactly that many steps run and
+    the sample is sized to take about budget_s; otherwise max_tiles tiles run
+    for as many steps as fill about budget_s."""
     from oracle import oracle as O
     rng = np.random.default_rng(12345)
-    # calibrate on one tile per arm
-    calib_tiles = np.array([0])
-    S0 = W.initial_state(w, calib_tiles)
-    slot0 = W.slot(w, 0, calib_tiles)
-    t0 = time.perf_counter()
-    for arm in w.arms:
-        cfg = O.OracleConfig(1, w.dk, w.dv, arm.bits, arm.group, w.delta, w.decay, arm.policy,
-                             arm.rounding)
-        st = O.init(cfg, S0)
-        O.step(st, *slot0, want_o=w.readout)
-    per_tile_step = max(time.perf_counter() - t0, 1e-6)
     threads = O.num_threads()
-    n = int(budget_s * threads / (per_tile_step * max(steps, 1)))
-    n = max(threads, min(n, max_tiles, w.tiles))
-    tiles = np.sort(rng.choice(w.tiles, size=n, replace=False))
-    S0 = W.initial_state(w, tiles)
-    states = []
-    for arm in w.arms:
-        cfg = O.OracleConfig(n, w.dk, w.dv, arm.bits, arm.group, w.delta, w.decay, arm.policy,
-                             arm.rounding)
-        states.append(O.init(cfg, S0))
+
+    def make(n):
+        tiles = np.sort(rng.choice(w.tiles, size=n, replace=False))
+        S0 = W.initial_state(w, tiles)
+        sts = []
+        for arm in w.arms:
+            cfg = O.OracleConfig(n, w.dk, w.dv, arm.bits, arm.group, w.delta, w.decay, arm.policy,
+                                 arm.rounding)
+            sts.append(O.init(cfg, S0))
+        return tiles, sts
+
+    # calibration: one step of a small sample (untimed warm-up of the oracle)
+    n0 = min(w.tiles, max(threads, 16))
+    tiles, sts = make(n0)
+    inp = W.slot(w, 0, tiles)
+    t0 = time.perf_counter()
+    for st in sts:
+        O.step(st, *inp, want_o=w.readout)
+    per_tile_step = max(time.perf_counter() - t0, 1e-6) / n0
+    if steps:
+        n = int(budget_s / (per_tile_step * steps))
+        n = max(min(threads, w.tiles), min(n, max_tiles, w.tiles))
+    else:
+        n = min(max_tiles, w.tiles)
+        steps = int(budget_s / (per_tile_step * n))
+        steps = max(2, min(steps, 100000))
+    tiles, sts = make(n)
     P = min(steps, 16)
     pool = [W.slot(w, t, tiles) for t in range(P)]
     t0 = time.perf_counter()
     for t in range(steps):
         inp = pool[t % P]
-        for st in states:
+        for st in sts:
             O.step(st, *inp, want_o=w.readout)
     dt = time.perf_counter() - t0
     rate = (n / w.tiles) * steps / dt
-    sample = f"{n} of {w.tiles} tiles (seeded random), {steps} steps, all {len(w.arms)} arms"
+    sample = (f"{n} of {w.tiles} tiles (seeded random sample), {steps} steps, all {len(w.arms)} arms; "
+              f"steps/s scaled by {w.tiles}/{n}")
     return rate, threads, sample, dt
 
 
@@ -288,26 +300,33 @@ def run_ours(args):
 
     # request groups so that all groups' states exceed 2x L2
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    per_group = sum(state_bytes(w, a) for a in arms)
-    G = args.groups or max(1, -(-2 * l2 // per_group))
-    while P % G:
-        G += 1
+    pool_bytes = P * sum(a[0].nbytes for a in host)
+
+    def groups_for(arm):
+        G = args.groups or max(1, -(-2 * l2 // state_bytes(w, arm)))
+        G = min(G, P)            # every group needs its own input slots in the cycle
+        while P % G:             # the captured cycle of P steps visits each group equally
+            G -= 1
+        return G
+
+    groups = [groups_for(a) for a in arms]
+    l2_resident = [g * state_bytes(w, a) + pool_bytes < 2 * l2 for g, a in zip(groups, arms)]
     S0 = torch.from_numpy(W.initial_state(w)).to(dev)
 
     cfgs = [Config(w.tiles, w.dk, w.dv, a.bits, a.group, w.delta, w.decay, a.policy, a.rounding)
             for a in arms]
-    states = [[QState(c, dev) for _ in range(G)] for c in cfgs]
+    states = [[QState(c, dev) for _ in range(g)] for c, g in zip(cfgs, groups)]
     outs = [torch.empty((w.tiles, w.dv), dtype=torch.float32, device=dev) if readout else None
             for _ in arms]
 
     def reinit():
         for ai, c in enumerate(cfgs):
-            for g in range(G):
-                states[ai][g].init(S0)
+            for st in states[ai]:
+                st.init(S0)
 
     def launch(ai, t):
         s = t % P
-        st = states[ai][t % G]
+        st = states[ai][t % len(states[ai])]
         st.step(pool[0][s], pool[1][s], pool[2][s], pool[3][s], pool[4][s], outs[ai])
 
     stream = torch.cuda.Stream(device=dev)
@@ -403,8 +422,13 @@ def run_ours(args):
             "step": f"one token for all {w.tiles} tiles under each arm ({len(arms)} launches)",
             "arms": [a.name for a in arms],
             "readout": readout,
-            "l2": f"inputs larger than L2: {G} request groups x {per_group / 1e6:.1f} MB state "
-                  f"+ {P} input slots rotated (L2 {l2 / 1e6:.0f} MB)",
+            "l2": "; ".join(
+                (f"{a.name}: L2-resident ({g} groups x {state_bytes(w, a) / 1e6:.3f} MB state, "
+                 f"smaller than L2)" if res else
+                 f"{a.name}: inputs larger than L2 ({g} request groups x "
+                 f"{state_bytes(w, a) / 1e6:.1f} MB state + {pool_bytes / 1e6:.0f} MB of input "
+                 f"slots rotated; L2 {l2 / 1e6:.0f} MB)")
+                for a, g, res in zip(arms, groups, l2_resident)),
             "parallelism": f"independent tile shards, {ws} GPU(s), no collective on the step",
         },
         "state_gbs": round(gbs, 1),
@@ -426,7 +450,7 @@ def run_ours(args):
         "clocks": clocks,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        rate, threads, sample, dt = oracle_sample_rate(w, steps=4, budget_s=args.cpu_budget)
+        rate, threads, sample, dt = oracle_sample_rate(w, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": round(rate, 4), "unit": "steps/s", "cores": threads,
                                 "kind": "oracle", "sample": sample, "seconds": round(dt, 2)}
     if rank == 0:
@@ -445,7 +469,6 @@ def run_e2e(args, w, arms, cfgs, states, dev, stream, dist, host, reinit):
 
     K = min(args.steps, args.e2e_steps)
     P = args.pool
-    G = len(states[0])
     T = w.tiles
     # one packed pinned buffer per slot: q | k | v | alpha | beta
     parts = [np.ascontiguousarray(a) for a in host]
@@ -465,7 +488,7 @@ def run_e2e(args, w, arms, cfgs, states, dev, stream, dist, host, reinit):
     def one(t):
         dbuf.copy_(packed[t % P], non_blocking=True)
         for ai in range(len(arms)):
-            states[ai][t % G].step(views[0] if readout else None, views[1], views[2], views[3],
+            states[ai][t % len(states[ai])].step(views[0] if readout else None, views[1], views[2], views[3],
                                    views[4], o_dev[ai] if readout else None)
         if readout:
             o_host.copy_(o_dev, non_blocking=True)
@@ -505,7 +528,7 @@ def run_reference(args):
     w = W.get(args.workload)
     from oracle import oracle as O
     # warm-up on a single tile (untimed), then the timed steps on a sample
-    rate, threads, sample, dt = oracle_sample_rate(w, steps=args.steps, budget_s=args.ref_budget)
+    rate, threads, sample, dt = oracle_sample_rate(w, budget_s=args.ref_budget, steps=args.steps)
     peak, _ = load_peak()
     bytes_step = sum(arm_bytes(w, a, w.readout) for a in w.arms)
     line = {

@@ -40,7 +40,11 @@
 
 namespace qs {
 
-constexpr int kThreads = 128;
+// Threads per CTA.
+#ifndef QS_THREADS
+#define QS_THREADS 128
+#endif
+constexpr int kThreads = QS_THREADS;
 
 // Resident CTAs per SM the register allocation targets (kThreads each);
 // the yoked kernel is held to fewer by its shared memory and gets more
@@ -55,6 +59,15 @@ constexpr int kThreads = 128;
 // shared memory for every row).
 #ifndef QS_Q_IN_REGS
 #define QS_Q_IN_REGS 0
+#endif
+// Keep the unit's k chunk in registers across rows (else re-read it from
+// shared memory at each use, which frees 32 registers per thread).
+#ifndef QS_K_IN_REGS
+#define QS_K_IN_REGS 1
+#endif
+// cp.async ring depth of the non-yoked kernels.
+#ifndef QS_STAGES
+#define QS_STAGES 4
 #endif
 // Rows a thread carries through the step together (1 or 2).
 #ifndef QS_ROWS_TOGETHER
@@ -445,8 +458,10 @@ __global__ void __launch_bounds__(kThreads, POLICY == 2 ? QS_MIN_BLOCKS_YOKED : 
     }
 
     // per-unit column vectors of this thread's chunk
-    float2 kk[16];
-    load_pairs(st + L.k, c, kk);
+    constexpr bool K_REG = QS_K_IN_REGS || YOKED || BDR;
+    float2 kk[K_REG ? 16 : 1];
+    if constexpr (K_REG) load_pairs(st + L.k, c, kk);
+    const float4* kp4 = reinterpret_cast<const float4*>(st + L.k) + c * (kChunkStride / 4);
     float2 qq[Q_REG ? 16 : 1];
     if constexpr (Q_REG) {
       if (readout) load_pairs(st + L.q, c, qq);
@@ -508,10 +523,22 @@ __global__ void __launch_bounds__(kThreads, POLICY == 2 ? QS_MIN_BLOCKS_YOKED : 
         float2 acc[NR];
 #pragma unroll
         for (int i = 0; i < NR; ++i) acc[i] = make_float2(0.0f, 0.0f);
+        if constexpr (K_REG) {
 #pragma unroll
-        for (int m = 0; m < 16; ++m)
+          for (int m = 0; m < 16; ++m)
 #pragma unroll
-          for (int i = 0; i < NR; ++i) acc[i] = __ffma2_rn(Sp[i][m], kk[m], acc[i]);
+            for (int i = 0; i < NR; ++i) acc[i] = __ffma2_rn(Sp[i][m], kk[m], acc[i]);
+        } else {
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const float4 t = kp4[m];
+#pragma unroll
+            for (int i = 0; i < NR; ++i) {
+              acc[i] = __ffma2_rn(Sp[i][2 * m], make_float2(t.x, t.y), acc[i]);
+              acc[i] = __ffma2_rn(Sp[i][2 * m + 1], make_float2(t.z, t.w), acc[i]);
+            }
+          }
+        }
 #pragma unroll
         for (int i = 0; i < NR; ++i) wcoef[i] = __fmul_rn(beta, __fsub_rn(v_i[i], row_tree<LPR>(acc[i])));
       } else {
@@ -519,10 +546,22 @@ __global__ void __launch_bounds__(kThreads, POLICY == 2 ? QS_MIN_BLOCKS_YOKED : 
         for (int i = 0; i < NR; ++i) wcoef[i] = __fmul_rn(beta, v_i[i]);
       }
       float2 x[NR][16];
+      if constexpr (K_REG) {
 #pragma unroll
-      for (int i = 0; i < NR; ++i)
+        for (int i = 0; i < NR; ++i)
 #pragma unroll
-        for (int m = 0; m < 16; ++m) x[i][m] = __ffma2_rn(f2(wcoef[i]), kk[m], Sp[i][m]);
+          for (int m = 0; m < 16; ++m) x[i][m] = __ffma2_rn(f2(wcoef[i]), kk[m], Sp[i][m]);
+      } else {
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const float4 t = kp4[m];
+#pragma unroll
+          for (int i = 0; i < NR; ++i) {
+            x[i][2 * m] = __ffma2_rn(f2(wcoef[i]), make_float2(t.x, t.y), Sp[i][2 * m]);
+            x[i][2 * m + 1] = __ffma2_rn(f2(wcoef[i]), make_float2(t.z, t.w), Sp[i][2 * m + 1]);
+          }
+        }
+      }
 
       // ---- a5: readout from the updated state
       if (readout) {

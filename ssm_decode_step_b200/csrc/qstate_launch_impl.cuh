@@ -9,7 +9,7 @@ namespace qs {
 
 // Stages of the cp.async ring per CTA.
 template <int POLICY>
-constexpr int step_stages() { return POLICY == 2 ? 3 : 4; }
+constexpr int step_stages() { return POLICY == 2 ? 3 : QS_STAGES; }
 
 // Rows per work unit: the largest of 128, 64, 32, 16 that divides dv and keeps
 // one stage within `budget` bytes (so that three or four CTAs fit per SM).
