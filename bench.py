@@ -381,6 +381,8 @@ def run_ours(args):
     arm_ms = max_over_ranks(dist, arm_ms, dev)
     total_ms = sum(arm_ms)
     clocks = sampler.summary()
+    fp32 = None if args.no_fp32 else run_fp32_state(args, w, dev, stream, dist, pool, host, S0, l2,
+                                                   pool_bytes)
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(args, w, arms, cfgs, states, dev, stream, dist, host, reinit)
@@ -446,6 +448,11 @@ def run_ours(args):
             "algorithmic_bytes_per_launch": dom_bytes,
         },
         "e2e": e2e,
+        "fp32_state": fp32 and dict(fp32, **{
+            "quantized_speedup": {a.name: round(fp32["us_per_launch"] / (arm_ms[i] * 1e3 / K), 3)
+                                  for i, a in enumerate(arms)},
+            "state_memory_ratio": {a.name: round(w.tiles * w.dv * w.dk * 4 / state_bytes(w, a), 3)
+                                   for a in arms}}),
         "gpu_launches": K * len(arms),
         "clocks": clocks,
     }
@@ -459,6 +466,76 @@ def run_ours(args):
         del g
     if dist is not None:
         dist.destroy_process_group()
+
+
+def fp32_bytes(w: W.Workload, readout: bool = True) -> int:
+    T, dk, dv = w.tiles, w.dk, w.dv
+    alpha = T * (dk if w.decay == "diagonal" else 1) * 4
+    return 2 * T * dv * dk * 4 + T * ((dk if readout else 0) + dk + dv) * 4 + alpha + T * 4 + \
+        (T * dv * 4 if readout else 0)
+
+
+def run_fp32_state(args, w, dev, stream, dist, pool, host, S0, l2, pool_bytes):
+    """The same steps on an FP32 state (qstate_fp32_decode_step): the
+    baseline of the quantized arms, timed the same way (CUDA graphs, events,
+    request groups sized past 2x L2).  Not part of the step."""
+    import torch
+    from ssm_decode_step_b200 import Config, qstate as Q
+    K, P = args.steps, args.pool
+    cfg = Config(w.tiles, w.dk, w.dv, 8, 32, w.delta, w.decay)
+    sb = w.tiles * w.dv * w.dk * 4
+    G = max(1, -(-2 * l2 // sb))
+    G = min(G, P)
+    while P % G:
+        G -= 1
+    states = [S0.clone() for _ in range(G)]
+    o = torch.empty((w.tiles, w.dv), dtype=torch.float32, device=dev) if w.readout else None
+
+    def launch(t):
+        s = t % P
+        Q.fp32_decode_step(cfg, states[t % G], pool[0][s], pool[1][s], pool[2][s], pool[3][s],
+                           pool[4][s], o, stream)
+
+    with torch.cuda.stream(stream):
+        for t in range(args.warmup):
+            launch(t)
+    stream.synchronize()
+    n_main, tail = divmod(K, P)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for t in range(P):
+            launch(t)
+    gt = None
+    if tail:
+        gt = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gt, stream=stream):
+            for t in range(tail):
+                launch(t)
+    with torch.cuda.stream(stream):
+        g.replay()
+    stream.synchronize()
+    for st in states:
+        st.copy_(S0)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(n_main):
+            g.replay()
+        if gt is not None:
+            gt.replay()
+        e1.record(stream)
+    stream.synchronize()
+    ms = max_over_ranks(dist, [e0.elapsed_time(e1)], dev)[0]
+    del g, gt
+    peak, _ = load_peak()
+    b = fp32_bytes(w, w.readout)
+    s = ms / 1e3 / K
+    return {"us_per_launch": round(s * 1e6, 3), "bytes_per_launch": b,
+            "gbs": round(b / s / 1e9, 1), "frac": round(b / s / 1e9 / peak, 4),
+            "l2": f"{G} request groups x {sb / 1e6:.1f} MB FP32 state + {pool_bytes / 1e6:.0f} MB inputs"}
 
 
 def run_e2e(args, w, arms, cfgs, states, dev, stream, dist, host, reinit):
@@ -571,6 +648,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
     ap.add_argument("--ref-budget", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fp32", action="store_true", help="skip the FP32-state comparison arm")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

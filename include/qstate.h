@@ -157,6 +157,16 @@ QS_API qs_status qstate_readout(const qs_config* cfg, const void* codes,
                          const float* scales, const float* q, float* o,
                          cudaStream_t stream);
 
+/* One decode step of the UNQUANTIZED recurrence (the same definition with
+ * the state kept in FP32: the baseline "FP32 state" the quantized state is
+ * measured against).  S [T][Dv][Dk] float, 32-byte aligned, updated in
+ * place: S <- (S * a) + w k^T with w as above (same fixed order); readout
+ * o = S_t q (o == NULL skips it; q may then be NULL).  Only num_tiles, dk,
+ * dv, delta and decay of cfg are used. */
+QS_API qs_status qstate_fp32_decode_step(const qs_config* cfg, float* S, const float* q,
+                                         const float* k, const float* v, const float* alpha,
+                                         const float* beta, float* o, cudaStream_t stream);
+
 /* Self-check of the library's fast arithmetic on the current GPU.  The
  * kernels compute the reciprocal of a scale and the division of a group
  * maximum by qmax with short fused multiply-add sequences; this compares

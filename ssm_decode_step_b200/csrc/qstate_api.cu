@@ -7,6 +7,7 @@
 #include <mutex>
 
 #include "../../include/qstate.h"
+#include "qstate_fp32.cuh"
 #include "qstate_launch.h"
 
 namespace qs {
@@ -234,6 +235,58 @@ qs_status qstate_decode_step(const qs_config* cfg, void* codes, float* scales, f
     e = cfg->dk == 64 ? dispatch_step<4, 64>(cfg, p, stream) : dispatch_step<4, 128>(cfg, p, stream);
   else
     e = cfg->dk == 64 ? dispatch_step<8, 64>(cfg, p, stream) : dispatch_step<8, 128>(cfg, p, stream);
+  return from_cuda(e);
+}
+
+qs_status qstate_fp32_decode_step(const qs_config* cfg, float* S, const float* q, const float* k,
+                                  const float* v, const float* alpha, const float* beta, float* o,
+                                  cudaStream_t stream) {
+  if (cfg == nullptr) return QS_ERR_INVALID_ARG;
+  // only the recurrence's fields matter here; check them through a quantized
+  // configuration that is always valid for storage
+  qs_config c = *cfg;
+  c.bits = 8;
+  c.group = 32;
+  c.policy = QS_SCALE_PERSISTENT;
+  c.rounding = QS_ROUND_NEAREST;
+  qs_status st = check_config(&c);
+  if (st != QS_OK) return st;
+  if (c.num_tiles == 0) return QS_OK;
+  const bool diag = c.decay == QS_DECAY_DIAGONAL;
+  if (!S || !k || !v || !alpha || !beta || (o && !q)) return QS_ERR_INVALID_ARG;
+  if (!aligned(S, 32) || !aligned(k, 16) || !aligned(v, 16) || (q && !aligned(q, 16)) ||
+      !aligned(alpha, diag ? 16 : 4) || !aligned(beta, 4) || (o && !aligned(o, 4)))
+    return QS_ERR_INVALID_ARG;
+  const Sizes s = sizes_of(&c);
+  const size_t state_bytes = static_cast<size_t>(c.num_tiles) * c.dv * c.dk * sizeof(float);
+  const Range w[2] = {range_of(S, state_bytes), range_of(o, o ? s.vec_v : 0)};
+  const Range r[5] = {range_of(q, q ? s.vec_k : 0), range_of(k, s.vec_k), range_of(v, s.vec_v),
+                      range_of(alpha, s.alpha), range_of(beta, s.tile_scalars)};
+  if (any_overlap(w, 2, r, 5)) return QS_ERR_INVALID_ARG;
+  qs::StepParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.shadow = S;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.alpha = alpha;
+  p.beta = beta;
+  p.o = o;
+  p.tiles = c.num_tiles;
+  p.dv = c.dv;
+  p.group = c.group;
+  const int sel = (c.dk == 128 ? 4 : 0) + (c.delta ? 2 : 0) + (diag ? 1 : 0);
+  cudaError_t e;
+  switch (sel) {
+    case 0: e = qs::launch_fp32_step<64, false, false>(p, stream); break;
+    case 1: e = qs::launch_fp32_step<64, false, true>(p, stream); break;
+    case 2: e = qs::launch_fp32_step<64, true, false>(p, stream); break;
+    case 3: e = qs::launch_fp32_step<64, true, true>(p, stream); break;
+    case 4: e = qs::launch_fp32_step<128, false, false>(p, stream); break;
+    case 5: e = qs::launch_fp32_step<128, false, true>(p, stream); break;
+    case 6: e = qs::launch_fp32_step<128, true, false>(p, stream); break;
+    default: e = qs::launch_fp32_step<128, true, true>(p, stream); break;
+  }
   return from_cuda(e);
 }
 

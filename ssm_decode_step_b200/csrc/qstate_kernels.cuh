@@ -93,6 +93,28 @@ struct StepParams {
   int group;
   int rb;              // rows per work unit (divides dv)
   int units_per_tile;  // dv / rb
+  int grid_tiles;      // gridDim.x / units_per_tile
+  int grid_part;       // gridDim.x % units_per_tile
+};
+
+// Work-unit cursor: unit = tile * units_per_tile + part, advanced by gridDim.x
+// without a division (the host precomputes the stride's tile / part split).
+struct UnitCursor {
+  int tile, part;
+  __device__ __forceinline__ UnitCursor(int unit, const StepParams& p)
+      : tile(unit / p.units_per_tile), part(unit % p.units_per_tile) {}
+  __device__ __forceinline__ void advance(const StepParams& p) {
+    part += p.grid_part;
+    tile += p.grid_tiles;
+    if (part >= p.units_per_tile) {
+      part -= p.units_per_tile;
+      ++tile;
+    }
+  }
+  // first global row of the unit
+  __device__ __forceinline__ size_t row0(const StepParams& p) const {
+    return static_cast<size_t>(tile) * p.dv + static_cast<size_t>(part) * p.rb;
+  }
 };
 
 // ---------------------------------------------------------------------------
@@ -198,12 +220,12 @@ __device__ __forceinline__ int vec_unit_offset(int i) { return (i >> 3) * (kChun
 // Issue the cp.async copies of one work unit into a stage.
 template <int BITS, int DK, bool DIAG, bool YOKED, bool WITH_STATE_UPDATE>
 __device__ __forceinline__ void stage_load(unsigned char* st, const StageLayout& L,
-                                           const StepParams& p, int unit) {
+                                           const StepParams& p, const UnitCursor& u) {
   constexpr int VU = DK / 4;  // 16-byte units per Dk vector
   const int tid = threadIdx.x;
   const int rb = p.rb;
-  const size_t tile = static_cast<size_t>(unit / p.units_per_tile);
-  const size_t row0 = tile * p.dv + static_cast<size_t>(unit % p.units_per_tile) * rb;
+  const size_t tile = static_cast<size_t>(u.tile);
+  const size_t row0 = u.row0(p);
   const int ng = DK / p.group;
   {
     const int n16 = rb * DK * BITS / 128;
@@ -421,29 +443,29 @@ __global__ void __launch_bounds__(kThreads, POLICY == 2 ? QS_MIN_BLOCKS_YOKED : 
   const int g = (32 * c) / p.group;
   const bool readout = p.o != nullptr;
   const bool writes_scale = (32 * c) % p.group == 0;
-  const int units = p.tiles * p.units_per_tile;
-
+  UnitCursor pre(blockIdx.x, p);  // next unit to stage
 #pragma unroll
   for (int s = 0; s < STAGES - 1; ++s) {
-    const int unit = blockIdx.x + s * gridDim.x;
-    if (unit < units) stage_load<BITS, DK, DIAG, YOKED, true>(smem + s * L.bytes, L, p, unit);
+    if (pre.tile < p.tiles) stage_load<BITS, DK, DIAG, YOKED, true>(smem + s * L.bytes, L, p, pre);
     cp_async_commit();
+    pre.advance(p);
   }
 
   int it = 0;
-  for (int unit = blockIdx.x; unit < units; unit += gridDim.x, ++it) {
-    {
-      const int pre = unit + (STAGES - 1) * gridDim.x;
-      if (pre < units)
-        stage_load<BITS, DK, DIAG, YOKED, true>(smem + ((it + STAGES - 1) % STAGES) * L.bytes, L, p,
-                                                pre);
-      cp_async_commit();
-    }
+  for (UnitCursor cur(blockIdx.x, p); cur.tile < p.tiles; cur.advance(p), ++it) {
+    if (pre.tile < p.tiles)
+      stage_load<BITS, DK, DIAG, YOKED, true>(smem + ((it + STAGES - 1) % STAGES) * L.bytes, L, p,
+                                              pre);
+    cp_async_commit();
+    pre.advance(p);
     cp_async_wait<STAGES - 1>();
     __syncthreads();
     unsigned char* st = smem + (it % STAGES) * L.bytes;
-    const size_t tile = static_cast<size_t>(unit / p.units_per_tile);
-    const size_t grow0 = tile * p.dv + static_cast<size_t>(unit % p.units_per_tile) * p.rb;
+    const size_t grow0 = cur.row0(p);
+    // per-unit global bases; rows below are 32-bit offsets from these
+    uint8_t* codes_u = p.codes + grow0 * (DK * BITS / 8) + c * (4 * CW);
+    float* scales_u = p.scales + grow0 * ng + g;
+    float* o_u = readout ? p.o + grow0 : nullptr;
 
     if constexpr (BDR) {
       // sign(k_j) per column, in the layout of k
@@ -588,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, POLICY == 2 ? QS_MIN_BLOCKS_YOKED : 
 #pragma unroll
         for (int i = 0; i < NR; ++i) {
           const float o = row_tree<LPR>(acc[i]);
-          if (c == 0 && valid[i]) p.o[grow0 + row[i]] = o;
+          if (c == 0 && valid[i]) o_u[row[i]] = o;
         }
       }
 
@@ -676,15 +698,14 @@ __global__ void __launch_bounds__(kThreads, POLICY == 2 ? QS_MIN_BLOCKS_YOKED : 
           for (int q = 0; q < CW; ++q) out[q] = 0u;
         }
         if (valid[i]) {
-          const size_t grow = grow0 + row[i];
-          uint8_t* cg = p.codes + grow * (DK * BITS / 8) + c * (4 * CW);
+          uint8_t* cg = codes_u + row[i] * (DK * BITS / 8);
           if constexpr (CW == 4) {
             *reinterpret_cast<uint4*>(cg) = make_uint4(out[0], out[1], out[2], out[3]);
           } else {
             st_global_v8(cg, out);
           }
           if constexpr (POLICY != 1) {
-            if (writes_scale) p.scales[grow * ng + g] = sp[i];
+            if (writes_scale) scales_u[row[i] * ng] = sp[i];
           }
         }
       }
@@ -708,28 +729,24 @@ __global__ void __launch_bounds__(kThreads, QS_MIN_BLOCKS) readout_kernel(StepPa
   const int c = tid % LPR, r0 = tid / LPR;
   const int ng = DK / p.group;
   const int g = (32 * c) / p.group;
-  const int units = p.tiles * p.units_per_tile;
-
+  UnitCursor pre(blockIdx.x, p);
 #pragma unroll
   for (int s = 0; s < STAGES - 1; ++s) {
-    const int unit = blockIdx.x + s * gridDim.x;
-    if (unit < units) stage_load<BITS, DK, false, false, false>(smem + s * L.bytes, L, p, unit);
+    if (pre.tile < p.tiles) stage_load<BITS, DK, false, false, false>(smem + s * L.bytes, L, p, pre);
     cp_async_commit();
+    pre.advance(p);
   }
   int it = 0;
-  for (int unit = blockIdx.x; unit < units; unit += gridDim.x, ++it) {
-    {
-      const int pre = unit + (STAGES - 1) * gridDim.x;
-      if (pre < units)
-        stage_load<BITS, DK, false, false, false>(smem + ((it + STAGES - 1) % STAGES) * L.bytes, L,
-                                                  p, pre);
-      cp_async_commit();
-    }
+  for (UnitCursor cur(blockIdx.x, p); cur.tile < p.tiles; cur.advance(p), ++it) {
+    if (pre.tile < p.tiles)
+      stage_load<BITS, DK, false, false, false>(smem + ((it + STAGES - 1) % STAGES) * L.bytes, L,
+                                                p, pre);
+    cp_async_commit();
+    pre.advance(p);
     cp_async_wait<STAGES - 1>();
     __syncthreads();
     unsigned char* st = smem + (it % STAGES) * L.bytes;
-    const size_t tile = static_cast<size_t>(unit / p.units_per_tile);
-    const size_t grow0 = tile * p.dv + static_cast<size_t>(unit % p.units_per_tile) * p.rb;
+    const size_t grow0 = cur.row0(p);
     float2 qq[16];
     load_pairs(st + L.q, c, qq);
 #pragma unroll 1

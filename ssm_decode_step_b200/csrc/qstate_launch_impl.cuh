@@ -48,7 +48,10 @@ static cudaError_t launch_persistent(K kernel, size_t smem, const StepParams& p,
   const long long units = static_cast<long long>(p.tiles) * p.units_per_tile;
   long long grid = static_cast<long long>(per_sm) * device_sm_count();
   if (grid > units) grid = units;
-  kernel<<<static_cast<int>(grid), kThreads, smem, stream>>>(p);
+  StepParams q = p;
+  q.grid_tiles = static_cast<int>(grid / p.units_per_tile);
+  q.grid_part = static_cast<int>(grid % p.units_per_tile);
+  kernel<<<static_cast<int>(grid), kThreads, smem, stream>>>(q);
   return cudaGetLastError();
 }
 

@@ -24,7 +24,7 @@ QS_OK, QS_ERR_INVALID_ARG, QS_ERR_UNSUPPORTED, QS_ERR_CUDA = 0, 1, 2, 3
 
 # Every entry point that include/qstate.h declares.
 EXPORTS = ("qstate_query_sizes", "qstate_init", "qstate_decode_step", "qstate_readout",
-           "qstate_selfcheck", "qstate_status_string", "qstate_version")
+           "qstate_fp32_decode_step", "qstate_selfcheck", "qstate_status_string", "qstate_version")
 
 
 class QStateError(RuntimeError):
@@ -56,8 +56,9 @@ def lib() -> ctypes.CDLL:
         L.qstate_decode_step.argtypes = [C, P, P, P, P, P, P, P, P, P, P]
         L.qstate_readout.argtypes = [C, P, P, P, P, P]
         L.qstate_selfcheck.argtypes = [P, P]
+        L.qstate_fp32_decode_step.argtypes = [C, P, P, P, P, P, P, P, P]
         for f in (L.qstate_query_sizes, L.qstate_init, L.qstate_decode_step, L.qstate_readout,
-                  L.qstate_selfcheck):
+                  L.qstate_selfcheck, L.qstate_fp32_decode_step):
             f.restype = ctypes.c_int
         L.qstate_status_string.argtypes = [ctypes.c_int]
         L.qstate_status_string.restype = ctypes.c_char_p
@@ -142,6 +143,14 @@ def readout(cfg: Config, codes, scales, q, o, stream=None) -> None:
     cc = cfg.c()
     _check(lib().qstate_readout(ctypes.byref(cc), _ptr(codes), _ptr(scales), _ptr(q), _ptr(o),
                                 _stream(stream)), "qstate_readout")
+
+
+def fp32_decode_step(cfg: Config, S, q, k, v, alpha, beta, o=None, stream=None) -> None:
+    """The unquantized FP32 recurrence, in place on S (float32 [T, dv, dk])."""
+    cc = cfg.c()
+    _check(lib().qstate_fp32_decode_step(ctypes.byref(cc), _ptr(S), _ptr(q), _ptr(k), _ptr(v),
+                                         _ptr(alpha), _ptr(beta), _ptr(o), _stream(stream)),
+           "qstate_fp32_decode_step")
 
 
 def selfcheck(stream=None):

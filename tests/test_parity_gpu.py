@@ -177,3 +177,28 @@ def test_workload_full_size_sampled(wname):
                      arm.rounding)
         rep = P.lockstep(cfg, S0, steps, tiles=tiles, label=f"{wname}-{arm.name}")
         assert rep.code_flips == 0, rep
+
+
+@pytest.mark.parametrize("dk,dv,delta,decay,T", [(128, 128, 1, "scalar", 333), (128, 64, 0, "diagonal", 77),
+                                                 (64, 64, 1, "diagonal", 5), (64, 48, 0, "scalar", 3),
+                                                 (128, 16, 1, "scalar", 9)])
+def test_fp32_state_step_matches_oracle_bit_for_bit(dk, dv, delta, decay, T):
+    """The unquantized FP32 decode step (qstate_fp32_decode_step) against the
+    oracle's FP32 recurrence: same fixed order, so states and readouts agree
+    bit for bit over several steps."""
+    import torch
+    from ssm_decode_step_b200 import qstate as Q
+    rng = np.random.default_rng(dk * 1000 + dv + T)
+    cfg = Config(T, dk, dv, 8, 32, delta, decay)
+    S0 = (rng.standard_normal((T, dv, dk)) * 0.3).astype(np.float32)
+    S_gpu = torch.from_numpy(S0.copy()).cuda()
+    S_ref = S0.copy()
+    ocfg = P.oracle_cfg(cfg)
+    for t, (q, k, v, a, b) in enumerate(P.random_steps(rng, T, dk, dv, decay, 6)):
+        o = torch.empty((T, dv), dtype=torch.float32, device="cuda")
+        dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+        Q.fp32_decode_step(cfg, S_gpu, dev(q), dev(k), dev(v), dev(a), dev(b), o if t % 2 == 0 else None)
+        o_ref = O.fp32_step(ocfg, S_ref, q, k, v, a, b)
+        assert np.array_equal(S_gpu.cpu().numpy(), S_ref), f"state differs at step {t}"
+        if t % 2 == 0:
+            assert np.array_equal(o.cpu().numpy(), o_ref), f"readout differs at step {t}"
