@@ -11,12 +11,15 @@ namespace qs {
 template <int POLICY>
 constexpr int step_stages() { return POLICY == 2 ? 3 : QS_STAGES; }
 
-// Rows per work unit: the largest of 128, 64, 32, 16 that divides dv and keeps
+// Rows per work unit: the largest of QS_RB_MAX (64), 32, 16 that divides dv and keeps
 // one stage within `budget` bytes (so that three or four CTAs fit per SM).
+#ifndef QS_RB_MAX
+#define QS_RB_MAX 64
+#endif
 inline int choose_rb(int bits, int dk, int dv, int group, bool diag, bool bdr, bool yoked) {
   const int budget = yoked ? 21 * 1024 : 13 * 1024;
   int best = 16;
-  for (int rb = 128; rb >= 16; rb /= 2) {
+  for (int rb = QS_RB_MAX; rb >= 16; rb /= 2) {
     if (dv % rb != 0) continue;
     if (StageLayout(bits, dk, rb, group, diag, bdr, yoked).bytes <= budget) return rb;
     best = rb;
