@@ -81,7 +81,7 @@
  *
  * Supported by this build: dk in {64, 128}; dv a multiple of 16 with
  * 16 <= dv <= 4096; bits in {4, 8}; group in {32, 64, 128} with
- * group <= dk; num_tiles >= 0 with num_tiles * dv / 16 < 2^31.
+ * group <= dk; num_tiles >= 0 with num_tiles * dv / 8 < 2^31.
  */
 #ifndef QSTATE_H
 #define QSTATE_H

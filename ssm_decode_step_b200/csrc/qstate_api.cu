@@ -79,7 +79,7 @@ qs_status check_config(const qs_config* c) {
   // what this build has kernels for
   if (c->dk != 64 && c->dk != 128) return QS_ERR_UNSUPPORTED;
   if (c->dv % 16 != 0 || c->dv > 4096) return QS_ERR_UNSUPPORTED;
-  if (static_cast<long long>(c->num_tiles) * (c->dv / 16) > 0x7fffffffLL) return QS_ERR_UNSUPPORTED;
+  if (static_cast<long long>(c->num_tiles) * (c->dv / 8) > 0x7fffffffLL) return QS_ERR_UNSUPPORTED;
   if (c->group != 32 && c->group != 64 && c->group != 128) return QS_ERR_UNSUPPORTED;
   return QS_OK;
 }

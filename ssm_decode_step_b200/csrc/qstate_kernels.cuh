@@ -1,23 +1,16 @@
-// Fused decode-step kernels for the quantized recurrent state (sm_100a).
+// Shared pieces of the quantized-state kernels (sm_100a): the element-level
+// arithmetic of the decode step, and the readout and quantization-start
+// kernels.  The step kernel itself is in qstate_step.cuh.
 //
 // The operation (LinQuant eq. (1) with readout o = S q, group-wise INT4/INT8
 // state, dynamic / persistent / yoked scales, nearest or Bounded Directional
 // Rounding) and its element-level FP32 definition are documented in
-// include/qstate.h.  This file is the CUDA realization of that definition.
+// include/qstate.h.
 //
-// Work decomposition.  Rows of a tile are independent: every reduction of
-// the step (u = S' k, o = x q, the group max) runs along one row.  A thread
-// owns a 32-column chunk c of a row (LPR = Dk/32 consecutive lanes per row),
-// so a row's reductions are in-thread chains plus log2(LPR) xor shuffles.
-// A work unit is a block of rb rows of one tile; a CTA of kThreads threads
-// takes one unit per iteration (persistent grid sized to the SMs), and
-// thread (r0, c) handles rows r0, r0 + RP, ... of the unit, keeping the
-// unit's k (and q) chunk in registers across those rows.
-//
-// Memory path.  Each unit's codes, scales, v, k, q (alpha, the FP32 shadow)
-// are staged into shared memory with 16-byte cp.async through an S-deep
-// ring per CTA, so S-1 units are in flight while one is computed; new codes
-// and scales leave as coalesced 16/32-byte stores straight from registers.
+// Ownership.  Rows of a tile are independent: every reduction of the step
+// (u = S' k, o = x q, the group max) runs along one row.  A thread owns a
+// 32-column chunk c of a row (LPR = Dk/32 consecutive lanes per row), so a
+// row's reductions are in-thread chains plus log2(LPR) xor shuffles.
 //
 // Arithmetic.  Each thread holds its chunk as 16 register pairs of adjacent
 // columns (2m, 2m+1) and works with the packed FP32 instructions of sm_100
@@ -31,8 +24,9 @@
 // a byte permute into the mantissa of 2^23 (exact) and rounded by adding
 // 1.5 * 2^23 inside one fused multiply-add (exact product, ties to even).
 //
-// No kernel here spins on a flag or barrier: the only waits are
-// cp.async.wait_group and __syncthreads, so nothing can hang.
+// The readout kernel stages work units of rb rows through a cp.async ring
+// per CTA.  No kernel here spins on a flag or barrier: the only waits are
+// cp.async.wait_group, __syncthreads and __syncwarp, so nothing can hang.
 #pragma once
 
 #include <cstdint>
@@ -55,23 +49,9 @@ constexpr int kThreads = QS_THREADS;
 #ifndef QS_MIN_BLOCKS_YOKED
 #define QS_MIN_BLOCKS_YOKED 3
 #endif
-// Keep the unit's q chunk in registers across rows (else re-read it from
-// shared memory for every row).
-#ifndef QS_Q_IN_REGS
-#define QS_Q_IN_REGS 0
-#endif
-// Keep the unit's k chunk in registers across rows (else re-read it from
-// shared memory at each use, which frees 32 registers per thread).
-#ifndef QS_K_IN_REGS
-#define QS_K_IN_REGS 1
-#endif
-// cp.async ring depth of the non-yoked kernels.
+// cp.async ring depth of the readout kernel.
 #ifndef QS_STAGES
 #define QS_STAGES 4
-#endif
-// Rows a thread carries through the step together (1 or 2).
-#ifndef QS_ROWS_TOGETHER
-#define QS_ROWS_TOGETHER 1
 #endif
 
 // 1.5 * 2^23: adding it to a float of magnitude < 2^22 leaves the nearest
@@ -413,306 +393,6 @@ __device__ __forceinline__ void bdr_chunk(float2 (&y)[16], const float2 (&Sp)[16
     y[m].x = fminf(fmaxf(yx, kOff - kQ), kOff + kQ);
     y[m].y = fminf(fmaxf(yy, kOff - kQ), kOff + kQ);
   }
-}
-
-// ---------------------------------------------------------------------------
-// the decode step
-// ---------------------------------------------------------------------------
-// POLICY: 0 dynamic, 1 persistent, 2 yoked.
-template <int BITS, int DK, int POLICY, bool BDR, bool DELTA, bool DIAG, int STAGES>
-__global__ void __launch_bounds__(kThreads, POLICY == 2 ? QS_MIN_BLOCKS_YOKED : QS_MIN_BLOCKS)
-    step_kernel(StepParams p) {
-  constexpr int LPR = DK / 32;
-  constexpr int RP = kThreads / LPR;  // rows per pass of the CTA
-  constexpr bool YOKED = POLICY == 2;
-  constexpr int CW = BITS;            // 32-bit words of codes per 32-column chunk
-  constexpr int QMAX = BITS == 4 ? 7 : 127;
-  constexpr float kQf = static_cast<float>(QMAX);
-  constexpr float kOff = kMagic + (BITS == 4 ? 8.0f : 128.0f);
-  // q stays in registers across the rows of a unit unless other per-column
-  // vectors need the registers
-  constexpr bool Q_REG = QS_Q_IN_REGS && !DIAG && !BDR && !YOKED;
-  // rows processed together by one thread (independent dependency chains)
-  constexpr int NR = (YOKED || BDR) ? 1 : QS_ROWS_TOGETHER;
-
-  extern __shared__ __align__(128) unsigned char smem[];
-  const StageLayout L(BITS, DK, p.rb, p.group, DIAG, BDR, YOKED);
-  const int tid = threadIdx.x;
-  const int c = tid % LPR, r0 = tid / LPR;
-  const int ng = DK / p.group;
-  const int g = (32 * c) / p.group;
-  const bool readout = p.o != nullptr;
-  const bool writes_scale = (32 * c) % p.group == 0;
-  UnitCursor pre(blockIdx.x, p);  // next unit to stage
-#pragma unroll
-  for (int s = 0; s < STAGES - 1; ++s) {
-    if (pre.tile < p.tiles) stage_load<BITS, DK, DIAG, YOKED, true>(smem + s * L.bytes, L, p, pre);
-    cp_async_commit();
-    pre.advance(p);
-  }
-
-  int it = 0;
-  for (UnitCursor cur(blockIdx.x, p); cur.tile < p.tiles; cur.advance(p), ++it) {
-    if (pre.tile < p.tiles)
-      stage_load<BITS, DK, DIAG, YOKED, true>(smem + ((it + STAGES - 1) % STAGES) * L.bytes, L, p,
-                                              pre);
-    cp_async_commit();
-    pre.advance(p);
-    cp_async_wait<STAGES - 1>();
-    __syncthreads();
-    unsigned char* st = smem + (it % STAGES) * L.bytes;
-    const size_t grow0 = cur.row0(p);
-    // per-unit global bases; rows below are 32-bit offsets from these
-    uint8_t* codes_u = p.codes + grow0 * (DK * BITS / 8) + c * (4 * CW);
-    float* scales_u = p.scales + grow0 * ng + g;
-    float* o_u = readout ? p.o + grow0 : nullptr;
-
-    if constexpr (BDR) {
-      // sign(k_j) per column, in the layout of k
-      const float* kvals = reinterpret_cast<const float*>(st + L.k);
-      float* ss = reinterpret_cast<float*>(st + L.sk);
-      for (int j = tid; j < DK; j += kThreads) {
-        const int pos = (j / 32) * kChunkStride + (j % 32);
-        const float kv = kvals[pos];
-        ss[pos] = kv > 0.0f ? 1.0f : (kv < 0.0f ? -1.0f : 0.0f);
-      }
-      __syncthreads();
-    }
-
-    // per-unit column vectors of this thread's chunk
-    constexpr bool K_REG = QS_K_IN_REGS || YOKED || BDR;
-    float2 kk[K_REG ? 16 : 1];
-    if constexpr (K_REG) load_pairs(st + L.k, c, kk);
-    const float4* kp4 = reinterpret_cast<const float4*>(st + L.k) + c * (kChunkStride / 4);
-    float2 qq[Q_REG ? 16 : 1];
-    if constexpr (Q_REG) {
-      if (readout) load_pairs(st + L.q, c, qq);
-    }
-    const float* miscf = reinterpret_cast<const float*>(st + L.misc);
-    const float beta = miscf[1];
-    const float a_scalar = DIAG ? 1.0f : miscf[0];
-
-    // NR rows of the unit at a time (rows rb0, rb0 + RP, ...): their chains
-    // are independent, so the scheduler can overlap them.  A missing second
-    // row repeats the first and is not stored.
-#pragma unroll 1
-    for (int rb0 = r0; rb0 < p.rb; rb0 += NR * RP) {
-      int row[NR];
-      bool valid[NR];
-#pragma unroll
-      for (int i = 0; i < NR; ++i) {
-        row[i] = rb0 + i * RP;
-        valid[i] = row[i] < p.rb;
-        if (!valid[i]) row[i] = rb0;
-      }
-      // ---- a1: load and unpack this thread's 32 codes of each row
-      float2 Sp[NR][16];
-      float s_old[NR], v_i[NR];
-#pragma unroll
-      for (int i = 0; i < NR; ++i) {
-        uint32_t w[CW];
-        const uint4* src = reinterpret_cast<const uint4*>(st + L.codes + (row[i] * LPR + c) * (4 * CW));
-#pragma unroll
-        for (int q = 0; q < CW / 4; ++q) {
-          const uint4 u = src[q];
-          w[4 * q + 0] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
-        }
-        s_old[i] = reinterpret_cast<const float*>(st + L.scales)[row[i] * ng + g];
-        v_i[i] = reinterpret_cast<const float*>(st + L.v)[row[i]];
-        decode_chunk<BITS>(w, Sp[i]);
-      }
-
-      // ---- a2: dequantize with the decayed scale, S' = c * (s * a)
-      if constexpr (DIAG) {
-        float2 aa[16];
-        load_pairs(st + L.a, c, aa);
-#pragma unroll
-        for (int i = 0; i < NR; ++i)
-#pragma unroll
-          for (int m = 0; m < 16; ++m) Sp[i][m] = __fmul2_rn(Sp[i][m], __fmul2_rn(f2(s_old[i]), aa[m]));
-      } else {
-#pragma unroll
-        for (int i = 0; i < NR; ++i) {
-          const float sa = __fmul_rn(s_old[i], a_scalar);
-#pragma unroll
-          for (int m = 0; m < 16; ++m) Sp[i][m] = __fmul2_rn(Sp[i][m], f2(sa));
-        }
-      }
-
-      // ---- a3/a4: key projection and rank-1 write
-      float wcoef[NR];
-      if constexpr (DELTA) {
-        float2 acc[NR];
-#pragma unroll
-        for (int i = 0; i < NR; ++i) acc[i] = make_float2(0.0f, 0.0f);
-        if constexpr (K_REG) {
-#pragma unroll
-          for (int m = 0; m < 16; ++m)
-#pragma unroll
-            for (int i = 0; i < NR; ++i) acc[i] = __ffma2_rn(Sp[i][m], kk[m], acc[i]);
-        } else {
-#pragma unroll
-          for (int m = 0; m < 8; ++m) {
-            const float4 t = kp4[m];
-#pragma unroll
-            for (int i = 0; i < NR; ++i) {
-              acc[i] = __ffma2_rn(Sp[i][2 * m], make_float2(t.x, t.y), acc[i]);
-              acc[i] = __ffma2_rn(Sp[i][2 * m + 1], make_float2(t.z, t.w), acc[i]);
-            }
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < NR; ++i) wcoef[i] = __fmul_rn(beta, __fsub_rn(v_i[i], row_tree<LPR>(acc[i])));
-      } else {
-#pragma unroll
-        for (int i = 0; i < NR; ++i) wcoef[i] = __fmul_rn(beta, v_i[i]);
-      }
-      float2 x[NR][16];
-      if constexpr (K_REG) {
-#pragma unroll
-        for (int i = 0; i < NR; ++i)
-#pragma unroll
-          for (int m = 0; m < 16; ++m) x[i][m] = __ffma2_rn(f2(wcoef[i]), kk[m], Sp[i][m]);
-      } else {
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const float4 t = kp4[m];
-#pragma unroll
-          for (int i = 0; i < NR; ++i) {
-            x[i][2 * m] = __ffma2_rn(f2(wcoef[i]), make_float2(t.x, t.y), Sp[i][2 * m]);
-            x[i][2 * m + 1] = __ffma2_rn(f2(wcoef[i]), make_float2(t.z, t.w), Sp[i][2 * m + 1]);
-          }
-        }
-      }
-
-      // ---- a5: readout from the updated state
-      if (readout) {
-        float2 acc[NR];
-#pragma unroll
-        for (int i = 0; i < NR; ++i) acc[i] = make_float2(0.0f, 0.0f);
-        if constexpr (Q_REG) {
-#pragma unroll
-          for (int m = 0; m < 16; ++m)
-#pragma unroll
-            for (int i = 0; i < NR; ++i) acc[i] = __ffma2_rn(x[i][m], qq[m], acc[i]);
-        } else {
-          const float4* qp4 = reinterpret_cast<const float4*>(st + L.q) + c * (kChunkStride / 4);
-#pragma unroll
-          for (int m = 0; m < 8; ++m) {
-            const float4 t = qp4[m];
-#pragma unroll
-            for (int i = 0; i < NR; ++i) {
-              acc[i] = __ffma2_rn(x[i][2 * m], make_float2(t.x, t.y), acc[i]);
-              acc[i] = __ffma2_rn(x[i][2 * m + 1], make_float2(t.z, t.w), acc[i]);
-            }
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < NR; ++i) {
-          const float o = row_tree<LPR>(acc[i]);
-          if (c == 0 && valid[i]) o_u[row[i]] = o;
-        }
-      }
-
-      // ---- a6/a7: scale selection (yoked shadow update)
-      float sp[NR];
-      if constexpr (POLICY == 0) {
-#pragma unroll
-        for (int i = 0; i < NR; ++i) sp[i] = div_qmax_rn<QMAX>(row_max<LPR>(chunk_absmax(x[i]), p.group));
-      } else if constexpr (POLICY == 1) {
-#pragma unroll
-        for (int i = 0; i < NR; ++i) sp[i] = s_old[i];
-      } else {
-        static_assert(NR == 1, "the yoked path handles one row at a time");
-        // shadow chunk from shared memory (swizzled 16-byte units), as pairs
-        const int rc = row[0] * LPR + c;
-        const float4* rs = reinterpret_cast<const float4*>(st + L.shadow + rc * 128);
-        float2 rr[16];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float4 t = rs[u ^ (rc & 7)];
-          rr[2 * u] = make_float2(t.x, t.y);
-          rr[2 * u + 1] = make_float2(t.z, t.w);
-        }
-        // R' = R * a
-        if constexpr (DIAG) {
-          float2 aa[16];
-          load_pairs(st + L.a, c, aa);
-#pragma unroll
-          for (int m = 0; m < 16; ++m) rr[m] = __fmul2_rn(rr[m], aa[m]);
-        } else {
-#pragma unroll
-          for (int m = 0; m < 16; ++m) rr[m] = __fmul2_rn(rr[m], f2(a_scalar));
-        }
-        float wr;
-        if constexpr (DELTA) {
-          float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-          for (int m = 0; m < 16; ++m) acc = __ffma2_rn(rr[m], kk[m], acc);
-          wr = __fmul_rn(beta, __fsub_rn(v_i[0], row_tree<LPR>(acc)));
-        } else {
-          wr = wcoef[0];
-        }
-#pragma unroll
-        for (int m = 0; m < 16; ++m) rr[m] = __ffma2_rn(f2(wr), kk[m], rr[m]);
-        float* rg = p.shadow + (grow0 + row[0]) * DK + 32 * c;
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          uint32_t ww[8];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            ww[2 * e] = __float_as_uint(rr[4 * h + e].x);
-            ww[2 * e + 1] = __float_as_uint(rr[4 * h + e].y);
-          }
-          st_global_v8(rg + 8 * h, ww);
-        }
-        sp[0] = div_qmax_rn<QMAX>(row_max<LPR>(chunk_absmax(rr), p.group));
-      }
-
-      // ---- a8/a9: round (and BDR), pack, store codes (and scales)
-#pragma unroll
-      for (int i = 0; i < NR; ++i) {
-        uint32_t out[CW];
-        if (sp[i] > 0.0f) {
-          const float inv = recip_rn(sp[i]);
-          bool clamp;
-          if constexpr (POLICY == 0) {
-            // |x| <= group max, so |x * inv| <= qmax(1 + 2^-23) rounds inside
-            // the range whenever the scale is a normal float below 2^126
-            clamp = !(sp[i] >= 0x1p-126f && sp[i] < 0x1p126f);
-          } else {
-            const float xm = chunk_absmax(x[i]);
-            clamp = !(__fmaf_rn(xm, inv, kOff) <= kOff + kQf);
-          }
-          float2 y[16];
-          round_chunk<BITS>(x[i], inv, clamp, y);
-          if constexpr (BDR) {
-            float2 sk[16];
-            load_pairs(st + L.sk, c, sk);
-            const float sw = wcoef[i] > 0.0f ? 1.0f : (wcoef[i] < 0.0f ? -1.0f : 0.0f);
-            bdr_chunk<BITS>(y, Sp[i], sk, sw, sp[i]);
-          }
-          pack_chunk<BITS>(y, out);
-        } else {
-#pragma unroll
-          for (int q = 0; q < CW; ++q) out[q] = 0u;
-        }
-        if (valid[i]) {
-          uint8_t* cg = codes_u + row[i] * (DK * BITS / 8);
-          if constexpr (CW == 4) {
-            *reinterpret_cast<uint4*>(cg) = make_uint4(out[0], out[1], out[2], out[3]);
-          } else {
-            st_global_v8(cg, out);
-          }
-          if constexpr (POLICY != 1) {
-            if (writes_scale) scales_u[row[i] * ng] = sp[i];
-          }
-        }
-      }
-    }
-    __syncthreads();
-  }
-  cp_async_wait<0>();
 }
 
 // ---------------------------------------------------------------------------

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include "qstate_kernels.cuh"
+#include "qstate_step.cuh"
 
 namespace qs {
 

@@ -7,12 +7,13 @@
 
 namespace qs {
 
-// Stages of the cp.async ring per CTA.
+// Ring depth of the step kernel (row blocks per lane).
 template <int POLICY>
-constexpr int step_stages() { return POLICY == 2 ? 3 : QS_STAGES; }
+constexpr int step_depth() { return POLICY == 2 ? QS_DEPTH_YOKED : QS_DEPTH; }
 
-// Rows per work unit: the largest of QS_RB_MAX (64), 32, 16 that divides dv and keeps
-// one stage within `budget` bytes (so that three or four CTAs fit per SM).
+// Rows per work unit of the readout kernel: the largest of QS_RB_MAX (64), 32,
+// 16 that divides dv and keeps one stage within `budget` bytes (so that three
+// or four CTAs fit per SM).
 #ifndef QS_RB_MAX
 #define QS_RB_MAX 64
 #endif
@@ -60,16 +61,40 @@ static cudaError_t launch_persistent(K kernel, size_t smem, const StepParams& p,
 
 template <int BITS, int DK, int POLICY, bool BDR, bool DELTA, bool DIAG>
 cudaError_t launch_step(const StepParams& p0, cudaStream_t stream) {
-  constexpr int S = step_stages<POLICY>();
-  auto kernel = step_kernel<BITS, DK, POLICY, BDR, DELTA, DIAG, S>;
+  constexpr int D = step_depth<POLICY>();
+  constexpr int RW = 32 / (DK / 32);  // rows per row block
+  constexpr int WARPS = kThreads / 32;
+  auto kernel = step_kernel<BITS, DK, POLICY, BDR, DELTA, DIAG, D>;
   static std::once_flag flag;
   cudaError_t err = allow_smem(kernel, flag);
   if (err != cudaSuccess) return err;
-  StepParams p = p0;
-  p.rb = choose_rb(BITS, DK, p.dv, p.group, DIAG, BDR, POLICY == 2);
-  p.units_per_tile = p.dv / p.rb;
-  const StageLayout L(BITS, DK, p.rb, p.group, DIAG, BDR, POLICY == 2);
-  return launch_persistent(kernel, static_cast<size_t>(S) * L.bytes, p, stream);
+  WarpStepParams p;
+  p.codes = p0.codes;
+  p.scales = p0.scales;
+  p.shadow = p0.shadow;
+  p.q = p0.q;
+  p.k = p0.k;
+  p.v = p0.v;
+  p.alpha = p0.alpha;
+  p.beta = p0.beta;
+  p.o = p0.o;
+  p.bpt = p0.dv / RW;
+  p.nblocks = p0.tiles * p.bpt;  // < 2^31 (checked by the caller)
+  p.group = p0.group;
+  // tile-vector slots: every tile that D consecutive row blocks can touch
+  p.ntv = (D - 1 + p.bpt - 1) / p.bpt + 1;
+  const WarpLayout L(BITS, DK, DIAG, BDR, POLICY == 2);
+  p.warp_bytes = L.bytes(D, p.ntv);
+  const size_t smem = static_cast<size_t>(p.warp_bytes) * WARPS;
+  int per_sm = 0;
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, smem);
+  if (err != cudaSuccess) return err;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  long long grid = static_cast<long long>(per_sm) * device_sm_count();
+  const long long need = (static_cast<long long>(p.nblocks) + WARPS - 1) / WARPS;
+  if (grid > need) grid = need;
+  kernel<<<static_cast<int>(grid), kThreads, smem, stream>>>(p);
+  return cudaGetLastError();
 }
 
 template <int BITS, int DK>
