@@ -63,7 +63,7 @@ template <int BITS, int DK, int POLICY, bool BDR, bool DELTA, bool DIAG>
 cudaError_t launch_step(const StepParams& p0, cudaStream_t stream) {
   constexpr int D = step_depth<POLICY>();
   constexpr int RW = 32 / (DK / 32);  // rows per row block
-  constexpr int WARPS = kThreads / 32;
+  constexpr int WARPS = kStepWarps;
   auto kernel = step_kernel<BITS, DK, POLICY, BDR, DELTA, DIAG, D>;
   static std::once_flag flag;
   cudaError_t err = allow_smem(kernel, flag);
@@ -87,13 +87,13 @@ cudaError_t launch_step(const StepParams& p0, cudaStream_t stream) {
   p.warp_bytes = L.bytes(D, p.ntv);
   const size_t smem = static_cast<size_t>(p.warp_bytes) * WARPS;
   int per_sm = 0;
-  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, smem);
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kStepThreads, smem);
   if (err != cudaSuccess) return err;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
   long long grid = static_cast<long long>(per_sm) * device_sm_count();
   const long long need = (static_cast<long long>(p.nblocks) + WARPS - 1) / WARPS;
   if (grid > need) grid = need;
-  kernel<<<static_cast<int>(grid), kThreads, smem, stream>>>(p);
+  kernel<<<static_cast<int>(grid), kStepThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 

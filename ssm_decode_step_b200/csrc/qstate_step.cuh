@@ -38,6 +38,26 @@ namespace qs {
 #ifndef QS_DEPTH_YOKED
 #define QS_DEPTH_YOKED 2
 #endif
+// Warps per CTA of the step kernel.  With one, everything derived from the
+// row-block cursor is uniform across the CTA, which the compiler keeps in
+// uniform registers and branches on without divergence bookkeeping.
+#ifndef QS_STEP_WARPS
+#define QS_STEP_WARPS 1
+#endif
+constexpr int kStepWarps = QS_STEP_WARPS;
+constexpr int kStepThreads = 32 * kStepWarps;
+// Read k from shared memory at each use instead of keeping the tile's k
+// chunk in 32 registers (non-yoked kernels).
+#ifndef QS_K_SMEM
+#define QS_K_SMEM 0
+#endif
+// Resident warps per SM the register allocation targets.
+#ifndef QS_STEP_WARPS_PER_SM
+#define QS_STEP_WARPS_PER_SM 16
+#endif
+#ifndef QS_STEP_WARPS_PER_SM_LOW
+#define QS_STEP_WARPS_PER_SM_LOW 12
+#endif
 
 struct WarpStepParams {
   uint8_t* codes;
@@ -208,7 +228,8 @@ __device__ __forceinline__ void issue_block(const BlockCursor<SLOT, DEPTH>& cur,
 
 // POLICY: 0 dynamic, 1 persistent, 2 yoked.
 template <int BITS, int DK, int POLICY, bool BDR, bool DELTA, bool DIAG, int DEPTH>
-__global__ void __launch_bounds__(kThreads, (POLICY == 2 || BDR) ? QS_MIN_BLOCKS_YOKED : QS_MIN_BLOCKS)
+__global__ void __launch_bounds__(kStepThreads, ((POLICY == 2 || BDR) ? QS_STEP_WARPS_PER_SM_LOW
+                                                                    : QS_STEP_WARPS_PER_SM) / kStepWarps)
     step_kernel(WarpStepParams p) {
   constexpr int LPR = DK / 32;
   constexpr int RW = 32 / LPR;
@@ -218,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, (POLICY == 2 || BDR) ? QS_MIN_BLOCKS
   constexpr int QMAX = BITS == 4 ? 7 : 127;
   constexpr float kQf = static_cast<float>(QMAX);
   constexpr float kOff = kMagic + (BITS == 4 ? 8.0f : 128.0f);
-  constexpr int WARPS = kThreads / 32;
+  constexpr int WARPS = kStepWarps;
   constexpr unsigned CSTRIDE = RW * DK * BITS / 8;  // code bytes per row block
   // ring-slot layout in bytes (the same as WarpLayout's)
   constexpr int O_SCALES = 32 * CB;
@@ -228,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, (POLICY == 2 || BDR) ? QS_MIN_BLOCKS
 
   extern __shared__ __align__(128) unsigned char smem[];
   const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
+  const int warp = WARPS == 1 ? 0 : threadIdx.x >> 5;
   const int c = lane % LPR, rr = lane / LPR;
   const WarpLayout L(BITS, DK, DIAG, BDR, YOKED);
   unsigned char* ring = smem + warp * p.warp_bytes;
@@ -280,7 +301,8 @@ __global__ void __launch_bounds__(kThreads, (POLICY == 2 || BDR) ? QS_MIN_BLOCKS
     pre.advance(bpt, L.tv, tv_end);
   }
 
-  float2 kk[16];
+  constexpr bool K_SMEM = QS_K_SMEM && !YOKED;
+  float2 kk[K_SMEM ? 1 : 16];
   float beta = 0.0f, a_scalar = 1.0f;
 
 #pragma unroll 1
@@ -300,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, (POLICY == 2 || BDR) ? QS_MIN_BLOCKS
     if (cur.tile_start) {
       // every lane's copies of the tile vectors have landed: publish them
       __syncwarp();
-      load_pairs(tv + L.k, c, kk);
+      if constexpr (!K_SMEM) load_pairs(tv + L.k, c, kk);
       const float* misc = reinterpret_cast<const float*>(tv + L.misc);
       beta = misc[1];
       a_scalar = DIAG ? 1.0f : misc[0];
@@ -308,9 +330,11 @@ __global__ void __launch_bounds__(kThreads, (POLICY == 2 || BDR) ? QS_MIN_BLOCKS
         // sign(k_j) per column, in the layout of k
         if (rr == 0) {
           float* ss = reinterpret_cast<float*>(tv + L.sk) + c * kChunkStride;
+          float2 kt[16];
+          load_pairs(tv + L.k, c, kt);
 #pragma unroll
           for (int m = 0; m < 16; ++m) {
-            const float2 kv = kk[m];
+            const float2 kv = kt[m];
             ss[2 * m] = kv.x > 0.0f ? 1.0f : (kv.x < 0.0f ? -1.0f : 0.0f);
             ss[2 * m + 1] = kv.y > 0.0f ? 1.0f : (kv.y < 0.0f ? -1.0f : 0.0f);
           }
@@ -346,18 +370,37 @@ __global__ void __launch_bounds__(kThreads, (POLICY == 2 || BDR) ? QS_MIN_BLOCKS
     }
 
     // ---- a3/a4: key projection and rank-1 write
+    const float4* kp4 = reinterpret_cast<const float4*>(tv + L.k) + c * (kChunkStride / 4);
     float wcoef;
     if constexpr (DELTA) {
       float2 acc = make_float2(0.0f, 0.0f);
+      if constexpr (K_SMEM) {
 #pragma unroll
-      for (int m = 0; m < 16; ++m) acc = __ffma2_rn(Sp[m], kk[m], acc);
+        for (int m = 0; m < 8; ++m) {
+          const float4 t = kp4[m];
+          acc = __ffma2_rn(Sp[2 * m], make_float2(t.x, t.y), acc);
+          acc = __ffma2_rn(Sp[2 * m + 1], make_float2(t.z, t.w), acc);
+        }
+      } else {
+#pragma unroll
+        for (int m = 0; m < 16; ++m) acc = __ffma2_rn(Sp[m], kk[m], acc);
+      }
       wcoef = __fmul_rn(beta, __fsub_rn(v_i, row_tree<LPR>(acc)));
     } else {
       wcoef = __fmul_rn(beta, v_i);
     }
     float2 x[16];
+    if constexpr (K_SMEM) {
 #pragma unroll
-    for (int m = 0; m < 16; ++m) x[m] = __ffma2_rn(f2(wcoef), kk[m], Sp[m]);
+      for (int m = 0; m < 8; ++m) {
+        const float4 t = kp4[m];
+        x[2 * m] = __ffma2_rn(f2(wcoef), make_float2(t.x, t.y), Sp[2 * m]);
+        x[2 * m + 1] = __ffma2_rn(f2(wcoef), make_float2(t.z, t.w), Sp[2 * m + 1]);
+      }
+    } else {
+#pragma unroll
+      for (int m = 0; m < 16; ++m) x[m] = __ffma2_rn(f2(wcoef), kk[m], Sp[m]);
+    }
 
     // ---- a5: readout from the updated state
     if (readout) {
