@@ -381,6 +381,7 @@ __device__ __forceinline__ void bdr_chunk(float2 (&y)[16], const float2 (&Sp)[16
                                           const float2 (&sk)[16], float sw, float sp) {
   constexpr float kOff = kMagic + (BITS == 4 ? 8.0f : 128.0f);
   constexpr float kQ = BITS == 4 ? 7.0f : 127.0f;
+  float hi = kOff, lo = kOff;
 #pragma unroll
   for (int m = 0; m < 16; ++m) {
     const float2 nf = __fadd2_rn(y[m], f2(-kOff));                   // n, exact
@@ -390,8 +391,18 @@ __device__ __forceinline__ void bdr_chunk(float2 (&y)[16], const float2 (&Sp)[16
     const float2 t = __fmul2_rn(e, sg);                              // > 0 iff reversed
     const float yx = t.x > 0.0f ? __fadd_rn(y[m].x, sg.x) : y[m].x;
     const float yy = t.y > 0.0f ? __fadd_rn(y[m].y, sg.y) : y[m].y;
-    y[m].x = fminf(fmaxf(yx, kOff - kQ), kOff + kQ);
-    y[m].y = fminf(fmaxf(yy, kOff - kQ), kOff + kQ);
+    y[m].x = yx;
+    y[m].y = yy;
+    hi = fmaxf(hi, fmaxf(yx, yy));
+    lo = fminf(lo, fminf(yx, yy));
+  }
+  // only a moved code can leave [-qmax, qmax]: clamp when the extremes show one did
+  if (hi > kOff + kQ || lo < kOff - kQ) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      y[i].x = fminf(fmaxf(y[i].x, kOff - kQ), kOff + kQ);
+      y[i].y = fminf(fmaxf(y[i].y, kOff - kQ), kOff + kQ);
+    }
   }
 }
 
