@@ -15,15 +15,17 @@
 // whatever the tile count.  Warps never wait for each other: there is no
 // block-level barrier in the kernel.
 //
-// Memory path.  Each lane copies the bytes it alone will read (its 16 or 32
-// code bytes, its scale, its row's v, its 128 shadow bytes) with cp.async
-// into a DEPTH-slot ring that is private to the lane, DEPTH - 1 row blocks
-// ahead of the one it computes, so its own cp.async.wait_group is the only
-// synchronisation those bytes need.  The per-tile vectors (k, q, diagonal
-// alpha, alpha, beta) go once per tile into one of `ntv` per-warp slots,
-// copied by all lanes together and published with __syncwarp; ntv covers
-// every tile that the prefetch window can span.  New codes, scales, shadow
-// and o leave straight from registers with 16/32-byte stores.
+// Memory path.  A two-slot cp.async ring per warp holds the next row block
+// while the current one is computed.  Every copy instruction reads 512
+// consecutive bytes across the warp (lane l copies the l-th 16-byte unit
+// of the block's codes or shadow, which may belong to another lane); the
+// warp publishes a slot with __syncwarp after its cp.async.wait_group and
+// again before the slot is refilled.  The per-tile vectors (k, q, diagonal
+// alpha, alpha, beta, sign(k) for BDR) go once per tile into one of `ntv`
+// per-warp slots; ntv covers every tile that the prefetch window can span.
+// New codes, scales, shadow and o leave straight from registers with
+// 16/32-byte stores.  One warp per CTA by default, so the row-block cursor
+// is uniform across the CTA.
 #pragma once
 
 #include "qstate_kernels.cuh"
