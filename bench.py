@@ -634,6 +634,101 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# recall over a decode horizon (a measurement of the quantized recurrence,
+# not a throughput figure)
+# ---------------------------------------------------------------------------
+def plant(S_w: np.ndarray, kstar: np.ndarray, vstar: np.ndarray) -> np.ndarray:
+    """S0 that maps the unit key k* to v* and agrees with S_w on the
+    complement of k*: S0 = S_w + (v* - S_w k*) k*^T, in float64 on the host,
+    rounded once to float32 (the probe the horizon measurement reads back)."""
+    S = S_w.astype(np.float64)
+    k = kstar.astype(np.float64)
+    v = vstar.astype(np.float64)
+    S += np.einsum("ti,tj->tij", v - np.einsum("tij,tj->ti", S, k), k)
+    return np.ascontiguousarray(S, dtype=np.float32)
+
+
+def run_recall(args):
+    """Plant (k*, v*) in S0, decode H distractor steps under every arm and the
+    FP32 state, and read S_t k* and ||S_t|| at power-of-two checkpoints
+    ("When Dynamic Scaling Fails": recall of a fact planted before
+    quantization began, as the decode horizon grows; the scale-state feedback
+    shows as norm inflation).  Prints one JSON line."""
+    import torch
+    from ssm_decode_step_b200 import qstate as Q
+    w = W.get("recall")
+    H, T, dk, dv = args.recall_steps, w.tiles, w.dk, w.dv
+    dev = torch.device("cuda")
+    torch.cuda.set_device(0)
+    kstar, vstar = W.probe(w)
+    S0 = plant(W.initial_state(w), kstar, vstar)
+    P = max(1, min(args.pool, H))
+    pool = [torch.from_numpy(a).to(dev) for a in W.pool(w, P)]
+    kst = torch.from_numpy(kstar).to(dev)
+    zk = torch.zeros((T, dk), dtype=torch.float32, device=dev)
+    zv = torch.zeros((T, dv), dtype=torch.float32, device=dev)
+    one = torch.ones(T, dtype=torch.float32, device=dev)
+    zero = torch.zeros(T, dtype=torch.float32, device=dev)
+    o = torch.empty((T, dv), dtype=torch.float32, device=dev)
+    nrm = torch.empty(T, dtype=torch.float64, device=dev)
+    marks = sorted({0, H} | {1 << i for i in range(40) if (1 << i) <= H})
+    launches = 0
+
+    def trajectory(step, probe):
+        nonlocal launches
+        rec, norms = [], []
+        t = 0
+        for m in marks:
+            while t < m:
+                step(t % P)
+                launches += 1
+                t += 1
+            probe()
+            launches += 2
+            torch.cuda.synchronize()
+            rec.append(o.cpu().numpy().astype(np.float64))
+            norms.append(nrm.cpu().numpy())
+        return np.stack(rec), np.stack(norms)
+
+    t0 = time.time()
+    cfg32 = Q.Config(T, dk, dv, 8, 32, w.delta, w.decay)
+    S = torch.from_numpy(S0.copy()).to(dev)
+    fp = trajectory(
+        lambda i: Q.fp32_decode_step(cfg32, S, None, pool[1][i], pool[2][i], pool[3][i], pool[4][i], None),
+        # readout with a zero update (alpha = 1, k = 0, beta = 0) leaves S unchanged
+        lambda: (Q.fp32_decode_step(cfg32, S, kst, zk, zv, one, zero, o), Q.fp32_sq_norms(cfg32, S, nrm)))
+    arms = {}
+    for arm in w.arms:
+        cfg = Q.Config(T, dk, dv, arm.bits, arm.group, w.delta, w.decay, arm.policy, arm.rounding)
+        st = Q.QState(cfg).init(torch.from_numpy(S0).to(dev))
+        arms[arm.name] = trajectory(
+            lambda i, st=st: st.step(None, pool[1][i], pool[2][i], pool[3][i], pool[4][i], None),
+            lambda st=st, cfg=cfg: (st.readout(kst, o), Q.state_sq_norms(cfg, st.codes, st.scales, nrm)))
+    elapsed = time.time() - t0
+
+    vs = vstar.astype(np.float64)
+    med = lambda a: [round(float(x), 6) for x in np.median(a, axis=1)]
+    rel = lambda r, ref: np.linalg.norm(r - ref, axis=-1) / np.linalg.norm(ref, axis=-1)
+    out = {"experiment": "recall over the decode horizon", "workload": w.description,
+           "tiles": T, "steps": H, "checkpoints": marks, "launches": launches,
+           "seconds": round(elapsed, 2),
+           "fp32": {"recall_err_vs_vstar": med(rel(fp[0], vs[None])),
+                    "state_norm": med(np.sqrt(fp[1]))},
+           "arms": {}}
+    for name, (r, n) in arms.items():
+        e = np.median(rel(r, fp[0]), axis=1)
+        bad = [m for m, x in zip(marks, e) if x > args.recall_tol]
+        out["arms"][name] = {
+            "recall_err_vs_fp32": [round(float(x), 6) for x in e],
+            "recall_err_vs_vstar": med(rel(r, vs[None])),
+            "norm_ratio_vs_fp32": med(np.sqrt(n / fp[1])),
+            "horizon": bad[0] if bad else None}
+    out["horizon_rule"] = (f"first checkpoint where the median over tiles of "
+                           f"||S_t k* - S_t^fp32 k*|| / ||S_t^fp32 k*|| exceeds {args.recall_tol}")
+    print(json.dumps(out))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -649,10 +744,16 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp32", action="store_true", help="skip the FP32-state comparison arm")
+    ap.add_argument("--recall", action="store_true",
+                    help="measure recall of a planted association over the decode horizon instead")
+    ap.add_argument("--recall-steps", type=int, default=32768)
+    ap.add_argument("--recall-tol", type=float, default=0.5)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.impl == "reference":
+    if args.recall:
+        run_recall(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

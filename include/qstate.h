@@ -32,11 +32,12 @@
  *                                            updated by the same steps
  *   if s'_ig > 0: n_ij = clamp(round_half_even(x_ij * (1/s'_ig)), +-qmax),
  *                 the product taken exactly; else n_ij = 0 for the group
- *   BDR: with sigma = sign(w_i) sign(k_j), if sigma > 0 and n s' < S'_ij
- *        then n += 1; if sigma < 0 and n s' > S'_ij then n -= 1; clamp.
- *        ("Preserving Updates in Low-Bit Recurrent State Quantization",
- *        abstract: elements whose rounding moves against their update are
- *        rounded one step toward it.)
+ *   BDR: with sigma = sign(w_i) sign(k_j) and d_ij = c_ij * s_ig the
+ *        element as stored before the step (no decay), if sigma > 0 and
+ *        n s' < d_ij then n += 1; if sigma < 0 and n s' > d_ij then
+ *        n -= 1; clamp.  ("Preserving Updates in Low-Bit Recurrent State
+ *        Quantization", abstract: a stored element whose value moves
+ *        against its update is rounded one step toward it.)
  * qmax = 2^(bits-1) - 1.  Dot products "." are evaluated in one fixed
  * order: each 32-column chunk is summed as two fused multiply-add chains
  * from +0 in column order, one over its even and one over its odd columns,
@@ -166,6 +167,22 @@ QS_API qs_status qstate_readout(const qs_config* cfg, const void* codes,
 QS_API qs_status qstate_fp32_decode_step(const qs_config* cfg, float* S, const float* q,
                                          const float* k, const float* v, const float* alpha,
                                          const float* beta, float* o, cudaStream_t stream);
+
+/* Squared Frobenius norm of every tile of the stored state, for tracking
+ * the state norm over a decode horizon (the norm inflation of per-token
+ * dynamic scaling: "When Dynamic Scaling Fails", abstract and project page,
+ * the feedback-loop passage).  out[t] = sum over (i, j) of d_ij^2 with
+ * d_ij = c_ij * s_ig formed in FP32 as in qstate_readout, each square and
+ * the sum in FP64 (summation order unspecified: the result is the exact
+ * sum up to FP64 rounding).  out: device array of num_tiles doubles,
+ * 8-byte aligned, written on `stream`. */
+QS_API qs_status qstate_state_sq_norms(const qs_config* cfg, const void* codes,
+                                       const float* scales, double* out, cudaStream_t stream);
+
+/* The same for an FP32 state S [T][Dv][Dk] (16-byte aligned): out[t] = sum
+ * of S_ij^2 in FP64.  Only num_tiles, dk and dv of cfg are used. */
+QS_API qs_status qstate_fp32_sq_norms(const qs_config* cfg, const float* S, double* out,
+                                      cudaStream_t stream);
 
 /* Self-check of the library's fast arithmetic on the current GPU.  The
  * kernels compute the reciprocal of a scale and the division of a group

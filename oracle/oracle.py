@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
             "qo_step": [C, P, P, P, P, P, P, P, P, P, P],
             "qo_readout": [C, P, P, P, P],
             "qo_fp32_step": [C, P, P, P, P, P, P, P],
+            "qo_sq_norms": [C, P, P, P],
+            "qo_fp32_sq_norms": [C, P, P],
         }.items():
             f = getattr(L, name)
             f.argtypes = args
@@ -202,3 +204,21 @@ def fp32_step(cfg: OracleConfig, S, q, k, v, alpha, beta, want_o=True):
     _ok(lib().qo_fp32_step(ctypes.byref(cc), _p(S), _p(q), _p(k), _p(v), _p(alpha),
                            _p(beta), _p(o)), "fp32_step")
     return o
+
+
+def sq_norms(st: State) -> np.ndarray:
+    """Squared Frobenius norm of each tile of the dequantized stored state (float64 [T])."""
+    cfg = st.cfg
+    out = np.empty(cfg.tiles, dtype=np.float64)
+    cc = cfg.c()
+    _ok(lib().qo_sq_norms(ctypes.byref(cc), _p(st.codes), _p(st.scales), _p(out)), "sq_norms")
+    return out
+
+
+def fp32_sq_norms(cfg: OracleConfig, S) -> np.ndarray:
+    """Squared Frobenius norm of each tile of an FP32 state (float64 [T])."""
+    S = _f32(S)
+    out = np.empty(cfg.tiles, dtype=np.float64)
+    cc = cfg.c()
+    _ok(lib().qo_fp32_sq_norms(ctypes.byref(cc), _p(S), _p(out)), "fp32_sq_norms")
+    return out

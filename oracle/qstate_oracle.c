@@ -142,9 +142,11 @@ static int32_t clamp_code(int32_t n, int qmax) {
   return n < -qmax ? -qmax : (n > qmax ? qmax : n);
 }
 
-/* Steps 6-8 for one row.  x: updated row; Sp: decayed row before the write
- * (the BDR reference); d: dequantized row before decay (used only by the
- * planted BDR_REFERENCE mistake); R: updated shadow row or NULL. */
+/* Steps 6-8 for one row.  x: updated row; d: the row as stored before this
+ * step, dequantized without decay (the BDR reference: a code's move is from
+ * its stored value before the step to its stored value after it); Sp:
+ * decayed row before the write (used only by the planted BDR_REFERENCE
+ * mistake); R: updated shadow row or NULL. */
 static void requantize_row(const qo_cfg* c, const float* x, const float* Sp,
                            const float* d, const float* R, float w,
                            const float* k, int32_t* crow, float* srow,
@@ -176,7 +178,7 @@ static void requantize_row(const qo_cfg* c, const float* x, const float* Sp,
         int32_t n = nearest_code(x[j], inv, qmax, pre ? &pre[j] : NULL);
         if (c->rounding == QO_ROUND_BDR) {
           float sigma = sign_of(w) * sign_of(k[j]);
-          float ref = (g_fault == QO_FAULT_BDR_REFERENCE) ? d[j] : Sp[j];
+          float ref = (g_fault == QO_FAULT_BDR_REFERENCE) ? Sp[j] : d[j];
           float dq = (float)n * s_new;
           if (sigma > 0.0f && dq < ref)
             n += 1;
@@ -282,6 +284,39 @@ int qo_readout(const qo_cfg* c, const int32_t* codes, const float* scales,
       }
       o[row] = qo_dot(d, q + (size_t)t * dk, dk);
     }
+  }
+  return 0;
+}
+
+int qo_sq_norms(const qo_cfg* c, const int32_t* codes, const float* scales, double* out) {
+  if (qo_check(c) || !codes || !scales || !out) return -1;
+  const int dk = c->dk, dv = c->dv, G = c->group, ng = dk / G;
+#pragma omp parallel for schedule(static)
+  for (int t = 0; t < c->tiles; ++t) {
+    double acc = 0.0;
+    for (int i = 0; i < dv; ++i) {
+      size_t row = (size_t)t * dv + i;
+      for (int j = 0; j < dk; ++j) {
+        double d = (double)((float)codes[row * dk + j] * scales[row * ng + j / G]);
+        acc += d * d;
+      }
+    }
+    out[t] = acc;
+  }
+  return 0;
+}
+
+int qo_fp32_sq_norms(const qo_cfg* c, const float* S, double* out) {
+  if (qo_check(c) || !S || !out) return -1;
+  const size_t n = (size_t)c->dv * c->dk;
+#pragma omp parallel for schedule(static)
+  for (int t = 0; t < c->tiles; ++t) {
+    double acc = 0.0;
+    for (size_t e = 0; e < n; ++e) {
+      double x = (double)S[(size_t)t * n + e];
+      acc += x * x;
+    }
+    out[t] = acc;
   }
   return 0;
 }

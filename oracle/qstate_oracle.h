@@ -96,6 +96,14 @@ int qo_fp32_step(const qo_cfg* c, float* S, const float* q, const float* k,
                  const float* v, const float* alpha, const float* beta,
                  float* o);
 
+/* Squared Frobenius norm of each tile, out[t] (doubles), summed in FP64 in
+ * row-major order: of the dequantized stored state (d = c * s in FP32, as in
+ * qo_readout), and of an FP32 state [tiles][dv][dk].  The state norm over a
+ * decode horizon is the quantity whose inflation under per-token dynamic
+ * scaling "When Dynamic Scaling Fails" reports (abstract, project page). */
+int qo_sq_norms(const qo_cfg* c, const int32_t* codes, const float* scales, double* out);
+int qo_fp32_sq_norms(const qo_cfg* c, const float* S, double* out);
+
 /* The fixed-order dot product used throughout (exposed for tests). */
 float qo_dot(const float* a, const float* b, int n);
 
@@ -109,7 +117,7 @@ enum {
   QO_FAULT_DECAY_SKIPPED = 3,   /* decay not applied                         */
   QO_FAULT_READ_K_FOR_Q = 4,    /* readout uses k instead of q               */
   QO_FAULT_GROUP_INDEX = 5,     /* scale of the wrong group used             */
-  QO_FAULT_BDR_REFERENCE = 6,   /* BDR measured from the stale value         */
+  QO_FAULT_BDR_REFERENCE = 6,   /* BDR measured from the decayed value S'    */
   QO_FAULT_ROUND_TRUNC = 7,     /* truncation instead of nearest rounding    */
   QO_FAULT_BETA_ON_V_ONLY = 8,  /* beta applied to v but not to the delta term */
   QO_FAULT_DIAG_DECAY_ROW = 9,  /* diagonal decay indexed by row, not column  */

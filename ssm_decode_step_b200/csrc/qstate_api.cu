@@ -9,6 +9,7 @@
 #include "../../include/qstate.h"
 #include "qstate_fp32.cuh"
 #include "qstate_launch.h"
+#include "qstate_norms.cuh"
 
 namespace qs {
 
@@ -317,6 +318,55 @@ qs_status qstate_readout(const qs_config* cfg, const void* codes, const float* s
   else
     e = cfg->dk == 64 ? qs::launch_readout<8, 64>(p, stream) : qs::launch_readout<8, 128>(p, stream);
   return from_cuda(e);
+}
+
+qs_status qstate_state_sq_norms(const qs_config* cfg, const void* codes, const float* scales,
+                                double* out, cudaStream_t stream) {
+  qs_status st = check_config(cfg);
+  if (st != QS_OK) return st;
+  if (cfg->num_tiles == 0) return QS_OK;
+  if (!codes || !scales || !out) return QS_ERR_INVALID_ARG;
+  if (!aligned(codes, 32) || !aligned(scales, 4) || !aligned(out, 8)) return QS_ERR_INVALID_ARG;
+  const Sizes s = sizes_of(cfg);
+  const Range w[1] = {range_of(out, static_cast<size_t>(cfg->num_tiles) * sizeof(double))};
+  const Range r[2] = {range_of(codes, s.codes), range_of(scales, s.scales)};
+  if (any_overlap(w, 1, r, 2)) return QS_ERR_INVALID_ARG;
+  const uint8_t* c8 = static_cast<const uint8_t*>(codes);
+  const dim3 grid(static_cast<unsigned>(cfg->num_tiles)), block(qs::kNormThreads);
+  if (cfg->bits == 4) {
+    if (cfg->dk == 64)
+      qs::state_sq_norm_kernel<4, 64><<<grid, block, 0, stream>>>(c8, scales, out, cfg->dv, cfg->group);
+    else
+      qs::state_sq_norm_kernel<4, 128><<<grid, block, 0, stream>>>(c8, scales, out, cfg->dv, cfg->group);
+  } else {
+    if (cfg->dk == 64)
+      qs::state_sq_norm_kernel<8, 64><<<grid, block, 0, stream>>>(c8, scales, out, cfg->dv, cfg->group);
+    else
+      qs::state_sq_norm_kernel<8, 128><<<grid, block, 0, stream>>>(c8, scales, out, cfg->dv, cfg->group);
+  }
+  return from_cuda(cudaGetLastError());
+}
+
+qs_status qstate_fp32_sq_norms(const qs_config* cfg, const float* S, double* out,
+                               cudaStream_t stream) {
+  if (cfg == nullptr) return QS_ERR_INVALID_ARG;
+  qs_config c = *cfg;
+  c.bits = 8;
+  c.group = 32;
+  c.policy = QS_SCALE_PERSISTENT;
+  c.rounding = QS_ROUND_NEAREST;
+  qs_status st = check_config(&c);
+  if (st != QS_OK) return st;
+  if (c.num_tiles == 0) return QS_OK;
+  if (!S || !out) return QS_ERR_INVALID_ARG;
+  if (!aligned(S, 16) || !aligned(out, 8)) return QS_ERR_INVALID_ARG;
+  const size_t elems = static_cast<size_t>(c.dv) * c.dk;
+  const Range w[1] = {range_of(out, static_cast<size_t>(c.num_tiles) * sizeof(double))};
+  const Range r[1] = {range_of(S, static_cast<size_t>(c.num_tiles) * elems * sizeof(float))};
+  if (any_overlap(w, 1, r, 1)) return QS_ERR_INVALID_ARG;
+  qs::fp32_sq_norm_kernel<<<static_cast<unsigned>(c.num_tiles), qs::kNormThreads, 0, stream>>>(
+      S, out, static_cast<long long>(elems));
+  return from_cuda(cudaGetLastError());
 }
 
 }  // extern "C"

@@ -375,22 +375,25 @@ __device__ __forceinline__ void round_chunk(const float2 (&x)[16], float inv, bo
 
 // Bounded Directional Rounding on rounded values y (see qstate.h): with
 // sigma = sign(w) sign(k_j), move n one step toward the update when n*s'
-// lies on the wrong side of the pre-update value S'.
+// lies on the wrong side of d, the element as stored before the step.
 template <int BITS>
-__device__ __forceinline__ void bdr_chunk(float2 (&y)[16], const float2 (&Sp)[16],
+__device__ __forceinline__ void bdr_chunk(float2 (&y)[16], const float2 (&d)[16],
                                           const float2 (&sk)[16], float sw, float sp) {
   constexpr float kOff = kMagic + (BITS == 4 ? 8.0f : 128.0f);
   constexpr float kQ = BITS == 4 ? 7.0f : 127.0f;
   float hi = kOff, lo = kOff;
 #pragma unroll
   for (int m = 0; m < 16; ++m) {
-    const float2 nf = __fadd2_rn(y[m], f2(-kOff));                   // n, exact
-    const float2 dq = __fmul2_rn(nf, f2(sp));                        // n * s'
-    const float2 e = __fadd2_rn(Sp[m], make_float2(-dq.x, -dq.y));  // sign of S' - n s'
-    const float2 sg = __fmul2_rn(sk[m], f2(sw));                     // sigma in {-1, 0, 1}
-    const float2 t = __fmul2_rn(e, sg);                              // > 0 iff reversed
-    const float yx = t.x > 0.0f ? __fadd_rn(y[m].x, sg.x) : y[m].x;
-    const float yy = t.y > 0.0f ? __fadd_rn(y[m].y, sg.y) : y[m].y;
+    // reversed iff sigma (n s') < sigma d; the products by sigma in
+    // {-1, 0, 1} are exact, and comparing the two rounded values directly
+    // (no subtraction after the product) leaves nothing to contract
+    const float2 nf = __fadd2_rn(y[m], f2(-kOff));   // n, exact
+    const float2 dq = __fmul2_rn(nf, f2(sp));        // n * s'
+    const float2 sg = __fmul2_rn(sk[m], f2(sw));     // sigma
+    const float2 a = __fmul2_rn(dq, sg);
+    const float2 b = __fmul2_rn(d[m], sg);
+    const float yx = a.x < b.x ? __fadd_rn(y[m].x, sg.x) : y[m].x;
+    const float yy = a.y < b.y ? __fadd_rn(y[m].y, sg.y) : y[m].y;
     y[m].x = yx;
     y[m].y = yy;
     hi = fmaxf(hi, fmaxf(yx, yy));

@@ -358,6 +358,12 @@ __global__ void __launch_bounds__(kStepThreads, ((POLICY == 2 || BDR) ? QS_STEP_
     const float v_i = reinterpret_cast<const float*>(s + O_V)[lane];
     float2 Sp[16];
     decode_chunk<BITS>(w, Sp);
+    // BDR's reference: the element as stored before the step, d = c * s
+    float2 dref[BDR ? 16 : 1];
+    if constexpr (BDR) {
+#pragma unroll
+      for (int m = 0; m < 16; ++m) dref[m] = __fmul2_rn(Sp[m], f2(s_old));
+    }
 
     // ---- a2: dequantize with the decayed scale, S' = c * (s * a)
     if constexpr (DIAG) {
@@ -501,7 +507,7 @@ __global__ void __launch_bounds__(kStepThreads, ((POLICY == 2 || BDR) ? QS_STEP_
       float2 sk[16];
       load_pairs(tv + L.sk, c, sk);
       const float sw = zero ? 0.0f : (wcoef > 0.0f ? 1.0f : (wcoef < 0.0f ? -1.0f : 0.0f));
-      bdr_chunk<BITS>(y, Sp, sk, sw, sp);
+      bdr_chunk<BITS>(y, dref, sk, sw, sp);
     }
     uint32_t out[CW];
     pack_chunk<BITS>(y, out);

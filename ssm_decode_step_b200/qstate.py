@@ -24,7 +24,8 @@ QS_OK, QS_ERR_INVALID_ARG, QS_ERR_UNSUPPORTED, QS_ERR_CUDA = 0, 1, 2, 3
 
 # Every entry point that include/qstate.h declares.
 EXPORTS = ("qstate_query_sizes", "qstate_init", "qstate_decode_step", "qstate_readout",
-           "qstate_fp32_decode_step", "qstate_selfcheck", "qstate_status_string", "qstate_version")
+           "qstate_fp32_decode_step", "qstate_state_sq_norms", "qstate_fp32_sq_norms",
+           "qstate_selfcheck", "qstate_status_string", "qstate_version")
 
 
 class QStateError(RuntimeError):
@@ -57,8 +58,11 @@ def lib() -> ctypes.CDLL:
         L.qstate_readout.argtypes = [C, P, P, P, P, P]
         L.qstate_selfcheck.argtypes = [P, P]
         L.qstate_fp32_decode_step.argtypes = [C, P, P, P, P, P, P, P, P]
+        L.qstate_state_sq_norms.argtypes = [C, P, P, P, P]
+        L.qstate_fp32_sq_norms.argtypes = [C, P, P, P]
         for f in (L.qstate_query_sizes, L.qstate_init, L.qstate_decode_step, L.qstate_readout,
-                  L.qstate_selfcheck, L.qstate_fp32_decode_step):
+                  L.qstate_selfcheck, L.qstate_fp32_decode_step, L.qstate_state_sq_norms,
+                  L.qstate_fp32_sq_norms):
             f.restype = ctypes.c_int
         L.qstate_status_string.argtypes = [ctypes.c_int]
         L.qstate_status_string.restype = ctypes.c_char_p
@@ -151,6 +155,20 @@ def fp32_decode_step(cfg: Config, S, q, k, v, alpha, beta, o=None, stream=None) 
     _check(lib().qstate_fp32_decode_step(ctypes.byref(cc), _ptr(S), _ptr(q), _ptr(k), _ptr(v),
                                          _ptr(alpha), _ptr(beta), _ptr(o), _stream(stream)),
            "qstate_fp32_decode_step")
+
+
+def state_sq_norms(cfg: Config, codes, scales, out, stream=None) -> None:
+    """out[t] (float64 [T]) = squared Frobenius norm of tile t of the stored state."""
+    cc = cfg.c()
+    _check(lib().qstate_state_sq_norms(ctypes.byref(cc), _ptr(codes), _ptr(scales), _ptr(out),
+                                       _stream(stream)), "qstate_state_sq_norms")
+
+
+def fp32_sq_norms(cfg: Config, S, out, stream=None) -> None:
+    """out[t] (float64 [T]) = squared Frobenius norm of tile t of an FP32 state."""
+    cc = cfg.c()
+    _check(lib().qstate_fp32_sq_norms(ctypes.byref(cc), _ptr(S), _ptr(out), _stream(stream)),
+           "qstate_fp32_sq_norms")
 
 
 def selfcheck(stream=None):

@@ -107,6 +107,12 @@ def _draw_slot(law: str, rng: np.random.Generator, T: int, dk: int, dv: int,
         v = rng.standard_normal((T, dv)) * s
         alpha = rng.uniform(0.8, 1.0, size=(T, dk))
         beta = np.ones((T,))
+    elif law == "recall":       # distractor steps of the recall-over-horizon measurement
+        q = rng.standard_normal((T, dk))
+        k = _unit_rows(rng.standard_normal((T, dk)))
+        v = rng.standard_normal((T, dv))
+        alpha = rng.uniform(0.999, 1.0, size=(T,))
+        beta = rng.uniform(0.0, 0.1, size=(T,))
     else:
         raise ValueError(law)
     if decay == "diagonal" and alpha.ndim == 1:
@@ -163,7 +169,19 @@ STACK = _reg(Workload(
     seed=4, layer_seeds=tuple(4000 + l for l in range(24)),
     s0_std=1.0 / np.sqrt(128.0), draw="gdn"))
 
-# Index in the order the workloads are listed for this step.
+RECALL = _reg(Workload(
+    name="recall", description="recall over a decode horizon, gated delta rule: B16 H16 "
+    "Dk=Dv=128, a probe association (k*, v*) planted in S0, then distractor steps with k "
+    "unit-norm, v~N(0,1), alpha~U(0.999,1), beta~U(0,0.1); INT8/INT4 dynamic, INT4 persistent, "
+    "yoked and BDR arms against the FP32 state; seed 5",
+    layers=1, batch=16, heads=16, dk=128, dv=128, steps=32768, delta=1, decay="scalar",
+    arms=(Arm(8, 32, "dynamic"), Arm(4, 32, "dynamic"), Arm(4, 32, "persistent"),
+          Arm(4, 32, "yoked"), Arm(4, 32, "persistent", "bdr"), Arm(4, 32, "dynamic", "bdr")),
+    seed=5, s0_std=1.0 / np.sqrt(128.0), draw="recall"))
+
+# Index in the order the workloads are listed for this step (the recall
+# measurement above is not one of them).
+
 ORDER: List[str] = ["tiny-gdn", "gdn", "mamba2", "gla", "stack24"]
 
 
@@ -220,3 +238,13 @@ def scaled_down(w: Workload, tiles_per_layer: int, layers: Optional[int] = None,
     seeds = None if w.layer_seeds is None else w.layer_seeds[:L]
     return replace(w, name=w.name + "-small", layers=L, batch=1, heads=tiles_per_layer,
                    layer_seeds=seeds, steps=w.steps if steps is None else steps)
+
+
+def probe(w: Workload, tiles: Optional[np.ndarray] = None):
+    """(k*, v*) of the recall measurement: per tile a unit-norm key and a
+    N(0, 1) value, from default_rng([seed, 3]) (float32 [T][dk], [T][dv])."""
+    rng = np.random.default_rng([w.seed, 3])
+    k = _unit_rows(rng.standard_normal((w.tiles, w.dk)))
+    v = rng.standard_normal((w.tiles, w.dv))
+    f = lambda a: np.ascontiguousarray(a if tiles is None else a[tiles], dtype=np.float32)
+    return f(k), f(v)

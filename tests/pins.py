@@ -328,55 +328,55 @@ def pin_zero_scale_group():
 
 
 def pin_bdr_bruteforce():
-    """BDR against brute force over every code: with sigma = sign(w) sign(k_j),
-    the chosen code is nearest or nearest + sigma; its dequantized value never
-    lies on the far side of the pre-update value S' from the update unless
-    clamped; it equals nearest when sigma = 0 or nearest does not reverse; and
-    otherwise it is the non-reversing code closest to the nearest one."""
+    """BDR against nearest rounding from the same state and inputs, element by
+    element: with sigma = sign(w) sign(k_j) and d = c * s the element as
+    stored before the step, BDR's own move is never against the update and
+    never more than one code step (the chosen code is nearest or
+    nearest + sigma, clamped); it equals nearest when sigma = 0 or when
+    nearest does not move the stored element against sigma; and where
+    nearest does, it is nearest + sigma unless that leaves [-qmax, qmax].
+    With a fixed scale and no decay nearest never moves an element against
+    its update, so BDR leaves every code alone; decay or a scale change are
+    what make reversals (checked both ways below)."""
     rng = _rng(22)
     T, dk, dv = 8, 32, 4
+    moved = 0
     for bits in (4, 8):
         for policy in ("persistent", "dynamic"):
-            qmax = (1 << (bits - 1)) - 1
-            cN = O.OracleConfig(T, dk, dv, bits, 16, 0, "diagonal", policy, "nearest")
-            cB = O.OracleConfig(T, dk, dv, bits, 16, 0, "diagonal", policy, "bdr")
-            S0 = (rng.standard_normal((T, dv, dk)) * 0.5).astype(F32)
-            B = O.init(cB, S0)
-            for _ in range(8):
-                q, k, v, a, b = _inputs(rng, T, dk, dv, "diagonal")
-                k[:, ::5] = 0.0          # some columns with no update
-                v[:, 0] = 0.0            # a row with no update
-                v = (v * 0.05).astype(F32)   # small updates: reversals are common
-                prev = B.copy()
-                # nearest rounding from the same state and inputs
-                Nst = O.State(cN, prev.codes.copy(), prev.scales.copy())
-                O.step(Nst, q, k, v, a, b, want_o=False)
-                O.step(B, q, k, v, a, b, want_o=False)
-                # S' = c * (s * a), the decayed scale first (as the step defines it)
-                sa = (np.repeat(prev.scales, 16, axis=-1) * a[:, None, :]).astype(F32)
-                Sp = (prev.codes.astype(F32) * sa).astype(F32)
-                w = (b[:, None] * v).astype(F32)
-                sigma = np.sign(w)[:, :, None] * np.sign(k)[:, None, :]
-                s_el = np.repeat(B.scales, 16, axis=-1)
-                n_near, n = Nst.codes, B.codes
-                assert np.array_equal(Nst.scales, B.scales)
-                step = n - n_near
-                assert np.all((step == 0) | (step == sigma))
-                dq = (n.astype(F32) * s_el).astype(F32)
-                reverse = ((sigma > 0) & (dq < Sp)) | ((sigma < 0) & (dq > Sp))
-                clamped = np.abs(n) == qmax
-                assert not np.any(reverse & ~clamped)
-                dqn = (n_near.astype(F32) * s_el).astype(F32)
-                near_rev = ((sigma > 0) & (dqn < Sp)) | ((sigma < 0) & (dqn > Sp))
-                assert np.all(n[~near_rev] == n_near[~near_rev])
-                # brute force: the smallest move in the update direction
-                live = near_rev & ~clamped & (s_el > 0)
-                for idx in zip(*np.nonzero(live)):
-                    sg = sigma[idx]
-                    cands = [c for c in range(-qmax, qmax + 1)
-                             if (F32(c) * s_el[idx] - Sp[idx]) * sg >= 0]
-                    best = min(cands, key=lambda c: abs(c - n_near[idx]))
-                    assert n[idx] == best
+            for decay_lo in (0.8, 1.0):
+                qmax = (1 << (bits - 1)) - 1
+                cN = O.OracleConfig(T, dk, dv, bits, 16, 0, "diagonal", policy, "nearest")
+                cB = O.OracleConfig(T, dk, dv, bits, 16, 0, "diagonal", policy, "bdr")
+                S0 = (rng.standard_normal((T, dv, dk)) * 0.5).astype(F32)
+                B = O.init(cB, S0)
+                for _ in range(8):
+                    q, k, v, a, b = _inputs(rng, T, dk, dv, "diagonal")
+                    if decay_lo == 1.0:
+                        a = np.ones_like(a)
+                    k[:, ::5] = 0.0          # some columns with no update
+                    v[:, 0] = 0.0            # a row with no update
+                    v = (v * 0.05).astype(F32)   # small updates: reversals are common
+                    prev = B.copy()
+                    Nst = O.State(cN, prev.codes.copy(), prev.scales.copy())
+                    O.step(Nst, q, k, v, a, b, want_o=False)
+                    O.step(B, q, k, v, a, b, want_o=False)
+                    d = (prev.codes.astype(F32) * np.repeat(prev.scales, 16, axis=-1)).astype(F32)
+                    w = (b[:, None] * v).astype(F32)
+                    sigma = np.sign(w)[:, :, None] * np.sign(k)[:, None, :]
+                    s_el = np.repeat(B.scales, 16, axis=-1)
+                    n_near, n = Nst.codes, B.codes
+                    assert np.array_equal(Nst.scales, B.scales)
+                    step = n - n_near
+                    assert np.all((step == 0) | (step == sigma))
+                    dqn = (n_near.astype(F32) * s_el).astype(F32)
+                    near_rev = (((sigma > 0) & (dqn < d)) | ((sigma < 0) & (dqn > d))) & (s_el > 0)
+                    assert np.all(n[~near_rev] == n_near[~near_rev])
+                    want = np.clip(n_near + sigma.astype(np.int64), -qmax, qmax)
+                    assert np.array_equal(n[near_rev], want[near_rev])
+                    if policy == "persistent" and decay_lo == 1.0:
+                        assert not np.any(near_rev)
+                    moved += int(np.count_nonzero(step))
+    assert moved > 0
 
 
 def pin_yoked_shadow_is_fp32_run():
@@ -545,6 +545,40 @@ def pin_dot_order():
             assert abs(float(O.dot(a, b)) - exact) <= bound
 
 
+def pin_sq_norms():
+    """State norms (the quantity the dynamic-scale norm inflation is measured
+    in): closed forms on constant and one-hot states, sign invariance, and
+    agreement with the squared readouts against the unit vectors e_j (which
+    return the dequantized columns exactly)."""
+    T, dk, dv, G = 3, 64, 16, 32
+    cfg = O.OracleConfig(T, dk, dv, 4, G, 1, "scalar", "persistent")
+    codes = np.full((T, dv, dk), 3, np.int32)
+    scales = np.full((T, dv, dk // G), 0.5, F32)
+    st = O.State(cfg, codes, scales)
+    assert np.array_equal(O.sq_norms(st), np.full(T, dv * dk * 2.25))
+    codes = np.zeros((T, dv, dk), np.int32)
+    codes[1, 5, 40] = -7
+    scales = np.full((T, dv, dk // G), 0.25, F32)
+    assert np.array_equal(O.sq_norms(O.State(cfg, codes, scales)), np.array([0.0, 3.0625, 0.0]))
+    rng = _rng(31)
+    codes = rng.integers(-7, 8, size=(T, dv, dk)).astype(np.int32)
+    scales = rng.uniform(0.01, 2.0, size=(T, dv, dk // G)).astype(F32)
+    st = O.State(cfg, codes, scales)
+    n = O.sq_norms(st)
+    assert np.array_equal(n, O.sq_norms(O.State(cfg, -codes, scales)))
+    cols = np.zeros(T)
+    for j in range(dk):
+        e = np.zeros((T, dk), F32)
+        e[:, j] = 1.0
+        o = O.readout(st, e).astype(np.float64)
+        cols += (o * o).sum(axis=1)
+    assert np.allclose(n, cols, rtol=1e-12, atol=0.0)
+    S = np.ones((T, dv, dk), F32)
+    assert np.array_equal(O.fp32_sq_norms(cfg, S), np.full(T, float(dv * dk)))
+    S = np.where(rng.integers(0, 2, size=(T, dv, dk)) == 1, F32(1.5), F32(-1.5)).astype(F32)
+    assert np.array_equal(O.fp32_sq_norms(cfg, S), np.full(T, dv * dk * 2.25))
+
+
 ALL_PINS = [
     pin_linear_write_sum_of_outer_products,
     pin_decay_closed_form,
@@ -566,4 +600,5 @@ ALL_PINS = [
     pin_worked_steps,
     pin_pack_layout,
     pin_dot_order,
+    pin_sq_norms,
 ]

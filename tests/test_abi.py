@@ -123,6 +123,20 @@ def test_readout_validation():
     assert lib.qstate_readout(ctypes.byref(c), A, 2 * A, 3 * A, A + 16, None) == Q.QS_ERR_INVALID_ARG
 
 
+def test_norms_validation():
+    # null, misaligned and overlapping arguments are rejected before any launch
+    c = _cfg().c()
+    lib = Q.lib()
+    assert lib.qstate_state_sq_norms(ctypes.byref(c), None, 2 * A, 8 * A, None) == Q.QS_ERR_INVALID_ARG
+    assert lib.qstate_state_sq_norms(ctypes.byref(c), A + 16, 2 * A, 8 * A, None) == Q.QS_ERR_INVALID_ARG
+    assert lib.qstate_state_sq_norms(ctypes.byref(c), A, 2 * A, 8 * A + 4, None) == Q.QS_ERR_INVALID_ARG
+    assert lib.qstate_state_sq_norms(ctypes.byref(c), A, 2 * A, A + 64, None) == Q.QS_ERR_INVALID_ARG
+    assert lib.qstate_fp32_sq_norms(ctypes.byref(c), None, 8 * A, None) == Q.QS_ERR_INVALID_ARG
+    assert lib.qstate_fp32_sq_norms(ctypes.byref(c), A + 4, 8 * A, None) == Q.QS_ERR_INVALID_ARG
+    assert lib.qstate_fp32_sq_norms(ctypes.byref(c), A, A + 64, None) == Q.QS_ERR_INVALID_ARG
+    assert lib.qstate_fp32_sq_norms(None, A, 8 * A, None) == Q.QS_ERR_INVALID_ARG
+
+
 def test_binding_raises():
     with pytest.raises(Q.QStateError):
         Q.query_sizes(_cfg(bits=5))

@@ -202,3 +202,28 @@ def test_fp32_state_step_matches_oracle_bit_for_bit(dk, dv, delta, decay, T):
         assert np.array_equal(S_gpu.cpu().numpy(), S_ref), f"state differs at step {t}"
         if t % 2 == 0:
             assert np.array_equal(o.cpu().numpy(), o_ref), f"readout differs at step {t}"
+
+
+@pytest.mark.parametrize("bits,dk,dv,group,T", [(4, 128, 128, 32, 37), (8, 128, 64, 64, 300),
+                                                (4, 64, 48, 64, 9), (8, 64, 16, 32, 5)])
+def test_state_norms(bits, dk, dv, group, T):
+    """qstate_state_sq_norms / qstate_fp32_sq_norms against the oracle's
+    FP64 sums (same terms, summation order differs: relative 1e-12)."""
+    import torch
+    from ssm_decode_step_b200 import qstate as Q
+    rng = np.random.default_rng(bits * 7 + dk + dv + T)
+    cfg = Config(T, dk, dv, bits, group, 1, "scalar", "dynamic")
+    S0 = (rng.standard_normal((T, dv, dk)) * 0.3).astype(np.float32)
+    gpu = P.GpuRun(cfg, S0)
+    ora = O.init(P.oracle_cfg(cfg), S0)
+    for q, k, v, a, b in P.random_steps(rng, T, dk, dv, "scalar", 3):
+        gpu.step(q, k, v, a, b)
+        O.step(ora, q, k, v, a, b)
+    c, s, _ = gpu.state()
+    P.compare_state(cfg, c, s, ora, None, "before norms")
+    out = torch.empty(T, dtype=torch.float64, device="cuda")
+    Q.state_sq_norms(cfg, gpu.st.codes, gpu.st.scales, out)
+    assert np.allclose(out.cpu().numpy(), O.sq_norms(ora), rtol=1e-12, atol=0.0)
+    S = torch.from_numpy(S0).cuda()
+    Q.fp32_sq_norms(cfg, S, out)
+    assert np.allclose(out.cpu().numpy(), O.fp32_sq_norms(P.oracle_cfg(cfg), S0), rtol=1e-12, atol=0.0)
