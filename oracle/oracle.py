@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
             "qo_readout": [C, P, P, P, P],
             "qo_fp32_step": [C, P, P, P, P, P, P, P],
             "qo_sq_norms": [C, P, P, P],
+            "qo_lrb_step": [C, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P],
             "qo_fp32_sq_norms": [C, P, P],
         }.items():
             f = getattr(L, name)
@@ -222,3 +223,41 @@ def fp32_sq_norms(cfg: OracleConfig, S) -> np.ndarray:
     cc = cfg.c()
     _ok(lib().qo_fp32_sq_norms(ctypes.byref(cc), _p(S), _p(out)), "fp32_sq_norms")
     return out
+
+
+class LrbBuffers:
+    """Low-Rank Bypass buffers of the oracle (see qo_lrb_step): accumulated
+    column decay A, decayed keys K and write coefficients U of the current
+    period, with the slot (position in the period) of the next step."""
+
+    def __init__(self, cfg: OracleConfig, rank: int):
+        self.rank = rank
+        self.slot = 0
+        self.A = np.ones((cfg.tiles, cfg.dk), np.float32)
+        self.K = np.zeros((cfg.tiles, rank, cfg.dk), np.float32)
+        self.U = np.zeros((cfg.tiles, rank, cfg.dv), np.float32)
+
+
+def lrb_step(st: State, buf: LrbBuffers, q, k, v, alpha, beta, want_o=True, want_pre=False):
+    """One Low-Rank Bypass step in place on (st, buf); returns o (and, if
+    asked, the exact pre-rounding values at a merge step, else None)."""
+    cfg = st.cfg
+    q, k, v, alpha, beta = map(_f32, (q, k, v, alpha, beta))
+    o = np.empty((cfg.tiles, cfg.dv), dtype=np.float32) if want_o else None
+    merge = buf.slot == buf.rank - 1
+    pre = np.full((cfg.tiles, cfg.dv, cfg.dk), np.nan) if (want_pre and merge) else None
+    A_out = None if merge else np.empty_like(buf.A)
+    K_out = None if merge else np.empty_like(buf.K)
+    cc = cfg.c()
+    _ok(lib().qo_lrb_step(ctypes.byref(cc), buf.rank, buf.slot, _p(st.codes), _p(st.scales),
+                          _p(st.shadow), _p(buf.A), _p(A_out), _p(buf.K), _p(K_out), _p(buf.U),
+                          _p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(o), _p(pre)), "lrb_step")
+    if merge:
+        buf.slot = 0
+        buf.A[:] = 1.0
+        buf.K[:] = 0.0
+        buf.U[:] = 0.0
+    else:
+        buf.A, buf.K = A_out, K_out
+        buf.slot += 1
+    return (o, pre) if want_pre else o

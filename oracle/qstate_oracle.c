@@ -24,9 +24,10 @@
  *                             else inv = 1/s', n = nearest integer to the exact
  *                             product x_j * inv (ties to even), clamped to
  *                             [-qmax, qmax]
- *   8. BDR (if selected)      sigma = sign(w) sign(k_j); if sigma > 0 and
- *                             n*s' < S'_j then n += 1; if sigma < 0 and
- *                             n*s' > S'_j then n -= 1; clamp again
+ *   8. BDR (if selected)      sigma = sign(w) sign(k_j), d_j = c_ij * s_ig
+ *                             (the element as stored before the step); if
+ *                             sigma > 0 and n*s' < d_j then n += 1; if
+ *                             sigma < 0 and n*s' > d_j then n -= 1; clamp
  *   9. store                  codes, and s' for dynamic / yoked
  * Dot products "." use qo_dot's fixed order (even / odd chains per 32
  * entries, pairwise tree over the chunks).
@@ -41,6 +42,7 @@
 #endif
 
 #define QO_MAX_DK 1024
+#define QO_MAX_RANK 32
 
 static int g_fault = QO_FAULT_NONE;
 
@@ -148,9 +150,8 @@ static int32_t clamp_code(int32_t n, int qmax) {
  * decayed row before the write (used only by the planted BDR_REFERENCE
  * mistake); R: updated shadow row or NULL. */
 static void requantize_row(const qo_cfg* c, const float* x, const float* Sp,
-                           const float* d, const float* R, float w,
-                           const float* k, int32_t* crow, float* srow,
-                           double* pre) {
+                           const float* d, const float* R, const float* sigma,
+                           int32_t* crow, float* srow, double* pre) {
   const int G = c->group, ng = c->dk / c->group, qmax = c->qmax;
   for (int g = 0; g < ng; ++g) {
     float s_new;
@@ -177,12 +178,11 @@ static void requantize_row(const qo_cfg* c, const float* x, const float* Sp,
       for (int j = g * G; j < (g + 1) * G; ++j) {
         int32_t n = nearest_code(x[j], inv, qmax, pre ? &pre[j] : NULL);
         if (c->rounding == QO_ROUND_BDR) {
-          float sigma = sign_of(w) * sign_of(k[j]);
           float ref = (g_fault == QO_FAULT_BDR_REFERENCE) ? Sp[j] : d[j];
           float dq = (float)n * s_new;
-          if (sigma > 0.0f && dq < ref)
+          if (sigma[j] > 0.0f && dq < ref)
             n += 1;
-          else if (sigma < 0.0f && dq > ref)
+          else if (sigma[j] < 0.0f && dq > ref)
             n -= 1;
           n = clamp_code(n, qmax);
         }
@@ -234,6 +234,7 @@ int qo_step(const qo_cfg* c, int32_t* codes, float* scales, float* shadow,
 #pragma omp parallel for schedule(static)
   for (int t = 0; t < c->tiles; ++t) {
     float d[QO_MAX_DK], Sp[QO_MAX_DK], x[QO_MAX_DK], Rp[QO_MAX_DK], Rn[QO_MAX_DK];
+    float sg[QO_MAX_DK];
     const float* kt = k + (size_t)t * dk;
     const float* qt = q ? q + (size_t)t * dk : NULL;
     for (int i = 0; i < dv; ++i) {
@@ -261,8 +262,106 @@ int qo_step(const qo_cfg* c, int32_t* codes, float* scales, float* shadow,
         R = Rn;
       }
       /* 6-9. scale, round, store */
-      requantize_row(c, x, Sp, d, R, w, kt, crow, srow,
-                     prequant ? prequant + row * dk : NULL);
+      for (int j = 0; j < dk; ++j) sg[j] = sign_of(w) * sign_of(kt[j]);
+      requantize_row(c, x, Sp, d, R, sg, crow, srow, prequant ? prequant + row * dk : NULL);
+    }
+  }
+  return 0;
+}
+
+int qo_lrb_step(const qo_cfg* c, int rank, int slot, int32_t* codes, float* scales,
+                float* shadow, const float* A_in, float* A_out, const float* K_in,
+                float* K_out, float* U, const float* q, const float* k, const float* v,
+                const float* alpha, const float* beta, float* o, double* prequant) {
+  if (qo_check(c) || rank < 1 || rank > QO_MAX_RANK || slot < 0 || slot >= rank) return -1;
+  if (!codes || !scales || !k || !v || !alpha || !beta || !U) return -1;
+  if (o && !q) return -1;
+  if (c->policy == QO_SCALE_YOKED && !shadow) return -1;
+  const int merge = slot == rank - 1;
+  if (slot > 0 && (!A_in || !K_in)) return -1;
+  if (!merge && (!A_out || !K_out)) return -1;
+  const int dk = c->dk, dv = c->dv, G = c->group, ng = dk / G;
+#pragma omp parallel for schedule(static)
+  for (int t = 0; t < c->tiles; ++t) {
+    float A[QO_MAX_DK], Kd[QO_MAX_RANK][QO_MAX_DK], kk[QO_MAX_RANK], kq[QO_MAX_RANK];
+    float d[QO_MAX_DK], Sp[QO_MAX_DK], x[QO_MAX_DK], M[QO_MAX_DK], Rp[QO_MAX_DK], Rn[QO_MAX_DK];
+    float sg[QO_MAX_DK];
+    const float* kt = k + (size_t)t * dk;
+    const float* qt = q ? q + (size_t)t * dk : NULL;
+    float* Ut = U + (size_t)t * rank * dv;
+    /* a. decay of the accumulated column factors and of the buffered keys */
+    for (int j = 0; j < dk; ++j) {
+      float a = decay_at(c, alpha, t, 0, j);
+      A[j] = (slot == 0 ? 1.0f : A_in[(size_t)t * dk + j]) * a;
+      for (int r = 0; r < slot; ++r) Kd[r][j] = K_in[((size_t)t * rank + r) * dk + j] * a;
+    }
+    /* b. the buffered keys against k and q */
+    for (int r = 0; r < slot; ++r) {
+      kk[r] = qo_dot(Kd[r], kt, dk);
+      kq[r] = qt ? qo_dot(Kd[r], qt, dk) : 0.0f;
+    }
+    const float kqn = qt ? qo_dot(kt, qt, dk) : 0.0f;
+    for (int i = 0; i < dv; ++i) {
+      size_t row = (size_t)t * dv + i;
+      int32_t* crow = codes + row * dk;
+      float* srow = scales + row * ng;
+      /* c. dequantize with the accumulated decay: S'_j = c * (s * A_j) */
+      for (int j = 0; j < dk; ++j) {
+        int g = j / G;
+        if (g_fault == QO_FAULT_GROUP_INDEX) g = (g + 1) % ng;
+        d[j] = (float)crow[j] * srow[g];
+        Sp[j] = (float)crow[j] * (srow[g] * A[j]);
+      }
+      /* d. write coefficient against the effective state S' + sum_r U_r K_r^T */
+      float w;
+      const float vi = v[row];
+      if (c->delta && g_fault != QO_FAULT_DROP_DELTA) {
+        float u = qo_dot(Sp, kt, dk);
+        for (int r = 0; r < slot; ++r) u = fmaf(Ut[(size_t)r * dv + i], kk[r], u);
+        w = (g_fault == QO_FAULT_BETA_ON_V_ONLY) ? beta[t] * vi - u : beta[t] * (vi - u);
+      } else {
+        w = beta[t] * vi;
+      }
+      if (g_fault == QO_FAULT_WRITE_SIGN) w = -w;
+      /* yoked shadow: the FP32 reference advances every step */
+      const float* R = NULL;
+      if (c->policy == QO_SCALE_YOKED) {
+        float* Rrow = shadow + row * dk;
+        for (int j = 0; j < dk; ++j) Rp[j] = Rrow[j] * decay_at(c, alpha, t, i, j);
+        row_write(c, Rp, kt, vi, beta[t], Rn);
+        memcpy(Rrow, Rn, sizeof(float) * dk);
+        R = Rn;
+      }
+      if (!merge) {
+        /* e. bypass: the write joins the buffer; the stored state is untouched */
+        if (o) {
+          float oi = qo_dot(Sp, g_fault == QO_FAULT_READ_K_FOR_Q ? kt : qt, dk);
+          for (int r = 0; r < slot; ++r) oi = fmaf(Ut[(size_t)r * dv + i], kq[r], oi);
+          o[row] = fmaf(w, kqn, oi);
+        }
+        Ut[(size_t)slot * dv + i] = w;
+      } else {
+        /* f. merge: x = S' + sum_r U_r K_r^T + w k^T, then requantize once */
+        for (int j = 0; j < dk; ++j) {
+          float xj = Sp[j], mj = 0.0f;
+          for (int r = 0; r < slot; ++r) {
+            const float ur = Ut[(size_t)r * dv + i];
+            xj = fmaf(ur, Kd[r][j], xj);
+            mj = fmaf(ur, Kd[r][j], mj);
+          }
+          x[j] = fmaf(w, kt[j], xj);
+          M[j] = fmaf(w, kt[j], mj);
+          sg[j] = sign_of(M[j]);
+        }
+        if (o) o[row] = qo_dot(x, g_fault == QO_FAULT_READ_K_FOR_Q ? kt : qt, dk);
+        requantize_row(c, x, Sp, d, R, sg, crow, srow, prequant ? prequant + row * dk : NULL);
+      }
+    }
+    if (!merge) {
+      memcpy(A_out + (size_t)t * dk, A, sizeof(float) * dk);
+      for (int r = 0; r < slot; ++r)
+        memcpy(K_out + ((size_t)t * rank + r) * dk, Kd[r], sizeof(float) * dk);
+      memcpy(K_out + ((size_t)t * rank + slot) * dk, kt, sizeof(float) * dk);
     }
   }
   return 0;

@@ -85,6 +85,35 @@ int qo_step(const qo_cfg* c, int32_t* codes, float* scales, float* shadow,
             const float* alpha, const float* beta, float* o,
             double* prequant);
 
+/* Low-Rank Bypass ("Preserving Updates in Low-Bit Recurrent State
+ * Quantization", abstract: small updates accumulate in a compact low-rank
+ * buffer that is periodically merged into the state).  Reading taken here:
+ * the buffer holds the last writes of the current period as rank-1 terms
+ * w k^T in FP32 (U [tiles][rank][dv], keys K [tiles][rank][dk] decayed in
+ * place), and the stored codes are not touched between merges; their decay
+ * accumulates per column in A [tiles][dk].  The period is `rank` steps; slot
+ * = position of this step in it (0 .. rank-1).  Per tile:
+ *   a. A_j = (slot ? A_in_j : 1) * a_j;  K'_r = K_in_r * a (r < slot)
+ *   b. kk_r = K'_r . k, kq_r = K'_r . q, kqn = k . q
+ *   c. S'_ij = c_ij * (s_ig * A_j)
+ *   d. u_i = S'_i . k, then u_i = fused(U_ri * kk_r + u_i) for r < slot;
+ *      w_i = beta (v_i - u_i) (delta 1) or beta v_i
+ *   e. slot < rank-1 (bypass): o_i = S'_i . q, then fused(U_ri kq_r + o_i)
+ *      for r < slot, then fused(w_i kqn + o_i); U_slot,i = w_i; A_out = A,
+ *      K_out_r = K'_r (r < slot), K_out_slot = k; codes and scales kept
+ *   f. slot = rank-1 (merge): x_ij = S'_ij, then fused(U_ri K'_rj + x_ij)
+ *      for r < slot, then fused(w_i k_j + x_ij); o_i = x_i . q; requantize x
+ *      as qo_step does, with BDR's sigma_ij = sign(M_ij), M_ij the same
+ *      chain from +0 (the accumulated update), and its reference the stored
+ *      element c_ij * s_ig.
+ * The yoked shadow advances by qo_step's rule at every step.  With rank 1
+ * every step is a merge and the step is qo_step's.  A_out, K_out may be NULL
+ * at a merge; A_in, K_in may be NULL at slot 0. */
+int qo_lrb_step(const qo_cfg* c, int rank, int slot, int32_t* codes, float* scales,
+                float* shadow, const float* A_in, float* A_out, const float* K_in,
+                float* K_out, float* U, const float* q, const float* k, const float* v,
+                const float* alpha, const float* beta, float* o, double* prequant);
+
 /* o = dequant(S) q with the state unchanged. */
 int qo_readout(const qo_cfg* c, const int32_t* codes, const float* scales,
                const float* q, float* o);

@@ -579,6 +579,121 @@ def pin_sq_norms():
     assert np.array_equal(O.fp32_sq_norms(cfg, S), np.full(T, dv * dk * 2.25))
 
 
+def pin_lrb_rank1_is_step():
+    """Low-Rank Bypass with a period of one step merges at every step, so it
+    must be the plain decode step bit for bit (codes, scales, shadow, o)."""
+    rng = _rng(41)
+    T, dk, dv = 4, 64, 16
+    for policy in ("dynamic", "persistent", "yoked"):
+        for rounding in ("nearest", "bdr"):
+            for decay, delta in (("scalar", 1), ("diagonal", 0)):
+                cfg = O.OracleConfig(T, dk, dv, 4, 32, delta, decay, policy, rounding)
+                S0 = (rng.standard_normal((T, dv, dk)) * 0.4).astype(F32)
+                a = O.init(cfg, S0)
+                b = a.copy()
+                buf = O.LrbBuffers(cfg, 1)
+                for _ in range(4):
+                    q, k, v, al, be = _inputs(rng, T, dk, dv, decay)
+                    v = (v * 0.2).astype(F32)
+                    oa = O.step(a, q, k, v, al, be)
+                    ob = O.lrb_step(b, buf, q, k, v, al, be)
+                    assert np.array_equal(oa, ob)
+                    assert np.array_equal(a.codes, b.codes) and np.array_equal(a.scales, b.scales)
+                    if a.shadow is not None:
+                        assert np.array_equal(a.shadow, b.shadow)
+
+
+def _lrb_effective(st, buf):
+    """S' + sum_r U_r K_r^T of the LRB state, in float64 (stored codes times
+    the accumulated decay, plus the buffered writes of the period)."""
+    cfg = st.cfg
+    d = st.codes.astype(np.float64) * np.repeat(st.scales.astype(np.float64), cfg.group, axis=-1)
+    S = d * buf.A.astype(np.float64)[:, None, :]
+    for r in range(buf.slot):
+        S += np.einsum("ti,tj->tij", buf.U[:, r].astype(np.float64), buf.K[:, r].astype(np.float64))
+    return S
+
+
+def pin_lrb_bypass_tracks_fp32():
+    """Between merges LRB quantizes nothing: the stored codes and scales stay
+    fixed and the effective state (stored state with its accumulated decay
+    plus the buffered rank-1 writes) follows the unquantized recurrence of
+    LinQuant eq. (1) from the dequantized state, readouts included."""
+    rng = _rng(42)
+    T, dk, dv, R = 3, 64, 16, 6
+    for decay, delta in (("scalar", 1), ("diagonal", 0), ("diagonal", 1)):
+        cfg = O.OracleConfig(T, dk, dv, 8, 32, delta, decay, "dynamic", "nearest")
+        st = O.init(cfg, (rng.standard_normal((T, dv, dk)) * 0.4).astype(F32))
+        codes0, scales0 = st.codes.copy(), st.scales.copy()
+        buf = O.LrbBuffers(cfg, R)
+        ref = (st.codes.astype(np.float64) *
+               np.repeat(st.scales.astype(np.float64), cfg.group, axis=-1))
+        for _ in range(R - 1):
+            q, k, v, al, be = _inputs(rng, T, dk, dv, decay)
+            o = O.lrb_step(st, buf, q, k, v, al, be)
+            a = _decay64(al, decay, dk)
+            ref = ref * a[:, None, :]
+            k64 = k.astype(np.float64)
+            u = np.einsum("tij,tj->ti", ref, k64) if delta else 0.0
+            w = be.astype(np.float64)[:, None] * (v.astype(np.float64) - u)
+            ref = ref + np.einsum("ti,tj->tij", w, k64)
+            o_ref = np.einsum("tij,tj->ti", ref, q.astype(np.float64))
+            assert np.array_equal(st.codes, codes0) and np.array_equal(st.scales, scales0)
+            eff = _lrb_effective(st, buf)
+            scale = np.abs(ref).max()
+            assert np.abs(eff - ref).max() <= 2e-6 * scale * (1 + buf.slot)
+            assert np.abs(o - o_ref).max() <= 2e-5 * np.abs(o_ref).max() * (1 + buf.slot)
+
+
+def pin_lrb_merge_closed_form():
+    """With no decay, a linear write and a persistent scale, the merge at the
+    end of a period requantizes the stored state plus the sum of the
+    period's writes: codes = nearest(clamped) of (d + sum_t beta_t v_t k_t^T)/s,
+    up to ties within FP32 rounding of a half step."""
+    rng = _rng(43)
+    T, dk, dv, R = 4, 64, 16, 5
+    cfg = O.OracleConfig(T, dk, dv, 4, 32, 0, "scalar", "persistent", "nearest")
+    st = O.init(cfg, (rng.standard_normal((T, dv, dk)) * 0.5).astype(F32))
+    s_el = np.repeat(st.scales.astype(np.float64), 32, axis=-1)
+    x = st.codes.astype(np.float64) * s_el
+    buf = O.LrbBuffers(cfg, R)
+    for _ in range(R):
+        q, k, v, al, be = _inputs(rng, T, dk, dv, "scalar", alpha=1.0)
+        v = (v * 0.1).astype(F32)
+        O.lrb_step(st, buf, q, k, v, al, be)
+        x += np.einsum("ti,tj->tij", be.astype(np.float64)[:, None] * v.astype(np.float64),
+                       k.astype(np.float64))
+    assert buf.slot == 0
+    p = x / s_el
+    want = np.clip(np.rint(p), -7, 7)
+    near_tie = np.abs(np.abs(p - np.floor(p)) - 0.5) < 1e-4
+    assert np.all((st.codes == want) | near_tie)
+    assert np.count_nonzero(st.codes != want) <= np.count_nonzero(near_tie)
+
+
+def pin_lrb_preserves_small_writes():
+    """The point of the bypass: a write of 0.3 code steps per step is rounded
+    away by every per-step requantization (persistent scale, no decay), but
+    survives when four of them accumulate in the buffer before one merge."""
+    T, dk, dv, R = 2, 32, 4, 4
+    cfg = O.OracleConfig(T, dk, dv, 8, 32, 0, "scalar", "persistent", "nearest")
+    S0 = np.zeros((T, dv, dk), F32)
+    S0[:, :, 0] = 127.0 / 64.0                      # scale 1/64 for every row
+    plain = O.init(cfg, S0)
+    lrb = plain.copy()
+    buf = O.LrbBuffers(cfg, R)
+    q = np.zeros((T, dk), F32)
+    k = np.zeros((T, dk), F32)
+    k[:, 5] = 1.0
+    v = np.full((T, dv), 0.3 / 64.0, F32)           # 0.3 steps of the 1/64 grid
+    one = np.ones(T, F32)
+    for _ in range(R):
+        O.step(plain, q, k, v, one, one, want_o=False)
+        O.lrb_step(lrb, buf, q, k, v, one, one, want_o=False)
+    assert np.all(plain.codes[:, :, 5] == 0)         # lost in rounding, every step
+    assert np.all(lrb.codes[:, :, 5] == 1)           # 4 x 0.3 = 1.2 steps -> 1
+
+
 ALL_PINS = [
     pin_linear_write_sum_of_outer_products,
     pin_decay_closed_form,
@@ -601,4 +716,8 @@ ALL_PINS = [
     pin_pack_layout,
     pin_dot_order,
     pin_sq_norms,
+    pin_lrb_rank1_is_step,
+    pin_lrb_bypass_tracks_fp32,
+    pin_lrb_merge_closed_form,
+    pin_lrb_preserves_small_writes,
 ]
