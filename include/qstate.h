@@ -168,6 +168,51 @@ QS_API qs_status qstate_fp32_decode_step(const qs_config* cfg, float* S, const f
                                          const float* k, const float* v, const float* alpha,
                                          const float* beta, float* o, cudaStream_t stream);
 
+/* Low-Rank Bypass ("Preserving Updates in Low-Bit Recurrent State
+ * Quantization", abstract: small updates are accumulated in a compact
+ * low-rank buffer whose elements are periodically merged into the state).
+ * Reading implemented here: over a period of `rank` steps the writes w k^T
+ * bypass the quantized state and are held in FP32 as rank-1 terms; the
+ * stored codes and scales are not touched between merges and their decay
+ * accumulates per column; the last step of the period merges the buffer
+ * into the state and requantizes it once with the configured scale policy
+ * and rounding.  Per tile, for the step at position `slot` of the period:
+ *   A_j    = (slot ? A_in_j : 1) * a_j;   K'_r = K_in_r * a   (r < slot)
+ *   kk_r   = K'_r . k,  kq_r = K'_r . q,  kqn = k . q
+ *   S'_ij  = c_ij * (s_ig * A_j)
+ *   u_i    = S'_i . k, then fused(U_ir * kk_r + u_i) for r < slot (delta 1)
+ *   w_i    = beta (v_i - u_i)  or  beta v_i
+ *   bypass (slot < rank-1): o_i = S'_i . q, fused(U_ir kq_r + o_i) for
+ *          r < slot, fused(w_i kqn + o_i); U_i,slot = w_i; A_out = A;
+ *          K_out_r = K'_r (r < slot), K_out_slot = k; codes, scales kept
+ *   merge  (slot = rank-1): x_ij = S'_ij, fused(U_ir K'_rj + x_ij) for
+ *          r < slot, fused(w_i k_j + x_ij); o_i = x_i . q; x is requantized
+ *          as by qstate_decode_step, with BDR's sigma_ij = sign(M_ij), M_ij
+ *          the same chain started from +0 (the update accumulated over the
+ *          period), and its reference the stored element c_ij * s_ig
+ * The yoked shadow advances by qstate_decode_step's rule at every step.
+ * rank 1 makes every step a merge: the step is then qstate_decode_step's
+ * (and is dispatched to it; no buffer is used).
+ * Buffers (the caller's, 16-byte aligned; sizes from qstate_lrb_query_sizes):
+ *   A_in, A_out [T][Dk] float   accumulated column decay (two copies: read
+ *                               one, write the other; A_in unused at slot 0,
+ *                               A_out unused at the merge)
+ *   K_in, K_out [T][rank][Dk]   buffered keys, decayed (same two copies)
+ *   U           [T][Dv][rpad]   buffered write coefficients, rpad = rank
+ *                               rounded up to a multiple of 4; column slot is
+ *                               written at bypass steps, columns < slot read
+ * Supported: 1 <= rank <= 16, 0 <= slot < rank; other fields as for
+ * qstate_decode_step.  The caller advances slot (0, 1, ..., rank-1, 0, ...)
+ * and swaps the A and K copies after every bypass step. */
+QS_API qs_status qstate_lrb_query_sizes(const qs_config* cfg, int rank, size_t* decay_bytes,
+                                        size_t* keys_bytes, size_t* coef_bytes);
+QS_API qs_status qstate_lrb_decode_step(const qs_config* cfg, int rank, int slot, void* codes,
+                                        float* scales, float* shadow, const float* A_in,
+                                        float* A_out, const float* K_in, float* K_out, float* U,
+                                        const float* q, const float* k, const float* v,
+                                        const float* alpha, const float* beta, float* o,
+                                        cudaStream_t stream);
+
 /* Squared Frobenius norm of every tile of the stored state, for tracking
  * the state norm over a decode horizon (the norm inflation of per-token
  * dynamic scaling: "When Dynamic Scaling Fails", abstract and project page,

@@ -235,7 +235,7 @@ class LrbBuffers:
         self.slot = 0
         self.A = np.ones((cfg.tiles, cfg.dk), np.float32)
         self.K = np.zeros((cfg.tiles, rank, cfg.dk), np.float32)
-        self.U = np.zeros((cfg.tiles, rank, cfg.dv), np.float32)
+        self.U = np.zeros((cfg.tiles, cfg.dv, rank), np.float32)
 
 
 def lrb_step(st: State, buf: LrbBuffers, q, k, v, alpha, beta, want_o=True, want_pre=False):

@@ -288,7 +288,7 @@ int qo_lrb_step(const qo_cfg* c, int rank, int slot, int32_t* codes, float* scal
     float sg[QO_MAX_DK];
     const float* kt = k + (size_t)t * dk;
     const float* qt = q ? q + (size_t)t * dk : NULL;
-    float* Ut = U + (size_t)t * rank * dv;
+    float* Ut = U + (size_t)t * dv * rank;
     /* a. decay of the accumulated column factors and of the buffered keys */
     for (int j = 0; j < dk; ++j) {
       float a = decay_at(c, alpha, t, 0, j);
@@ -317,7 +317,7 @@ int qo_lrb_step(const qo_cfg* c, int rank, int slot, int32_t* codes, float* scal
       const float vi = v[row];
       if (c->delta && g_fault != QO_FAULT_DROP_DELTA) {
         float u = qo_dot(Sp, kt, dk);
-        for (int r = 0; r < slot; ++r) u = fmaf(Ut[(size_t)r * dv + i], kk[r], u);
+        for (int r = 0; r < slot; ++r) u = fmaf(Ut[(size_t)i * rank + r], kk[r], u);
         w = (g_fault == QO_FAULT_BETA_ON_V_ONLY) ? beta[t] * vi - u : beta[t] * (vi - u);
       } else {
         w = beta[t] * vi;
@@ -336,16 +336,16 @@ int qo_lrb_step(const qo_cfg* c, int rank, int slot, int32_t* codes, float* scal
         /* e. bypass: the write joins the buffer; the stored state is untouched */
         if (o) {
           float oi = qo_dot(Sp, g_fault == QO_FAULT_READ_K_FOR_Q ? kt : qt, dk);
-          for (int r = 0; r < slot; ++r) oi = fmaf(Ut[(size_t)r * dv + i], kq[r], oi);
+          for (int r = 0; r < slot; ++r) oi = fmaf(Ut[(size_t)i * rank + r], kq[r], oi);
           o[row] = fmaf(w, kqn, oi);
         }
-        Ut[(size_t)slot * dv + i] = w;
+        Ut[(size_t)i * rank + slot] = w;
       } else {
         /* f. merge: x = S' + sum_r U_r K_r^T + w k^T, then requantize once */
         for (int j = 0; j < dk; ++j) {
           float xj = Sp[j], mj = 0.0f;
           for (int r = 0; r < slot; ++r) {
-            const float ur = Ut[(size_t)r * dv + i];
+            const float ur = Ut[(size_t)i * rank + r];
             xj = fmaf(ur, Kd[r][j], xj);
             mj = fmaf(ur, Kd[r][j], mj);
           }

@@ -89,7 +89,7 @@ int qo_step(const qo_cfg* c, int32_t* codes, float* scales, float* shadow,
  * Quantization", abstract: small updates accumulate in a compact low-rank
  * buffer that is periodically merged into the state).  Reading taken here:
  * the buffer holds the last writes of the current period as rank-1 terms
- * w k^T in FP32 (U [tiles][rank][dv], keys K [tiles][rank][dk] decayed in
+ * w k^T in FP32 (U [tiles][dv][rank], keys K [tiles][rank][dk] decayed in
  * place), and the stored codes are not touched between merges; their decay
  * accumulates per column in A [tiles][dk].  The period is `rank` steps; slot
  * = position of this step in it (0 .. rank-1).  Per tile:
@@ -98,8 +98,8 @@ int qo_step(const qo_cfg* c, int32_t* codes, float* scales, float* shadow,
  *   c. S'_ij = c_ij * (s_ig * A_j)
  *   d. u_i = S'_i . k, then u_i = fused(U_ri * kk_r + u_i) for r < slot;
  *      w_i = beta (v_i - u_i) (delta 1) or beta v_i
- *   e. slot < rank-1 (bypass): o_i = S'_i . q, then fused(U_ri kq_r + o_i)
- *      for r < slot, then fused(w_i kqn + o_i); U_slot,i = w_i; A_out = A,
+ *   e. slot < rank-1 (bypass): o_i = S'_i . q, then fused(U_ir kq_r + o_i)
+ *      for r < slot, then fused(w_i kqn + o_i); U_i,slot = w_i; A_out = A,
  *      K_out_r = K'_r (r < slot), K_out_slot = k; codes and scales kept
  *   f. slot = rank-1 (merge): x_ij = S'_ij, then fused(U_ri K'_rj + x_ij)
  *      for r < slot, then fused(w_i k_j + x_ij); o_i = x_i . q; requantize x

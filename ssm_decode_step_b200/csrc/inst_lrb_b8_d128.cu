@@ -1,0 +1,6 @@
+// Low-Rank Bypass kernel instances for 8-bit codes and Dk = 128.
+#include "qstate_launch_impl.cuh"
+
+namespace qs {
+QS_INSTANTIATE_LRB(8, 128)
+}  // namespace qs

@@ -134,6 +134,41 @@ cudaError_t dispatch_step(const qs_config* c, const qs::StepParams& p, cudaStrea
   }
 }
 
+template <int BITS, int DK>
+cudaError_t dispatch_lrb(const qs_config* c, const qs::LrbParams& p, bool merge, cudaStream_t s) {
+  using namespace qs;
+  const bool bdr = c->rounding == QS_ROUND_BDR, delta = c->delta == 1, diag = c->decay == QS_DECAY_DIAGONAL;
+  const int T = c->num_tiles, dv = c->dv;
+  if (!merge) {
+    const int sel = (c->policy == QS_SCALE_YOKED ? 4 : 0) + (delta ? 2 : 0) + (diag ? 1 : 0);
+    switch (sel) {
+      case 0: return launch_lrb<BITS, DK, 0, false, false, false, false>(p, T, dv, s);
+      case 1: return launch_lrb<BITS, DK, 0, false, false, true, false>(p, T, dv, s);
+      case 2: return launch_lrb<BITS, DK, 0, false, true, false, false>(p, T, dv, s);
+      case 3: return launch_lrb<BITS, DK, 0, false, true, true, false>(p, T, dv, s);
+      case 4: return launch_lrb<BITS, DK, 2, false, false, false, false>(p, T, dv, s);
+      case 5: return launch_lrb<BITS, DK, 2, false, false, true, false>(p, T, dv, s);
+      case 6: return launch_lrb<BITS, DK, 2, false, true, false, false>(p, T, dv, s);
+      default: return launch_lrb<BITS, DK, 2, false, true, true, false>(p, T, dv, s);
+    }
+  }
+  const int sel = (c->policy * 8) + (bdr ? 4 : 0) + (delta ? 2 : 0) + (diag ? 1 : 0);
+  switch (sel) {
+#define QS_CASE(P, R, DE, DI) \
+  case (P * 8 + R * 4 + DE * 2 + DI): return launch_lrb<BITS, DK, P, R, DE, DI, true>(p, T, dv, s);
+    QS_CASE(0, 0, 0, 0) QS_CASE(0, 0, 0, 1) QS_CASE(0, 0, 1, 0) QS_CASE(0, 0, 1, 1)
+    QS_CASE(0, 1, 0, 0) QS_CASE(0, 1, 0, 1) QS_CASE(0, 1, 1, 0) QS_CASE(0, 1, 1, 1)
+    QS_CASE(1, 0, 0, 0) QS_CASE(1, 0, 0, 1) QS_CASE(1, 0, 1, 0) QS_CASE(1, 0, 1, 1)
+    QS_CASE(1, 1, 0, 0) QS_CASE(1, 1, 0, 1) QS_CASE(1, 1, 1, 0) QS_CASE(1, 1, 1, 1)
+    QS_CASE(2, 0, 0, 0) QS_CASE(2, 0, 0, 1) QS_CASE(2, 0, 1, 0) QS_CASE(2, 0, 1, 1)
+    QS_CASE(2, 1, 0, 0) QS_CASE(2, 1, 0, 1) QS_CASE(2, 1, 1, 0) QS_CASE(2, 1, 1, 1)
+#undef QS_CASE
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+int lrb_rpad(int rank) { return (rank + 3) / 4 * 4; }
+
 }  // namespace
 
 extern "C" {
@@ -317,6 +352,89 @@ qs_status qstate_readout(const qs_config* cfg, const void* codes, const float* s
     e = cfg->dk == 64 ? qs::launch_readout<4, 64>(p, stream) : qs::launch_readout<4, 128>(p, stream);
   else
     e = cfg->dk == 64 ? qs::launch_readout<8, 64>(p, stream) : qs::launch_readout<8, 128>(p, stream);
+  return from_cuda(e);
+}
+
+qs_status qstate_lrb_query_sizes(const qs_config* cfg, int rank, size_t* decay_bytes,
+                                 size_t* keys_bytes, size_t* coef_bytes) {
+  qs_status st = check_config(cfg);
+  if (st != QS_OK) return st;
+  if (rank < 1 || rank > qs::kLrbMaxRank) return QS_ERR_UNSUPPORTED;
+  const size_t T = static_cast<size_t>(cfg->num_tiles);
+  if (decay_bytes) *decay_bytes = T * cfg->dk * sizeof(float);
+  if (keys_bytes) *keys_bytes = T * rank * cfg->dk * sizeof(float);
+  if (coef_bytes) *coef_bytes = T * cfg->dv * lrb_rpad(rank) * sizeof(float);
+  return QS_OK;
+}
+
+qs_status qstate_lrb_decode_step(const qs_config* cfg, int rank, int slot, void* codes,
+                                 float* scales, float* shadow, const float* A_in, float* A_out,
+                                 const float* K_in, float* K_out, float* U, const float* q,
+                                 const float* k, const float* v, const float* alpha,
+                                 const float* beta, float* o, cudaStream_t stream) {
+  qs_status st = check_config(cfg);
+  if (st != QS_OK) return st;
+  if (rank < 1 || rank > qs::kLrbMaxRank) return QS_ERR_UNSUPPORTED;
+  if (slot < 0 || slot >= rank) return QS_ERR_INVALID_ARG;
+  if (rank == 1)
+    return qstate_decode_step(cfg, codes, scales, shadow, q, k, v, alpha, beta, o, stream);
+  if (cfg->num_tiles == 0) return QS_OK;
+  const bool merge = slot == rank - 1;
+  const bool yoked = cfg->policy == QS_SCALE_YOKED;
+  const bool diag = cfg->decay == QS_DECAY_DIAGONAL;
+  if (!codes || !scales || !k || !v || !alpha || !beta || !U || (yoked && !shadow) || (o && !q))
+    return QS_ERR_INVALID_ARG;
+  if (slot > 0 && (!A_in || !K_in)) return QS_ERR_INVALID_ARG;
+  if (!merge && (!A_out || !K_out)) return QS_ERR_INVALID_ARG;
+  if (!aligned(codes, 32) || !aligned(scales, 16) || !aligned(k, 16) || !aligned(v, 16) ||
+      (q && !aligned(q, 16)) || (yoked && !aligned(shadow, 32)) || !aligned(alpha, diag ? 16 : 4) ||
+      !aligned(beta, 4) || (o && !aligned(o, 4)) || !aligned(U, 16) ||
+      (A_in && slot > 0 && !aligned(A_in, 16)) || (K_in && slot > 0 && !aligned(K_in, 16)) ||
+      (!merge && (!aligned(A_out, 16) || !aligned(K_out, 16))))
+    return QS_ERR_INVALID_ARG;
+  const Sizes s = sizes_of(cfg);
+  size_t a_b = 0, k_b = 0, u_b = 0;
+  qstate_lrb_query_sizes(cfg, rank, &a_b, &k_b, &u_b);
+  const Range w[6] = {range_of(codes, s.codes), range_of(scales, s.scales),
+                      range_of(yoked ? shadow : nullptr, s.shadow), range_of(o, o ? s.vec_v : 0),
+                      range_of(U, u_b), range_of(merge ? nullptr : A_out, merge ? 0 : a_b)};
+  const Range r[7] = {range_of(q, q ? s.vec_k : 0), range_of(k, s.vec_k), range_of(v, s.vec_v),
+                      range_of(alpha, s.alpha), range_of(beta, s.tile_scalars),
+                      range_of(slot > 0 ? A_in : nullptr, slot > 0 ? a_b : 0),
+                      range_of(slot > 0 ? K_in : nullptr, slot > 0 ? k_b : 0)};
+  if (any_overlap(w, 6, r, 7)) return QS_ERR_INVALID_ARG;
+  if (!merge) {
+    const Range w2[1] = {range_of(K_out, k_b)};
+    const Range r2[2] = {range_of(slot > 0 ? K_in : nullptr, slot > 0 ? k_b : 0), w[0]};
+    if (any_overlap(w2, 1, r2, 2)) return QS_ERR_INVALID_ARG;
+    for (int i = 0; i < 6; ++i)
+      if (overlap(w2[0], w[i])) return QS_ERR_INVALID_ARG;
+  }
+  qs::LrbParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.codes = static_cast<uint8_t*>(codes);
+  p.scales = scales;
+  p.shadow = yoked ? shadow : nullptr;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.alpha = alpha;
+  p.beta = beta;
+  p.o = o;
+  p.A_in = A_in;
+  p.A_out = A_out;
+  p.K_in = K_in;
+  p.K_out = K_out;
+  p.U = U;
+  p.group = cfg->group;
+  p.rank = rank;
+  p.rpad = lrb_rpad(rank);
+  p.slot = slot;
+  cudaError_t e;
+  if (cfg->bits == 4)
+    e = cfg->dk == 64 ? dispatch_lrb<4, 64>(cfg, p, merge, stream) : dispatch_lrb<4, 128>(cfg, p, merge, stream);
+  else
+    e = cfg->dk == 64 ? dispatch_lrb<8, 64>(cfg, p, merge, stream) : dispatch_lrb<8, 128>(cfg, p, merge, stream);
   return from_cuda(e);
 }
 

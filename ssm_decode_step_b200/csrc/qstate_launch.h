@@ -8,6 +8,7 @@
 
 #include "qstate_kernels.cuh"
 #include "qstate_step.cuh"
+#include "qstate_lrb.cuh"
 
 namespace qs {
 
@@ -16,6 +17,10 @@ cudaError_t launch_step(const StepParams& p, cudaStream_t stream);
 
 template <int BITS, int DK>
 cudaError_t launch_readout(const StepParams& p, cudaStream_t stream);
+
+// Low-Rank Bypass step; p carries pointers, group, rank, rpad and slot.
+template <int BITS, int DK, int POLICY, bool BDR, bool DELTA, bool DIAG, bool MERGE>
+cudaError_t launch_lrb(const LrbParams& p, int tiles, int dv, cudaStream_t stream);
 
 template <int BITS, int DK>
 cudaError_t launch_init(const float* S0, uint8_t* codes, float* scales, float* shadow,

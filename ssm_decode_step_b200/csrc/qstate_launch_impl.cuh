@@ -97,6 +97,33 @@ cudaError_t launch_step(const StepParams& p0, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+template <int BITS, int DK, int POLICY, bool BDR, bool DELTA, bool DIAG, bool MERGE>
+cudaError_t launch_lrb(const LrbParams& p0, int tiles, int dv, cudaStream_t stream) {
+  constexpr int D = 2;
+  constexpr int RW = 32 / (DK / 32);
+  constexpr int WARPS = kStepWarps;
+  auto kernel = lrb_step_kernel<BITS, DK, POLICY, BDR, DELTA, DIAG, MERGE, D>;
+  static std::once_flag flag;
+  cudaError_t err = allow_smem(kernel, flag);
+  if (err != cudaSuccess) return err;
+  LrbParams p = p0;
+  p.bpt = dv / RW;
+  p.nblocks = tiles * p.bpt;
+  p.ntv = (D - 1 + p.bpt - 1) / p.bpt + 1;
+  const LrbLayout L(BITS, DK, DIAG, POLICY == 2, MERGE, p.rank, p.rpad);
+  p.warp_bytes = L.bytes(D, p.ntv);
+  const size_t smem = static_cast<size_t>(p.warp_bytes) * WARPS;
+  int per_sm = 0;
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kStepThreads, smem);
+  if (err != cudaSuccess) return err;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  long long grid = static_cast<long long>(per_sm) * device_sm_count();
+  const long long need = (static_cast<long long>(p.nblocks) + WARPS - 1) / WARPS;
+  if (grid > need) grid = need;
+  kernel<<<static_cast<int>(grid), kStepThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
 template <int BITS, int DK>
 cudaError_t launch_readout(const StepParams& p0, cudaStream_t stream) {
   constexpr int S = 4;
@@ -140,5 +167,28 @@ cudaError_t launch_init(const float* S0, uint8_t* codes, float* scales, float* s
   template cudaError_t launch_readout<B, D>(const StepParams&, cudaStream_t);        \
   template cudaError_t launch_init<B, D>(const float*, uint8_t*, float*, float*, long long, int, \
                                          cudaStream_t);
+
+#define QS_INSTANTIATE_LRB1(B, D, P, R, DE, DI, M) \
+  template cudaError_t launch_lrb<B, D, P, R, DE, DI, M>(const LrbParams&, int, int, cudaStream_t);
+
+// bypass steps requantize nothing, so only the yoked shadow distinguishes
+// the policies there (0 stands for dynamic and persistent)
+#define QS_INSTANTIATE_LRB(B, D)                                                                \
+  QS_INSTANTIATE_LRB1(B, D, 0, false, false, false, false) QS_INSTANTIATE_LRB1(B, D, 0, false, false, true, false) \
+  QS_INSTANTIATE_LRB1(B, D, 0, false, true, false, false)  QS_INSTANTIATE_LRB1(B, D, 0, false, true, true, false)  \
+  QS_INSTANTIATE_LRB1(B, D, 2, false, false, false, false) QS_INSTANTIATE_LRB1(B, D, 2, false, false, true, false) \
+  QS_INSTANTIATE_LRB1(B, D, 2, false, true, false, false)  QS_INSTANTIATE_LRB1(B, D, 2, false, true, true, false)  \
+  QS_INSTANTIATE_LRB1(B, D, 0, false, false, false, true) QS_INSTANTIATE_LRB1(B, D, 0, false, false, true, true) \
+  QS_INSTANTIATE_LRB1(B, D, 0, false, true, false, true)  QS_INSTANTIATE_LRB1(B, D, 0, false, true, true, true)  \
+  QS_INSTANTIATE_LRB1(B, D, 0, true, false, false, true)  QS_INSTANTIATE_LRB1(B, D, 0, true, false, true, true)  \
+  QS_INSTANTIATE_LRB1(B, D, 0, true, true, false, true)   QS_INSTANTIATE_LRB1(B, D, 0, true, true, true, true)   \
+  QS_INSTANTIATE_LRB1(B, D, 1, false, false, false, true) QS_INSTANTIATE_LRB1(B, D, 1, false, false, true, true) \
+  QS_INSTANTIATE_LRB1(B, D, 1, false, true, false, true)  QS_INSTANTIATE_LRB1(B, D, 1, false, true, true, true)  \
+  QS_INSTANTIATE_LRB1(B, D, 1, true, false, false, true)  QS_INSTANTIATE_LRB1(B, D, 1, true, false, true, true)  \
+  QS_INSTANTIATE_LRB1(B, D, 1, true, true, false, true)   QS_INSTANTIATE_LRB1(B, D, 1, true, true, true, true)   \
+  QS_INSTANTIATE_LRB1(B, D, 2, false, false, false, true) QS_INSTANTIATE_LRB1(B, D, 2, false, false, true, true) \
+  QS_INSTANTIATE_LRB1(B, D, 2, false, true, false, true)  QS_INSTANTIATE_LRB1(B, D, 2, false, true, true, true)  \
+  QS_INSTANTIATE_LRB1(B, D, 2, true, false, false, true)  QS_INSTANTIATE_LRB1(B, D, 2, true, false, true, true)  \
+  QS_INSTANTIATE_LRB1(B, D, 2, true, true, false, true)   QS_INSTANTIATE_LRB1(B, D, 2, true, true, true, true)
 
 }  // namespace qs

@@ -24,7 +24,8 @@ QS_OK, QS_ERR_INVALID_ARG, QS_ERR_UNSUPPORTED, QS_ERR_CUDA = 0, 1, 2, 3
 
 # Every entry point that include/qstate.h declares.
 EXPORTS = ("qstate_query_sizes", "qstate_init", "qstate_decode_step", "qstate_readout",
-           "qstate_fp32_decode_step", "qstate_state_sq_norms", "qstate_fp32_sq_norms",
+           "qstate_fp32_decode_step", "qstate_lrb_query_sizes", "qstate_lrb_decode_step",
+           "qstate_state_sq_norms", "qstate_fp32_sq_norms",
            "qstate_selfcheck", "qstate_status_string", "qstate_version")
 
 
@@ -58,11 +59,13 @@ def lib() -> ctypes.CDLL:
         L.qstate_readout.argtypes = [C, P, P, P, P, P]
         L.qstate_selfcheck.argtypes = [P, P]
         L.qstate_fp32_decode_step.argtypes = [C, P, P, P, P, P, P, P, P]
+        L.qstate_lrb_query_sizes.argtypes = [C, ctypes.c_int, sz, sz, sz]
+        L.qstate_lrb_decode_step.argtypes = [C, ctypes.c_int, ctypes.c_int] + [P] * 15
         L.qstate_state_sq_norms.argtypes = [C, P, P, P, P]
         L.qstate_fp32_sq_norms.argtypes = [C, P, P, P]
         for f in (L.qstate_query_sizes, L.qstate_init, L.qstate_decode_step, L.qstate_readout,
                   L.qstate_selfcheck, L.qstate_fp32_decode_step, L.qstate_state_sq_norms,
-                  L.qstate_fp32_sq_norms):
+                  L.qstate_fp32_sq_norms, L.qstate_lrb_query_sizes, L.qstate_lrb_decode_step):
             f.restype = ctypes.c_int
         L.qstate_status_string.argtypes = [ctypes.c_int]
         L.qstate_status_string.restype = ctypes.c_char_p
@@ -155,6 +158,56 @@ def fp32_decode_step(cfg: Config, S, q, k, v, alpha, beta, o=None, stream=None) 
     _check(lib().qstate_fp32_decode_step(ctypes.byref(cc), _ptr(S), _ptr(q), _ptr(k), _ptr(v),
                                          _ptr(alpha), _ptr(beta), _ptr(o), _stream(stream)),
            "qstate_fp32_decode_step")
+
+
+def lrb_query_sizes(cfg: Config, rank: int):
+    """(decay_bytes, keys_bytes, coef_bytes) of the Low-Rank Bypass buffers."""
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    cc = cfg.c()
+    _check(lib().qstate_lrb_query_sizes(ctypes.byref(cc), rank, ctypes.byref(a), ctypes.byref(b),
+                                        ctypes.byref(c)), "qstate_lrb_query_sizes")
+    return a.value, b.value, c.value
+
+
+def lrb_decode_step(cfg: Config, rank: int, slot: int, codes, scales, shadow, A_in, A_out, K_in,
+                    K_out, U, q, k, v, alpha, beta, o=None, stream=None) -> None:
+    cc = cfg.c()
+    _check(lib().qstate_lrb_decode_step(ctypes.byref(cc), rank, slot, _ptr(codes), _ptr(scales),
+                                        _ptr(shadow), _ptr(A_in), _ptr(A_out), _ptr(K_in),
+                                        _ptr(K_out), _ptr(U), _ptr(q), _ptr(k), _ptr(v),
+                                        _ptr(alpha), _ptr(beta), _ptr(o), _stream(stream)),
+           "qstate_lrb_decode_step")
+
+
+class LrbBuffers:
+    """Low-Rank Bypass buffers of one state family (qstate_lrb_decode_step):
+    two copies of the accumulated decay A and of the buffered keys K (read one,
+    write the other), the coefficients U, and the slot of the next step."""
+
+    def __init__(self, cfg: Config, rank: int, device=None):
+        import torch
+        dev = torch.device("cuda") if device is None else torch.device(device)
+        self.cfg, self.rank, self.slot, self.cur = cfg, rank, 0, 0
+        self.rpad = (rank + 3) // 4 * 4
+        T = cfg.num_tiles
+        z = lambda *shape: torch.zeros(shape, dtype=torch.float32, device=dev)
+        self.A = [z(T, cfg.dk), z(T, cfg.dk)]
+        self.K = [z(T, rank, cfg.dk), z(T, rank, cfg.dk)]
+        self.U = z(T, cfg.dv, self.rpad)
+        a, b, c = lrb_query_sizes(cfg, rank)
+        assert a == 4 * self.A[0].numel() and b == 4 * self.K[0].numel() and c == 4 * self.U.numel()
+
+    def step(self, st: "QState", q, k, v, alpha, beta, o=None, stream=None):
+        i, j = self.cur, 1 - self.cur
+        lrb_decode_step(self.cfg, self.rank, self.slot, st.codes, st.scales, st.shadow,
+                        self.A[i], self.A[j], self.K[i], self.K[j], self.U, q, k, v, alpha, beta,
+                        o, stream)
+        if self.slot == self.rank - 1:
+            self.slot = 0
+        else:
+            self.slot += 1
+            self.cur = j
+        return o
 
 
 def state_sq_norms(cfg: Config, codes, scales, out, stream=None) -> None:

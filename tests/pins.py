@@ -610,7 +610,7 @@ def _lrb_effective(st, buf):
     d = st.codes.astype(np.float64) * np.repeat(st.scales.astype(np.float64), cfg.group, axis=-1)
     S = d * buf.A.astype(np.float64)[:, None, :]
     for r in range(buf.slot):
-        S += np.einsum("ti,tj->tij", buf.U[:, r].astype(np.float64), buf.K[:, r].astype(np.float64))
+        S += np.einsum("ti,tj->tij", buf.U[:, :, r].astype(np.float64), buf.K[:, r].astype(np.float64))
     return S
 
 

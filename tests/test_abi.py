@@ -137,6 +137,34 @@ def test_norms_validation():
     assert lib.qstate_fp32_sq_norms(None, A, 8 * A, None) == Q.QS_ERR_INVALID_ARG
 
 
+def _lrb(rank, slot, **ptrs):
+    p = dict(codes=A, scales=2 * A, shadow=None, A_in=10 * A, A_out=11 * A, K_in=12 * A,
+             K_out=13 * A, U=14 * A, q=3 * A, k=4 * A, v=5 * A, alpha=6 * A, beta=7 * A, o=8 * A)
+    p.update(ptrs)
+    c = _cfg().c()
+    return Q.lib().qstate_lrb_decode_step(ctypes.byref(c), rank, slot, p["codes"], p["scales"],
+                                          p["shadow"], p["A_in"], p["A_out"], p["K_in"], p["K_out"],
+                                          p["U"], p["q"], p["k"], p["v"], p["alpha"], p["beta"],
+                                          p["o"], None)
+
+
+def test_lrb_validation():
+    # rejected before any launch: unsupported rank, slot outside the period,
+    # missing or misaligned buffers, buffers overlapping the state
+    assert _lrb(0, 0) == Q.QS_ERR_UNSUPPORTED
+    assert _lrb(17, 0) == Q.QS_ERR_UNSUPPORTED
+    assert _lrb(4, 4) == Q.QS_ERR_INVALID_ARG
+    assert _lrb(4, -1) == Q.QS_ERR_INVALID_ARG
+    assert _lrb(4, 1, U=None) == Q.QS_ERR_INVALID_ARG
+    assert _lrb(4, 1, A_in=None) == Q.QS_ERR_INVALID_ARG
+    assert _lrb(4, 1, K_out=None) == Q.QS_ERR_INVALID_ARG
+    assert _lrb(4, 1, U=14 * A + 4) == Q.QS_ERR_INVALID_ARG
+    assert _lrb(4, 1, A_out=A + 64) == Q.QS_ERR_INVALID_ARG
+    assert _lrb(4, 1, K_out=12 * A) == Q.QS_ERR_INVALID_ARG
+    cfg = _cfg()
+    assert Q.lrb_query_sizes(cfg, 6) == (4 * 128 * 4, 4 * 6 * 128 * 4, 4 * 128 * 8 * 4)
+
+
 def test_binding_raises():
     with pytest.raises(Q.QStateError):
         Q.query_sizes(_cfg(bits=5))
