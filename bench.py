@@ -383,6 +383,9 @@ def run_ours(args):
     clocks = sampler.summary()
     fp32 = None if args.no_fp32 else run_fp32_state(args, w, dev, stream, dist, pool, host, S0, l2,
                                                    pool_bytes)
+    plain_us = {a.name: arm_ms[i] * 1e3 / K for i, a in enumerate(arms)}
+    lrb = None if args.lrb_rank <= 1 else run_lrb(args, w, dev, stream, dist, pool, S0, l2,
+                                                   pool_bytes, plain_us)
 
     # ---- end to end through the public API with host buffers
     e2e = run_e2e(args, w, arms, cfgs, states, dev, stream, dist, host, reinit)
@@ -453,6 +456,7 @@ def run_ours(args):
                                   for i, a in enumerate(arms)},
             "state_memory_ratio": {a.name: round(w.tiles * w.dv * w.dk * 4 / state_bytes(w, a), 3)
                                    for a in arms}}),
+        "lrb": lrb,
         "gpu_launches": K * len(arms),
         "clocks": clocks,
     }
@@ -536,6 +540,98 @@ def run_fp32_state(args, w, dev, stream, dist, pool, host, S0, l2, pool_bytes):
     return {"us_per_launch": round(s * 1e6, 3), "bytes_per_launch": b,
             "gbs": round(b / s / 1e9, 1), "frac": round(b / s / 1e9 / peak, 4),
             "l2": f"{G} request groups x {sb / 1e6:.1f} MB FP32 state + {pool_bytes / 1e6:.0f} MB inputs"}
+
+
+def lrb_bytes(w: W.Workload, arm: W.Arm, rank: int, slot: int, readout: bool = True) -> int:
+    """Algorithmic bytes of one Low-Rank Bypass step at position `slot` of
+    its period: the stored state is read at every step and written only at
+    the merge; the accumulated decay and the buffered keys are read (and
+    written at bypass steps), the coefficients read for slots < slot and
+    written for the slot."""
+    T, dk, dv = w.tiles, w.dk, w.dv
+    merge = slot == rank - 1
+    codes = T * dv * dk * arm.bits // 8
+    scales = T * dv * (dk // arm.group) * 4
+    b = codes + scales
+    if merge:
+        b += codes + (scales if arm.policy != "persistent" else 0)
+    b += T * (2 * dk + dv + 2) * 4 + (T * dk * 4 if w.decay == "diagonal" else 0)
+    b += T * dv * 4 if readout else 0
+    b += (T * dk * 4 if slot > 0 else 0) + (0 if merge else T * dk * 4)      # A in / out
+    b += T * slot * dk * 4 + (0 if merge else T * (slot + 1) * dk * 4)      # K in / out
+    b += T * dv * slot * 4 + (0 if merge else T * dv * 4)                    # U read / write
+    if arm.policy == "yoked":
+        b += 2 * T * dv * dk * 4
+    return b
+
+
+def run_lrb(args, w, dev, stream, dist, pool, S0, l2, pool_bytes, plain_us):
+    """Every arm of the workload again with Low-Rank Bypass of rank R
+    (qstate_lrb_decode_step): R - 1 bypass steps and one merge per period,
+    timed over whole periods the same way as the arms (CUDA graphs, events,
+    request groups past 2x L2).  Reported per step, averaged over the period.
+    Not part of the step."""
+    import torch
+    from ssm_decode_step_b200 import Config, QState, qstate as Q
+    R, P = args.lrb_rank, args.pool
+    out = {"rank": R}
+    peak, _ = load_peak()
+    for arm in w.arms:
+        cfg = Config(w.tiles, w.dk, w.dv, arm.bits, arm.group, w.delta, w.decay, arm.policy,
+                     arm.rounding)
+        a_b, k_b, u_b = Q.lrb_query_sizes(cfg, R)
+        gb = state_bytes(w, arm) + 2 * a_b + 2 * k_b + u_b
+        G = max(1, -(-2 * l2 // gb))
+        groups = []
+        for _ in range(G):
+            st = QState(cfg, dev).init(S0)
+            groups.append((st, Q.LrbBuffers(cfg, R, dev)))
+        o = torch.empty((w.tiles, w.dv), dtype=torch.float32, device=dev) if w.readout else None
+        # one graph = one period of every group; inputs keep cycling the pool
+        order = [(gi, slot) for slot in range(R) for gi in range(G)]
+
+        def launch(t, gi, slot):
+            st, b = groups[gi]
+            i = slot % 2
+            sl = t % P
+            Q.lrb_decode_step(cfg, R, slot, st.codes, st.scales, st.shadow, b.A[i], b.A[1 - i],
+                              b.K[i], b.K[1 - i], b.U, pool[0][sl], pool[1][sl], pool[2][sl],
+                              pool[3][sl], pool[4][sl], o, stream)
+
+        with torch.cuda.stream(stream):
+            for t, (gi, slot) in enumerate(order):
+                launch(t, gi, slot)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for t, (gi, slot) in enumerate(order):
+                launch(t, gi, slot)
+        reps = max(1, args.steps // len(order))
+        for st, _ in groups:
+            st.init(S0)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if dist is not None:
+            dist.barrier()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        ms = max_over_ranks(dist, [e0.elapsed_time(e1)], dev)[0]
+        del g
+        steps = reps * len(order)
+        sec = ms / 1e3 / steps
+        b = sum(lrb_bytes(w, arm, R, sl, w.readout) for sl in range(R)) / R
+        out[arm.name] = {"us_per_step": round(sec * 1e6, 3), "bytes_per_step": int(b),
+                         "gbs": round(b / sec / 1e9, 1), "frac": round(b / sec / 1e9 / peak, 4),
+                         "speedup_vs_plain": round(plain_us[arm.name] / (sec * 1e6), 3),
+                         "l2": f"{G} request groups x {gb / 1e6:.1f} MB (state + buffers)",
+                         "steps": steps}
+        del groups
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_e2e(args, w, arms, cfgs, states, dev, stream, dist, host, reinit):
@@ -650,11 +746,17 @@ def plant(S_w: np.ndarray, kstar: np.ndarray, vstar: np.ndarray) -> np.ndarray:
 
 
 def run_recall(args):
-    """Plant (k*, v*) in S0, decode H distractor steps under every arm and the
-    FP32 state, and read S_t k* and ||S_t|| at power-of-two checkpoints
+    """Plant (k*, v*) in S0, decode H distractor steps under every arm (and,
+    with --recall-lrb R, the same arms with Low-Rank Bypass of rank R) and
+    the FP32 state, and read the fact back at power-of-two checkpoints
     ("When Dynamic Scaling Fails": recall of a fact planted before
-    quantization began, as the decode horizon grows; the scale-state feedback
-    shows as norm inflation).  Prints one JSON line."""
+    quantization began, as the decode horizon grows; the scale-state
+    feedback shows as norm inflation).  The read is each step's own readout
+    with q = k*: o_t = S_t k* from the updated state (for a Low-Rank Bypass
+    arm, the stored state with its accumulated decay plus the buffer).  The
+    state norm is that of the stored state (qstate_state_sq_norms); for a
+    bypass arm it is taken at the ends of periods only, where the buffer has
+    just been merged.  Prints one JSON line."""
     import torch
     from ssm_decode_step_b200 import qstate as Q
     w = W.get("recall")
@@ -675,17 +777,26 @@ def run_recall(args):
     marks = sorted({0, H} | {1 << i for i in range(40) if (1 << i) <= H})
     launches = 0
 
-    def trajectory(step, probe):
+    def trajectory(step, probe0, norms_at):
+        """step(t, want_o) advances one step (readout into o with q = k* when
+        want_o); probe0() reads the state before the first step."""
         nonlocal launches
         rec, norms = [], []
         t = 0
         for m in marks:
+            if m == 0:
+                probe0()
+                launches += 2
             while t < m:
-                step(t % P)
-                launches += 1
                 t += 1
-            probe()
-            launches += 2
+                step(t - 1, t == m)
+                launches += 1
+            if m > 0:
+                if norms_at(m):
+                    norms_at(m)(nrm)
+                    launches += 1
+                else:
+                    nrm.fill_(float("nan"))
             torch.cuda.synchronize()
             rec.append(o.cpu().numpy().astype(np.float64))
             norms.append(nrm.cpu().numpy())
@@ -695,24 +806,43 @@ def run_recall(args):
     cfg32 = Q.Config(T, dk, dv, 8, 32, w.delta, w.decay)
     S = torch.from_numpy(S0.copy()).to(dev)
     fp = trajectory(
-        lambda i: Q.fp32_decode_step(cfg32, S, None, pool[1][i], pool[2][i], pool[3][i], pool[4][i], None),
-        # readout with a zero update (alpha = 1, k = 0, beta = 0) leaves S unchanged
-        lambda: (Q.fp32_decode_step(cfg32, S, kst, zk, zv, one, zero, o), Q.fp32_sq_norms(cfg32, S, nrm)))
+        lambda i, want: Q.fp32_decode_step(cfg32, S, kst, pool[1][i % P], pool[2][i % P],
+                                           pool[3][i % P], pool[4][i % P], o if want else None),
+        # before the first step: a zero update (alpha = 1, k = 0, beta = 0) leaves S unchanged
+        lambda: (Q.fp32_decode_step(cfg32, S, kst, zk, zv, one, zero, o), Q.fp32_sq_norms(cfg32, S, nrm)),
+        lambda m: (lambda out: Q.fp32_sq_norms(cfg32, S, out)))
     arms = {}
-    for arm in w.arms:
+    runs = [(arm, 1) for arm in w.arms]
+    if args.recall_lrb > 1:
+        runs += [(arm, args.recall_lrb) for arm in w.arms if arm.policy != "yoked"]
+    for arm, R in runs:
         cfg = Q.Config(T, dk, dv, arm.bits, arm.group, w.delta, w.decay, arm.policy, arm.rounding)
         st = Q.QState(cfg).init(torch.from_numpy(S0).to(dev))
-        arms[arm.name] = trajectory(
-            lambda i, st=st: st.step(None, pool[1][i], pool[2][i], pool[3][i], pool[4][i], None),
-            lambda st=st, cfg=cfg: (st.readout(kst, o), Q.state_sq_norms(cfg, st.codes, st.scales, nrm)))
+        name = arm.name if R == 1 else f"{arm.name}+lrb{R}"
+        if R == 1:
+            stepf = (lambda i, want, st=st: st.step(kst, pool[1][i % P], pool[2][i % P],
+                                                     pool[3][i % P], pool[4][i % P],
+                                                     o if want else None))
+            norms_at = lambda m, st=st, cfg=cfg: (lambda out: Q.state_sq_norms(cfg, st.codes, st.scales, out))
+        else:
+            buf = Q.LrbBuffers(cfg, R)
+            stepf = (lambda i, want, st=st, buf=buf: buf.step(st, kst, pool[1][i % P], pool[2][i % P],
+                                                               pool[3][i % P], pool[4][i % P],
+                                                               o if want else None))
+            norms_at = (lambda m, st=st, cfg=cfg, R=R:
+                        (lambda out: Q.state_sq_norms(cfg, st.codes, st.scales, out)) if m % R == 0 else None)
+        arms[name] = trajectory(
+            stepf,
+            lambda st=st, cfg=cfg: (st.readout(kst, o), Q.state_sq_norms(cfg, st.codes, st.scales, nrm)),
+            norms_at)
     elapsed = time.time() - t0
 
     vs = vstar.astype(np.float64)
-    med = lambda a: [round(float(x), 6) for x in np.median(a, axis=1)]
+    med = lambda a: [None if not np.isfinite(x) else round(float(x), 6) for x in np.median(a, axis=1)]
     rel = lambda r, ref: np.linalg.norm(r - ref, axis=-1) / np.linalg.norm(ref, axis=-1)
     out = {"experiment": "recall over the decode horizon", "workload": w.description,
            "tiles": T, "steps": H, "checkpoints": marks, "launches": launches,
-           "seconds": round(elapsed, 2),
+           "seconds": round(elapsed, 2), "read": "each step's readout with q = k*",
            "fp32": {"recall_err_vs_vstar": med(rel(fp[0], vs[None])),
                     "state_norm": med(np.sqrt(fp[1]))},
            "arms": {}}
@@ -744,10 +874,14 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp32", action="store_true", help="skip the FP32-state comparison arm")
+    ap.add_argument("--lrb-rank", type=int, default=8,
+                    help="also time every arm with Low-Rank Bypass of this rank (0: skip)")
     ap.add_argument("--recall", action="store_true",
                     help="measure recall of a planted association over the decode horizon instead")
     ap.add_argument("--recall-steps", type=int, default=32768)
     ap.add_argument("--recall-tol", type=float, default=0.5)
+    ap.add_argument("--recall-lrb", type=int, default=8,
+                    help="also run the non-yoked arms with Low-Rank Bypass of this rank (0: skip)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -196,7 +196,9 @@ QS_API qs_status qstate_fp32_decode_step(const qs_config* cfg, float* S, const f
  * Buffers (the caller's, 16-byte aligned; sizes from qstate_lrb_query_sizes):
  *   A_in, A_out [T][Dk] float   accumulated column decay (two copies: read
  *                               one, write the other; A_in unused at slot 0,
- *                               A_out unused at the merge)
+ *                               A_out unused at the merge; under scalar decay
+ *                               every column holds the same value, as the
+ *                               library writes it, and column 0 is read)
  *   K_in, K_out [T][rank][Dk]   buffered keys, decayed (same two copies)
  *   U           [T][Dv][rpad]   buffered write coefficients, rpad = rank
  *                               rounded up to a multiple of 4; column slot is

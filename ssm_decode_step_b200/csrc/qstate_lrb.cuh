@@ -68,7 +68,7 @@ struct LrbLayout {
     q = off;    off += vec;
     a = off;    off += diag ? vec : 0;
     A = off;    off += vec;
-    Kb = off;   off += merge ? rank * vec : 0;
+    Kb = off;   off += rank * vec;
     kdot = off; off += rpad * 4;
     qdot = off; off += rpad * 4;
     misc = off; off += 16;  // alpha, beta, k . q
@@ -109,6 +109,17 @@ __device__ __forceinline__ void lrb_issue_block(const BlockCursor<SLOT, DEPTH>& 
       if (lane == 0) cp4<0>(tv + L.misc, p.alpha + t);
     }
     if (lane == 1) cp4<4>(tv + L.misc, p.beta + t);
+    if (p.slot > 0) {
+      // the accumulated decay and the buffered keys of this tile
+      const int vec = (DK / 32) * kChunkStride * 4;
+      if (lane < VU)
+        cp16<0>(tv + L.A + static_cast<uint32_t>(vec_unit_offset(lane)), p.A_in + t * DK + 4 * lane);
+      const float* kin = p.K_in + t * p.rank * DK;
+      for (int i = lane; i < p.slot * VU; i += 32) {
+        const int r = i / VU, u = i % VU;
+        cp16<0>(tv + L.Kb + r * vec + static_cast<uint32_t>(vec_unit_offset(u)), kin + r * DK + 4 * u);
+      }
+    }
   }
   const uint32_t s4 = ring4 + cur.slot;
   const uint8_t* cs = codes_blk + static_cast<size_t>(cur.blk) * CSTRIDE;
@@ -262,19 +273,15 @@ __global__ void __launch_bounds__(kStepThreads, ((POLICY == 2 || BDR || MERGE) ?
         for (int m = 0; m < 16; ++m) aa[m] = f2(a_scalar);
       }
       if (rr == 0) {
-        // A = A_in * a for this chunk; k . q
+        // A = A_in * a for this chunk (A_in staged in the slot)
         float2 A[16];
         if (slot == 0) {
 #pragma unroll
           for (int m = 0; m < 16; ++m) A[m] = aa[m];
         } else {
-          const float4* src = reinterpret_cast<const float4*>(p.A_in + t * DK + 32 * c);
+          load_pairs(tv + L.A, c, A);
 #pragma unroll
-          for (int m = 0; m < 8; ++m) {
-            const float4 x = src[m];
-            A[2 * m] = __fmul2_rn(make_float2(x.x, x.y), aa[2 * m]);
-            A[2 * m + 1] = __fmul2_rn(make_float2(x.z, x.w), aa[2 * m + 1]);
-          }
+          for (int m = 0; m < 16; ++m) A[m] = __fmul2_rn(A[m], aa[m]);
         }
         float* dA = reinterpret_cast<float*>(tv + L.A) + c * kChunkStride;
 #pragma unroll
@@ -301,14 +308,12 @@ __global__ void __launch_bounds__(kStepThreads, ((POLICY == 2 || BDR || MERGE) ?
       for (int r0 = 0; r0 < slot; r0 += RW) {
         const int r = r0 + rr;
         const bool live = r < slot;
+        // K'_r = K_in_r * a (K_in_r staged in the slot; decayed in place below)
         float2 Kr[16];
-        const float4* src = reinterpret_cast<const float4*>(p.K_in + (t * p.rank + (live ? r : 0)) * DK + 32 * c);
+        const int vec = LPR * kChunkStride * 4;
+        load_pairs(tv + L.Kb + (live ? r : 0) * vec, c, Kr);
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const float4 x = live ? src[m] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-          Kr[2 * m] = __fmul2_rn(make_float2(x.x, x.y), aa[2 * m]);
-          Kr[2 * m + 1] = __fmul2_rn(make_float2(x.z, x.w), aa[2 * m + 1]);
-        }
+        for (int m = 0; m < 16; ++m) Kr[m] = live ? __fmul2_rn(Kr[m], aa[m]) : make_float2(0.0f, 0.0f);
         const float dk_ = chunk_dot<LPR>(Kr, kk);
         float dq_ = 0.0f;
         if (readout) {
@@ -321,7 +326,7 @@ __global__ void __launch_bounds__(kStepThreads, ((POLICY == 2 || BDR || MERGE) ?
             reinterpret_cast<float*>(tv + L.kdot)[r] = dk_;
             reinterpret_cast<float*>(tv + L.qdot)[r] = dq_;
           }
-          if constexpr (MERGE) {
+          {
             float* dK = reinterpret_cast<float*>(tv + L.Kb) + r * (LPR * kChunkStride) + c * kChunkStride;
 #pragma unroll
             for (int m = 0; m < 16; ++m) {
@@ -362,19 +367,38 @@ __global__ void __launch_bounds__(kStepThreads, ((POLICY == 2 || BDR || MERGE) ?
 #pragma unroll
       for (int m = 0; m < 16; ++m) dref[m] = __fmul2_rn(Sp[m], f2(s_old));
     }
-    {
+    if constexpr (DIAG) {
       float2 A[16];
       load_pairs(tv + L.A, c, A);
 #pragma unroll
       for (int m = 0; m < 16; ++m) Sp[m] = __fmul2_rn(Sp[m], __fmul2_rn(f2(s_old), A[m]));
+    } else {
+      // scalar decay: every A_j of the tile holds the same product of the
+      // alphas, so s * A_j is one product per row (the same bits)
+      const float sa = __fmul_rn(s_old, reinterpret_cast<const float*>(tv + L.A)[0]);
+#pragma unroll
+      for (int m = 0; m < 16; ++m) Sp[m] = __fmul2_rn(Sp[m], f2(sa));
+    }
+
+    // ---- the buffer's terms of u and o, U_ir kk_r and U_ir kq_r (r < slot),
+    // continuing each chain from its dot product over S'
+    float u_acc = 0.0f, o_acc = 0.0f;
+    if (DELTA) u_acc = chunk_dot<LPR>(Sp, kk);
+    float2 qq[16];
+    if (readout && !MERGE) {
+      load_pairs(tv + L.q, c, qq);
+      o_acc = chunk_dot<LPR>(Sp, qq);
+    }
+    for (int r = 0; r < slot; ++r) {
+      const float urr = ur[r];
+      if (DELTA) u_acc = __fmaf_rn(urr, kdot[r], u_acc);
+      if (readout && !MERGE) o_acc = __fmaf_rn(urr, qdot[r], o_acc);
     }
 
     // ---- write coefficient against S' + sum_r U_r K'_r^T
     float wcoef;
     if constexpr (DELTA) {
-      float u = chunk_dot<LPR>(Sp, kk);
-      for (int r = 0; r < slot; ++r) u = __fmaf_rn(ur[r], kdot[r], u);
-      wcoef = __fmul_rn(beta, __fsub_rn(v_i, u));
+      wcoef = __fmul_rn(beta, __fsub_rn(v_i, u_acc));
     } else {
       wcoef = __fmul_rn(beta, v_i);
     }
@@ -423,11 +447,7 @@ __global__ void __launch_bounds__(kStepThreads, ((POLICY == 2 || BDR || MERGE) ?
     if constexpr (!MERGE) {
       // ---- bypass: the write joins the buffer, the stored state is kept
       if (readout) {
-        float2 qq[16];
-        load_pairs(tv + L.q, c, qq);
-        float o = chunk_dot<LPR>(Sp, qq);
-        for (int r = 0; r < slot; ++r) o = __fmaf_rn(ur[r], qdot[r], o);
-        o = __fmaf_rn(wcoef, kqn, o);
+        const float o = __fmaf_rn(wcoef, kqn, o_acc);
         if (c == 0) o_l[blk * RW] = o;
       }
       if (c == 0) p.U[row * p.rpad + slot] = wcoef;

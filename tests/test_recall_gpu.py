@@ -38,12 +38,17 @@ def test_fp32_probe_leaves_state_unchanged():
 
 
 def test_recall_measurement_runs(capsys):
-    args = argparse.Namespace(recall_steps=16, pool=8, recall_tol=0.5)
+    args = argparse.Namespace(recall_steps=16, pool=8, recall_tol=0.5, recall_lrb=4)
     bench.run_recall(args)
     line = capsys.readouterr().out.strip().splitlines()[-1]
     d = json.loads(line)
     assert d["checkpoints"] == [0, 1, 2, 4, 8, 16]
-    assert set(d["arms"]) == {a.name for a in W.get("recall").arms}
+    names = {a.name for a in W.get("recall").arms}
+    names |= {a.name + "+lrb4" for a in W.get("recall").arms if a.policy != "yoked"}
+    assert set(d["arms"]) == names
+    # a bypass arm's stored-state norm is taken at the ends of periods only
+    assert d["arms"]["int4-g32-persistent+lrb4"]["norm_ratio_vs_fp32"][1] is None
+    assert d["arms"]["int4-g32-persistent+lrb4"]["norm_ratio_vs_fp32"][3] is not None
     # at t = 0 every arm holds the planted state up to its quantization error
     assert d["fp32"]["recall_err_vs_vstar"][0] < 1e-5
     assert d["arms"]["int8-g32-dynamic"]["recall_err_vs_fp32"][0] < 0.05
