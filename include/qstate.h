@@ -215,6 +215,31 @@ QS_API qs_status qstate_lrb_decode_step(const qs_config* cfg, int rank, int slot
                                         const float* alpha, const float* beta, float* o,
                                         cudaStream_t stream);
 
+/* Chunkwise prefill of an FP32 state over `length` tokens, for the linear
+ * write (delta = 0) with scalar decay (the Mamba-2 family whose chunkwise
+ * realization LinQuant gives: Low-Precision Chunkwise Realization, state
+ * write / state pass / state read / local score / intra-chunk output) or
+ * diagonal decay (the GLA family, the same contractions per channel).  It
+ * computes, for every tile, the token-by-token recurrence
+ *   S_t = S_{t-1} Lambda_t + beta_t v_t k_t^T,   o_t = S_t q_t
+ * regrouped in chunks of 32 tokens (exact in real arithmetic; in FP32 the
+ * summation order differs from the token-by-token order, so results agree
+ * with qstate_fp32_decode_step applied token by token to within FP32
+ * rounding, not bit for bit).  The state it leaves is the S0 that
+ * qstate_init quantizes for the decode path.
+ *   S      [T][Dv][Dk] float, in: state before the first token (e.g. zeros),
+ *          out: state after the last
+ *   q, k   [T][length][Dk] float;  v [T][length][Dv] float
+ *   alpha  [T][length] (QS_DECAY_SCALAR) or [T][length][Dk] (diagonal), in (0, 1]
+ *   beta   [T][length] float
+ *   o      [T][length][Dv] float, or NULL to skip the outputs
+ * Only num_tiles, dk, dv, delta and decay of cfg are used; delta must be 0
+ * (the delta rule's chunkwise form is not built), dv <= 128.  Under
+ * diagonal decay a chunk may decay a channel by at most e^-170. */
+QS_API qs_status qstate_prefill(const qs_config* cfg, int length, float* S, const float* q,
+                                const float* k, const float* v, const float* alpha,
+                                const float* beta, float* o, cudaStream_t stream);
+
 /* Squared Frobenius norm of every tile of the stored state, for tracking
  * the state norm over a decode horizon (the norm inflation of per-token
  * dynamic scaling: "When Dynamic Scaling Fails", abstract and project page,

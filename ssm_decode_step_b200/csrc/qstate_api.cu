@@ -438,6 +438,49 @@ qs_status qstate_lrb_decode_step(const qs_config* cfg, int rank, int slot, void*
   return from_cuda(e);
 }
 
+qs_status qstate_prefill(const qs_config* cfg, int length, float* S, const float* q,
+                         const float* k, const float* v, const float* alpha, const float* beta,
+                         float* o, cudaStream_t stream) {
+  if (cfg == nullptr) return QS_ERR_INVALID_ARG;
+  qs_config c = *cfg;
+  c.bits = 8;
+  c.group = 32;
+  c.policy = QS_SCALE_PERSISTENT;
+  c.rounding = QS_ROUND_NEAREST;
+  qs_status st = check_config(&c);
+  if (st != QS_OK) return st;
+  if (c.delta != 0 || c.dv > 128) return QS_ERR_UNSUPPORTED;
+  if (length < 0) return QS_ERR_INVALID_ARG;
+  if (c.num_tiles == 0 || length == 0) return QS_OK;
+  const bool diag = c.decay == QS_DECAY_DIAGONAL;
+  if (!S || !q || !k || !v || !alpha || !beta) return QS_ERR_INVALID_ARG;
+  if (!aligned(S, 4) || !aligned(q, 4) || !aligned(k, 4) || !aligned(v, 4) || !aligned(alpha, 4) ||
+      !aligned(beta, 4) || (o && !aligned(o, 4)))
+    return QS_ERR_INVALID_ARG;
+  const size_t T = static_cast<size_t>(c.num_tiles), L = static_cast<size_t>(length);
+  const Range w[2] = {range_of(S, T * c.dv * c.dk * 4), range_of(o, o ? T * L * c.dv * 4 : 0)};
+  const Range r[5] = {range_of(q, T * L * c.dk * 4), range_of(k, T * L * c.dk * 4),
+                      range_of(v, T * L * c.dv * 4), range_of(alpha, T * L * (diag ? c.dk : 1) * 4),
+                      range_of(beta, T * L * 4)};
+  if (any_overlap(w, 2, r, 5)) return QS_ERR_INVALID_ARG;
+  qs::PrefillParams p;
+  p.S = S;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.alpha = alpha;
+  p.beta = beta;
+  p.o = o;
+  p.L = length;
+  p.dv = c.dv;
+  cudaError_t e;
+  if (c.dk == 64)
+    e = diag ? qs::launch_prefill<64, true>(p, c.num_tiles, stream) : qs::launch_prefill<64, false>(p, c.num_tiles, stream);
+  else
+    e = diag ? qs::launch_prefill<128, true>(p, c.num_tiles, stream) : qs::launch_prefill<128, false>(p, c.num_tiles, stream);
+  return from_cuda(e);
+}
+
 qs_status qstate_state_sq_norms(const qs_config* cfg, const void* codes, const float* scales,
                                 double* out, cudaStream_t stream) {
   qs_status st = check_config(cfg);

@@ -9,6 +9,7 @@
 #include "qstate_kernels.cuh"
 #include "qstate_step.cuh"
 #include "qstate_lrb.cuh"
+#include "qstate_prefill.cuh"
 
 namespace qs {
 
@@ -25,6 +26,10 @@ cudaError_t launch_lrb(const LrbParams& p, int tiles, int dv, cudaStream_t strea
 template <int BITS, int DK>
 cudaError_t launch_init(const float* S0, uint8_t* codes, float* scales, float* shadow,
                         long long rows, int group, cudaStream_t stream);
+
+// Chunkwise prefill (delta = 0) of `tiles` tiles.
+template <int DK, bool DIAG>
+cudaError_t launch_prefill(const PrefillParams& p, int tiles, cudaStream_t stream);
 
 // Streaming multiprocessors of the current device (queried once per device).
 int device_sm_count();

@@ -124,6 +124,17 @@ cudaError_t launch_lrb(const LrbParams& p0, int tiles, int dv, cudaStream_t stre
   return cudaGetLastError();
 }
 
+template <int DK, bool DIAG>
+cudaError_t launch_prefill(const PrefillParams& p, int tiles, cudaStream_t stream) {
+  auto kernel = prefill_kernel<DK, DIAG>;
+  static std::once_flag flag;
+  cudaError_t err = allow_smem(kernel, flag);
+  if (err != cudaSuccess) return err;
+  const PrefillLayout L(DK, p.dv, DIAG);
+  kernel<<<tiles, kPrefillThreads, static_cast<size_t>(L.total) * sizeof(float), stream>>>(p);
+  return cudaGetLastError();
+}
+
 template <int BITS, int DK>
 cudaError_t launch_readout(const StepParams& p0, cudaStream_t stream) {
   constexpr int S = 4;
@@ -167,6 +178,10 @@ cudaError_t launch_init(const float* S0, uint8_t* codes, float* scales, float* s
   template cudaError_t launch_readout<B, D>(const StepParams&, cudaStream_t);        \
   template cudaError_t launch_init<B, D>(const float*, uint8_t*, float*, float*, long long, int, \
                                          cudaStream_t);
+
+#define QS_INSTANTIATE_PREFILL(D)                                                   \
+  template cudaError_t launch_prefill<D, false>(const PrefillParams&, int, cudaStream_t); \
+  template cudaError_t launch_prefill<D, true>(const PrefillParams&, int, cudaStream_t);
 
 #define QS_INSTANTIATE_LRB1(B, D, P, R, DE, DI, M) \
   template cudaError_t launch_lrb<B, D, P, R, DE, DI, M>(const LrbParams&, int, int, cudaStream_t);

@@ -1,0 +1,224 @@
+// Chunkwise prefill of the linear-write recurrence (delta = 0) on an FP32
+// state: qstate_prefill.  The state S_0 that the quantized decode path then
+// starts from (LinQuant, Low-Precision Chunkwise Realization, for the
+// Mamba-2 family: state write, state pass, state read, local score,
+// intra-chunk output; here in FP32, with the diagonal decay of the GLA
+// family as the per-channel extension).
+//
+// Per tile, tokens are taken in chunks of C = 32.  With Lam_t the running
+// sum of log(alpha) over the chunk's tokens up to t (per channel for
+// diagonal decay) and S the state at the chunk's start:
+//   o_t   = (S (q_t * e^{Lam_t})) + sum_{s <= t} A_ts beta_s v_s
+//   A_ts  = sum_j q_tj k_sj e^{Lam_tj - Lam_sj}
+//   S_new = S * e^{Lam_C} + sum_s beta_s v_s (k_s * e^{Lam_C - Lam_s})^T
+// which is the token-by-token recurrence S_t = S_{t-1} Lambda_t + beta_t v_t
+// k_t^T, o_t = S_t q_t regrouped (exactly in real arithmetic).  Under scalar
+// decay A_ts = (q_t . k_s) e^{Lam_t - Lam_s}; under diagonal decay the
+// factor is split around the chunk's middle token m as
+// (q_t e^{Lam_t - Lam_m}) . (k_s e^{Lam_m - Lam_s}), which stays in range
+// while a chunk decays any channel by less than e^{-170}.
+//
+// One CTA per tile, 256 threads; the state stays in shared memory (rows
+// padded to Dk + 1 floats) for the whole sequence.  Only the state pass is
+// sequential; tiles are independent.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace qs {
+
+constexpr int kPrefillChunk = 32;
+constexpr int kPrefillThreads = 256;
+
+struct PrefillParams {
+  float* S;            // [T][dv][dk], in: initial state, out: state after the L tokens
+  const float* q;      // [T][L][dk]
+  const float* k;      // [T][L][dk]
+  const float* v;      // [T][L][dv]
+  const float* alpha;  // [T][L] (scalar) or [T][L][dk] (diagonal)
+  const float* beta;   // [T][L]
+  float* o;            // [T][L][dv] or nullptr
+  int L;
+  int dv;
+};
+
+// Shared-memory layout (floats) of one CTA.
+struct PrefillLayout {
+  int S, qbar, kbar, qt, kh, v, lam, A, beta, elam, total;
+  __host__ __device__ PrefillLayout(int dk, int dv, bool diag) {
+    constexpr int C = kPrefillChunk;
+    int off = 0;
+    S = off;    off += dv * (dk + 1);
+    qbar = off; off += dk * C;           // [j][t]: q_t * e^{Lam_t}
+    kbar = off; off += C * dk;           // [s][j]: k_s * e^{Lam_C - Lam_s}
+    qt = off;   off += diag ? C * dk : 0;  // [t][j]: q_t * e^{Lam_t - Lam_m}
+    kh = off;   off += diag ? C * dk : 0;  // [s][j]: k_s * e^{Lam_m - Lam_s}
+    v = off;    off += C * dv;           // [s][i]
+    lam = off;  off += diag ? C * dk : C;  // [t][j] or [t]
+    A = off;    off += C * C;            // [t][s], beta_s folded in
+    beta = off; off += C;
+    elam = off; off += diag ? dk : 1;    // e^{Lam_C} per channel
+    total = off;
+  }
+};
+
+template <int DK, bool DIAG>
+__global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(PrefillParams p) {
+  constexpr int C = kPrefillChunk;
+  constexpr int NT = kPrefillThreads;
+  extern __shared__ __align__(16) float sm[];
+  const int dv = p.dv;
+  const PrefillLayout Ly(DK, dv, DIAG);
+  float* S = sm + Ly.S;
+  float* qbar = sm + Ly.qbar;
+  float* kbar = sm + Ly.kbar;
+  float* qt = sm + Ly.qt;
+  float* kh = sm + Ly.kh;
+  float* V = sm + Ly.v;
+  float* lam = sm + Ly.lam;
+  float* A = sm + Ly.A;
+  float* bt = sm + Ly.beta;
+  float* elam = sm + Ly.elam;
+  const int tid = threadIdx.x;
+  const size_t tile = blockIdx.x;
+  constexpr int SP = DK + 1;  // padded state row
+
+  float* Sg = p.S + tile * dv * DK;
+  for (int e = tid; e < dv * DK; e += NT) S[(e / DK) * SP + (e % DK)] = Sg[e];
+
+  for (int c0 = 0; c0 < p.L; c0 += C) {
+    const int Ce = min(C, p.L - c0);
+    const size_t tok0 = tile * p.L + c0;
+    __syncthreads();
+    // ---- chunk inputs
+    for (int e = tid; e < C * dv; e += NT) {
+      const int s = e / dv, i = e % dv;
+      V[e] = s < Ce ? p.v[(tok0 + s) * dv + i] : 0.0f;
+    }
+    if (tid < C) bt[tid] = tid < Ce ? p.beta[tok0 + tid] : 0.0f;
+    // ---- running log-decay over the chunk
+    if constexpr (DIAG) {
+      for (int j = tid; j < DK; j += NT) {
+        float acc = 0.0f;
+        for (int t = 0; t < C; ++t) {
+          if (t < Ce) acc += logf(p.alpha[(tok0 + t) * DK + j]);
+          lam[t * DK + j] = acc;
+        }
+        elam[j] = expf(acc);
+      }
+    } else {
+      if (tid < 32) {
+        float x = tid < Ce ? logf(p.alpha[tok0 + tid]) : 0.0f;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+          const float y = __shfl_up_sync(0xffffffffu, x, d);
+          if (tid >= d) x += y;
+        }
+        lam[tid] = x;
+        const float total = __shfl_sync(0xffffffffu, x, 31);
+        if (tid == 0) elam[0] = expf(total);
+      }
+    }
+    __syncthreads();
+    // ---- decayed copies of q and k
+    const int m = (Ce - 1) / 2;
+    for (int e = tid; e < C * DK; e += NT) {
+      const int t = e / DK, j = e % DK;
+      const bool live = t < Ce;
+      const float qv = live ? p.q[(tok0 + t) * DK + j] : 0.0f;
+      const float kv = live ? p.k[(tok0 + t) * DK + j] : 0.0f;
+      if constexpr (DIAG) {
+        const float lt = lam[t * DK + j], lC = lam[(C - 1) * DK + j], lm = lam[m * DK + j];
+        qbar[j * C + t] = qv * expf(lt);
+        kbar[t * DK + j] = kv * expf(lC - lt);
+        qt[t * DK + j] = qv * expf(lt - lm);
+        kh[t * DK + j] = kv * expf(lm - lt);
+      } else {
+        const float lt = lam[t], lC = lam[C - 1];
+        qbar[j * C + t] = qv * expf(lt);
+        kbar[t * DK + j] = kv * expf(lC - lt);
+      }
+    }
+    __syncthreads();
+    // ---- local scores A_ts (s <= t), beta_s folded in
+    for (int e = tid; e < C * C; e += NT) {
+      const int t = e / C, s = e % C;
+      float a = 0.0f;
+      if (s <= t && t < Ce) {
+        if constexpr (DIAG) {
+          const float* x = qt + t * DK;
+          const float* y = kh + s * DK;
+          for (int j = 0; j < DK; ++j) a = fmaf(x[j], y[j], a);
+        } else {
+          const float* x = p.q + (tok0 + t) * DK;
+          const float* y = p.k + (tok0 + s) * DK;
+          for (int j = 0; j < DK; ++j) a = fmaf(__ldg(x + j), __ldg(y + j), a);
+          a *= expf(lam[t] - lam[s]);
+        }
+        a *= bt[s];
+      }
+      A[e] = a;
+    }
+    __syncthreads();
+    // ---- outputs: state read + intra-chunk output
+    if (p.o != nullptr) {
+      for (int e = tid; e < dv * (C / 8); e += NT) {
+        const int i = e % dv, tg = e / dv;  // 8 tokens per thread
+        float acc[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc[u] = 0.0f;
+        const float* srow = S + i * SP;
+        for (int j = 0; j < DK; ++j) {
+          const float sv = srow[j];
+          const float4 a0 = *reinterpret_cast<const float4*>(qbar + j * C + 8 * tg);
+          const float4 a1 = *reinterpret_cast<const float4*>(qbar + j * C + 8 * tg + 4);
+          acc[0] = fmaf(sv, a0.x, acc[0]); acc[1] = fmaf(sv, a0.y, acc[1]);
+          acc[2] = fmaf(sv, a0.z, acc[2]); acc[3] = fmaf(sv, a0.w, acc[3]);
+          acc[4] = fmaf(sv, a1.x, acc[4]); acc[5] = fmaf(sv, a1.y, acc[5]);
+          acc[6] = fmaf(sv, a1.z, acc[6]); acc[7] = fmaf(sv, a1.w, acc[7]);
+        }
+        for (int s = 0; s < C; ++s) {
+          const float vs = V[s * dv + i];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) acc[u] = fmaf(A[(8 * tg + u) * C + s], vs, acc[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int t = 8 * tg + u;
+          if (t < Ce) p.o[(tok0 + t) * dv + i] = acc[u];
+        }
+      }
+      __syncthreads();
+    }
+    // ---- state pass: S = S e^{Lam_C} + sum_s beta_s v_s kbar_s^T
+    {
+      constexpr int JW = 16;  // columns per thread
+      for (int e = tid; e < dv * (DK / JW); e += NT) {
+        const int i = e % dv, jb = (e / dv) * JW;
+        float acc[JW];
+        float* srow = S + i * SP + jb;
+#pragma unroll
+        for (int u = 0; u < JW; ++u) acc[u] = srow[u] * elam[DIAG ? jb + u : 0];
+        for (int s = 0; s < Ce; ++s) {
+          const float w = bt[s] * V[s * dv + i];
+          const float4* kr = reinterpret_cast<const float4*>(kbar + s * DK + jb);
+#pragma unroll
+          for (int u4 = 0; u4 < JW / 4; ++u4) {
+            const float4 kv = kr[u4];
+            acc[4 * u4 + 0] = fmaf(w, kv.x, acc[4 * u4 + 0]);
+            acc[4 * u4 + 1] = fmaf(w, kv.y, acc[4 * u4 + 1]);
+            acc[4 * u4 + 2] = fmaf(w, kv.z, acc[4 * u4 + 2]);
+            acc[4 * u4 + 3] = fmaf(w, kv.w, acc[4 * u4 + 3]);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < JW; ++u) srow[u] = acc[u];
+      }
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < dv * DK; e += NT) Sg[e] = S[(e / DK) * SP + (e % DK)];
+}
+
+}  // namespace qs

@@ -25,6 +25,7 @@ QS_OK, QS_ERR_INVALID_ARG, QS_ERR_UNSUPPORTED, QS_ERR_CUDA = 0, 1, 2, 3
 # Every entry point that include/qstate.h declares.
 EXPORTS = ("qstate_query_sizes", "qstate_init", "qstate_decode_step", "qstate_readout",
            "qstate_fp32_decode_step", "qstate_lrb_query_sizes", "qstate_lrb_decode_step",
+           "qstate_prefill",
            "qstate_state_sq_norms", "qstate_fp32_sq_norms",
            "qstate_selfcheck", "qstate_status_string", "qstate_version")
 
@@ -61,11 +62,13 @@ def lib() -> ctypes.CDLL:
         L.qstate_fp32_decode_step.argtypes = [C, P, P, P, P, P, P, P, P]
         L.qstate_lrb_query_sizes.argtypes = [C, ctypes.c_int, sz, sz, sz]
         L.qstate_lrb_decode_step.argtypes = [C, ctypes.c_int, ctypes.c_int] + [P] * 15
+        L.qstate_prefill.argtypes = [C, ctypes.c_int] + [P] * 8
         L.qstate_state_sq_norms.argtypes = [C, P, P, P, P]
         L.qstate_fp32_sq_norms.argtypes = [C, P, P, P]
         for f in (L.qstate_query_sizes, L.qstate_init, L.qstate_decode_step, L.qstate_readout,
                   L.qstate_selfcheck, L.qstate_fp32_decode_step, L.qstate_state_sq_norms,
-                  L.qstate_fp32_sq_norms, L.qstate_lrb_query_sizes, L.qstate_lrb_decode_step):
+                  L.qstate_fp32_sq_norms, L.qstate_lrb_query_sizes, L.qstate_lrb_decode_step,
+                  L.qstate_prefill):
             f.restype = ctypes.c_int
         L.qstate_status_string.argtypes = [ctypes.c_int]
         L.qstate_status_string.restype = ctypes.c_char_p
@@ -208,6 +211,16 @@ class LrbBuffers:
             self.slot += 1
             self.cur = j
         return o
+
+
+def prefill(cfg: Config, length: int, S, q, k, v, alpha, beta, o=None, stream=None) -> None:
+    """Chunkwise prefill (delta = 0) of the FP32 state S [T][dv][dk] over
+    `length` tokens: q, k [T][L][dk], v [T][L][dv], alpha [T][L] or
+    [T][L][dk], beta [T][L]; o [T][L][dv] or None."""
+    cc = cfg.c()
+    _check(lib().qstate_prefill(ctypes.byref(cc), length, _ptr(S), _ptr(q), _ptr(k), _ptr(v),
+                                _ptr(alpha), _ptr(beta), _ptr(o), _stream(stream)),
+           "qstate_prefill")
 
 
 def state_sq_norms(cfg: Config, codes, scales, out, stream=None) -> None:

@@ -165,6 +165,19 @@ def test_lrb_validation():
     assert Q.lrb_query_sizes(cfg, 6) == (4 * 128 * 4, 4 * 6 * 128 * 4, 4 * 128 * 8 * 4)
 
 
+def test_prefill_validation():
+    lib = Q.lib()
+    pre = lambda cfg, L, **kw: lib.qstate_prefill(ctypes.byref(cfg.c()), L, kw.get("S", A), kw.get("q", 2 * A),
+                                                  kw.get("k", 3 * A), kw.get("v", 4 * A), kw.get("a", 5 * A),
+                                                  kw.get("b", 6 * A), kw.get("o", 7 * A), None)
+    assert pre(_cfg(delta=1), 8) == Q.QS_ERR_UNSUPPORTED
+    assert pre(_cfg(delta=0, dv=256), 8) == Q.QS_ERR_UNSUPPORTED
+    assert pre(_cfg(delta=0), -1) == Q.QS_ERR_INVALID_ARG
+    assert pre(_cfg(delta=0), 8, S=None) == Q.QS_ERR_INVALID_ARG
+    assert pre(_cfg(delta=0), 8, o=A + 64) == Q.QS_ERR_INVALID_ARG
+    assert pre(_cfg(delta=0), 0, S=None) == Q.QS_OK
+
+
 def test_binding_raises():
     with pytest.raises(Q.QStateError):
         Q.query_sizes(_cfg(bits=5))
