@@ -859,6 +859,67 @@ def run_recall(args):
     print(json.dumps(out))
 
 
+def prefill_flops(dk: int, dv: int, L: int, C: int = 32) -> int:
+    """Algorithmic FLOPs of the chunkwise prefill of one tile over L tokens:
+    per chunk of c tokens, the state read 2 c dk dv, the local scores c^2 dk
+    (the causal half of 2 c^2 dk), the intra-chunk outputs c^2 dv and the
+    state pass 2 c dk dv + dk dv."""
+    f = 0
+    for c0 in range(0, L, C):
+        c = min(C, L - c0)
+        f += 4 * c * dk * dv + c * c * (dk + dv) + dk * dv
+    return f
+
+
+def run_prefill(args):
+    """Time qstate_prefill over `--prefill` tokens for every tile of the
+    workload (inputs drawn from its laws, slot t mod P for token t), from a
+    zero state, with outputs.  Prints one JSON line: tokens/s and the
+    achieved FP32 rate against the FP32 FMA peak of the SMs (148 SMs x 128
+    lanes x 2 FLOPs x the SM clock sampled during the run)."""
+    import torch
+    from ssm_decode_step_b200 import Config, qstate as Q
+    w = W.get(args.workload)
+    if w.delta != 0:
+        raise SystemExit("the chunkwise prefill covers the linear write (delta = 0) workloads")
+    L, P = args.prefill, max(1, min(args.pool, args.prefill))
+    dev = torch.device("cuda")
+    T = w.tiles
+    slots = [W.slot(w, t) for t in range(P)]
+    idx = np.arange(L) % P
+    arrs = [np.ascontiguousarray(np.stack([s[i] for s in slots], axis=1)[:, idx]) for i in range(5)]
+    q, k, v, a, b = (torch.from_numpy(x).to(dev) for x in arrs)
+    cfg = Config(T, w.dk, w.dv, 8, 32, 0, w.decay)
+    S = torch.zeros((T, w.dv, w.dk), dtype=torch.float32, device=dev)
+    o = torch.empty((T, L, w.dv), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        Q.prefill(cfg, L, S, q, k, v, a, b, o)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as sampler:
+        e0.record(stream)
+        for _ in range(args.steps):
+            S.zero_()
+            Q.prefill(cfg, L, S, q, k, v, a, b, o)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    clocks = sampler.summary()
+    sec = e0.elapsed_time(e1) / 1e3 / args.steps
+    flops = T * prefill_flops(w.dk, w.dv, L)
+    mhz = clocks.get("sm_mhz") or 1965
+    peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+    print(json.dumps({
+        "experiment": "chunkwise prefill (qstate_prefill)", "workload": w.description,
+        "tiles": T, "tokens_per_tile": L, "launches": args.steps,
+        "ms_per_prefill": round(sec * 1e3, 4), "tokens_per_s": round(T * L / sec, 1),
+        "tflops": round(flops / sec / 1e12, 3), "fp32_peak_tflops": round(peak, 2),
+        "frac_of_fp32_peak": round(flops / sec / 1e12 / peak, 4), "bound": "alu",
+        "note": "FLOPs are the chunkwise algorithm's (prefill_flops); the zeroing of S between "
+                "launches is inside the timed region (one memset of the state)",
+        "clocks": clocks}))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -876,6 +937,8 @@ def main():
     ap.add_argument("--no-fp32", action="store_true", help="skip the FP32-state comparison arm")
     ap.add_argument("--lrb-rank", type=int, default=8,
                     help="also time every arm with Low-Rank Bypass of this rank (0: skip)")
+    ap.add_argument("--prefill", type=int, default=0,
+                    help="time the chunkwise prefill over this many tokens per tile instead")
     ap.add_argument("--recall", action="store_true",
                     help="measure recall of a planted association over the decode horizon instead")
     ap.add_argument("--recall-steps", type=int, default=32768)
@@ -887,6 +950,8 @@ def main():
         ap.error("--warmup must be at least 3")
     if args.recall:
         run_recall(args)
+    elif args.prefill > 0:
+        run_prefill(args)
     elif args.impl == "reference":
         run_reference(args)
     else:

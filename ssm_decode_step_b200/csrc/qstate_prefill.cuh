@@ -52,8 +52,8 @@ struct PrefillLayout {
     S = off;    off += dv * (dk + 1);
     qbar = off; off += dk * C;           // [j][t]: q_t * e^{Lam_t}
     kbar = off; off += C * dk;           // [s][j]: k_s * e^{Lam_C - Lam_s}
-    qt = off;   off += diag ? C * dk : 0;  // [t][j]: q_t * e^{Lam_t - Lam_m}
-    kh = off;   off += diag ? C * dk : 0;  // [s][j]: k_s * e^{Lam_m - Lam_s}
+    qt = off;   off += C * (dk + 4);     // [t][j]: q_t (* e^{Lam_t - Lam_m} when diagonal)
+    kh = off;   off += C * (dk + 4);     // [s][j]: k_s (* e^{Lam_m - Lam_s} when diagonal)
     v = off;    off += C * dv;           // [s][i]
     lam = off;  off += diag ? C * dk : C;  // [t][j] or [t]
     A = off;    off += C * C;            // [t][s], beta_s folded in
@@ -64,7 +64,7 @@ struct PrefillLayout {
 };
 
 template <int DK, bool DIAG>
-__global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(PrefillParams p) {
+__global__ void __launch_bounds__(kPrefillThreads, 2) prefill_kernel(PrefillParams p) {
   constexpr int C = kPrefillChunk;
   constexpr int NT = kPrefillThreads;
   extern __shared__ __align__(16) float sm[];
@@ -83,6 +83,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(PrefillPara
   const int tid = threadIdx.x;
   const size_t tile = blockIdx.x;
   constexpr int SP = DK + 1;  // padded state row
+  constexpr int QP = DK + 4;  // padded q / k row (16-byte aligned, no bank conflicts)
+  static_assert(kPrefillThreads == 8 * 32 && kPrefillChunk == 32, "8 warps x 4 tokens, 32 keys");
 
   float* Sg = p.S + tile * dv * DK;
   for (int e = tid; e < dv * DK; e += NT) S[(e / DK) * SP + (e % DK)] = Sg[e];
@@ -132,33 +134,46 @@ __global__ void __launch_bounds__(kPrefillThreads, 1) prefill_kernel(PrefillPara
         const float lt = lam[t * DK + j], lC = lam[(C - 1) * DK + j], lm = lam[m * DK + j];
         qbar[j * C + t] = qv * expf(lt);
         kbar[t * DK + j] = kv * expf(lC - lt);
-        qt[t * DK + j] = qv * expf(lt - lm);
-        kh[t * DK + j] = kv * expf(lm - lt);
+        qt[t * QP + j] = qv * expf(lt - lm);
+        kh[t * QP + j] = kv * expf(lm - lt);
       } else {
         const float lt = lam[t], lC = lam[C - 1];
         qbar[j * C + t] = qv * expf(lt);
         kbar[t * DK + j] = kv * expf(lC - lt);
+        qt[t * QP + j] = qv;
+        kh[t * QP + j] = kv;
       }
     }
     __syncthreads();
-    // ---- local scores A_ts (s <= t), beta_s folded in
-    for (int e = tid; e < C * C; e += NT) {
-      const int t = e / C, s = e % C;
-      float a = 0.0f;
-      if (s <= t && t < Ce) {
-        if constexpr (DIAG) {
-          const float* x = qt + t * DK;
-          const float* y = kh + s * DK;
-          for (int j = 0; j < DK; ++j) a = fmaf(x[j], y[j], a);
-        } else {
-          const float* x = p.q + (tok0 + t) * DK;
-          const float* y = p.k + (tok0 + s) * DK;
-          for (int j = 0; j < DK; ++j) a = fmaf(__ldg(x + j), __ldg(y + j), a);
-          a *= expf(lam[t] - lam[s]);
+    // ---- local scores A_ts (s <= t), beta_s folded in: warp w takes tokens
+    // t = 4w .. 4w+3, lane s one key; float4 steps along Dk
+    {
+      const int lane = tid & 31, w = tid >> 5;
+      const int s = lane;
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      const float4* kr = reinterpret_cast<const float4*>(kh + s * QP);
+      for (int j4 = 0; j4 < DK / 4; ++j4) {
+        const float4 kv = kr[j4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 qv = reinterpret_cast<const float4*>(qt + (4 * w + u) * QP)[j4];
+          acc[u] = fmaf(qv.x, kv.x, acc[u]);
+          acc[u] = fmaf(qv.y, kv.y, acc[u]);
+          acc[u] = fmaf(qv.z, kv.z, acc[u]);
+          acc[u] = fmaf(qv.w, kv.w, acc[u]);
         }
-        a *= bt[s];
       }
-      A[e] = a;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int t = 4 * w + u;
+        float a = 0.0f;
+        if (s <= t && t < Ce) {
+          a = acc[u];
+          if constexpr (!DIAG) a *= expf(lam[t] - lam[s]);
+          a *= bt[s];
+        }
+        A[t * C + s] = a;
+      }
     }
     __syncthreads();
     // ---- outputs: state read + intra-chunk output
