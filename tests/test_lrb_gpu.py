@@ -22,6 +22,7 @@ CASES = [
     (4, 64, 16, 64, 0, "scalar", "yoked", "bdr", 7, 6),
     (8, 128, 32, 128, 1, "diagonal", "yoked", "bdr", 5, 7),
     (4, 128, 16, 32, 1, "diagonal", "persistent", "nearest", 3, 12),
+    (4, 128, 4096, 32, 1, "scalar", "persistent", "bdr", 2, 4),   # the largest Dv
 ]
 
 

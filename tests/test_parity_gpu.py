@@ -227,3 +227,29 @@ def test_state_norms(bits, dk, dv, group, T):
     S = torch.from_numpy(S0).cuda()
     Q.fp32_sq_norms(cfg, S, out)
     assert np.allclose(out.cpu().numpy(), O.fp32_sq_norms(P.oracle_cfg(cfg), S0), rtol=1e-12, atol=0.0)
+
+
+@pytest.mark.parametrize("bits,dk,policy,rounding", [(4, 128, "dynamic", "bdr"), (8, 64, "yoked", "nearest")])
+def test_maximum_dv(bits, dk, policy, rounding):
+    """The largest supported value dimension (Dv = 4096) on a few tiles."""
+    rng = np.random.default_rng(bits + dk)
+    T, dv = 3, 4096
+    cfg = Config(T, dk, dv, bits, 32, 1, "scalar", policy, rounding)
+    S0 = (rng.standard_normal((T, dv, dk)) * 0.3).astype(np.float32)
+    steps = P.random_steps(rng, T, dk, dv, "scalar", 2)
+    rep = P.lockstep(cfg, S0, steps, label=f"dv4096-int{bits}-{policy}")
+    assert rep.code_flips == 0
+
+
+def test_many_tiles_sampled():
+    """300,000 tiles (the row-block sequence far past one grid's worth of
+    warps, ragged against it), checked on sampled tiles including the last."""
+    rng = np.random.default_rng(17)
+    T, dk, dv = 300_000, 64, 16
+    cfg = Config(T, dk, dv, 4, 32, 1, "diagonal", "persistent", "bdr")
+    S0 = (rng.standard_normal((T, dv, dk)) * 0.3).astype(np.float32)
+    steps = P.random_steps(rng, T, dk, dv, "diagonal", 2)
+    tiles = np.sort(rng.choice(T, size=24, replace=False))
+    tiles[-1] = T - 1
+    rep = P.lockstep(cfg, S0, steps, tiles=tiles, label="300k tiles")
+    assert rep.code_flips == 0
