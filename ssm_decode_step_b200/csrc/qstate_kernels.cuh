@@ -1,6 +1,6 @@
 // Shared pieces of the quantized-state kernels (sm_100a): the element-level
-// arithmetic of the decode step, and the readout and quantization-start
-// kernels.  The step kernel itself is in qstate_step.cuh.
+// arithmetic of the decode step and the quantization-start kernel.  The
+// step and readout kernels are in qstate_step.cuh.
 //
 // The operation (LinQuant eq. (1) with readout o = S q, group-wise INT4/INT8
 // state, dynamic / persistent / yoked scales, nearest or Bounded Directional
@@ -24,8 +24,7 @@
 // a byte permute into the mantissa of 2^23 (exact) and rounded by adding
 // 1.5 * 2^23 inside one fused multiply-add (exact product, ties to even).
 //
-// The readout kernel stages work units of rb rows through a cp.async ring
-// per CTA.  No kernel here spins on a flag or barrier: the only waits are
+// No kernel here spins on a flag or barrier: the only waits are
 // cp.async.wait_group, __syncthreads and __syncwarp, so nothing can hang.
 #pragma once
 
@@ -40,18 +39,9 @@ namespace qs {
 #endif
 constexpr int kThreads = QS_THREADS;
 
-// Resident CTAs per SM the register allocation targets (kThreads each);
-// the yoked kernel is held to fewer by its shared memory and gets more
-// registers instead.
+// Resident CTAs per SM the register allocation targets (kThreads each).
 #ifndef QS_MIN_BLOCKS
 #define QS_MIN_BLOCKS 4
-#endif
-#ifndef QS_MIN_BLOCKS_YOKED
-#define QS_MIN_BLOCKS_YOKED 3
-#endif
-// cp.async ring depth of the readout kernel.
-#ifndef QS_STAGES
-#define QS_STAGES 4
 #endif
 
 // 1.5 * 2^23: adding it to a float of magnitude < 2^22 leaves the nearest
@@ -165,7 +155,7 @@ __device__ __forceinline__ float div_qmax_rn(float m) {
 }
 
 // ---------------------------------------------------------------------------
-// work units and the shared-memory stage layout (identical on host and device)
+// staged vectors (layout identical on host and device)
 // ---------------------------------------------------------------------------
 
 __host__ __device__ __forceinline__ int align_up(int x, int a) { return (x + a - 1) / a * a; }
@@ -174,79 +164,8 @@ __host__ __device__ __forceinline__ int align_up(int x, int a) { return (x + a -
 // LPR chunks of a row start in different banks).
 constexpr int kChunkStride = 36;
 
-struct StageLayout {
-  int codes, scales, v, k, q, a, sk, misc, shadow, bytes;
-
-  __host__ __device__ StageLayout(int bits, int dk, int rb, int group, bool diag, bool bdr,
-                                  bool yoked) {
-    const int vec = (dk / 32) * kChunkStride * 4;
-    int off = 0;
-    codes = off;  off = align_up(off + rb * dk * bits / 8, 16);
-    scales = off; off = align_up(off + rb * (dk / group) * 4, 16);
-    v = off;      off = align_up(off + rb * 4, 16);
-    k = off;      off += vec;
-    q = off;      off += vec;
-    a = off;      off += diag ? vec : 0;
-    sk = off;     off += bdr ? vec : 0;
-    misc = off;   off += 16;
-    shadow = off; off += yoked ? rb * dk * 4 : 0;
-    bytes = align_up(off, 128);
-  }
-};
-
 // 16-byte unit i of a staged Dk vector lands in chunk i/8 at the padded stride.
 __device__ __forceinline__ int vec_unit_offset(int i) { return (i >> 3) * (kChunkStride * 4) + (i & 7) * 16; }
-
-// Issue the cp.async copies of one work unit into a stage.
-template <int BITS, int DK, bool DIAG, bool YOKED, bool WITH_STATE_UPDATE>
-__device__ __forceinline__ void stage_load(unsigned char* st, const StageLayout& L,
-                                           const StepParams& p, const UnitCursor& u) {
-  constexpr int VU = DK / 4;  // 16-byte units per Dk vector
-  const int tid = threadIdx.x;
-  const int rb = p.rb;
-  const size_t tile = static_cast<size_t>(u.tile);
-  const size_t row0 = u.row0(p);
-  const int ng = DK / p.group;
-  {
-    const int n16 = rb * DK * BITS / 128;
-    const uint8_t* g = p.codes + row0 * (DK * BITS / 8);
-    for (int i = tid; i < n16; i += kThreads) cp_async16(st + L.codes + 16 * i, g + 16 * i);
-  }
-  {
-    const int n16 = rb * ng / 4;
-    const float* g = p.scales + row0 * ng;
-    for (int i = tid; i < n16; i += kThreads) cp_async16(st + L.scales + 16 * i, g + 4 * i);
-  }
-  // the per-tile vectors k, q, alpha (diagonal): one 16-byte unit per thread
-  for (int i = tid; i < 3 * VU; i += kThreads) {
-    const int which = i / VU, u = i % VU;
-    if (which == 0) {
-      if (WITH_STATE_UPDATE) cp_async16(st + L.k + vec_unit_offset(u), p.k + tile * DK + 4 * u);
-    } else if (which == 1) {
-      if (p.o != nullptr) cp_async16(st + L.q + vec_unit_offset(u), p.q + tile * DK + 4 * u);
-    } else {
-      if (WITH_STATE_UPDATE && DIAG) cp_async16(st + L.a + vec_unit_offset(u), p.alpha + tile * DK + 4 * u);
-    }
-  }
-  if constexpr (WITH_STATE_UPDATE) {
-    for (int i = tid; i < rb / 4; i += kThreads) cp_async16(st + L.v + 16 * i, p.v + row0 + 4 * i);
-    if (tid == kThreads - 1) {
-      float* misc = reinterpret_cast<float*>(st + L.misc);
-      if constexpr (!DIAG) cp_async4(misc + 0, p.alpha + tile);
-      cp_async4(misc + 1, p.beta + tile);
-    }
-  }
-  if constexpr (YOKED) {
-    // 16-byte unit u of local row-chunk rc lands at unit position u ^ (rc & 7)
-    // so that the 8 lanes of a quarter-warp read 8 different bank groups.
-    const int n16 = rb * DK / 4;
-    const float* g = p.shadow + row0 * DK;
-    for (int i = tid; i < n16; i += kThreads) {
-      const int rc = i >> 3, u = i & 7;
-      cp_async16(st + L.shadow + rc * 128 + 16 * (u ^ (rc & 7)), g + 4 * i);
-    }
-  }
-}
 
 // Load a staged Dk vector's chunk c as 16 pairs (2m, 2m+1).
 __device__ __forceinline__ void load_pairs(const unsigned char* base, int c, float2 (&v)[16]) {
@@ -407,63 +326,6 @@ __device__ __forceinline__ void bdr_chunk(float2 (&y)[16], const float2 (&d)[16]
       y[i].y = fminf(fmaxf(y[i].y, kOff - kQ), kOff + kQ);
     }
   }
-}
-
-// ---------------------------------------------------------------------------
-// readout of the stored state (no update): o = (c * s) . q
-// ---------------------------------------------------------------------------
-template <int BITS, int DK, int STAGES>
-__global__ void __launch_bounds__(kThreads, QS_MIN_BLOCKS) readout_kernel(StepParams p) {
-  constexpr int LPR = DK / 32;
-  constexpr int RP = kThreads / LPR;
-  constexpr int CW = BITS;
-  extern __shared__ __align__(128) unsigned char smem[];
-  const StageLayout L(BITS, DK, p.rb, p.group, false, false, false);
-  const int tid = threadIdx.x;
-  const int c = tid % LPR, r0 = tid / LPR;
-  const int ng = DK / p.group;
-  const int g = (32 * c) / p.group;
-  UnitCursor pre(blockIdx.x, p);
-#pragma unroll
-  for (int s = 0; s < STAGES - 1; ++s) {
-    if (pre.tile < p.tiles) stage_load<BITS, DK, false, false, false>(smem + s * L.bytes, L, p, pre);
-    cp_async_commit();
-    pre.advance(p);
-  }
-  int it = 0;
-  for (UnitCursor cur(blockIdx.x, p); cur.tile < p.tiles; cur.advance(p), ++it) {
-    if (pre.tile < p.tiles)
-      stage_load<BITS, DK, false, false, false>(smem + ((it + STAGES - 1) % STAGES) * L.bytes, L,
-                                                p, pre);
-    cp_async_commit();
-    pre.advance(p);
-    cp_async_wait<STAGES - 1>();
-    __syncthreads();
-    unsigned char* st = smem + (it % STAGES) * L.bytes;
-    const size_t grow0 = cur.row0(p);
-    float2 qq[16];
-    load_pairs(st + L.q, c, qq);
-#pragma unroll 1
-    for (int r = r0; r < p.rb; r += RP) {
-      uint32_t w[CW];
-      const uint4* src = reinterpret_cast<const uint4*>(st + L.codes + (r * LPR + c) * (4 * CW));
-#pragma unroll
-      for (int q = 0; q < CW / 4; ++q) {
-        const uint4 u = src[q];
-        w[4 * q + 0] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
-      }
-      const float s = reinterpret_cast<const float*>(st + L.scales)[r * ng + g];
-      float2 d[16];
-      decode_chunk<BITS>(w, d);
-      float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-      for (int m = 0; m < 16; ++m) acc = __ffma2_rn(__fmul2_rn(d[m], f2(s)), qq[m], acc);
-      const float o = row_tree<LPR>(acc);
-      if (c == 0) p.o[grow0 + r] = o;
-    }
-    __syncthreads();
-  }
-  cp_async_wait<0>();
 }
 
 // ---------------------------------------------------------------------------

@@ -11,23 +11,6 @@ namespace qs {
 template <int POLICY>
 constexpr int step_depth() { return POLICY == 2 ? QS_DEPTH_YOKED : QS_DEPTH; }
 
-// Rows per work unit of the readout kernel: the largest of QS_RB_MAX (64), 32,
-// 16 that divides dv and keeps one stage within `budget` bytes (so that three
-// or four CTAs fit per SM).
-#ifndef QS_RB_MAX
-#define QS_RB_MAX 64
-#endif
-inline int choose_rb(int bits, int dk, int dv, int group, bool diag, bool bdr, bool yoked) {
-  const int budget = yoked ? 21 * 1024 : 13 * 1024;
-  int best = 16;
-  for (int rb = QS_RB_MAX; rb >= 16; rb /= 2) {
-    if (dv % rb != 0) continue;
-    if (StageLayout(bits, dk, rb, group, diag, bdr, yoked).bytes <= budget) return rb;
-    best = rb;
-  }
-  return best;
-}
-
 // Allow the kernel the device's full opt-in shared memory (once per kernel).
 template <typename K>
 static cudaError_t allow_smem(K kernel, std::once_flag& flag) {
@@ -59,6 +42,21 @@ static cudaError_t launch_persistent(K kernel, size_t smem, const StepParams& p,
   return cudaGetLastError();
 }
 
+// Launch a one-warp-per-range kernel (step, Low-Rank Bypass step, readout):
+// as many CTAs as stay resident on all SMs, at most one warp per row block.
+template <typename K, typename P>
+static cudaError_t launch_warps(K kernel, const P& p, size_t smem, cudaStream_t stream) {
+  int per_sm = 0;
+  cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kStepThreads, smem);
+  if (err != cudaSuccess) return err;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  long long grid = static_cast<long long>(per_sm) * device_sm_count();
+  const long long need = (static_cast<long long>(p.nblocks) + kStepWarps - 1) / kStepWarps;
+  if (grid > need) grid = need;
+  kernel<<<static_cast<int>(grid), kStepThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
 template <int BITS, int DK, int POLICY, bool BDR, bool DELTA, bool DIAG>
 cudaError_t launch_step(const StepParams& p0, cudaStream_t stream) {
   constexpr int D = step_depth<POLICY>();
@@ -85,16 +83,7 @@ cudaError_t launch_step(const StepParams& p0, cudaStream_t stream) {
   p.ntv = (D - 1 + p.bpt - 1) / p.bpt + 1;
   const WarpLayout L(BITS, DK, DIAG, BDR, POLICY == 2);
   p.warp_bytes = L.bytes(D, p.ntv);
-  const size_t smem = static_cast<size_t>(p.warp_bytes) * WARPS;
-  int per_sm = 0;
-  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kStepThreads, smem);
-  if (err != cudaSuccess) return err;
-  if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  long long grid = static_cast<long long>(per_sm) * device_sm_count();
-  const long long need = (static_cast<long long>(p.nblocks) + WARPS - 1) / WARPS;
-  if (grid > need) grid = need;
-  kernel<<<static_cast<int>(grid), kStepThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_warps(kernel, p, static_cast<size_t>(p.warp_bytes) * WARPS, stream);
 }
 
 template <int BITS, int DK, int POLICY, bool BDR, bool DELTA, bool DIAG, bool MERGE>
@@ -112,16 +101,7 @@ cudaError_t launch_lrb(const LrbParams& p0, int tiles, int dv, cudaStream_t stre
   p.ntv = (D - 1 + p.bpt - 1) / p.bpt + 1;
   const LrbLayout L(BITS, DK, DIAG, POLICY == 2, MERGE, p.rank, p.rpad);
   p.warp_bytes = L.bytes(D, p.ntv);
-  const size_t smem = static_cast<size_t>(p.warp_bytes) * WARPS;
-  int per_sm = 0;
-  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kStepThreads, smem);
-  if (err != cudaSuccess) return err;
-  if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  long long grid = static_cast<long long>(per_sm) * device_sm_count();
-  const long long need = (static_cast<long long>(p.nblocks) + WARPS - 1) / WARPS;
-  if (grid > need) grid = need;
-  kernel<<<static_cast<int>(grid), kStepThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_warps(kernel, p, static_cast<size_t>(p.warp_bytes) * WARPS, stream);
 }
 
 template <int DK, bool DIAG>
@@ -137,16 +117,24 @@ cudaError_t launch_prefill(const PrefillParams& p, int tiles, cudaStream_t strea
 
 template <int BITS, int DK>
 cudaError_t launch_readout(const StepParams& p0, cudaStream_t stream) {
-  constexpr int S = 4;
-  auto kernel = readout_kernel<BITS, DK, S>;
+  constexpr int D = QS_DEPTH;
+  constexpr int RW = 32 / (DK / 32);
+  auto kernel = readout_kernel<BITS, DK, D>;
   static std::once_flag flag;
   cudaError_t err = allow_smem(kernel, flag);
   if (err != cudaSuccess) return err;
-  StepParams p = p0;
-  p.rb = choose_rb(BITS, DK, p.dv, p.group, false, false, false);
-  p.units_per_tile = p.dv / p.rb;
-  const StageLayout L(BITS, DK, p.rb, p.group, false, false, false);
-  return launch_persistent(kernel, static_cast<size_t>(S) * L.bytes, p, stream);
+  WarpStepParams p{};
+  p.codes = p0.codes;
+  p.scales = p0.scales;
+  p.q = p0.q;
+  p.o = p0.o;
+  p.bpt = p0.dv / RW;
+  p.nblocks = p0.tiles * p.bpt;
+  p.group = p0.group;
+  p.ntv = (D - 1 + p.bpt - 1) / p.bpt + 1;
+  const WarpLayout L(BITS, DK, false, false, false);
+  p.warp_bytes = L.bytes(D, p.ntv);
+  return launch_warps(kernel, p, static_cast<size_t>(p.warp_bytes) * kStepWarps, stream);
 }
 
 template <int BITS, int DK>

@@ -48,11 +48,6 @@ namespace qs {
 #endif
 constexpr int kStepWarps = QS_STEP_WARPS;
 constexpr int kStepThreads = 32 * kStepWarps;
-// Read k from shared memory at each use instead of keeping the tile's k
-// chunk in 32 registers (non-yoked kernels).
-#ifndef QS_K_SMEM
-#define QS_K_SMEM 0
-#endif
 // Resident warps per SM the register allocation targets.
 #ifndef QS_STEP_WARPS_PER_SM
 #define QS_STEP_WARPS_PER_SM 16
@@ -167,7 +162,7 @@ struct BlockCursor {
 // Issue the copies of row block cur.blk into ring slot cur.slot (ring16,
 // ring4, code8, shadow8: this lane's destinations in slot 0) and, at a tile
 // start, the tile's vectors into the warp's slot cur.tv.
-template <int BITS, int DK, bool DIAG, bool YOKED, int SLOT, int DEPTH>
+template <int BITS, int DK, bool DIAG, bool YOKED, int SLOT, int DEPTH, bool UPDATE = true>
 __device__ __forceinline__ void issue_block(const BlockCursor<SLOT, DEPTH>& cur, const WarpStepParams& p,
                                             const WarpLayout& L, uint32_t ring16, uint32_t ring4,
                                             uint32_t code8, uint32_t shadow8, uint32_t tvs, int lane,
@@ -190,14 +185,16 @@ __device__ __forceinline__ void issue_block(const BlockCursor<SLOT, DEPTH>& cur,
     const size_t t = cur.tile;
     if (lane < VU) {
       const uint32_t u = tv + static_cast<uint32_t>(vec_unit_offset(lane));
-      cp16<0>(u + L.k, p.k + t * DK + 4 * lane);
+      if constexpr (UPDATE) cp16<0>(u + L.k, p.k + t * DK + 4 * lane);
       if (readout) cp16<0>(u + L.q, p.q + t * DK + 4 * lane);
-      if constexpr (DIAG) cp16<0>(u + L.a, p.alpha + t * DK + 4 * lane);
+      if constexpr (UPDATE && DIAG) cp16<0>(u + L.a, p.alpha + t * DK + 4 * lane);
     }
-    if constexpr (!DIAG) {
+    if constexpr (UPDATE && !DIAG) {
       if (lane == 0) cp4<0>(tv + L.misc, p.alpha + t);
     }
-    if (lane == 1) cp4<4>(tv + L.misc, p.beta + t);
+    if constexpr (UPDATE) {
+      if (lane == 1) cp4<4>(tv + L.misc, p.beta + t);
+    }
   }
   // Every copy instruction below reads 512 consecutive bytes across the
   // warp: lane l copies the l-th 16-byte unit, which may belong to another
@@ -212,7 +209,7 @@ __device__ __forceinline__ void issue_block(const BlockCursor<SLOT, DEPTH>& cur,
     cp16<256>(code8 + cur.slot, cs + 512);
   }
   cp4<O_SCALES>(s4, scales_l + static_cast<size_t>(cur.blk) * sstride);
-  cp4<O_V>(s4, v_l + static_cast<size_t>(cur.blk) * RW);
+  if constexpr (UPDATE) cp4<O_V>(s4, v_l + static_cast<size_t>(cur.blk) * RW);
   if constexpr (YOKED) {
     // unit G = 32 i + lane is unit G & 7 of lane G >> 3's 128 bytes
     const uint32_t d = shadow8 + cur.slot;
@@ -303,8 +300,7 @@ __global__ void __launch_bounds__(kStepThreads, ((POLICY == 2 || BDR) ? QS_STEP_
     pre.advance(bpt, L.tv, tv_end);
   }
 
-  constexpr bool K_SMEM = QS_K_SMEM && !YOKED;
-  float2 kk[K_SMEM ? 1 : 16];
+  float2 kk[16];
   float beta = 0.0f, a_scalar = 1.0f;
 
 #pragma unroll 1
@@ -324,7 +320,7 @@ __global__ void __launch_bounds__(kStepThreads, ((POLICY == 2 || BDR) ? QS_STEP_
     if (cur.tile_start) {
       // every lane's copies of the tile vectors have landed: publish them
       __syncwarp();
-      if constexpr (!K_SMEM) load_pairs(tv + L.k, c, kk);
+      load_pairs(tv + L.k, c, kk);
       const float* misc = reinterpret_cast<const float*>(tv + L.misc);
       beta = misc[1];
       a_scalar = DIAG ? 1.0f : misc[0];
@@ -378,37 +374,18 @@ __global__ void __launch_bounds__(kStepThreads, ((POLICY == 2 || BDR) ? QS_STEP_
     }
 
     // ---- a3/a4: key projection and rank-1 write
-    const float4* kp4 = reinterpret_cast<const float4*>(tv + L.k) + c * (kChunkStride / 4);
     float wcoef;
     if constexpr (DELTA) {
       float2 acc = make_float2(0.0f, 0.0f);
-      if constexpr (K_SMEM) {
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const float4 t = kp4[m];
-          acc = __ffma2_rn(Sp[2 * m], make_float2(t.x, t.y), acc);
-          acc = __ffma2_rn(Sp[2 * m + 1], make_float2(t.z, t.w), acc);
-        }
-      } else {
-#pragma unroll
-        for (int m = 0; m < 16; ++m) acc = __ffma2_rn(Sp[m], kk[m], acc);
-      }
+      for (int m = 0; m < 16; ++m) acc = __ffma2_rn(Sp[m], kk[m], acc);
       wcoef = __fmul_rn(beta, __fsub_rn(v_i, row_tree<LPR>(acc)));
     } else {
       wcoef = __fmul_rn(beta, v_i);
     }
     float2 x[16];
-    if constexpr (K_SMEM) {
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const float4 t = kp4[m];
-        x[2 * m] = __ffma2_rn(f2(wcoef), make_float2(t.x, t.y), Sp[2 * m]);
-        x[2 * m + 1] = __ffma2_rn(f2(wcoef), make_float2(t.z, t.w), Sp[2 * m + 1]);
-      }
-    } else {
-#pragma unroll
-      for (int m = 0; m < 16; ++m) x[m] = __ffma2_rn(f2(wcoef), kk[m], Sp[m]);
-    }
+    for (int m = 0; m < 16; ++m) x[m] = __ffma2_rn(f2(wcoef), kk[m], Sp[m]);
 
     // ---- a5: readout from the updated state
     if (readout) {
@@ -520,6 +497,100 @@ __global__ void __launch_bounds__(kStepThreads, ((POLICY == 2 || BDR) ? QS_STEP_
     if constexpr (POLICY != 1) {
       if (writes_scale) scales_l[blk * sstride] = sp;
     }
+  }
+  cp_async_wait<0>();
+}
+
+// Readout of the stored state without changing it (qstate_readout):
+// o_i = d_i . q with d = c * s, on the step kernel's layout (row-block
+// ranges per warp, the ring carrying codes and scales, q once per tile).
+template <int BITS, int DK, int DEPTH>
+__global__ void __launch_bounds__(kStepThreads, QS_STEP_WARPS_PER_SM / kStepWarps)
+    readout_kernel(WarpStepParams p) {
+  constexpr int LPR = DK / 32;
+  constexpr int RW = 32 / LPR;
+  constexpr int CW = BITS;
+  constexpr int CB = 4 * BITS;
+  constexpr int WARPS = kStepWarps;
+  constexpr int O_SCALES = 32 * CB;
+  constexpr int O_V = O_SCALES + 128;
+  constexpr int SLOT = O_V + 128;
+
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int lane = threadIdx.x & 31;
+  const int warp = WARPS == 1 ? 0 : threadIdx.x >> 5;
+  const int c = lane % LPR, rr = lane / LPR;
+  const WarpLayout L(BITS, DK, false, false, false);
+  unsigned char* ring = smem + warp * p.warp_bytes;
+  unsigned char* tvs = ring + DEPTH * SLOT;
+  const uint32_t ring16 = smem_addr(ring) + 16 * lane;
+  const uint32_t ring4 = smem_addr(ring) + 4 * lane;
+  const uint32_t code8 = smem_addr(ring) + 512 * (lane & 1) + 16 * (lane >> 1);
+  const uint32_t tvs_s = smem_addr(tvs);
+  const int tv_end = p.ntv * L.tv;
+  const unsigned ng = DK / p.group;
+  const unsigned g = (32 * c) / p.group;
+
+  const long long gw = static_cast<long long>(blockIdx.x) * WARPS + warp;
+  const long long nw = static_cast<long long>(gridDim.x) * WARPS;
+  const unsigned b0 = static_cast<unsigned>(gw * p.nblocks / nw);
+  const unsigned b1 = static_cast<unsigned>((gw + 1) * p.nblocks / nw);
+  if (b0 >= b1) return;
+  const unsigned bpt = static_cast<unsigned>(p.bpt);
+  const uint8_t* codes_blk = p.codes + 16 * lane;
+  const unsigned sstride = RW * ng;
+  const float* scales_l = p.scales + rr * ng + g;
+  float* o_l = p.o + rr;
+
+  BlockCursor<SLOT, DEPTH> pre;
+  pre.blk = b0;
+  pre.tile = b0 / bpt;
+  pre.next_tile = (pre.tile + 1) * bpt;
+  pre.slot = 0;
+  pre.tv = 0;
+  pre.tile_start = true;
+  BlockCursor<SLOT, DEPTH> cur = pre;
+#pragma unroll
+  for (int i = 0; i < DEPTH - 1; ++i) {
+    if (pre.blk < b1)
+      issue_block<BITS, DK, false, false, SLOT, DEPTH, false>(pre, p, L, ring16, ring4, code8, 0u, tvs_s,
+                                                              lane, codes_blk, scales_l, sstride,
+                                                              nullptr, nullptr, true);
+    cp_async_commit();
+    pre.advance(bpt, L.tv, tv_end);
+  }
+  float2 qq[16];
+#pragma unroll 1
+  for (; cur.blk < b1; cur.advance(bpt, L.tv, tv_end)) {
+    if constexpr (CB == 32) __syncwarp();
+    if (pre.blk < b1)
+      issue_block<BITS, DK, false, false, SLOT, DEPTH, false>(pre, p, L, ring16, ring4, code8, 0u, tvs_s,
+                                                              lane, codes_blk, scales_l, sstride,
+                                                              nullptr, nullptr, true);
+    cp_async_commit();
+    pre.advance(bpt, L.tv, tv_end);
+    cp_async_wait<DEPTH - 1>();
+    if constexpr (CB == 32) __syncwarp();
+    const unsigned char* tv = tvs + cur.tv;
+    if (cur.tile_start) {
+      __syncwarp();
+      load_pairs(tv + L.q, c, qq);
+    }
+    const unsigned char* s = ring + cur.slot;
+    uint32_t w[CW];
+#pragma unroll
+    for (int h = 0; h < CW / 4; ++h) {
+      const uint4 u = reinterpret_cast<const uint4*>(s + h * 512)[lane];
+      w[4 * h + 0] = u.x; w[4 * h + 1] = u.y; w[4 * h + 2] = u.z; w[4 * h + 3] = u.w;
+    }
+    const float sc = reinterpret_cast<const float*>(s + O_SCALES)[lane];
+    float2 d[16];
+    decode_chunk<BITS>(w, d);
+    float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int m = 0; m < 16; ++m) acc = __ffma2_rn(__fmul2_rn(d[m], f2(sc)), qq[m], acc);
+    const float o = row_tree<LPR>(acc);
+    if (c == 0) o_l[static_cast<size_t>(cur.blk) * RW] = o;
   }
   cp_async_wait<0>();
 }
