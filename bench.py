@@ -894,12 +894,21 @@ def prefill_flops(dk: int, dv: int, L: int, C: int = 32) -> int:
     return f
 
 
+def prefill_bytes(dk: int, dv: int, L: int, diag: bool) -> int:
+    """Algorithmic HBM bytes of the prefill of one tile: q, k, v, alpha,
+    beta read, o written, the FP32 state read and written."""
+    return 4 * (L * (2 * dk + dv) + L * (dk if diag else 1) + L + L * dv + 2 * dv * dk)
+
+
 def run_prefill(args):
-    """Time qstate_prefill over `--prefill` tokens for every tile of the
+    """Time both prefill paths over `--prefill` tokens for every tile of the
     workload (inputs drawn from its laws, slot t mod P for token t), from a
-    zero state, with outputs.  Prints one JSON line: tokens/s and the
-    achieved FP32 rate against the FP32 FMA peak of the SMs (148 SMs x 128
-    lanes x 2 FLOPs x the SM clock sampled during the run)."""
+    zero state, with outputs: qstate_prefill (FP32 on the CUDA cores, against
+    the FP32 FMA peak of 148 SMs x 128 lanes x 2 FLOPs x the sampled SM
+    clock) and qstate_prefill_tf32 (tensor cores, against the measured HBM
+    copy bandwidth: its algorithmic bytes per launch / launch time, and its
+    contraction FLOPs against the TF32 tensor peak, taken as half the
+    measured bf16 peak, the nominal dense ratio).  Prints one JSON line."""
     import torch
     from ssm_decode_step_b200 import Config, qstate as Q
     w = W.get(args.workload)
@@ -916,31 +925,54 @@ def run_prefill(args):
     S = torch.zeros((T, w.dv, w.dk), dtype=torch.float32, device=dev)
     o = torch.empty((T, L, w.dv), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
-    for _ in range(args.warmup):
-        Q.prefill(cfg, L, S, q, k, v, a, b, o)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(torch.cuda.current_device()) as sampler:
-        e0.record(stream)
-        for _ in range(args.steps):
-            S.zero_()
-            Q.prefill(cfg, L, S, q, k, v, a, b, o)
-        e1.record(stream)
+    hbm_peak, hbm_src = load_peak()
+    try:
+        with open(PEAKS_FILE) as f:
+            tf32_peak, tf32_src = 0.5 * float(json.load(f)["bf16_tflops"]), "measured bf16 x 0.5"
+    except Exception:
+        tf32_peak, tf32_src = 0.5 * 1590.0, "fallback bf16 x 0.5"
+    out = {"experiment": "chunkwise prefill", "workload": w.description, "tiles": T,
+           "tokens_per_tile": L, "launches": args.steps,
+           "note": "the zeroing of S before every launch is inside the timed region (one memset)"}
+    before = Q.prefill_tf32_timeouts()
+    for name, fn in (("fp32", Q.prefill), ("tf32", Q.prefill_tf32)):
+        for _ in range(args.warmup):
+            fn(cfg, L, S, q, k, v, a, b, o)
         torch.cuda.synchronize()
-    clocks = sampler.summary()
-    sec = e0.elapsed_time(e1) / 1e3 / args.steps
-    flops = T * prefill_flops(w.dk, w.dv, L)
-    mhz = clocks.get("sm_mhz") or 1965
-    peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
-    print(json.dumps({
-        "experiment": "chunkwise prefill (qstate_prefill)", "workload": w.description,
-        "tiles": T, "tokens_per_tile": L, "launches": args.steps,
-        "ms_per_prefill": round(sec * 1e3, 4), "tokens_per_s": round(T * L / sec, 1),
-        "tflops": round(flops / sec / 1e12, 3), "fp32_peak_tflops": round(peak, 2),
-        "frac_of_fp32_peak": round(flops / sec / 1e12 / peak, 4), "bound": "alu",
-        "note": "FLOPs are the chunkwise algorithm's (prefill_flops); the zeroing of S between "
-                "launches is inside the timed region (one memset of the state)",
-        "clocks": clocks}))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(torch.cuda.current_device()) as sampler:
+            e0.record(stream)
+            for _ in range(args.steps):
+                S.zero_()
+                fn(cfg, L, S, q, k, v, a, b, o)
+            e1.record(stream)
+            torch.cuda.synchronize()
+        clocks = sampler.summary()
+        sec = e0.elapsed_time(e1) / 1e3 / args.steps
+        mhz = clocks.get("sm_mhz") or 1965
+        if name == "fp32":
+            flops = T * prefill_flops(w.dk, w.dv, L)
+            peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+            out[name] = {"kernel": "prefill_kernel (CUDA cores, FP32)", "ms_per_prefill": round(sec * 1e3, 4),
+                         "tokens_per_s": round(T * L / sec, 1), "tflops": round(flops / sec / 1e12, 3),
+                         "fp32_peak_tflops": round(peak, 2),
+                         "frac_of_fp32_peak": round(flops / sec / 1e12 / peak, 4), "bound": "alu",
+                         "flops": "prefill_flops (chunks of 32)", "clocks": clocks}
+        else:
+            flops = T * prefill_flops(w.dk, w.dv, L, C=64)
+            nbytes = T * prefill_bytes(w.dk, w.dv, L, w.decay == "diagonal")
+            gbs = nbytes / sec / 1e9
+            out[name] = {"kernel": "prefill_tc_kernel (tcgen05 TF32, accumulators in tensor memory)",
+                         "ms_per_prefill": round(sec * 1e3, 4), "tokens_per_s": round(T * L / sec, 1),
+                         "bytes_per_launch": nbytes, "gbs": round(gbs, 1), "hbm_peak_gbs": hbm_peak,
+                         "hbm_peak_source": hbm_src, "frac_of_hbm_peak": round(gbs / hbm_peak, 4),
+                         "bound": "hbm", "tflops": round(flops / sec / 1e12, 3),
+                         "tf32_peak_tflops": round(tf32_peak, 1), "tf32_peak_source": tf32_src,
+                         "frac_of_tf32_peak": round(flops / sec / 1e12 / tf32_peak, 4),
+                         "flops": "prefill_flops (chunks of 64)", "clocks": clocks,
+                         "speedup_vs_fp32": round(out["fp32"]["ms_per_prefill"] / (sec * 1e3), 2)}
+    out["tf32"]["timeouts"] = Q.prefill_tf32_timeouts() - before
+    print(json.dumps(out))
 
 
 def main():

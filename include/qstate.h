@@ -240,6 +240,27 @@ QS_API qs_status qstate_prefill(const qs_config* cfg, int length, float* S, cons
                                 const float* k, const float* v, const float* alpha,
                                 const float* beta, float* o, cudaStream_t stream);
 
+/* The same prefill with its four contractions on the tensor cores
+ * (tcgen05.mma, kind::tf32, FP32 accumulators in tensor memory; chunks of
+ * 64 tokens; the state stays in tensor memory for the whole sequence).
+ * The operands of every contraction are rounded to TF32 (10 explicit
+ * mantissa bits, round to nearest) and the state is read at TF32
+ * precision by the state read, so results agree with the FP32 recurrence
+ * to about 2^-10 of the magnitudes summed, not to FP32 rounding: every
+ * element of S and o is within 2^-8 of the same recurrence run on |S0|,
+ * |q|, |k|, |v| (the sum of the magnitudes of its terms).  Arguments,
+ * validation and the range condition on the decay are those of
+ * qstate_prefill, with S, q and k 16-byte aligned.  A wait for the tensor
+ * cores that does not end (a bounded poll) makes the CTA free its tensor
+ * memory and return; qstate_prefill_tf32_timeouts reports the count. */
+QS_API qs_status qstate_prefill_tf32(const qs_config* cfg, int length, float* S, const float* q,
+                                     const float* k, const float* v, const float* alpha,
+                                     const float* beta, float* o, cudaStream_t stream);
+
+/* Number of CTAs of qstate_prefill_tf32 whose wait for the tensor cores gave
+ * up since the library was loaded (current device; synchronous). */
+QS_API qs_status qstate_prefill_tf32_timeouts(unsigned int* count);
+
 /* Squared Frobenius norm of every tile of the stored state, for tracking
  * the state norm over a decode horizon (the norm inflation of per-token
  * dynamic scaling: "When Dynamic Scaling Fails", abstract and project page,

@@ -438,9 +438,14 @@ qs_status qstate_lrb_decode_step(const qs_config* cfg, int rank, int slot, void*
   return from_cuda(e);
 }
 
-qs_status qstate_prefill(const qs_config* cfg, int length, float* S, const float* q,
-                         const float* k, const float* v, const float* alpha, const float* beta,
-                         float* o, cudaStream_t stream) {
+namespace {
+
+// Validation shared by the two prefill paths; fills p and reports whether
+// there is work to launch.
+qs_status prefill_args(const qs_config* cfg, int length, float* S, const float* q, const float* k,
+                       const float* v, const float* alpha, const float* beta, float* o, uintptr_t align,
+                       qs_config* out, qs::PrefillParams* p, bool* work) {
+  *work = false;
   if (cfg == nullptr) return QS_ERR_INVALID_ARG;
   qs_config c = *cfg;
   c.bits = 8;
@@ -454,8 +459,8 @@ qs_status qstate_prefill(const qs_config* cfg, int length, float* S, const float
   if (c.num_tiles == 0 || length == 0) return QS_OK;
   const bool diag = c.decay == QS_DECAY_DIAGONAL;
   if (!S || !q || !k || !v || !alpha || !beta) return QS_ERR_INVALID_ARG;
-  if (!aligned(S, 4) || !aligned(q, 4) || !aligned(k, 4) || !aligned(v, 4) || !aligned(alpha, 4) ||
-      !aligned(beta, 4) || (o && !aligned(o, 4)))
+  if (!aligned(S, align) || !aligned(q, align) || !aligned(k, align) || !aligned(v, 4) ||
+      !aligned(alpha, 4) || !aligned(beta, 4) || (o && !aligned(o, 4)))
     return QS_ERR_INVALID_ARG;
   const size_t T = static_cast<size_t>(c.num_tiles), L = static_cast<size_t>(length);
   const Range w[2] = {range_of(S, T * c.dv * c.dk * 4), range_of(o, o ? T * L * c.dv * 4 : 0)};
@@ -463,22 +468,68 @@ qs_status qstate_prefill(const qs_config* cfg, int length, float* S, const float
                       range_of(v, T * L * c.dv * 4), range_of(alpha, T * L * (diag ? c.dk : 1) * 4),
                       range_of(beta, T * L * 4)};
   if (any_overlap(w, 2, r, 5)) return QS_ERR_INVALID_ARG;
+  p->S = S;
+  p->q = q;
+  p->k = k;
+  p->v = v;
+  p->alpha = alpha;
+  p->beta = beta;
+  p->o = o;
+  p->L = length;
+  p->dv = c.dv;
+  *out = c;
+  *work = true;
+  return QS_OK;
+}
+
+}  // namespace
+
+qs_status qstate_prefill(const qs_config* cfg, int length, float* S, const float* q,
+                         const float* k, const float* v, const float* alpha, const float* beta,
+                         float* o, cudaStream_t stream) {
+  qs_config c;
   qs::PrefillParams p;
-  p.S = S;
-  p.q = q;
-  p.k = k;
-  p.v = v;
-  p.alpha = alpha;
-  p.beta = beta;
-  p.o = o;
-  p.L = length;
-  p.dv = c.dv;
+  bool work;
+  const qs_status st = prefill_args(cfg, length, S, q, k, v, alpha, beta, o, 4, &c, &p, &work);
+  if (st != QS_OK || !work) return st;
+  const bool diag = c.decay == QS_DECAY_DIAGONAL;
   cudaError_t e;
   if (c.dk == 64)
     e = diag ? qs::launch_prefill<64, true>(p, c.num_tiles, stream) : qs::launch_prefill<64, false>(p, c.num_tiles, stream);
   else
     e = diag ? qs::launch_prefill<128, true>(p, c.num_tiles, stream) : qs::launch_prefill<128, false>(p, c.num_tiles, stream);
   return from_cuda(e);
+}
+
+// Tensor-memory waits of the TF32 prefill that gave up (per device).
+__device__ unsigned int qs_tc_timeouts = 0;
+
+qs_status qstate_prefill_tf32(const qs_config* cfg, int length, float* S, const float* q,
+                              const float* k, const float* v, const float* alpha, const float* beta,
+                              float* o, cudaStream_t stream) {
+  qs_config c;
+  qs::PrefillParams p;
+  bool work;
+  const qs_status st = prefill_args(cfg, length, S, q, k, v, alpha, beta, o, 16, &c, &p, &work);
+  if (st != QS_OK || !work) return st;
+  unsigned int* timeouts = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&timeouts), qs_tc_timeouts);
+  if (e != cudaSuccess) return from_cuda(e);
+  const bool diag = c.decay == QS_DECAY_DIAGONAL;
+  const int T = c.num_tiles;
+#define QS_TC(DK, M) (diag ? qs::launch_prefill_tc<DK, M, true>(p, T, timeouts, stream) \
+                           : qs::launch_prefill_tc<DK, M, false>(p, T, timeouts, stream))
+  if (c.dk == 64)
+    e = c.dv <= 64 ? QS_TC(64, 64) : QS_TC(64, 128);
+  else
+    e = c.dv <= 64 ? QS_TC(128, 64) : QS_TC(128, 128);
+#undef QS_TC
+  return from_cuda(e);
+}
+
+qs_status qstate_prefill_tf32_timeouts(unsigned int* count) {
+  if (count == nullptr) return QS_ERR_INVALID_ARG;
+  return from_cuda(cudaMemcpyFromSymbol(count, qs_tc_timeouts, sizeof(unsigned int)));
 }
 
 qs_status qstate_state_sq_norms(const qs_config* cfg, const void* codes, const float* scales,

@@ -137,6 +137,25 @@ cudaError_t launch_readout(const StepParams& p0, cudaStream_t stream) {
   return launch_warps(kernel, p, static_cast<size_t>(p.warp_bytes) * kStepWarps, stream);
 }
 
+template <int DK, int MDV, bool DIAG>
+cudaError_t launch_prefill_tc(const PrefillParams& p, int tiles, unsigned int* timeouts,
+                              cudaStream_t stream) {
+  auto kernel = prefill_tc_kernel<DK, MDV, DIAG>;
+  static std::once_flag flag;
+  cudaError_t err = allow_smem(kernel, flag);
+  if (err != cudaSuccess) return err;
+  const size_t smem = static_cast<size_t>(TcLayout(DK, DIAG).bytes());
+  int per_sm = 0;
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kTcThreads, smem);
+  if (err != cudaSuccess) return err;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  if (per_sm > 2) per_sm = 2;  // two 256-column tensor-memory allocations per SM
+  long long grid = static_cast<long long>(per_sm) * device_sm_count();
+  if (grid > tiles) grid = tiles;
+  kernel<<<static_cast<int>(grid), kTcThreads, smem, stream>>>(p, tiles, timeouts);
+  return cudaGetLastError();
+}
+
 template <int BITS, int DK>
 cudaError_t launch_init(const float* S0, uint8_t* codes, float* scales, float* shadow,
                         long long rows, int group, cudaStream_t stream) {
@@ -167,9 +186,14 @@ cudaError_t launch_init(const float* S0, uint8_t* codes, float* scales, float* s
   template cudaError_t launch_init<B, D>(const float*, uint8_t*, float*, float*, long long, int, \
                                          cudaStream_t);
 
+#define QS_INSTANTIATE_PREFILL_TC(D, M, DI) \
+  template cudaError_t launch_prefill_tc<D, M, DI>(const PrefillParams&, int, unsigned int*, cudaStream_t);
+
 #define QS_INSTANTIATE_PREFILL(D)                                                   \
   template cudaError_t launch_prefill<D, false>(const PrefillParams&, int, cudaStream_t); \
-  template cudaError_t launch_prefill<D, true>(const PrefillParams&, int, cudaStream_t);
+  template cudaError_t launch_prefill<D, true>(const PrefillParams&, int, cudaStream_t);  \
+  QS_INSTANTIATE_PREFILL_TC(D, 64, false) QS_INSTANTIATE_PREFILL_TC(D, 64, true)          \
+  QS_INSTANTIATE_PREFILL_TC(D, 128, false) QS_INSTANTIATE_PREFILL_TC(D, 128, true)
 
 #define QS_INSTANTIATE_LRB1(B, D, P, R, DE, DI, M) \
   template cudaError_t launch_lrb<B, D, P, R, DE, DI, M>(const LrbParams&, int, int, cudaStream_t);

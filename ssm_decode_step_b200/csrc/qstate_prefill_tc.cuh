@@ -1,0 +1,473 @@
+// Chunkwise prefill on the fifth-generation tensor cores (qstate_prefill_tc):
+// the same recurrence and regrouping as prefill_kernel (qstate_prefill.cuh),
+// with the four contractions of a chunk issued as tcgen05.mma in TF32 and
+// accumulated in FP32 in tensor memory (LinQuant, Low-Precision Chunkwise
+// Realization: local score, state read, intra-chunk output, state write;
+// the state pass is the FP32 decay of the accumulator).
+//
+// One CTA (4 warps) per tile at a time, persistent over tiles; chunks of
+// C = 64 tokens.  Tensor memory (256 columns per CTA):
+//   S   columns [0, Dk)     the FP32 state, row i of Dv in the lane of an
+//                           M = MDV accumulator; it stays there for the
+//                           whole sequence and is the A operand of the
+//                           state read (read from tensor memory)
+//   X   columns [128, 192)  local scores D[t][s] (M = 64), then the output
+//                           O^T[i][t] (M = MDV)
+//   VT  columns [192, 256)  v^T[i][s] (A operand of the intra-chunk output
+//                           and of the state write)
+// Shared memory holds the B operands (and the A operand of the scores) in
+// the K-major, unswizzled core-matrix layout: element (r, k) of an R x K
+// operand at byte (r/8)*32K + (k/4)*128 + (r%8)*16 + (k%4)*4.
+//
+// Per chunk, with Lam the running log-decay (inclusive; per channel under
+// diagonal decay) and m the chunk's middle token:
+//   scores  D[t][s] = sum_j Qs[t][j] Ks[s][j]          (M=64, N=64, K=Dk)
+//           Qs = q (scalar) or q e^{Lam_t - Lam_m}; Ks = k or k e^{Lam_m - Lam_s}
+//   A[t][s] = D[t][s] (e^{Lam_t - Lam_s} under scalar decay) beta_s, s <= t
+//   output  O^T[i][t] = sum_j S[i][j] Qb[t][j] + sum_s VT[i][s] A[t][s]
+//           Qb = q e^{Lam_t}                            (M=Dv, N=64)
+//   state   S <- S e^{Lam_C} (in place, FP32) then
+//           S[i][j] += sum_s VT[i][s] KbT[j][s],  KbT = beta_s k_s e^{Lam_C - Lam_s}
+//
+// Operands are rounded to TF32 (round to nearest, ties away) before they
+// are stored; the state operand of the state read is the FP32 accumulator,
+// which the tensor core reads at TF32 precision (low mantissa bits
+// dropped).  Every mbarrier wait is bounded: on a timeout the kernel counts
+// it in `timeouts`, frees its tensor memory and returns.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "qstate_prefill.cuh"
+
+namespace qs {
+
+constexpr int kTcChunk = 64;
+constexpr int kTcThreads = 128;
+constexpr int kTcCols = 256;
+constexpr int kTcColS = 0, kTcColX = 128, kTcColV = 192;
+// Shared memory per CTA is at least this, so that at most two CTAs (two
+// 256-column tensor-memory allocations) share an SM.
+constexpr int kTcMinSmem = 80 * 1024;
+// mbarrier polls before a wait gives up (each poll may suspend the thread
+// for a bounded, system-dependent time).
+constexpr long long kTcSpinLimit = 1ll << 22;
+
+struct TcLayout {
+  int qs, ks, qb, kbt, lam, beta, lamc, misc, total;
+  __host__ __device__ TcLayout(int dk, bool diag) {
+    constexpr int C = kTcChunk;
+    int off = 0;
+    qs = off;   off += C * dk * 4;   // A operand of the scores
+    ks = off;   off += C * dk * 4;   // B operand of the scores, then A[t][s]
+    qb = off;   off += C * dk * 4;   // B operand of the state read
+    kbt = off;  off += dk * C * 4;   // B operand of the state write
+    lam = off;  off += diag ? C * (dk + 4) * 4 : C * 4;  // Lam[t][j] (row stride dk+4) or Lam[t]
+    beta = off; off += C * 4;
+    lamc = off; off += diag ? 2 * dk * 4 : 16;           // Lam_C and e^{Lam_C} per channel
+    misc = off; off += 16;                               // mbarrier, tensor-memory base
+    total = off;
+  }
+  __host__ __device__ int bytes() const { return total > kTcMinSmem ? total : kTcMinSmem; }
+};
+
+namespace tc {
+
+__device__ __forceinline__ uint32_t saddr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// byte offset of element (r, k) of a K-major operand with K columns
+__device__ __forceinline__ uint32_t cm_off(int r, int k, int K) {
+  return static_cast<uint32_t>((r >> 3) * (K * 32) + (k >> 2) * 128 + (r & 7) * 16 + (k & 3) * 4);
+}
+
+// Shared-memory matrix descriptor, K-major without swizzle: start address,
+// 128 bytes between the two core matrices of one MMA's K step (leading
+// byte offset), sbo bytes between 8-row groups (stride byte offset),
+// descriptor version 1.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t sbo) {
+  uint64_t d = static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(128u >> 4) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;
+}
+
+// Instruction descriptor: FP32 accumulator, TF32 A and B, both K-major.
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d),
+      "r"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t mbar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+               : "memory");
+}
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_init(uint32_t mbar) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(mbar) : "memory");
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// Wait for the phase with the given parity to complete; false after
+// kTcSpinLimit polls.
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
+  for (long long i = 0; i < kTcSpinLimit; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(mbar), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ float tf32(float x) {
+  uint32_t y;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(y) : "f"(x));
+  return __uint_as_float(y);
+}
+
+// 16 consecutive columns of this warp's 32 lanes (one register per column).
+__device__ __forceinline__ void tm_ld16(uint32_t addr, float (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];"
+      : "=f"(r[0]), "=f"(r[1]), "=f"(r[2]), "=f"(r[3]), "=f"(r[4]), "=f"(r[5]), "=f"(r[6]),
+        "=f"(r[7]), "=f"(r[8]), "=f"(r[9]), "=f"(r[10]), "=f"(r[11]), "=f"(r[12]), "=f"(r[13]),
+        "=f"(r[14]), "=f"(r[15])
+      : "r"(addr));
+}
+__device__ __forceinline__ void tm_st16(uint32_t addr, const float (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(addr),
+      "f"(r[0]), "f"(r[1]), "f"(r[2]), "f"(r[3]), "f"(r[4]), "f"(r[5]), "f"(r[6]), "f"(r[7]),
+      "f"(r[8]), "f"(r[9]), "f"(r[10]), "f"(r[11]), "f"(r[12]), "f"(r[13]), "f"(r[14]), "f"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void st_shared4(unsigned char* base, uint32_t off, float a, float b, float c,
+                                           float d) {
+  *reinterpret_cast<float4*>(base + off) = make_float4(a, b, c, d);
+}
+
+}  // namespace tc
+
+// Row of an M-row accumulator held by lane `lane` of warp `warp`: M = 128
+// puts row r in lane r; M = 64 puts rows 16w .. 16w+15 in lanes 32w .. 32w+15.
+template <int M>
+__device__ __forceinline__ int tc_row(int warp, int lane) {
+  return M == 128 ? 32 * warp + lane : (lane < 16 ? 16 * warp + lane : -1);
+}
+
+template <int DK, int MDV, bool DIAG>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    prefill_tc_kernel(PrefillParams p, int tiles, unsigned int* timeouts) {
+  using namespace tc;
+  constexpr int C = kTcChunk;
+  constexpr int LS = DK + 4;  // row stride of the diagonal-decay Lam table
+  static_assert(DK == 64 || DK == 128, "Dk");
+  static_assert(MDV == 64 || MDV == 128, "accumulator rows");
+  extern __shared__ __align__(1024) unsigned char tsm[];
+  const TcLayout Ly(DK, DIAG);
+  unsigned char* sQs = tsm + Ly.qs;
+  unsigned char* sKs = tsm + Ly.ks;  // then the scores A[t][s]
+  unsigned char* sQb = tsm + Ly.qb;
+  unsigned char* sKbT = tsm + Ly.kbt;
+  float* lam = reinterpret_cast<float*>(tsm + Ly.lam);
+  float* bt = reinterpret_cast<float*>(tsm + Ly.beta);
+  float* lamc = reinterpret_cast<float*>(tsm + Ly.lamc);  // [0, DK): Lam_C; [DK, 2DK): e^{Lam_C}
+  uint64_t* mbar_p = reinterpret_cast<uint64_t*>(tsm + Ly.misc);
+  volatile uint32_t* tslot = reinterpret_cast<volatile uint32_t*>(tsm + Ly.misc + 8);
+  volatile int* failed = reinterpret_cast<volatile int*>(tsm + Ly.misc + 12);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int dv = p.dv;
+  const uint32_t mbar = saddr(mbar_p);
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     saddr(const_cast<uint32_t*>(tslot))),
+                 "r"(kTcCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (tid == 0) {
+    mbar_init(mbar);
+    *failed = 0;
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tbase = *tslot;
+  const uint32_t tw = tbase + (static_cast<uint32_t>(32 * warp) << 16);  // this warp's lanes
+  uint32_t phase = 0;
+  const int irow = tc_row<MDV>(warp, lane);      // state / output row of this lane
+  const bool ivalid = irow >= 0 && irow < dv;
+  const int trow = tc_row<64>(warp, lane);       // score row of this lane
+
+  // Issue-side helper: wait for the MMAs committed last; on a timeout every
+  // thread leaves through `done`.
+  auto wait_mma = [&]() -> bool {
+    if (!mbar_wait(mbar, phase)) *failed = 1;
+    phase ^= 1u;
+    __syncthreads();
+    fence_after();
+    return *failed == 0;
+  };
+
+  for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+    // ---- initial state into tensor memory
+    {
+      const float* src = p.S + (static_cast<size_t>(tile) * dv + (ivalid ? irow : 0)) * DK;
+#pragma unroll 1
+      for (int c = 0; c < DK; c += 16) {
+        float r[16];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 x = ivalid ? __ldg(reinterpret_cast<const float4*>(src + c) + u)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+          r[4 * u] = x.x; r[4 * u + 1] = x.y; r[4 * u + 2] = x.z; r[4 * u + 3] = x.w;
+        }
+        tm_st16(tw + kTcColS + c, r);
+      }
+      wait_st();
+    }
+
+#pragma unroll 1
+    for (int c0 = 0; c0 < p.L; c0 += C) {
+      const int Ce = min(C, p.L - c0);
+      const size_t tok0 = static_cast<size_t>(tile) * p.L + c0;
+      // previous chunk's readers of lam / beta / KbT are done (the state
+      // write it fed has completed)
+      __syncthreads();
+
+      // ---- beta and the running log-decay
+      if (tid < C) bt[tid] = tid < Ce ? p.beta[tok0 + tid] : 0.0f;
+      if constexpr (DIAG) {
+        for (int j = tid; j < DK; j += kTcThreads) {
+          float acc = 0.0f;
+#pragma unroll 4
+          for (int t = 0; t < C; ++t) {
+            if (t < Ce) acc += logf(p.alpha[(tok0 + t) * DK + j]);
+            lam[t * LS + j] = acc;
+          }
+          lamc[j] = acc;
+          lamc[DK + j] = expf(acc);
+        }
+      } else {
+        if (warp == 0) {
+          float x0 = lane < Ce ? logf(p.alpha[tok0 + lane]) : 0.0f;
+          float x1 = 32 + lane < Ce ? logf(p.alpha[tok0 + 32 + lane]) : 0.0f;
+#pragma unroll
+          for (int d = 1; d < 32; d <<= 1) {
+            const float y0 = __shfl_up_sync(0xffffffffu, x0, d);
+            const float y1 = __shfl_up_sync(0xffffffffu, x1, d);
+            if (lane >= d) { x0 += y0; x1 += y1; }
+          }
+          x1 += __shfl_sync(0xffffffffu, x0, 31);
+          lam[lane] = x0;
+          lam[32 + lane] = x1;
+          if (lane == 31) { lamc[0] = x1; lamc[1] = expf(x1); }
+        }
+      }
+      __syncthreads();
+
+      // ---- operands: Qs, Ks, Qb ([t][j], 8 tokens x 16 columns per warp step)
+      const int m = (Ce - 1) / 2;
+#pragma unroll 1
+      for (int it = warp; it < 8 * (DK / 16); it += 4) {
+        const int t = 8 * (it & 7) + (lane & 7);
+        const int j = 16 * (it >> 3) + 4 * (lane >> 3);
+        float4 qv = make_float4(0.f, 0.f, 0.f, 0.f), kv = qv;
+        if (t < Ce) {
+          qv = __ldg(reinterpret_cast<const float4*>(p.q + (tok0 + t) * DK + j));
+          kv = __ldg(reinterpret_cast<const float4*>(p.k + (tok0 + t) * DK + j));
+        }
+        const uint32_t o = cm_off(t, j, DK);
+        if constexpr (DIAG) {
+          const float4 lt = *reinterpret_cast<const float4*>(lam + t * LS + j);
+          const float4 lm = *reinterpret_cast<const float4*>(lam + m * LS + j);
+          st_shared4(sQs, o, tf32(qv.x * expf(lt.x - lm.x)), tf32(qv.y * expf(lt.y - lm.y)),
+                     tf32(qv.z * expf(lt.z - lm.z)), tf32(qv.w * expf(lt.w - lm.w)));
+          st_shared4(sKs, o, tf32(kv.x * expf(lm.x - lt.x)), tf32(kv.y * expf(lm.y - lt.y)),
+                     tf32(kv.z * expf(lm.z - lt.z)), tf32(kv.w * expf(lm.w - lt.w)));
+          st_shared4(sQb, o, tf32(qv.x * expf(lt.x)), tf32(qv.y * expf(lt.y)), tf32(qv.z * expf(lt.z)),
+                     tf32(qv.w * expf(lt.w)));
+        } else {
+          const float e = expf(lam[t]);
+          st_shared4(sQs, o, tf32(qv.x), tf32(qv.y), tf32(qv.z), tf32(qv.w));
+          st_shared4(sKs, o, tf32(kv.x), tf32(kv.y), tf32(kv.z), tf32(kv.w));
+          st_shared4(sQb, o, tf32(qv.x * e), tf32(qv.y * e), tf32(qv.z * e), tf32(qv.w * e));
+        }
+      }
+      // ---- KbT[j][s] = beta_s k_sj e^{Lam_C - Lam_s} (8 channels x 16 tokens per warp step)
+#pragma unroll 1
+      for (int it = warp; it < (DK / 8) * (C / 16); it += 4) {
+        const int j = 8 * (it % (DK / 8)) + (lane & 7);
+        const int s = 16 * (it / (DK / 8)) + 4 * (lane >> 3);
+        float w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float kv = s + u < Ce ? __ldg(p.k + (tok0 + s + u) * DK + j) : 0.0f;
+          const float ld = DIAG ? lamc[j] - lam[(s + u) * LS + j] : lam[C - 1] - lam[s + u];
+          w[u] = tf32(kv * (bt[s + u] * expf(ld)));
+        }
+        st_shared4(sKbT, cm_off(j, s, C), w[0], w[1], w[2], w[3]);
+      }
+      // ---- VT[i][s] into tensor memory
+#pragma unroll 1
+      for (int s0 = 0; s0 < C; s0 += 16) {
+        float r[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          r[u] = (ivalid && s0 + u < Ce) ? tf32(__ldg(p.v + (tok0 + s0 + u) * dv + irow)) : 0.0f;
+        tm_st16(tw + kTcColV + s0, r);
+      }
+      fence_async_smem();
+      wait_st();
+      fence_before();
+      __syncthreads();
+
+      // ---- local scores
+      if (tid == 0) {
+        fence_after();
+        constexpr uint32_t id = idesc_tf32(64, C);
+#pragma unroll
+        for (int kk = 0; kk < DK / 8; ++kk)
+          mma_ss(tbase + kTcColX, sdesc(saddr(sQs) + 256 * kk, DK * 32), sdesc(saddr(sKs) + 256 * kk, DK * 32),
+                 id, kk > 0);
+        mma_commit(mbar);
+      }
+      if (!wait_mma()) goto done;
+
+      // ---- A[t][s] (into the Ks region: the scores have read it)
+#pragma unroll 1
+      for (int s0 = 0; s0 < C; s0 += 16) {
+        float r[16];
+        tm_ld16(tw + kTcColX + s0, r);
+        wait_ld();
+        if (trow >= 0) {
+          const int t = trow;
+#pragma unroll
+          for (int u = 0; u < 16; u += 4) {
+            float a[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int s = s0 + u + e;
+              float x = 0.0f;
+              if (s <= t && t < Ce) {
+                x = r[u + e];
+                if constexpr (!DIAG) x *= expf(lam[t] - lam[s]);
+                x *= bt[s];
+              }
+              a[e] = tf32(x);
+            }
+            st_shared4(sKs, cm_off(t, s0 + u, C), a[0], a[1], a[2], a[3]);
+          }
+        }
+      }
+      fence_async_smem();
+      fence_before();
+      __syncthreads();
+
+      // ---- outputs: state read + intra-chunk output, O^T in X
+      if (tid == 0) {
+        fence_after();
+        constexpr uint32_t id = idesc_tf32(MDV, C);
+#pragma unroll
+        for (int kk = 0; kk < DK / 8; ++kk)
+          mma_ts(tbase + kTcColX, tbase + kTcColS + 8 * kk, sdesc(saddr(sQb) + 256 * kk, DK * 32), id, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < C / 8; ++kk)
+          mma_ts(tbase + kTcColX, tbase + kTcColV + 8 * kk, sdesc(saddr(sKs) + 256 * kk, C * 32), id, 1u);
+        mma_commit(mbar);
+      }
+      if (!wait_mma()) goto done;
+#pragma unroll 1
+      for (int t0 = 0; t0 < C; t0 += 16) {
+        float r[16];
+        tm_ld16(tw + kTcColX + t0, r);
+        wait_ld();
+        if (ivalid && p.o != nullptr) {
+#pragma unroll
+          for (int u = 0; u < 16; ++u)
+            if (t0 + u < Ce) p.o[(tok0 + t0 + u) * dv + irow] = r[u];
+        }
+      }
+      // ---- state pass: S <- S e^{Lam_C} (the state read above has completed)
+#pragma unroll 1
+      for (int c = 0; c < DK; c += 16) {
+        float r[16];
+        tm_ld16(tw + kTcColS + c, r);
+        wait_ld();
+#pragma unroll
+        for (int u = 0; u < 16; ++u) r[u] *= DIAG ? lamc[DK + c + u] : lamc[1];
+        tm_st16(tw + kTcColS + c, r);
+      }
+      wait_st();
+      fence_before();
+      __syncthreads();
+      // ---- state write: S += VT KbT^T
+      if (tid == 0) {
+        fence_after();
+        constexpr uint32_t id = idesc_tf32(MDV, DK);
+#pragma unroll
+        for (int kk = 0; kk < C / 8; ++kk)
+          mma_ts(tbase + kTcColS, tbase + kTcColV + 8 * kk, sdesc(saddr(sKbT) + 256 * kk, C * 32), id, 1u);
+        mma_commit(mbar);
+      }
+      if (!wait_mma()) goto done;
+    }
+
+    // ---- final state out of tensor memory
+    {
+      float* dst = p.S + (static_cast<size_t>(tile) * dv + (ivalid ? irow : 0)) * DK;
+#pragma unroll 1
+      for (int c = 0; c < DK; c += 16) {
+        float r[16];
+        tm_ld16(tw + kTcColS + c, r);
+        wait_ld();
+        if (ivalid) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            reinterpret_cast<float4*>(dst + c)[u] = make_float4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
+        }
+      }
+      fence_before();
+    }
+  }
+
+done:
+  __syncthreads();
+  if (tid == 0 && *failed) atomicAdd(timeouts, 1u);
+  fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(kTcCols) : "memory");
+}
+
+}  // namespace qs

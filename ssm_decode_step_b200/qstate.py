@@ -25,7 +25,7 @@ QS_OK, QS_ERR_INVALID_ARG, QS_ERR_UNSUPPORTED, QS_ERR_CUDA = 0, 1, 2, 3
 # Every entry point that include/qstate.h declares.
 EXPORTS = ("qstate_query_sizes", "qstate_init", "qstate_decode_step", "qstate_readout",
            "qstate_fp32_decode_step", "qstate_lrb_query_sizes", "qstate_lrb_decode_step",
-           "qstate_prefill",
+           "qstate_prefill", "qstate_prefill_tf32", "qstate_prefill_tf32_timeouts",
            "qstate_state_sq_norms", "qstate_fp32_sq_norms",
            "qstate_selfcheck", "qstate_status_string", "qstate_version")
 
@@ -63,12 +63,14 @@ def lib() -> ctypes.CDLL:
         L.qstate_lrb_query_sizes.argtypes = [C, ctypes.c_int, sz, sz, sz]
         L.qstate_lrb_decode_step.argtypes = [C, ctypes.c_int, ctypes.c_int] + [P] * 15
         L.qstate_prefill.argtypes = [C, ctypes.c_int] + [P] * 8
+        L.qstate_prefill_tf32.argtypes = [C, ctypes.c_int] + [P] * 8
+        L.qstate_prefill_tf32_timeouts.argtypes = [P]
         L.qstate_state_sq_norms.argtypes = [C, P, P, P, P]
         L.qstate_fp32_sq_norms.argtypes = [C, P, P, P]
         for f in (L.qstate_query_sizes, L.qstate_init, L.qstate_decode_step, L.qstate_readout,
                   L.qstate_selfcheck, L.qstate_fp32_decode_step, L.qstate_state_sq_norms,
                   L.qstate_fp32_sq_norms, L.qstate_lrb_query_sizes, L.qstate_lrb_decode_step,
-                  L.qstate_prefill):
+                  L.qstate_prefill, L.qstate_prefill_tf32, L.qstate_prefill_tf32_timeouts):
             f.restype = ctypes.c_int
         L.qstate_status_string.argtypes = [ctypes.c_int]
         L.qstate_status_string.restype = ctypes.c_char_p
@@ -221,6 +223,22 @@ def prefill(cfg: Config, length: int, S, q, k, v, alpha, beta, o=None, stream=No
     _check(lib().qstate_prefill(ctypes.byref(cc), length, _ptr(S), _ptr(q), _ptr(k), _ptr(v),
                                 _ptr(alpha), _ptr(beta), _ptr(o), _stream(stream)),
            "qstate_prefill")
+
+
+def prefill_tf32(cfg: Config, length: int, S, q, k, v, alpha, beta, o=None, stream=None) -> None:
+    """The same prefill on the tensor cores (TF32 operands, FP32 accumulators);
+    S, q and k 16-byte aligned."""
+    cc = cfg.c()
+    _check(lib().qstate_prefill_tf32(ctypes.byref(cc), length, _ptr(S), _ptr(q), _ptr(k), _ptr(v),
+                                     _ptr(alpha), _ptr(beta), _ptr(o), _stream(stream)),
+           "qstate_prefill_tf32")
+
+
+def prefill_tf32_timeouts() -> int:
+    """CTAs of prefill_tf32 whose bounded wait for the tensor cores gave up."""
+    n = ctypes.c_uint(0)
+    _check(lib().qstate_prefill_tf32_timeouts(ctypes.byref(n)), "qstate_prefill_tf32_timeouts")
+    return n.value
 
 
 def state_sq_norms(cfg: Config, codes, scales, out, stream=None) -> None:

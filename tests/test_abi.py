@@ -178,6 +178,27 @@ def test_prefill_validation():
     assert pre(_cfg(delta=0), 0, S=None) == Q.QS_OK
 
 
+def test_prefill_tf32_validation():
+    """The tensor-core prefill takes the same arguments as qstate_prefill and
+    also needs S, q and k 16-byte aligned (rejected before any launch)."""
+    lib = Q.lib()
+    pre = lambda cfg, L, **kw: lib.qstate_prefill_tf32(
+        ctypes.byref(cfg.c()), L, kw.get("S", A), kw.get("q", 2 * A), kw.get("k", 3 * A),
+        kw.get("v", 4 * A), kw.get("a", 5 * A), kw.get("b", 6 * A), kw.get("o", 7 * A), None)
+    assert pre(_cfg(delta=1), 8) == Q.QS_ERR_UNSUPPORTED
+    assert pre(_cfg(delta=0, dv=256), 8) == Q.QS_ERR_UNSUPPORTED
+    assert pre(_cfg(delta=0), -1) == Q.QS_ERR_INVALID_ARG
+    assert pre(_cfg(delta=0), 8, S=None) == Q.QS_ERR_INVALID_ARG
+    assert pre(_cfg(delta=0), 8, S=A + 4) == Q.QS_ERR_INVALID_ARG
+    assert pre(_cfg(delta=0), 8, q=2 * A + 8) == Q.QS_ERR_INVALID_ARG
+    assert pre(_cfg(delta=0), 8, k=3 * A + 4) == Q.QS_ERR_INVALID_ARG
+    assert pre(_cfg(delta=0), 8, o=A + 64) == Q.QS_ERR_INVALID_ARG
+    assert pre(_cfg(delta=0), 0, S=None) == Q.QS_OK
+    with pytest.raises(Q.QStateError):
+        lib_call = lib.qstate_prefill_tf32_timeouts(None)
+        Q._check(lib_call, "qstate_prefill_tf32_timeouts")
+
+
 def test_binding_raises():
     with pytest.raises(Q.QStateError):
         Q.query_sizes(_cfg(bits=5))

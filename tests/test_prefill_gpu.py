@@ -1,5 +1,6 @@
-"""GPU checks of the chunkwise prefill (qstate_prefill, delta = 0) against the
-oracle's token-by-token FP32 recurrence (qo_fp32_step per token).
+"""GPU checks of the chunkwise prefill (qstate_prefill and its tensor-core
+form qstate_prefill_tf32, delta = 0) against the oracle's token-by-token FP32
+recurrence (qo_fp32_step per token).
 
 The chunkwise form regroups the same sums, so the two agree to FP32 rounding
 rather than bit for bit.  Tolerance: every state element within 1e-4 of the
@@ -10,7 +11,16 @@ dk + 32 = 160 (1e-5), cancellation makes the error relative to the largest
 result a few times that, and the decay factors come from exp of running log
 sums instead of running products (a few ulp times |log decay|).  Observed
 worst case over these inputs: 2.6e-5 (the Mamba-2-shaped law, unnormalized
-keys); the assertion message reports it."""
+keys); the assertion message reports it.
+
+The tensor-core form rounds every operand to TF32 (relative error 2^-11 per
+operand, 2^-10 for the state, which the state read takes at TF32 precision
+by dropping mantissa bits), so each product carries at most about 2^-10 +
+2^-11 + 2^-11 = 2^-9 of its magnitude, and the FP32 accumulation adds
+n * 2^-24 (n <= 192).  Errors of the state carry into later chunks with the
+decay and stay relative to the magnitudes.  Bound checked: every element
+within 2^-8 of the same recurrence run on |S0|, |q|, |k|, |v| (the sum of
+the magnitudes of its terms), twice the estimate."""
 import numpy as np
 import pytest
 
@@ -20,6 +30,7 @@ from ssm_decode_step_b200 import Config, workloads as W
 pytestmark = pytest.mark.gpu
 
 TOL = 1e-4
+TOL_TF32 = 2.0 ** -8
 
 # (dk, dv, decay, tiles, length, with_o)
 CASES = [
@@ -101,3 +112,70 @@ def test_prefill_on_workload_laws(wname):
     o = torch.empty((T, L, w.dv), dtype=torch.float32, device="cuda")
     Q.prefill(cfg, L, S, dev(q), dev(k), dev(v), dev(a), dev(b), o)
     _check(S.cpu().numpy(), S_ref, o.cpu().numpy(), o_ref)
+
+
+TF32_CASES = [
+    (128, 64, "scalar", 13, 100, True),
+    (128, 128, "diagonal", 7, 77, True),
+    (64, 48, "scalar", 5, 32, True),
+    (64, 16, "diagonal", 3, 1, True),
+    (128, 32, "diagonal", 4, 33, False),
+    (64, 64, "scalar", 2, 257, True),
+    (128, 112, "scalar", 3, 64, True),
+    (64, 128, "diagonal", 2, 65, True),
+    (128, 128, "scalar", 300, 130, True),
+]
+
+
+def _check_bound(name, gpu, ref, mag):
+    err = np.abs(gpu.astype(np.float64) - ref)
+    bound = TOL_TF32 * mag.astype(np.float64) + 1e-30
+    worst = float((err / bound).max())
+    assert worst <= 1.0, f"{name}: worst error / bound {worst:.3g} (bound 2^-8 of magnitudes)"
+    return worst
+
+
+@pytest.mark.parametrize("case", TF32_CASES, ids=_id)
+def test_prefill_tf32_within_bound(case):
+    import torch
+    from ssm_decode_step_b200 import qstate as Q
+    dk, dv, decay, T, L, with_o = case
+    rng = np.random.default_rng(7 * dk + dv + T + L)
+    S0 = (rng.standard_normal((T, dv, dk)) * 0.1).astype(np.float32)
+    q, k, v, a, b = _inputs(rng, T, L, dk, dv, decay)
+    S_ref, o_ref = _reference(T, dk, dv, decay, S0, q, k, v, a, b)
+    S_mag, o_mag = _reference(T, dk, dv, decay, np.abs(S0), np.abs(q), np.abs(k), np.abs(v), a, b)
+    cfg = Config(T, dk, dv, 8, 32, 0, decay)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    S = dev(S0)
+    o = torch.empty((T, L, dv), dtype=torch.float32, device="cuda") if with_o else None
+    before = Q.prefill_tf32_timeouts()
+    Q.prefill_tf32(cfg, L, S, dev(q), dev(k), dev(v), dev(a), dev(b), o)
+    torch.cuda.synchronize()
+    assert Q.prefill_tf32_timeouts() == before
+    _check_bound("state", S.cpu().numpy(), S_ref, S_mag)
+    if with_o:
+        _check_bound("outputs", o.cpu().numpy(), o_ref, o_mag)
+
+
+@pytest.mark.parametrize("wname", ["mamba2", "gla"])
+def test_prefill_tf32_on_workload_laws(wname):
+    """The Mamba-2- and GLA-shaped laws (64 tiles, 256 tokens from a zero
+    state), the tensor-core form against the same bound."""
+    import torch
+    from ssm_decode_step_b200 import qstate as Q
+    w = W.scaled_down(W.get(wname), 64)
+    T, L = w.tiles, 256
+    slots = [W.slot(w, t) for t in range(L)]
+    q, k, v, a, b = (np.ascontiguousarray(np.stack([s[i] for s in slots], axis=1)) for i in range(5))
+    S0 = np.zeros((T, w.dv, w.dk), np.float32)
+    S_ref, o_ref = _reference(T, w.dk, w.dv, w.decay, S0, q, k, v, a, b)
+    S_mag, o_mag = _reference(T, w.dk, w.dv, w.decay, S0, np.abs(q), np.abs(k), np.abs(v), a, b)
+    cfg = Config(T, w.dk, w.dv, 8, 32, 0, w.decay)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    S = dev(S0)
+    o = torch.empty((T, L, w.dv), dtype=torch.float32, device="cuda")
+    Q.prefill_tf32(cfg, L, S, dev(q), dev(k), dev(v), dev(a), dev(b), o)
+    torch.cuda.synchronize()
+    _check_bound("state", S.cpu().numpy(), S_ref, S_mag)
+    _check_bound("outputs", o.cpu().numpy(), o_ref, o_mag)
