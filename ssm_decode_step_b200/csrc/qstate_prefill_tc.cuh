@@ -5,8 +5,11 @@
 // Realization: local score, state read, intra-chunk output, state write;
 // the state pass is the FP32 decay of the accumulator).
 //
-// One CTA (4 warps) per tile at a time, persistent over tiles; chunks of
-// C = 64 tokens.  Tensor memory (256 columns per CTA):
+// One CTA per tile at a time, persistent over tiles; chunks of C = 64
+// tokens; 8 warps, two per quadrant of tensor-memory lanes (each takes half
+// of the columns).  Each thread holds the next chunk's inputs in registers:
+// their loads are issued before the current chunk's contractions and land
+// while those and the epilogues run.  Tensor memory (256 columns per CTA):
 //   S   columns [0, Dk)     the FP32 state, row i of Dv in the lane of an
 //                           M = MDV accumulator; it stays there for the
 //                           whole sequence and is the A operand of the
@@ -28,6 +31,8 @@
 //           Qb = q e^{Lam_t}                            (M=Dv, N=64)
 //   state   S <- S e^{Lam_C} (in place, FP32) then
 //           S[i][j] += sum_s VT[i][s] KbT[j][s],  KbT = beta_s k_s e^{Lam_C - Lam_s}
+//           (KbT is formed from the staged Ks, so k is rounded to TF32 twice
+//           on this path)
 //
 // Operands are rounded to TF32 (round to nearest, ties away) before they
 // are stored; the state operand of the state read is the FP32 accumulator,
@@ -44,7 +49,7 @@
 namespace qs {
 
 constexpr int kTcChunk = 64;
-constexpr int kTcThreads = 128;
+constexpr int kTcThreads = 256;
 constexpr int kTcCols = 256;
 constexpr int kTcColS = 0, kTcColX = 128, kTcColV = 192;
 // Shared memory per CTA is at least this, so that at most two CTAs (two
@@ -177,21 +182,62 @@ __device__ __forceinline__ void st_shared4(unsigned char* base, uint32_t off, fl
 
 }  // namespace tc
 
-// Row of an M-row accumulator held by lane `lane` of warp `warp`: M = 128
-// puts row r in lane r; M = 64 puts rows 16w .. 16w+15 in lanes 32w .. 32w+15.
+// Row of an M-row accumulator held by lane `lane` of a warp of quadrant
+// qd (warp % 4): M = 128 puts row r in lane r; M = 64 puts rows
+// 16 qd .. 16 qd + 15 in lanes 32 qd .. 32 qd + 15.
 template <int M>
-__device__ __forceinline__ int tc_row(int warp, int lane) {
-  return M == 128 ? 32 * warp + lane : (lane < 16 ? 16 * warp + lane : -1);
+__device__ __forceinline__ int tc_row(int qd, int lane) {
+  return M == 128 ? 32 * qd + lane : (lane < 16 ? 16 * qd + lane : -1);
+}
+
+// One chunk's inputs held in registers by one thread: its Qs/Ks/Qb items
+// (8 tokens x 16 columns per warp step, a float4 of q and of k per lane),
+// its half of v^T's row, and the scalar decay and beta of one token.
+template <int DK>
+struct TcInputs {
+  static constexpr int IQ = DK / 16;
+  float4 q[IQ], k[IQ];
+  float v[kTcChunk / 2];
+  float a0, a1, b;
+};
+
+template <int DK>
+__device__ __forceinline__ void tc_load(TcInputs<DK>& in, const PrefillParams& p, size_t tok0, int Ce,
+                                        int warp, int lane, int irow, bool ivalid, bool diag) {
+  constexpr int C = kTcChunk;
+#pragma unroll
+  for (int i = 0; i < TcInputs<DK>::IQ; ++i) {
+    const int it = warp + 8 * i;
+    const int t = 8 * (it & 7) + (lane & 7);
+    const int j = 16 * (it >> 3) + 4 * (lane >> 3);
+    in.q[i] = in.k[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (t < Ce) {
+      in.q[i] = __ldg(reinterpret_cast<const float4*>(p.q + (tok0 + t) * DK + j));
+      in.k[i] = __ldg(reinterpret_cast<const float4*>(p.k + (tok0 + t) * DK + j));
+    }
+  }
+  const int s0 = (C / 2) * (warp >> 2);
+#pragma unroll
+  for (int u = 0; u < C / 2; ++u)
+    in.v[u] = (ivalid && s0 + u < Ce) ? __ldg(p.v + (tok0 + s0 + u) * p.dv + irow) : 0.0f;
+  in.a0 = in.a1 = 1.0f;
+  if (!diag && warp == 0) {
+    if (lane < Ce) in.a0 = __ldg(p.alpha + tok0 + lane);
+    if (32 + lane < Ce) in.a1 = __ldg(p.alpha + tok0 + 32 + lane);
+  }
+  const int tid = 32 * warp + lane;
+  in.b = tid < Ce ? __ldg(p.beta + tok0 + tid) : 0.0f;
 }
 
 template <int DK, int MDV, bool DIAG>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kTcThreads, DK == 64 ? 2 : 1)
     prefill_tc_kernel(PrefillParams p, int tiles, unsigned int* timeouts) {
   using namespace tc;
   constexpr int C = kTcChunk;
   constexpr int LS = DK + 4;  // row stride of the diagonal-decay Lam table
   static_assert(DK == 64 || DK == 128, "Dk");
   static_assert(MDV == 64 || MDV == 128, "accumulator rows");
+  static_assert(kTcThreads == 256, "8 warps: two per tensor-memory lane quadrant");
   extern __shared__ __align__(1024) unsigned char tsm[];
   const TcLayout Ly(DK, DIAG);
   unsigned char* sQs = tsm + Ly.qs;
@@ -206,6 +252,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   volatile int* failed = reinterpret_cast<volatile int*>(tsm + Ly.misc + 12);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qd = warp & 3;   // tensor-memory lane quadrant of this warp
+  const int half = warp >> 2;  // which half of the columns this warp takes
   const int dv = p.dv;
   const uint32_t mbar = saddr(mbar_p);
 
@@ -224,14 +272,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   fence_after();
   const uint32_t tbase = *tslot;
-  const uint32_t tw = tbase + (static_cast<uint32_t>(32 * warp) << 16);  // this warp's lanes
+  const uint32_t tw = tbase + (static_cast<uint32_t>(32 * qd) << 16);  // this warp's lanes
   uint32_t phase = 0;
-  const int irow = tc_row<MDV>(warp, lane);      // state / output row of this lane
+  const int irow = tc_row<MDV>(qd, lane);  // state / output row of this lane
   const bool ivalid = irow >= 0 && irow < dv;
-  const int trow = tc_row<64>(warp, lane);       // score row of this lane
+  const int trow = tc_row<64>(qd, lane);   // score row of this lane
+  const int nch = (p.L + C - 1) / C;
 
-  // Issue-side helper: wait for the MMAs committed last; on a timeout every
-  // thread leaves through `done`.
+  // wait for the MMAs committed last; on a timeout every thread leaves
   auto wait_mma = [&]() -> bool {
     if (!mbar_wait(mbar, phase)) *failed = 1;
     phase ^= 1u;
@@ -240,12 +288,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     return *failed == 0;
   };
 
-  for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-    // ---- initial state into tensor memory
-    {
+  int tile = blockIdx.x, ch = 0;
+  TcInputs<DK> in;
+  if (tile < tiles) tc_load<DK>(in, p, static_cast<size_t>(tile) * p.L, min(C, p.L), warp, lane, irow, ivalid, DIAG);
+
+  while (tile < tiles) {
+    const int c0 = ch * C;
+    const int Ce = min(C, p.L - c0);
+    const size_t tok0 = static_cast<size_t>(tile) * p.L + c0;
+
+    // ---- initial state of the tile into tensor memory (this warp's rows, half the columns)
+    if (ch == 0) {
       const float* src = p.S + (static_cast<size_t>(tile) * dv + (ivalid ? irow : 0)) * DK;
-#pragma unroll 1
-      for (int c = 0; c < DK; c += 16) {
+#pragma unroll
+      for (int c = half * (DK / 2); c < (half + 1) * (DK / 2); c += 16) {
         float r[16];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -257,198 +313,210 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       wait_st();
     }
+    // the previous chunk's readers of lam, beta and the operands are done
+    __syncthreads();
 
-#pragma unroll 1
-    for (int c0 = 0; c0 < p.L; c0 += C) {
-      const int Ce = min(C, p.L - c0);
-      const size_t tok0 = static_cast<size_t>(tile) * p.L + c0;
-      // previous chunk's readers of lam / beta / KbT are done (the state
-      // write it fed has completed)
-      __syncthreads();
+    // ---- beta and the running log-decay
+    if (tid < C) bt[tid] = in.b;
+    if constexpr (DIAG) {
+      for (int j = tid; j < DK; j += kTcThreads) {
+        float acc = 0.0f;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float x[C / 2];
+#pragma unroll
+          for (int u = 0; u < C / 2; ++u) {
+            const int t = (C / 2) * hh + u;
+            x[u] = t < Ce ? __ldg(p.alpha + (tok0 + t) * DK + j) : 1.0f;
+          }
+#pragma unroll
+          for (int u = 0; u < C / 2; ++u) {
+            acc += logf(x[u]);
+            lam[((C / 2) * hh + u) * LS + j] = acc;
+          }
+        }
+        lamc[j] = acc;
+        lamc[DK + j] = expf(acc);
+      }
+    } else {
+      if (warp == 0) {
+        float x0 = logf(in.a0), x1 = logf(in.a1);
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+          const float y0 = __shfl_up_sync(0xffffffffu, x0, d);
+          const float y1 = __shfl_up_sync(0xffffffffu, x1, d);
+          if (lane >= d) { x0 += y0; x1 += y1; }
+        }
+        x1 += __shfl_sync(0xffffffffu, x0, 31);
+        lam[lane] = x0;
+        lam[32 + lane] = x1;
+        if (lane == 31) { lamc[0] = x1; lamc[1] = expf(x1); }
+      }
+    }
+    __syncthreads();
 
-      // ---- beta and the running log-decay
-      if (tid < C) bt[tid] = tid < Ce ? p.beta[tok0 + tid] : 0.0f;
+    // ---- operands Qs, Ks, Qb from the registers
+    const int m = (Ce - 1) / 2;
+#pragma unroll
+    for (int i = 0; i < TcInputs<DK>::IQ; ++i) {
+      const int it = warp + 8 * i;
+      const int t = 8 * (it & 7) + (lane & 7);
+      const int j = 16 * (it >> 3) + 4 * (lane >> 3);
+      const float4 qv = in.q[i], kv = in.k[i];
+      const uint32_t o = cm_off(t, j, DK);
       if constexpr (DIAG) {
-        for (int j = tid; j < DK; j += kTcThreads) {
-          float acc = 0.0f;
-#pragma unroll 4
-          for (int t = 0; t < C; ++t) {
-            if (t < Ce) acc += logf(p.alpha[(tok0 + t) * DK + j]);
-            lam[t * LS + j] = acc;
-          }
-          lamc[j] = acc;
-          lamc[DK + j] = expf(acc);
-        }
+        const float4 lt = *reinterpret_cast<const float4*>(lam + t * LS + j);
+        const float4 lm = *reinterpret_cast<const float4*>(lam + m * LS + j);
+        st_shared4(sQs, o, tf32(qv.x * expf(lt.x - lm.x)), tf32(qv.y * expf(lt.y - lm.y)),
+                   tf32(qv.z * expf(lt.z - lm.z)), tf32(qv.w * expf(lt.w - lm.w)));
+        st_shared4(sKs, o, tf32(kv.x * expf(lm.x - lt.x)), tf32(kv.y * expf(lm.y - lt.y)),
+                   tf32(kv.z * expf(lm.z - lt.z)), tf32(kv.w * expf(lm.w - lt.w)));
+        st_shared4(sQb, o, tf32(qv.x * expf(lt.x)), tf32(qv.y * expf(lt.y)), tf32(qv.z * expf(lt.z)),
+                   tf32(qv.w * expf(lt.w)));
       } else {
-        if (warp == 0) {
-          float x0 = lane < Ce ? logf(p.alpha[tok0 + lane]) : 0.0f;
-          float x1 = 32 + lane < Ce ? logf(p.alpha[tok0 + 32 + lane]) : 0.0f;
-#pragma unroll
-          for (int d = 1; d < 32; d <<= 1) {
-            const float y0 = __shfl_up_sync(0xffffffffu, x0, d);
-            const float y1 = __shfl_up_sync(0xffffffffu, x1, d);
-            if (lane >= d) { x0 += y0; x1 += y1; }
-          }
-          x1 += __shfl_sync(0xffffffffu, x0, 31);
-          lam[lane] = x0;
-          lam[32 + lane] = x1;
-          if (lane == 31) { lamc[0] = x1; lamc[1] = expf(x1); }
-        }
+        const float e = expf(lam[t]);
+        st_shared4(sQs, o, tf32(qv.x), tf32(qv.y), tf32(qv.z), tf32(qv.w));
+        st_shared4(sKs, o, tf32(kv.x), tf32(kv.y), tf32(kv.z), tf32(kv.w));
+        st_shared4(sQb, o, tf32(qv.x * e), tf32(qv.y * e), tf32(qv.z * e), tf32(qv.w * e));
       }
-      __syncthreads();
-
-      // ---- operands: Qs, Ks, Qb ([t][j], 8 tokens x 16 columns per warp step)
-      const int m = (Ce - 1) / 2;
-#pragma unroll 1
-      for (int it = warp; it < 8 * (DK / 16); it += 4) {
-        const int t = 8 * (it & 7) + (lane & 7);
-        const int j = 16 * (it >> 3) + 4 * (lane >> 3);
-        float4 qv = make_float4(0.f, 0.f, 0.f, 0.f), kv = qv;
-        if (t < Ce) {
-          qv = __ldg(reinterpret_cast<const float4*>(p.q + (tok0 + t) * DK + j));
-          kv = __ldg(reinterpret_cast<const float4*>(p.k + (tok0 + t) * DK + j));
-        }
-        const uint32_t o = cm_off(t, j, DK);
-        if constexpr (DIAG) {
-          const float4 lt = *reinterpret_cast<const float4*>(lam + t * LS + j);
-          const float4 lm = *reinterpret_cast<const float4*>(lam + m * LS + j);
-          st_shared4(sQs, o, tf32(qv.x * expf(lt.x - lm.x)), tf32(qv.y * expf(lt.y - lm.y)),
-                     tf32(qv.z * expf(lt.z - lm.z)), tf32(qv.w * expf(lt.w - lm.w)));
-          st_shared4(sKs, o, tf32(kv.x * expf(lm.x - lt.x)), tf32(kv.y * expf(lm.y - lt.y)),
-                     tf32(kv.z * expf(lm.z - lt.z)), tf32(kv.w * expf(lm.w - lt.w)));
-          st_shared4(sQb, o, tf32(qv.x * expf(lt.x)), tf32(qv.y * expf(lt.y)), tf32(qv.z * expf(lt.z)),
-                     tf32(qv.w * expf(lt.w)));
-        } else {
-          const float e = expf(lam[t]);
-          st_shared4(sQs, o, tf32(qv.x), tf32(qv.y), tf32(qv.z), tf32(qv.w));
-          st_shared4(sKs, o, tf32(kv.x), tf32(kv.y), tf32(kv.z), tf32(kv.w));
-          st_shared4(sQb, o, tf32(qv.x * e), tf32(qv.y * e), tf32(qv.z * e), tf32(qv.w * e));
-        }
+    }
+    // ---- VT[i][s] into tensor memory (this warp's rows, half the tokens)
+#pragma unroll
+    for (int u = 0; u < C / 2; u += 16) {
+      float r[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) r[e] = tf32(in.v[u + e]);
+      tm_st16(tw + kTcColV + (C / 2) * half + u, r);
+    }
+    __syncthreads();  // Ks complete
+    // ---- KbT[j][s] = Ks[s][j] beta_s e^{Lam_C - Lam_s} / (e^{Lam_m - Lam_s} under diagonal decay)
+#pragma unroll
+    for (int i = 0; i < DK / 16; ++i) {
+      const int it = warp + 8 * i;
+      const int j = 8 * (it % (DK / 8)) + (lane & 7);
+      const int s = 16 * (it / (DK / 8)) + 4 * (lane >> 3);
+      float w[4];
+      if constexpr (DIAG) {
+        const float f = expf(lamc[j] - lam[m * LS + j]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          w[u] = tf32(*reinterpret_cast<const float*>(sKs + cm_off(s + u, j, DK)) * (f * bt[s + u]));
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          w[u] = tf32(*reinterpret_cast<const float*>(sKs + cm_off(s + u, j, DK)) *
+                      (bt[s + u] * expf(lam[C - 1] - lam[s + u])));
       }
-      // ---- KbT[j][s] = beta_s k_sj e^{Lam_C - Lam_s} (8 channels x 16 tokens per warp step)
-#pragma unroll 1
-      for (int it = warp; it < (DK / 8) * (C / 16); it += 4) {
-        const int j = 8 * (it % (DK / 8)) + (lane & 7);
-        const int s = 16 * (it / (DK / 8)) + 4 * (lane >> 3);
-        float w[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float kv = s + u < Ce ? __ldg(p.k + (tok0 + s + u) * DK + j) : 0.0f;
-          const float ld = DIAG ? lamc[j] - lam[(s + u) * LS + j] : lam[C - 1] - lam[s + u];
-          w[u] = tf32(kv * (bt[s + u] * expf(ld)));
-        }
-        st_shared4(sKbT, cm_off(j, s, C), w[0], w[1], w[2], w[3]);
-      }
-      // ---- VT[i][s] into tensor memory
-#pragma unroll 1
-      for (int s0 = 0; s0 < C; s0 += 16) {
-        float r[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u)
-          r[u] = (ivalid && s0 + u < Ce) ? tf32(__ldg(p.v + (tok0 + s0 + u) * dv + irow)) : 0.0f;
-        tm_st16(tw + kTcColV + s0, r);
-      }
-      fence_async_smem();
-      wait_st();
-      fence_before();
-      __syncthreads();
-
-      // ---- local scores
-      if (tid == 0) {
-        fence_after();
-        constexpr uint32_t id = idesc_tf32(64, C);
-#pragma unroll
-        for (int kk = 0; kk < DK / 8; ++kk)
-          mma_ss(tbase + kTcColX, sdesc(saddr(sQs) + 256 * kk, DK * 32), sdesc(saddr(sKs) + 256 * kk, DK * 32),
-                 id, kk > 0);
-        mma_commit(mbar);
-      }
-      if (!wait_mma()) goto done;
-
-      // ---- A[t][s] (into the Ks region: the scores have read it)
-#pragma unroll 1
-      for (int s0 = 0; s0 < C; s0 += 16) {
-        float r[16];
-        tm_ld16(tw + kTcColX + s0, r);
-        wait_ld();
-        if (trow >= 0) {
-          const int t = trow;
-#pragma unroll
-          for (int u = 0; u < 16; u += 4) {
-            float a[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int s = s0 + u + e;
-              float x = 0.0f;
-              if (s <= t && t < Ce) {
-                x = r[u + e];
-                if constexpr (!DIAG) x *= expf(lam[t] - lam[s]);
-                x *= bt[s];
-              }
-              a[e] = tf32(x);
-            }
-            st_shared4(sKs, cm_off(t, s0 + u, C), a[0], a[1], a[2], a[3]);
-          }
-        }
-      }
-      fence_async_smem();
-      fence_before();
-      __syncthreads();
-
-      // ---- outputs: state read + intra-chunk output, O^T in X
-      if (tid == 0) {
-        fence_after();
-        constexpr uint32_t id = idesc_tf32(MDV, C);
-#pragma unroll
-        for (int kk = 0; kk < DK / 8; ++kk)
-          mma_ts(tbase + kTcColX, tbase + kTcColS + 8 * kk, sdesc(saddr(sQb) + 256 * kk, DK * 32), id, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < C / 8; ++kk)
-          mma_ts(tbase + kTcColX, tbase + kTcColV + 8 * kk, sdesc(saddr(sKs) + 256 * kk, C * 32), id, 1u);
-        mma_commit(mbar);
-      }
-      if (!wait_mma()) goto done;
-#pragma unroll 1
-      for (int t0 = 0; t0 < C; t0 += 16) {
-        float r[16];
-        tm_ld16(tw + kTcColX + t0, r);
-        wait_ld();
-        if (ivalid && p.o != nullptr) {
-#pragma unroll
-          for (int u = 0; u < 16; ++u)
-            if (t0 + u < Ce) p.o[(tok0 + t0 + u) * dv + irow] = r[u];
-        }
-      }
-      // ---- state pass: S <- S e^{Lam_C} (the state read above has completed)
-#pragma unroll 1
-      for (int c = 0; c < DK; c += 16) {
-        float r[16];
-        tm_ld16(tw + kTcColS + c, r);
-        wait_ld();
-#pragma unroll
-        for (int u = 0; u < 16; ++u) r[u] *= DIAG ? lamc[DK + c + u] : lamc[1];
-        tm_st16(tw + kTcColS + c, r);
-      }
-      wait_st();
-      fence_before();
-      __syncthreads();
-      // ---- state write: S += VT KbT^T
-      if (tid == 0) {
-        fence_after();
-        constexpr uint32_t id = idesc_tf32(MDV, DK);
-#pragma unroll
-        for (int kk = 0; kk < C / 8; ++kk)
-          mma_ts(tbase + kTcColS, tbase + kTcColV + 8 * kk, sdesc(saddr(sKbT) + 256 * kk, C * 32), id, 1u);
-        mma_commit(mbar);
-      }
-      if (!wait_mma()) goto done;
+      st_shared4(sKbT, cm_off(j, s, C), w[0], w[1], w[2], w[3]);
     }
 
-    // ---- final state out of tensor memory
-    {
+    // ---- the next chunk's inputs: loads in flight while this chunk computes
+    int ntile = tile, nchk = ch + 1;
+    if (nchk == nch) { nchk = 0; ntile += gridDim.x; }
+    if (ntile < tiles)
+      tc_load<DK>(in, p, static_cast<size_t>(ntile) * p.L + nchk * C, min(C, p.L - nchk * C), warp, lane,
+                  irow, ivalid, DIAG);
+
+    fence_async_smem();
+    wait_st();
+    fence_before();
+    __syncthreads();
+
+    // ---- local scores
+    if (tid == 0) {
+      fence_after();
+      constexpr uint32_t id = idesc_tf32(64, C);
+#pragma unroll
+      for (int kk = 0; kk < DK / 8; ++kk)
+        mma_ss(tbase + kTcColX, sdesc(saddr(sQs) + 256 * kk, DK * 32), sdesc(saddr(sKs) + 256 * kk, DK * 32),
+               id, kk > 0);
+      mma_commit(mbar);
+    }
+    if (!wait_mma()) break;
+
+    // ---- A[t][s] (into the Ks region: the scores have read it)
+#pragma unroll
+    for (int s0 = (C / 2) * half; s0 < (C / 2) * (half + 1); s0 += 16) {
+      float r[16];
+      tm_ld16(tw + kTcColX + s0, r);
+      wait_ld();
+      if (trow >= 0) {
+        const int t = trow;
+#pragma unroll
+        for (int u = 0; u < 16; u += 4) {
+          float a[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int s = s0 + u + e;
+            float x = 0.0f;
+            if (s <= t && t < Ce) {
+              x = r[u + e];
+              if constexpr (!DIAG) x *= expf(lam[t] - lam[s]);
+              x *= bt[s];
+            }
+            a[e] = tf32(x);
+          }
+          st_shared4(sKs, cm_off(t, s0 + u, C), a[0], a[1], a[2], a[3]);
+        }
+      }
+    }
+    fence_async_smem();
+    fence_before();
+    __syncthreads();
+
+    // ---- outputs: state read + intra-chunk output, O^T in X
+    if (tid == 0) {
+      fence_after();
+      constexpr uint32_t id = idesc_tf32(MDV, C);
+#pragma unroll
+      for (int kk = 0; kk < DK / 8; ++kk)
+        mma_ts(tbase + kTcColX, tbase + kTcColS + 8 * kk, sdesc(saddr(sQb) + 256 * kk, DK * 32), id, kk > 0);
+#pragma unroll
+      for (int kk = 0; kk < C / 8; ++kk)
+        mma_ts(tbase + kTcColX, tbase + kTcColV + 8 * kk, sdesc(saddr(sKs) + 256 * kk, C * 32), id, 1u);
+      mma_commit(mbar);
+    }
+    if (!wait_mma()) break;
+#pragma unroll
+    for (int t0 = (C / 2) * half; t0 < (C / 2) * (half + 1); t0 += 16) {
+      float r[16];
+      tm_ld16(tw + kTcColX + t0, r);
+      wait_ld();
+      if (ivalid && p.o != nullptr) {
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          if (t0 + u < Ce) p.o[(tok0 + t0 + u) * dv + irow] = r[u];
+      }
+    }
+    // ---- state pass: S <- S e^{Lam_C} (the state read above has completed)
+#pragma unroll
+    for (int c = half * (DK / 2); c < (half + 1) * (DK / 2); c += 16) {
+      float r[16];
+      tm_ld16(tw + kTcColS + c, r);
+      wait_ld();
+#pragma unroll
+      for (int u = 0; u < 16; ++u) r[u] *= DIAG ? lamc[DK + c + u] : lamc[1];
+      tm_st16(tw + kTcColS + c, r);
+    }
+    wait_st();
+    fence_before();
+    __syncthreads();
+    // ---- state write: S += VT KbT^T
+    if (tid == 0) {
+      fence_after();
+      constexpr uint32_t id = idesc_tf32(MDV, DK);
+#pragma unroll
+      for (int kk = 0; kk < C / 8; ++kk)
+        mma_ts(tbase + kTcColS, tbase + kTcColV + 8 * kk, sdesc(saddr(sKbT) + 256 * kk, C * 32), id, 1u);
+      mma_commit(mbar);
+    }
+    if (!wait_mma()) break;
+
+    // ---- final state of the tile out of tensor memory
+    if (ch == nch - 1) {
       float* dst = p.S + (static_cast<size_t>(tile) * dv + (ivalid ? irow : 0)) * DK;
-#pragma unroll 1
-      for (int c = 0; c < DK; c += 16) {
+#pragma unroll
+      for (int c = half * (DK / 2); c < (half + 1) * (DK / 2); c += 16) {
         float r[16];
         tm_ld16(tw + kTcColS + c, r);
         wait_ld();
@@ -458,11 +526,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             reinterpret_cast<float4*>(dst + c)[u] = make_float4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
         }
       }
-      fence_before();
     }
+    tile = ntile;
+    ch = nchk;
   }
 
-done:
   __syncthreads();
   if (tid == 0 && *failed) atomicAdd(timeouts, 1u);
   fence_after();
