@@ -249,8 +249,9 @@ QS_API qs_status qstate_prefill(const qs_config* cfg, int length, float* S, cons
  * to about 2^-10 of the magnitudes summed, not to FP32 rounding: every
  * element of S and o is within 2^-8 of the same recurrence run on |S0|,
  * |q|, |k|, |v| (the sum of the magnitudes of its terms).  Arguments,
- * validation and the range condition on the decay are those of
- * qstate_prefill, with S, q and k 16-byte aligned.  A wait for the tensor
+ * validation are those of qstate_prefill, with S, q and k 16-byte aligned;
+ * under either decay a chunk of 64 tokens may decay a channel by at most
+ * e^-170 (the decay factors are split around the chunk's middle token).  A wait for the tensor
  * cores that does not end (a bounded poll) makes the CTA free its tensor
  * memory and return; qstate_prefill_tf32_timeouts reports the count. */
 QS_API qs_status qstate_prefill_tf32(const qs_config* cfg, int length, float* S, const float* q,

@@ -149,7 +149,7 @@ cudaError_t launch_prefill_tc(const PrefillParams& p, int tiles, unsigned int* t
   err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kTcThreads, smem);
   if (err != cudaSuccess) return err;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
-  if (per_sm > 2) per_sm = 2;  // two 256-column tensor-memory allocations per SM
+  if (per_sm > 2) per_sm = 2;  // at most two 256-column tensor-memory allocations per SM
   long long grid = static_cast<long long>(per_sm) * device_sm_count();
   if (grid > tiles) grid = tiles;
   kernel<<<static_cast<int>(grid), kTcThreads, smem, stream>>>(p, tiles, timeouts);

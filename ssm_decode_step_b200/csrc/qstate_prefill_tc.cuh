@@ -1,4 +1,4 @@
-// Chunkwise prefill on the fifth-generation tensor cores (qstate_prefill_tc):
+// Chunkwise prefill on the fifth-generation tensor cores (qstate_prefill_tf32):
 // the same recurrence and regrouping as prefill_kernel (qstate_prefill.cuh),
 // with the four contractions of a chunk issued as tcgen05.mma in TF32 and
 // accumulated in FP32 in tensor memory (LinQuant, Low-Precision Chunkwise
@@ -6,8 +6,8 @@
 // the state pass is the FP32 decay of the accumulator).
 //
 // One CTA per tile at a time, persistent over tiles; chunks of C = 64
-// tokens; 8 warps, two per quadrant of tensor-memory lanes (each takes half
-// of the columns).  Each thread holds the next chunk's inputs in registers:
+// tokens; 16 warps, four per quadrant of tensor-memory lanes (each takes a
+// quarter of the columns).  Each thread holds the next chunk's inputs in registers:
 // their loads are issued before the current chunk's contractions and land
 // while those and the epilogues run.  Tensor memory (256 columns per CTA):
 //   S   columns [0, Dk)     the FP32 state, row i of Dv in the lane of an
@@ -18,21 +18,25 @@
 //                           O^T[i][t] (M = MDV)
 //   VT  columns [192, 256)  v^T[i][s] (A operand of the intra-chunk output
 //                           and of the state write)
-// Shared memory holds the B operands (and the A operand of the scores) in
-// the K-major, unswizzled core-matrix layout: element (r, k) of an R x K
-// operand at byte (r/8)*32K + (k/4)*128 + (r%8)*16 + (k%4)*4.
+// Shared memory holds the smem operands in the K-major, unswizzled
+// core-matrix layout: element (r, k) of an R x K operand at byte
+// (r/8)*32K + (k/4)*128 + (r%8)*16 + (k%4)*4.
 //
 // Per chunk, with Lam the running log-decay (inclusive; per channel under
-// diagonal decay) and m the chunk's middle token:
+// diagonal decay), m the chunk's middle token and C its last:
+//   Qs = q e^{Lam_t - Lam_m},  Ks = k e^{Lam_m - Lam_s}
 //   scores  D[t][s] = sum_j Qs[t][j] Ks[s][j]          (M=64, N=64, K=Dk)
-//           Qs = q (scalar) or q e^{Lam_t - Lam_m}; Ks = k or k e^{Lam_m - Lam_s}
-//   A[t][s] = D[t][s] (e^{Lam_t - Lam_s} under scalar decay) beta_s, s <= t
-//   output  O^T[i][t] = sum_j S[i][j] Qb[t][j] + sum_s VT[i][s] A[t][s]
-//           Qb = q e^{Lam_t}                            (M=Dv, N=64)
-//   state   S <- S e^{Lam_C} (in place, FP32) then
-//           S[i][j] += sum_s VT[i][s] KbT[j][s],  KbT = beta_s k_s e^{Lam_C - Lam_s}
-//           (KbT is formed from the staged Ks, so k is rounded to TF32 twice
-//           on this path)
+//           = sum_j q_tj k_sj e^{Lam_tj - Lam_sj}
+//   output  o_t = S (q_t e^{Lam_t}) + sum_{s<=t} D[t][s] beta_s v_s
+//     scalar decay:   O^T = e^{Lam_m} (S Qs^T + VT A^T), A = D beta_s e^{-Lam_m}
+//     diagonal decay: S <- S e^{Lam_m} (per column, in tensor memory) first,
+//                     then O^T = S Qs^T + VT A^T, A = D beta_s
+//   state   S <- S e^{Lam_C - Lam_m} (diagonal) or S e^{Lam_C} (scalar), then
+//           S[i][j] += sum_s VT[i][s] KbT[j][s],  KbT = Ks[s][j] beta_s e^{Lam_C - Lam_m}
+//           (= beta_s k_sj e^{Lam_C - Lam_s}; KbT is formed from the staged
+//           Ks, so k is rounded to TF32 twice on this path)
+// The factors e^{+-(Lam_t - Lam_m)} stay in range while a chunk decays a
+// channel by at most e^-170.
 //
 // Operands are rounded to TF32 (round to nearest, ties away) before they
 // are stored; the state operand of the state read is the FP32 accumulator,
@@ -49,7 +53,7 @@
 namespace qs {
 
 constexpr int kTcChunk = 64;
-constexpr int kTcThreads = 256;
+constexpr int kTcThreads = 512;
 constexpr int kTcCols = 256;
 constexpr int kTcColS = 0, kTcColX = 128, kTcColV = 192;
 // Shared memory per CTA is at least this, so that at most two CTAs (two
@@ -60,18 +64,21 @@ constexpr int kTcMinSmem = 80 * 1024;
 constexpr long long kTcSpinLimit = 1ll << 22;
 
 struct TcLayout {
-  int qs, ks, qb, kbt, lam, beta, lamc, misc, total;
+  int qs, ks, kbt, lam, beta, lamc, part, misc, total;
   __host__ __device__ TcLayout(int dk, bool diag) {
     constexpr int C = kTcChunk;
     int off = 0;
-    qs = off;   off += C * dk * 4;   // A operand of the scores
+    qs = off;   off += C * dk * 4;   // A operand of the scores, B operand of the state read
     ks = off;   off += C * dk * 4;   // B operand of the scores, then A[t][s]
-    qb = off;   off += C * dk * 4;   // B operand of the state read
     kbt = off;  off += dk * C * 4;   // B operand of the state write
-    lam = off;  off += diag ? C * (dk + 4) * 4 : C * 4;  // Lam[t][j] (row stride dk+4) or Lam[t]
+    // diagonal: Lam[t][j] (row stride dk + 4); scalar: Lam[t], e^{Lam_t - Lam_m}, e^{Lam_m - Lam_t}
+    lam = off;  off += diag ? C * (dk + 4) * 4 : 3 * C * 4;
     beta = off; off += C * 4;
-    lamc = off; off += diag ? 2 * dk * 4 : 16;           // Lam_C and e^{Lam_C} per channel
-    misc = off; off += 16;                               // mbarrier, tensor-memory base
+    // diagonal: per channel e^{Lam_C - Lam_m}, e^{Lam_m}; scalar: e^{Lam_C - Lam_m},
+    // e^{Lam_C}, e^{Lam_m}, e^{-Lam_m}
+    lamc = off; off += diag ? 2 * dk * 4 : 16;
+    part = off; off += diag ? kTcThreads * 4 : 0;  // diagonal: per-thread partial log sums
+    misc = off; off += 16;           // mbarrier, tensor-memory base, failure flag
     total = off;
   }
   __host__ __device__ int bytes() const { return total > kTcMinSmem ? total : kTcMinSmem; }
@@ -190,14 +197,17 @@ __device__ __forceinline__ int tc_row(int qd, int lane) {
   return M == 128 ? 32 * qd + lane : (lane < 16 ? 16 * qd + lane : -1);
 }
 
-// One chunk's inputs held in registers by one thread: its Qs/Ks/Qb items
-// (8 tokens x 16 columns per warp step, a float4 of q and of k per lane),
-// its half of v^T's row, and the scalar decay and beta of one token.
+// One chunk's inputs held in registers by one thread: its Qs/Ks items (8
+// tokens x 16 columns per warp step, a float4 of q and of k per lane), a
+// quarter of its row of v^T, the diagonal decays of TP tokens of one
+// channel, the scalar decays of two tokens and beta of one.
 template <int DK>
 struct TcInputs {
-  static constexpr int IQ = DK / 16;
+  static constexpr int IQ = DK / 32;
+  static constexpr int TP = kTcChunk * DK / kTcThreads;  // tokens per thread of the diagonal scan
   float4 q[IQ], k[IQ];
-  float v[kTcChunk / 2];
+  float v[kTcChunk / 4];
+  float al[TP];
   float a0, a1, b;
 };
 
@@ -205,9 +215,10 @@ template <int DK>
 __device__ __forceinline__ void tc_load(TcInputs<DK>& in, const PrefillParams& p, size_t tok0, int Ce,
                                         int warp, int lane, int irow, bool ivalid, bool diag) {
   constexpr int C = kTcChunk;
+  constexpr int TP = TcInputs<DK>::TP;
 #pragma unroll
   for (int i = 0; i < TcInputs<DK>::IQ; ++i) {
-    const int it = warp + 8 * i;
+    const int it = warp + 16 * i;
     const int t = 8 * (it & 7) + (lane & 7);
     const int j = 16 * (it >> 3) + 4 * (lane >> 3);
     in.q[i] = in.k[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -216,44 +227,50 @@ __device__ __forceinline__ void tc_load(TcInputs<DK>& in, const PrefillParams& p
       in.k[i] = __ldg(reinterpret_cast<const float4*>(p.k + (tok0 + t) * DK + j));
     }
   }
-  const int s0 = (C / 2) * (warp >> 2);
+  const int s0 = (C / 4) * (warp >> 2);
 #pragma unroll
-  for (int u = 0; u < C / 2; ++u)
+  for (int u = 0; u < C / 4; ++u)
     in.v[u] = (ivalid && s0 + u < Ce) ? __ldg(p.v + (tok0 + s0 + u) * p.dv + irow) : 0.0f;
+  const int tid = 32 * warp + lane;
+  if (diag) {
+    const int j = tid % DK, t0 = TP * (tid / DK);
+#pragma unroll
+    for (int u = 0; u < TP; ++u) in.al[u] = t0 + u < Ce ? __ldg(p.alpha + (tok0 + t0 + u) * DK + j) : 1.0f;
+  }
   in.a0 = in.a1 = 1.0f;
   if (!diag && warp == 0) {
     if (lane < Ce) in.a0 = __ldg(p.alpha + tok0 + lane);
     if (32 + lane < Ce) in.a1 = __ldg(p.alpha + tok0 + 32 + lane);
   }
-  const int tid = 32 * warp + lane;
   in.b = tid < Ce ? __ldg(p.beta + tok0 + tid) : 0.0f;
 }
 
 template <int DK, int MDV, bool DIAG>
-__global__ void __launch_bounds__(kTcThreads, DK == 64 ? 2 : 1)
+__global__ void __launch_bounds__(kTcThreads, 1)
     prefill_tc_kernel(PrefillParams p, int tiles, unsigned int* timeouts) {
   using namespace tc;
   constexpr int C = kTcChunk;
   constexpr int LS = DK + 4;  // row stride of the diagonal-decay Lam table
   static_assert(DK == 64 || DK == 128, "Dk");
   static_assert(MDV == 64 || MDV == 128, "accumulator rows");
-  static_assert(kTcThreads == 256, "8 warps: two per tensor-memory lane quadrant");
+  static_assert(kTcThreads == 512, "16 warps: four per tensor-memory lane quadrant");
   extern __shared__ __align__(1024) unsigned char tsm[];
   const TcLayout Ly(DK, DIAG);
   unsigned char* sQs = tsm + Ly.qs;
   unsigned char* sKs = tsm + Ly.ks;  // then the scores A[t][s]
-  unsigned char* sQb = tsm + Ly.qb;
   unsigned char* sKbT = tsm + Ly.kbt;
   float* lam = reinterpret_cast<float*>(tsm + Ly.lam);
+  float* fq = lam + C;      // scalar: e^{Lam_t - Lam_m}
+  float* fk = lam + 2 * C;  // scalar: e^{Lam_m - Lam_t}
   float* bt = reinterpret_cast<float*>(tsm + Ly.beta);
-  float* lamc = reinterpret_cast<float*>(tsm + Ly.lamc);  // [0, DK): Lam_C; [DK, 2DK): e^{Lam_C}
+  float* lamc = reinterpret_cast<float*>(tsm + Ly.lamc);
   uint64_t* mbar_p = reinterpret_cast<uint64_t*>(tsm + Ly.misc);
   volatile uint32_t* tslot = reinterpret_cast<volatile uint32_t*>(tsm + Ly.misc + 8);
   volatile int* failed = reinterpret_cast<volatile int*>(tsm + Ly.misc + 12);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qd = warp & 3;   // tensor-memory lane quadrant of this warp
-  const int half = warp >> 2;  // which half of the columns this warp takes
+  const int qt = warp >> 2;  // which quarter of the columns this warp takes
   const int dv = p.dv;
   const uint32_t mbar = saddr(mbar_p);
 
@@ -278,14 +295,29 @@ __global__ void __launch_bounds__(kTcThreads, DK == 64 ? 2 : 1)
   const bool ivalid = irow >= 0 && irow < dv;
   const int trow = tc_row<64>(qd, lane);   // score row of this lane
   const int nch = (p.L + C - 1) / C;
+  const int cS0 = qt * (DK / 4), cS1 = cS0 + DK / 4;  // this warp's state columns
 
-  // wait for the MMAs committed last; on a timeout every thread leaves
+  // Wait for the MMAs committed last: warp 0 polls, the barrier releases the
+  // others.  On a timeout every thread leaves.
   auto wait_mma = [&]() -> bool {
-    if (!mbar_wait(mbar, phase)) *failed = 1;
+    if (warp == 0 && !mbar_wait(mbar, phase)) *failed = 1;
     phase ^= 1u;
     __syncthreads();
     fence_after();
     return *failed == 0;
+  };
+  // Scale this warp's state columns in tensor memory (per column under
+  // diagonal decay: f[c]; scalar: f[0]).
+  auto scale_state = [&](const float* f) {
+#pragma unroll
+    for (int c = cS0; c < cS1; c += 16) {
+      float r[16];
+      tm_ld16(tw + kTcColS + c, r);
+      wait_ld();
+#pragma unroll
+      for (int u = 0; u < 16; ++u) r[u] *= DIAG ? f[c + u] : f[0];
+      tm_st16(tw + kTcColS + c, r);
+    }
   };
 
   int tile = blockIdx.x, ch = 0;
@@ -296,12 +328,13 @@ __global__ void __launch_bounds__(kTcThreads, DK == 64 ? 2 : 1)
     const int c0 = ch * C;
     const int Ce = min(C, p.L - c0);
     const size_t tok0 = static_cast<size_t>(tile) * p.L + c0;
+    const int m = (Ce - 1) / 2;
 
-    // ---- initial state of the tile into tensor memory (this warp's rows, half the columns)
+    // ---- initial state of the tile into tensor memory (this warp's rows, a quarter of the columns)
     if (ch == 0) {
       const float* src = p.S + (static_cast<size_t>(tile) * dv + (ivalid ? irow : 0)) * DK;
 #pragma unroll
-      for (int c = half * (DK / 2); c < (half + 1) * (DK / 2); c += 16) {
+      for (int c = cS0; c < cS1; c += 16) {
         float r[16];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -316,27 +349,31 @@ __global__ void __launch_bounds__(kTcThreads, DK == 64 ? 2 : 1)
     // the previous chunk's readers of lam, beta and the operands are done
     __syncthreads();
 
-    // ---- beta and the running log-decay
+    // ---- beta, the running log-decay and the decay factors
     if (tid < C) bt[tid] = in.b;
     if constexpr (DIAG) {
-      for (int j = tid; j < DK; j += kTcThreads) {
-        float acc = 0.0f;
+      // thread (j, part) scans TP tokens of channel j; the parts' totals are
+      // then added in order
+      constexpr int TP = TcInputs<DK>::TP;
+      float* psum = reinterpret_cast<float*>(tsm + Ly.part);
+      const int j = tid % DK, pt = tid / DK;
+      float acc = 0.0f, loc[TP];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float x[C / 2];
+      for (int u = 0; u < TP; ++u) {
+        acc += logf(in.al[u]);
+        loc[u] = acc;
+      }
+      psum[pt * DK + j] = acc;
+      __syncthreads();
+      float off = 0.0f;
+      for (int q2 = 0; q2 < pt; ++q2) off += psum[q2 * DK + j];
 #pragma unroll
-          for (int u = 0; u < C / 2; ++u) {
-            const int t = (C / 2) * hh + u;
-            x[u] = t < Ce ? __ldg(p.alpha + (tok0 + t) * DK + j) : 1.0f;
-          }
-#pragma unroll
-          for (int u = 0; u < C / 2; ++u) {
-            acc += logf(x[u]);
-            lam[((C / 2) * hh + u) * LS + j] = acc;
-          }
-        }
-        lamc[j] = acc;
-        lamc[DK + j] = expf(acc);
+      for (int u = 0; u < TP; ++u) lam[(pt * TP + u) * LS + j] = loc[u] + off;
+      __syncthreads();
+      if (tid < DK) {
+        const float lC = lam[(C - 1) * LS + tid], lm = lam[m * LS + tid];
+        lamc[tid] = expf(lC - lm);
+        lamc[DK + tid] = expf(lm);
       }
     } else {
       if (warp == 0) {
@@ -348,18 +385,28 @@ __global__ void __launch_bounds__(kTcThreads, DK == 64 ? 2 : 1)
           if (lane >= d) { x0 += y0; x1 += y1; }
         }
         x1 += __shfl_sync(0xffffffffu, x0, 31);
+        const float lC = __shfl_sync(0xffffffffu, x1, 31);
+        const float lm = __shfl_sync(0xffffffffu, m < 32 ? x0 : x1, m & 31);
         lam[lane] = x0;
         lam[32 + lane] = x1;
-        if (lane == 31) { lamc[0] = x1; lamc[1] = expf(x1); }
+        fq[lane] = expf(x0 - lm);
+        fq[32 + lane] = expf(x1 - lm);
+        fk[lane] = expf(lm - x0);
+        fk[32 + lane] = expf(lm - x1);
+        if (lane == 0) {
+          lamc[0] = expf(lC - lm);
+          lamc[1] = expf(lC);
+          lamc[2] = expf(lm);
+          lamc[3] = expf(-lm);
+        }
       }
     }
     __syncthreads();
 
-    // ---- operands Qs, Ks, Qb from the registers
-    const int m = (Ce - 1) / 2;
+    // ---- operands Qs, Ks from the registers
 #pragma unroll
     for (int i = 0; i < TcInputs<DK>::IQ; ++i) {
-      const int it = warp + 8 * i;
+      const int it = warp + 16 * i;
       const int t = 8 * (it & 7) + (lane & 7);
       const int j = 16 * (it >> 3) + 4 * (lane >> 3);
       const float4 qv = in.q[i], kv = in.k[i];
@@ -371,42 +418,33 @@ __global__ void __launch_bounds__(kTcThreads, DK == 64 ? 2 : 1)
                    tf32(qv.z * expf(lt.z - lm.z)), tf32(qv.w * expf(lt.w - lm.w)));
         st_shared4(sKs, o, tf32(kv.x * expf(lm.x - lt.x)), tf32(kv.y * expf(lm.y - lt.y)),
                    tf32(kv.z * expf(lm.z - lt.z)), tf32(kv.w * expf(lm.w - lt.w)));
-        st_shared4(sQb, o, tf32(qv.x * expf(lt.x)), tf32(qv.y * expf(lt.y)), tf32(qv.z * expf(lt.z)),
-                   tf32(qv.w * expf(lt.w)));
       } else {
-        const float e = expf(lam[t]);
-        st_shared4(sQs, o, tf32(qv.x), tf32(qv.y), tf32(qv.z), tf32(qv.w));
-        st_shared4(sKs, o, tf32(kv.x), tf32(kv.y), tf32(kv.z), tf32(kv.w));
-        st_shared4(sQb, o, tf32(qv.x * e), tf32(qv.y * e), tf32(qv.z * e), tf32(qv.w * e));
+        const float eq = fq[t], ek = fk[t];
+        st_shared4(sQs, o, tf32(qv.x * eq), tf32(qv.y * eq), tf32(qv.z * eq), tf32(qv.w * eq));
+        st_shared4(sKs, o, tf32(kv.x * ek), tf32(kv.y * ek), tf32(kv.z * ek), tf32(kv.w * ek));
       }
     }
-    // ---- VT[i][s] into tensor memory (this warp's rows, half the tokens)
-#pragma unroll
-    for (int u = 0; u < C / 2; u += 16) {
+    // ---- VT[i][s] into tensor memory (this warp's rows, a quarter of the tokens)
+    {
       float r[16];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) r[e] = tf32(in.v[u + e]);
-      tm_st16(tw + kTcColV + (C / 2) * half + u, r);
+      for (int e = 0; e < 16; ++e) r[e] = tf32(in.v[e]);
+      tm_st16(tw + kTcColV + (C / 4) * qt, r);
     }
+    // ---- diagonal decay: S <- S e^{Lam_m} for the state read
+    if constexpr (DIAG) scale_state(lamc + DK);
     __syncthreads();  // Ks complete
-    // ---- KbT[j][s] = Ks[s][j] beta_s e^{Lam_C - Lam_s} / (e^{Lam_m - Lam_s} under diagonal decay)
+    // ---- KbT[j][s] = Ks[s][j] beta_s e^{Lam_C - Lam_m}
 #pragma unroll
-    for (int i = 0; i < DK / 16; ++i) {
-      const int it = warp + 8 * i;
+    for (int i = 0; i < DK / 32; ++i) {
+      const int it = warp + 16 * i;
       const int j = 8 * (it % (DK / 8)) + (lane & 7);
       const int s = 16 * (it / (DK / 8)) + 4 * (lane >> 3);
+      const float f = DIAG ? lamc[j] : lamc[0];
       float w[4];
-      if constexpr (DIAG) {
-        const float f = expf(lamc[j] - lam[m * LS + j]);
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          w[u] = tf32(*reinterpret_cast<const float*>(sKs + cm_off(s + u, j, DK)) * (f * bt[s + u]));
-      } else {
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          w[u] = tf32(*reinterpret_cast<const float*>(sKs + cm_off(s + u, j, DK)) *
-                      (bt[s + u] * expf(lam[C - 1] - lam[s + u])));
-      }
+      for (int u = 0; u < 4; ++u)
+        w[u] = tf32(*reinterpret_cast<const float*>(sKs + cm_off(s + u, j, DK)) * (f * bt[s + u]));
       st_shared4(sKbT, cm_off(j, s, C), w[0], w[1], w[2], w[3]);
     }
 
@@ -435,28 +473,25 @@ __global__ void __launch_bounds__(kTcThreads, DK == 64 ? 2 : 1)
     if (!wait_mma()) break;
 
     // ---- A[t][s] (into the Ks region: the scores have read it)
+    {
+      const float sa = DIAG ? 1.0f : lamc[3];
 #pragma unroll
-    for (int s0 = (C / 2) * half; s0 < (C / 2) * (half + 1); s0 += 16) {
-      float r[16];
-      tm_ld16(tw + kTcColX + s0, r);
-      wait_ld();
-      if (trow >= 0) {
-        const int t = trow;
+      for (int s0 = (C / 4) * qt; s0 < (C / 4) * (qt + 1); s0 += 16) {
+        float r[16];
+        tm_ld16(tw + kTcColX + s0, r);
+        wait_ld();
+        if (trow >= 0) {
+          const int t = trow;
 #pragma unroll
-        for (int u = 0; u < 16; u += 4) {
-          float a[4];
+          for (int u = 0; u < 16; u += 4) {
+            float a[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int s = s0 + u + e;
-            float x = 0.0f;
-            if (s <= t && t < Ce) {
-              x = r[u + e];
-              if constexpr (!DIAG) x *= expf(lam[t] - lam[s]);
-              x *= bt[s];
+            for (int e = 0; e < 4; ++e) {
+              const int s = s0 + u + e;
+              a[e] = (s <= t && t < Ce) ? tf32(r[u + e] * (bt[s] * sa)) : 0.0f;
             }
-            a[e] = tf32(x);
+            st_shared4(sKs, cm_off(t, s0 + u, C), a[0], a[1], a[2], a[3]);
           }
-          st_shared4(sKs, cm_off(t, s0 + u, C), a[0], a[1], a[2], a[3]);
         }
       }
     }
@@ -470,34 +505,29 @@ __global__ void __launch_bounds__(kTcThreads, DK == 64 ? 2 : 1)
       constexpr uint32_t id = idesc_tf32(MDV, C);
 #pragma unroll
       for (int kk = 0; kk < DK / 8; ++kk)
-        mma_ts(tbase + kTcColX, tbase + kTcColS + 8 * kk, sdesc(saddr(sQb) + 256 * kk, DK * 32), id, kk > 0);
+        mma_ts(tbase + kTcColX, tbase + kTcColS + 8 * kk, sdesc(saddr(sQs) + 256 * kk, DK * 32), id, kk > 0);
 #pragma unroll
       for (int kk = 0; kk < C / 8; ++kk)
         mma_ts(tbase + kTcColX, tbase + kTcColV + 8 * kk, sdesc(saddr(sKs) + 256 * kk, C * 32), id, 1u);
       mma_commit(mbar);
     }
     if (!wait_mma()) break;
+    {
+      const float so = DIAG ? 1.0f : lamc[2];
 #pragma unroll
-    for (int t0 = (C / 2) * half; t0 < (C / 2) * (half + 1); t0 += 16) {
-      float r[16];
-      tm_ld16(tw + kTcColX + t0, r);
-      wait_ld();
-      if (ivalid && p.o != nullptr) {
+      for (int t0 = (C / 4) * qt; t0 < (C / 4) * (qt + 1); t0 += 16) {
+        float r[16];
+        tm_ld16(tw + kTcColX + t0, r);
+        wait_ld();
+        if (ivalid && p.o != nullptr) {
 #pragma unroll
-        for (int u = 0; u < 16; ++u)
-          if (t0 + u < Ce) p.o[(tok0 + t0 + u) * dv + irow] = r[u];
+          for (int u = 0; u < 16; ++u)
+            if (t0 + u < Ce) p.o[(tok0 + t0 + u) * dv + irow] = DIAG ? r[u] : r[u] * so;
+        }
       }
     }
-    // ---- state pass: S <- S e^{Lam_C} (the state read above has completed)
-#pragma unroll
-    for (int c = half * (DK / 2); c < (half + 1) * (DK / 2); c += 16) {
-      float r[16];
-      tm_ld16(tw + kTcColS + c, r);
-      wait_ld();
-#pragma unroll
-      for (int u = 0; u < 16; ++u) r[u] *= DIAG ? lamc[DK + c + u] : lamc[1];
-      tm_st16(tw + kTcColS + c, r);
-    }
+    // ---- state pass (the state read above has completed)
+    scale_state(DIAG ? lamc : lamc + 1);
     wait_st();
     fence_before();
     __syncthreads();
@@ -516,7 +546,7 @@ __global__ void __launch_bounds__(kTcThreads, DK == 64 ? 2 : 1)
     if (ch == nch - 1) {
       float* dst = p.S + (static_cast<size_t>(tile) * dv + (ivalid ? irow : 0)) * DK;
 #pragma unroll
-      for (int c = half * (DK / 2); c < (half + 1) * (DK / 2); c += 16) {
+      for (int c = cS0; c < cS1; c += 16) {
         float r[16];
         tm_ld16(tw + kTcColS + c, r);
         wait_ld();
