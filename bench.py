@@ -83,12 +83,20 @@ def state_bytes(w: W.Workload, arm: W.Arm) -> int:
     return b
 
 
+# The sources the decode-step kernel is compiled from: a committed traffic
+# figure stays valid while none of them changes.
+STEP_SOURCES = ("qstate_step.cuh", "qstate_kernels.cuh", "qstate_launch.h", "qstate_launch_impl.cuh",
+                "inst_b4_d128.cu", "inst_b4_d64.cu", "inst_b8_d128.cu", "inst_b8_d64.cu")
+
+
 def source_sha() -> str:
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "ssm_decode_step_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, f), "rb") as fh:
+    pkg = os.path.join(ROOT, "ssm_decode_step_b200")
+    for f in STEP_SOURCES:
+        with open(os.path.join(pkg, "csrc", f), "rb") as fh:
             h.update(f.encode() + fh.read())
+    with open(os.path.join(pkg, "build.py"), "rb") as fh:
+        h.update(b"build.py" + fh.read())
     return h.hexdigest()[:16]
 
 
@@ -912,6 +920,8 @@ def run_prefill(args):
     import torch
     from ssm_decode_step_b200 import Config, qstate as Q
     w = W.get(args.workload)
+    if args.prefill_tiles > 0:
+        w = W.scaled_down(w, args.prefill_tiles, layers=1)
     if w.delta != 0:
         raise SystemExit("the chunkwise prefill covers the linear write (delta = 0) workloads")
     L, P = args.prefill, max(1, min(args.pool, args.prefill))
@@ -994,6 +1004,8 @@ def main():
                     help="also time every arm with Low-Rank Bypass of this rank (0: skip)")
     ap.add_argument("--prefill", type=int, default=0,
                     help="time the chunkwise prefill over this many tokens per tile instead")
+    ap.add_argument("--prefill-tiles", type=int, default=0,
+                    help="with --prefill: that many tiles of the workload's laws (0: all)")
     ap.add_argument("--recall", action="store_true",
                     help="measure recall of a planted association over the decode horizon instead")
     ap.add_argument("--recall-steps", type=int, default=32768)
