@@ -8,8 +8,12 @@
 // One CTA per tile at a time, persistent over tiles; chunks of C = 64
 // tokens; 16 warps, four per quadrant of tensor-memory lanes (each takes a
 // quarter of the columns).  Each thread holds the next chunk's inputs in registers:
-// their loads are issued before the current chunk's contractions and land
-// while those and the epilogues run.  Tensor memory (256 columns per CTA):
+// their loads are issued once the current chunk's output contraction is
+// issued and land while it, the state pass and write and the epilogues run.
+// Within a chunk KbT is formed while the scores contraction runs and the
+// outputs are written while the state write runs; the next chunk's staging
+// overlaps that state write, which is waited for only before VT and the
+// state are touched again.  Tensor memory (256 columns per CTA):
 //   S   columns [0, Dk)     the FP32 state, row i of Dv in the lane of an
 //                           M = MDV accumulator; it stays there for the
 //                           whole sequence and is the A operand of the
@@ -321,6 +325,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   };
 
   int tile = blockIdx.x, ch = 0;
+  bool pending = false;  // the state write of the previous chunk is in flight
   TcInputs<DK> in;
   if (tile < tiles) tc_load<DK>(in, p, static_cast<size_t>(tile) * p.L, min(C, p.L), warp, lane, irow, ivalid, DIAG);
 
@@ -424,6 +429,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         st_shared4(sKs, o, tf32(kv.x * ek), tf32(kv.y * ek), tf32(kv.z * ek), tf32(kv.w * ek));
       }
     }
+    // ---- the previous chunk's state write has read VT and KbT and written S
+    if (pending) {
+      if (!wait_mma()) break;
+      pending = false;
+    }
     // ---- VT[i][s] into tensor memory (this warp's rows, a quarter of the tokens)
     {
       float r[16];
@@ -433,8 +443,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     // ---- diagonal decay: S <- S e^{Lam_m} for the state read
     if constexpr (DIAG) scale_state(lamc + DK);
-    __syncthreads();  // Ks complete
-    // ---- KbT[j][s] = Ks[s][j] beta_s e^{Lam_C - Lam_m}
+    fence_async_smem();
+    wait_st();
+    fence_before();
+    __syncthreads();  // Qs, Ks, VT complete
+
+    // ---- local scores
+    if (tid == 0) {
+      fence_after();
+      constexpr uint32_t id = idesc_tf32(64, C);
+#pragma unroll
+      for (int kk = 0; kk < DK / 8; ++kk)
+        mma_ss(tbase + kTcColX, sdesc(saddr(sQs) + 256 * kk, DK * 32), sdesc(saddr(sKs) + 256 * kk, DK * 32),
+               id, kk > 0);
+      mma_commit(mbar);
+    }
+    // ---- while the scores run: KbT[j][s] = Ks[s][j] beta_s e^{Lam_C - Lam_m}
 #pragma unroll
     for (int i = 0; i < DK / 32; ++i) {
       const int it = warp + 16 * i;
@@ -447,30 +471,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         w[u] = tf32(*reinterpret_cast<const float*>(sKs + cm_off(s + u, j, DK)) * (f * bt[s + u]));
       st_shared4(sKbT, cm_off(j, s, C), w[0], w[1], w[2], w[3]);
     }
-
-    // ---- the next chunk's inputs: loads in flight while this chunk computes
-    int ntile = tile, nchk = ch + 1;
-    if (nchk == nch) { nchk = 0; ntile += gridDim.x; }
-    if (ntile < tiles)
-      tc_load<DK>(in, p, static_cast<size_t>(ntile) * p.L + nchk * C, min(C, p.L - nchk * C), warp, lane,
-                  irow, ivalid, DIAG);
-
     fence_async_smem();
-    wait_st();
-    fence_before();
-    __syncthreads();
-
-    // ---- local scores
-    if (tid == 0) {
-      fence_after();
-      constexpr uint32_t id = idesc_tf32(64, C);
-#pragma unroll
-      for (int kk = 0; kk < DK / 8; ++kk)
-        mma_ss(tbase + kTcColX, sdesc(saddr(sQs) + 256 * kk, DK * 32), sdesc(saddr(sKs) + 256 * kk, DK * 32),
-               id, kk > 0);
-      mma_commit(mbar);
-    }
-    if (!wait_mma()) break;
+    if (!wait_mma()) break;  // scores done; every warp is done with Ks
 
     // ---- A[t][s] (into the Ks region: the scores have read it)
     {
@@ -511,7 +513,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mma_ts(tbase + kTcColX, tbase + kTcColV + 8 * kk, sdesc(saddr(sKs) + 256 * kk, C * 32), id, 1u);
       mma_commit(mbar);
     }
+    // ---- the next chunk's loads, in flight from here to the next chunk's staging
+    int ntile = tile, nchk = ch + 1;
+    if (nchk == nch) { nchk = 0; ntile += gridDim.x; }
+    if (ntile < tiles)
+      tc_load<DK>(in, p, static_cast<size_t>(ntile) * p.L + nchk * C, min(C, p.L - nchk * C), warp, lane,
+                  irow, ivalid, DIAG);
     if (!wait_mma()) break;
+    // ---- state pass (the state read above has completed)
+    scale_state(DIAG ? lamc : lamc + 1);
+    wait_st();
+    fence_before();
+    __syncthreads();
+    // ---- state write: S += VT KbT^T, in flight while the outputs are written
+    if (tid == 0) {
+      fence_after();
+      constexpr uint32_t id = idesc_tf32(MDV, DK);
+#pragma unroll
+      for (int kk = 0; kk < C / 8; ++kk)
+        mma_ts(tbase + kTcColS, tbase + kTcColV + 8 * kk, sdesc(saddr(sKbT) + 256 * kk, C * 32), id, 1u);
+      mma_commit(mbar);
+    }
+    pending = true;
     {
       const float so = DIAG ? 1.0f : lamc[2];
 #pragma unroll
@@ -526,24 +549,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
     }
-    // ---- state pass (the state read above has completed)
-    scale_state(DIAG ? lamc : lamc + 1);
-    wait_st();
     fence_before();
-    __syncthreads();
-    // ---- state write: S += VT KbT^T
-    if (tid == 0) {
-      fence_after();
-      constexpr uint32_t id = idesc_tf32(MDV, DK);
-#pragma unroll
-      for (int kk = 0; kk < C / 8; ++kk)
-        mma_ts(tbase + kTcColS, tbase + kTcColV + 8 * kk, sdesc(saddr(sKbT) + 256 * kk, C * 32), id, 1u);
-      mma_commit(mbar);
-    }
-    if (!wait_mma()) break;
 
     // ---- final state of the tile out of tensor memory
     if (ch == nch - 1) {
+      if (!wait_mma()) break;
+      pending = false;
       float* dst = p.S + (static_cast<size_t>(tile) * dv + (ivalid ? irow : 0)) * DK;
 #pragma unroll
       for (int c = cS0; c < cS1; c += 16) {
