@@ -203,15 +203,14 @@ __device__ __forceinline__ int tc_row(int qd, int lane) {
 
 // One chunk's inputs held in registers by one thread: its Qs/Ks items (8
 // tokens x 16 columns per warp step, a float4 of q and of k per lane), a
-// quarter of its row of v^T, the diagonal decays of TP tokens of one
-// channel, the scalar decays of two tokens and beta of one.
+// quarter of its row of v^T, the scalar decays of two tokens and beta of
+// one (diagonal decays are loaded when the chunk's scan runs).
 template <int DK>
 struct TcInputs {
   static constexpr int IQ = DK / 32;
   static constexpr int TP = kTcChunk * DK / kTcThreads;  // tokens per thread of the diagonal scan
   float4 q[IQ], k[IQ];
   float v[kTcChunk / 4];
-  float al[TP];
   float a0, a1, b;
 };
 
@@ -236,11 +235,6 @@ __device__ __forceinline__ void tc_load(TcInputs<DK>& in, const PrefillParams& p
   for (int u = 0; u < C / 4; ++u)
     in.v[u] = (ivalid && s0 + u < Ce) ? __ldg(p.v + (tok0 + s0 + u) * p.dv + irow) : 0.0f;
   const int tid = 32 * warp + lane;
-  if (diag) {
-    const int j = tid % DK, t0 = TP * (tid / DK);
-#pragma unroll
-    for (int u = 0; u < TP; ++u) in.al[u] = t0 + u < Ce ? __ldg(p.alpha + (tok0 + t0 + u) * DK + j) : 1.0f;
-  }
   in.a0 = in.a1 = 1.0f;
   if (!diag && warp == 0) {
     if (lane < Ce) in.a0 = __ldg(p.alpha + tok0 + lane);
@@ -365,7 +359,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       float acc = 0.0f, loc[TP];
 #pragma unroll
       for (int u = 0; u < TP; ++u) {
-        acc += logf(in.al[u]);
+        const int t = pt * TP + u;
+        loc[u] = t < Ce ? __ldg(p.alpha + (tok0 + t) * DK + j) : 1.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < TP; ++u) {
+        acc += logf(loc[u]);
         loc[u] = acc;
       }
       psum[pt * DK + j] = acc;
