@@ -84,7 +84,7 @@ def state_bytes(w: W.Workload, arm: W.Arm) -> int:
 
 
 # The sources the decode-step kernel is compiled from: a committed traffic
-# figure stays valid while none of them changes.
+# figure stays valid while none of them, nor the nvcc flags, changes.
 STEP_SOURCES = ("qstate_step.cuh", "qstate_kernels.cuh", "qstate_launch.h", "qstate_launch_impl.cuh",
                 "inst_b4_d128.cu", "inst_b4_d64.cu", "inst_b8_d128.cu", "inst_b8_d64.cu")
 
@@ -95,8 +95,8 @@ def source_sha() -> str:
     for f in STEP_SOURCES:
         with open(os.path.join(pkg, "csrc", f), "rb") as fh:
             h.update(f.encode() + fh.read())
-    with open(os.path.join(pkg, "build.py"), "rb") as fh:
-        h.update(b"build.py" + fh.read())
+    from ssm_decode_step_b200 import build as B
+    h.update(" ".join(B.NVFLAGS).encode())
     return h.hexdigest()[:16]
 
 

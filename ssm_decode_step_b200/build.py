@@ -42,9 +42,17 @@ def _deps():
     return [os.path.join(CSRC, f) for f in os.listdir(CSRC)] + [HEADER, __file__]
 
 
+STAMP = LIB + ".flags"
+
+
 def _up_to_date() -> bool:
-    if not os.path.exists(LIB):
+    """The library exists, is newer than every source, and was built with
+    the same nvcc flags."""
+    if not (os.path.exists(LIB) and os.path.exists(STAMP)):
         return False
+    with open(STAMP) as f:
+        if f.read() != " ".join(NVFLAGS):
+            return False
     t = os.path.getmtime(LIB)
     return all(os.path.getmtime(d) <= t for d in _deps())
 
@@ -76,6 +84,8 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stderr}")
     os.replace(tmp, LIB)
+    with open(STAMP, "w") as f:
+        f.write(" ".join(NVFLAGS))
     return LIB
 
 
