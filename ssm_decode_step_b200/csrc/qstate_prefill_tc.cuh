@@ -3,42 +3,38 @@
 // with the four contractions of a chunk issued as tcgen05.mma in TF32 and
 // accumulated in FP32 in tensor memory (LinQuant, Low-Precision Chunkwise
 // Realization: local score, state read, intra-chunk output, state write;
-// the state pass is the FP32 decay of the accumulator).
+// the state pass is an FP32 scale of the accumulator).
 //
 // One CTA per tile at a time, persistent over tiles; chunks of C = 64
 // tokens; 16 warps, four per quadrant of tensor-memory lanes (each takes a
-// quarter of the columns).  Each thread holds the next chunk's inputs in registers:
-// their loads are issued once the current chunk's output contraction is
-// issued and land while it, the state pass and write and the epilogues run.
-// Within a chunk KbT is formed while the scores contraction runs and the
-// outputs are written while the state write runs; the next chunk's staging
-// overlaps that state write, which is waited for only before VT and the
-// state are touched again.  Tensor memory (256 columns per CTA):
+// quarter of the columns).  Each thread holds the next chunk's inputs in
+// registers: their loads are issued once the current chunk's output
+// contraction is issued and land while it, the state write and the
+// epilogues run.  Tensor memory (256 columns per CTA):
 //   S   columns [0, Dk)     the FP32 state, row i of Dv in the lane of an
-//                           M = MDV accumulator; it stays there for the
-//                           whole sequence and is the A operand of the
-//                           state read (read from tensor memory)
+//                           M = MDV accumulator, held pre-scaled (below);
+//                           it stays there for the whole sequence and is the
+//                           A operand of the state read
 //   X   columns [128, 192)  local scores D[t][s] (M = 64), then the output
 //                           O^T[i][t] (M = MDV)
-//   VT  columns [192, 256)  v^T[i][s] (A operand of the intra-chunk output
-//                           and of the state write)
-// Shared memory holds the smem operands in the K-major, unswizzled
-// core-matrix layout: element (r, k) of an R x K operand at byte
-// (r/8)*32K + (k/4)*128 + (r%8)*16 + (k%4)*4.
+//   VT  columns [192, 256)  beta_s v^T[i][s] (A operand of the intra-chunk
+//                           output and of the state write)
+// Shared memory holds the smem operands unswizzled, element (r, k) of an
+// R x K K-major operand at byte (r/8)*32K + (k/4)*128 + (r%8)*16 + (k%4)*4.
 //
 // Per chunk, with Lam the running log-decay (inclusive; per channel under
 // diagonal decay), m the chunk's middle token and C its last:
 //   Qs = q e^{Lam_t - Lam_m},  Ks = k e^{Lam_m - Lam_s}
-//   scores  D[t][s] = sum_j Qs[t][j] Ks[s][j]          (M=64, N=64, K=Dk)
-//           = sum_j q_tj k_sj e^{Lam_tj - Lam_sj}
-//   output  o_t = S (q_t e^{Lam_t}) + sum_{s<=t} D[t][s] beta_s v_s
-//     scalar decay:   O^T = e^{Lam_m} (S Qs^T + VT A^T), A = D beta_s e^{-Lam_m}
-//     diagonal decay: S <- S e^{Lam_m} (per column, in tensor memory) first,
-//                     then O^T = S Qs^T + VT A^T, A = D beta_s
-//   state   S <- S e^{Lam_C - Lam_m} (diagonal) or S e^{Lam_C} (scalar), then
-//           S[i][j] += sum_s VT[i][s] KbT[j][s],  KbT = Ks[s][j] beta_s e^{Lam_C - Lam_m}
-//           (= beta_s k_sj e^{Lam_C - Lam_s}; KbT is formed from the staged
-//           Ks, so k is rounded to TF32 twice on this path)
+//   S is held as P = S_in e^{Lam_m} (column j scaled by e^{Lam_mj})
+//   scores  D[t][s] = sum_j Qs[t][j] Ks[s][j] = q_t . k_s e^{Lam_t - Lam_s}
+//                                                     (M=64, N=64, K=Dk)
+//   output  O^T = P Qs^T + VT A^T,  A = D masked to s <= t   (M=Dv, N=64)
+//           (= S_in q_t e^{Lam_t} + sum_{s<=t} D[t][s] beta_s v_s)
+//   state   P += VT KbT^T with KbT[j][s] = Ks[s][j], an exact transposed copy
+//           formed while the scores run (M=Dv, N=Dk, K=64); then
+//           S_out = P e^{Lam_C - Lam_m}, folded into the next chunk's
+//           pre-scale (one FP32 pass over S per chunk) or into the store of
+//           the tile's final state.
 // The factors e^{+-(Lam_t - Lam_m)} stay in range while a chunk decays a
 // channel by at most e^-170.
 //
@@ -68,21 +64,22 @@ constexpr int kTcMinSmem = 80 * 1024;
 constexpr long long kTcSpinLimit = 1ll << 22;
 
 struct TcLayout {
-  int qs, ks, kbt, lam, beta, lamc, part, misc, total;
+  int qs, ks, kbt, a, lam, beta, lamc, part, misc, total;
   __host__ __device__ TcLayout(int dk, bool diag) {
     constexpr int C = kTcChunk;
     int off = 0;
     qs = off;   off += C * dk * 4;   // A operand of the scores, B operand of the state read
-    ks = off;   off += C * dk * 4;   // B operand of the scores, then A[t][s]
-    kbt = off;  off += dk * C * 4;   // B operand of the state write
+    ks = off;   off += C * dk * 4;   // Ks: B operand of the scores
+    kbt = off;  off += dk * C * 4;   // KbT[j][s] = Ks[s][j]: B operand of the state write
+    a = off;    off += C * C * 4;    // local scores A[t][s], B operand of the intra-chunk output
     // diagonal: Lam[t][j] (row stride dk + 4); scalar: Lam[t], e^{Lam_t - Lam_m}, e^{Lam_m - Lam_t}
     lam = off;  off += diag ? C * (dk + 4) * 4 : 3 * C * 4;
     beta = off; off += C * 4;
-    // diagonal: per channel e^{Lam_C - Lam_m}, e^{Lam_m}; scalar: e^{Lam_C - Lam_m},
-    // e^{Lam_C}, e^{Lam_m}, e^{-Lam_m}
-    lamc = off; off += diag ? 2 * dk * 4 : 16;
+    // per channel (diagonal) or one value (scalar): e^{Lam_m}, e^{Lam_C - Lam_m} of this
+    // chunk and e^{Lam_C - Lam_m} of the previous chunk
+    lamc = off; off += diag ? 3 * dk * 4 : 16;
     part = off; off += diag ? kTcThreads * 4 : 0;  // diagonal: per-thread partial log sums
-    misc = off; off += 16;           // mbarrier, tensor-memory base, failure flag
+    misc = off; off += 16;                         // mbarrier, tensor-memory base, failure flag
     total = off;
   }
   __host__ __device__ int bytes() const { return total > kTcMinSmem ? total : kTcMinSmem; }
@@ -249,19 +246,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   using namespace tc;
   constexpr int C = kTcChunk;
   constexpr int LS = DK + 4;  // row stride of the diagonal-decay Lam table
+  constexpr int NF = DIAG ? DK : 1;  // decay factors per chunk
   static_assert(DK == 64 || DK == 128, "Dk");
   static_assert(MDV == 64 || MDV == 128, "accumulator rows");
   static_assert(kTcThreads == 512, "16 warps: four per tensor-memory lane quadrant");
   extern __shared__ __align__(1024) unsigned char tsm[];
   const TcLayout Ly(DK, DIAG);
   unsigned char* sQs = tsm + Ly.qs;
-  unsigned char* sKs = tsm + Ly.ks;  // then the scores A[t][s]
+  unsigned char* sKs = tsm + Ly.ks;
   unsigned char* sKbT = tsm + Ly.kbt;
+  unsigned char* sA = tsm + Ly.a;
   float* lam = reinterpret_cast<float*>(tsm + Ly.lam);
   float* fq = lam + C;      // scalar: e^{Lam_t - Lam_m}
   float* fk = lam + 2 * C;  // scalar: e^{Lam_m - Lam_t}
   float* bt = reinterpret_cast<float*>(tsm + Ly.beta);
-  float* lamc = reinterpret_cast<float*>(tsm + Ly.lamc);
+  float* pre = reinterpret_cast<float*>(tsm + Ly.lamc);  // e^{Lam_m}
+  float* post = pre + NF;                                 // e^{Lam_C - Lam_m}
+  float* carry = pre + 2 * NF;                            // the previous chunk's post
   uint64_t* mbar_p = reinterpret_cast<uint64_t*>(tsm + Ly.misc);
   volatile uint32_t* tslot = reinterpret_cast<volatile uint32_t*>(tsm + Ly.misc + 8);
   volatile int* failed = reinterpret_cast<volatile int*>(tsm + Ly.misc + 12);
@@ -304,22 +305,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     fence_after();
     return *failed == 0;
   };
-  // Scale this warp's state columns in tensor memory (per column under
-  // diagonal decay: f[c]; scalar: f[0]).
-  auto scale_state = [&](const float* f) {
-#pragma unroll
-    for (int c = cS0; c < cS1; c += 16) {
-      float r[16];
-      tm_ld16(tw + kTcColS + c, r);
-      wait_ld();
-#pragma unroll
-      for (int u = 0; u < 16; ++u) r[u] *= DIAG ? f[c + u] : f[0];
-      tm_st16(tw + kTcColS + c, r);
-    }
-  };
 
   int tile = blockIdx.x, ch = 0;
-  bool pending = false;  // the state write of the previous chunk is in flight
+  bool pending = false;   // the state write of the previous chunk is in flight
   TcInputs<DK> in;
   if (tile < tiles) tc_load<DK>(in, p, static_cast<size_t>(tile) * p.L, min(C, p.L), warp, lane, irow, ivalid, DIAG);
 
@@ -329,31 +317,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const size_t tok0 = static_cast<size_t>(tile) * p.L + c0;
     const int m = (Ce - 1) / 2;
 
-    // ---- initial state of the tile into tensor memory (this warp's rows, a quarter of the columns)
-    if (ch == 0) {
-      const float* src = p.S + (static_cast<size_t>(tile) * dv + (ivalid ? irow : 0)) * DK;
-#pragma unroll
-      for (int c = cS0; c < cS1; c += 16) {
-        float r[16];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float4 x = ivalid ? __ldg(reinterpret_cast<const float4*>(src + c) + u)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-          r[4 * u] = x.x; r[4 * u + 1] = x.y; r[4 * u + 2] = x.z; r[4 * u + 3] = x.w;
-        }
-        tm_st16(tw + kTcColS + c, r);
-      }
-      wait_st();
-    }
-    // the previous chunk's readers of lam, beta and the operands are done
+    // the previous chunk's readers of lam, beta and the factors are done
     __syncthreads();
 
-    // ---- beta, the running log-decay and the decay factors
+    // ---- beta, the running log-decay and the decay factors (post moves to carry)
     if (tid < C) bt[tid] = in.b;
     if constexpr (DIAG) {
       // thread (j, part) scans TP tokens of channel j; the parts' totals are
       // then added in order
-      constexpr int TP = TcInputs<DK>::TP;
+      constexpr int TP = C * DK / kTcThreads;
       float* psum = reinterpret_cast<float*>(tsm + Ly.part);
       const int j = tid % DK, pt = tid / DK;
       float acc = 0.0f, loc[TP];
@@ -376,8 +348,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       __syncthreads();
       if (tid < DK) {
         const float lC = lam[(C - 1) * LS + tid], lm = lam[m * LS + tid];
-        lamc[tid] = expf(lC - lm);
-        lamc[DK + tid] = expf(lm);
+        carry[tid] = ch == 0 ? 1.0f : post[tid];
+        pre[tid] = expf(lm);
+        post[tid] = expf(lC - lm);
       }
     } else {
       if (warp == 0) {
@@ -398,21 +371,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         fk[lane] = expf(lm - x0);
         fk[32 + lane] = expf(lm - x1);
         if (lane == 0) {
-          lamc[0] = expf(lC - lm);
-          lamc[1] = expf(lC);
-          lamc[2] = expf(lm);
-          lamc[3] = expf(-lm);
+          carry[0] = ch == 0 ? 1.0f : post[0];
+          pre[0] = expf(lm);
+          post[0] = expf(lC - lm);
         }
       }
     }
     __syncthreads();
 
-    // ---- operands Qs, Ks from the registers
+    // ---- operands Qs, Ks from the registers (the previous chunk's state
+    // write reads KbT and VT only)
 #pragma unroll
     for (int i = 0; i < TcInputs<DK>::IQ; ++i) {
-      const int it = warp + 16 * i;
-      const int t = 8 * (it & 7) + (lane & 7);
-      const int j = 16 * (it >> 3) + 4 * (lane >> 3);
+      const int itm = warp + 16 * i;
+      const int t = 8 * (itm & 7) + (lane & 7);
+      const int j = 16 * (itm >> 3) + 4 * (lane >> 3);
       const float4 qv = in.q[i], kv = in.k[i];
       const uint32_t o = cm_off(t, j, DK);
       if constexpr (DIAG) {
@@ -428,24 +401,52 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         st_shared4(sKs, o, tf32(kv.x * ek), tf32(kv.y * ek), tf32(kv.z * ek), tf32(kv.w * ek));
       }
     }
+
     // ---- the previous chunk's state write has read VT and KbT and written S
     if (pending) {
       if (!wait_mma()) break;
       pending = false;
     }
-    // ---- VT[i][s] into tensor memory (this warp's rows, a quarter of the tokens)
+    // ---- the initial state of a tile into tensor memory
+    if (ch == 0) {
+      const float* src = p.S + (static_cast<size_t>(tile) * dv + (ivalid ? irow : 0)) * DK;
+#pragma unroll
+      for (int c = cS0; c < cS1; c += 16) {
+        float r[16];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 x = ivalid ? __ldg(reinterpret_cast<const float4*>(src + c) + u)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+          r[4 * u] = x.x; r[4 * u + 1] = x.y; r[4 * u + 2] = x.z; r[4 * u + 3] = x.w;
+        }
+        tm_st16(tw + kTcColS + c, r);
+      }
+      wait_st();
+    }
+    // ---- state pass: P <- P e^{Lam_C - Lam_m} (previous chunk) e^{Lam_m} (this chunk)
+#pragma unroll
+    for (int c = cS0; c < cS1; c += 16) {
+      float r[16];
+      tm_ld16(tw + kTcColS + c, r);
+      wait_ld();
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int f = DIAG ? c + u : 0;
+        r[u] *= carry[f] * pre[f];
+      }
+      tm_st16(tw + kTcColS + c, r);
+    }
+    // ---- VT[i][s] = beta_s v_si into tensor memory (this warp's rows, a quarter of the tokens)
     {
       float r[16];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) r[e] = tf32(in.v[e]);
+      for (int e = 0; e < 16; ++e) r[e] = tf32(bt[(C / 4) * qt + e] * in.v[e]);
       tm_st16(tw + kTcColV + (C / 4) * qt, r);
     }
-    // ---- diagonal decay: S <- S e^{Lam_m} for the state read
-    if constexpr (DIAG) scale_state(lamc + DK);
     fence_async_smem();
     wait_st();
     fence_before();
-    __syncthreads();  // Qs, Ks, VT complete
+    __syncthreads();  // Qs, Ks, VT, S complete
 
     // ---- local scores
     if (tid == 0) {
@@ -457,42 +458,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                id, kk > 0);
       mma_commit(mbar);
     }
-    // ---- while the scores run: KbT[j][s] = Ks[s][j] beta_s e^{Lam_C - Lam_m}
+    // ---- while the scores run: KbT[j][s] = Ks[s][j] (an exact copy)
 #pragma unroll
     for (int i = 0; i < DK / 32; ++i) {
-      const int it = warp + 16 * i;
-      const int j = 8 * (it % (DK / 8)) + (lane & 7);
-      const int s = 16 * (it / (DK / 8)) + 4 * (lane >> 3);
-      const float f = DIAG ? lamc[j] : lamc[0];
+      const int itm = warp + 16 * i;
+      const int j = 8 * (itm % (DK / 8)) + (lane & 7);
+      const int s = 16 * (itm / (DK / 8)) + 4 * (lane >> 3);
       float w[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        w[u] = tf32(*reinterpret_cast<const float*>(sKs + cm_off(s + u, j, DK)) * (f * bt[s + u]));
+      for (int u = 0; u < 4; ++u) w[u] = *reinterpret_cast<const float*>(sKs + cm_off(s + u, j, DK));
       st_shared4(sKbT, cm_off(j, s, C), w[0], w[1], w[2], w[3]);
     }
     fence_async_smem();
-    if (!wait_mma()) break;  // scores done; every warp is done with Ks
+    if (!wait_mma()) break;
 
-    // ---- A[t][s] (into the Ks region: the scores have read it)
-    {
-      const float sa = DIAG ? 1.0f : lamc[3];
+    // ---- A[t][s] = D[t][s] for s <= t
 #pragma unroll
-      for (int s0 = (C / 4) * qt; s0 < (C / 4) * (qt + 1); s0 += 16) {
-        float r[16];
-        tm_ld16(tw + kTcColX + s0, r);
-        wait_ld();
-        if (trow >= 0) {
-          const int t = trow;
+    for (int s0 = (C / 4) * qt; s0 < (C / 4) * (qt + 1); s0 += 16) {
+      float r[16];
+      tm_ld16(tw + kTcColX + s0, r);
+      wait_ld();
+      if (trow >= 0) {
+        const int t = trow;
 #pragma unroll
-          for (int u = 0; u < 16; u += 4) {
-            float a[4];
+        for (int u = 0; u < 16; u += 4) {
+          float a[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int s = s0 + u + e;
-              a[e] = (s <= t && t < Ce) ? tf32(r[u + e] * (bt[s] * sa)) : 0.0f;
-            }
-            st_shared4(sKs, cm_off(t, s0 + u, C), a[0], a[1], a[2], a[3]);
-          }
+          for (int e = 0; e < 4; ++e) a[e] = (s0 + u + e <= t && t < Ce) ? tf32(r[u + e]) : 0.0f;
+          st_shared4(sA, cm_off(t, s0 + u, C), a[0], a[1], a[2], a[3]);
         }
       }
     }
@@ -509,7 +502,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mma_ts(tbase + kTcColX, tbase + kTcColS + 8 * kk, sdesc(saddr(sQs) + 256 * kk, DK * 32), id, kk > 0);
 #pragma unroll
       for (int kk = 0; kk < C / 8; ++kk)
-        mma_ts(tbase + kTcColX, tbase + kTcColV + 8 * kk, sdesc(saddr(sKs) + 256 * kk, C * 32), id, 1u);
+        mma_ts(tbase + kTcColX, tbase + kTcColV + 8 * kk, sdesc(saddr(sA) + 256 * kk, C * 32), id, 1u);
       mma_commit(mbar);
     }
     // ---- the next chunk's loads, in flight from here to the next chunk's staging
@@ -519,12 +512,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_load<DK>(in, p, static_cast<size_t>(ntile) * p.L + nchk * C, min(C, p.L - nchk * C), warp, lane,
                   irow, ivalid, DIAG);
     if (!wait_mma()) break;
-    // ---- state pass (the state read above has completed)
-    scale_state(DIAG ? lamc : lamc + 1);
-    wait_st();
-    fence_before();
-    __syncthreads();
-    // ---- state write: S += VT KbT^T, in flight while the outputs are written
+
+    // ---- state write: P += VT Ks^T, in flight while the outputs are written
     if (tid == 0) {
       fence_after();
       constexpr uint32_t id = idesc_tf32(MDV, DK);
@@ -534,23 +523,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mma_commit(mbar);
     }
     pending = true;
-    {
-      const float so = DIAG ? 1.0f : lamc[2];
+    if (p.o != nullptr) {
 #pragma unroll
       for (int t0 = (C / 4) * qt; t0 < (C / 4) * (qt + 1); t0 += 16) {
         float r[16];
         tm_ld16(tw + kTcColX + t0, r);
         wait_ld();
-        if (ivalid && p.o != nullptr) {
+        if (ivalid) {
 #pragma unroll
           for (int u = 0; u < 16; ++u)
-            if (t0 + u < Ce) p.o[(tok0 + t0 + u) * dv + irow] = DIAG ? r[u] : r[u] * so;
+            if (t0 + u < Ce) p.o[(tok0 + t0 + u) * dv + irow] = r[u];
         }
       }
     }
     fence_before();
 
-    // ---- final state of the tile out of tensor memory
+    // ---- final state of the tile: S_out = P e^{Lam_C - Lam_m}
     if (ch == nch - 1) {
       if (!wait_mma()) break;
       pending = false;
@@ -562,10 +550,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         wait_ld();
         if (ivalid) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-            reinterpret_cast<float4*>(dst + c)[u] = make_float4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
+          for (int u = 0; u < 4; ++u) {
+            const int f = DIAG ? c + 4 * u : 0;
+            reinterpret_cast<float4*>(dst + c)[u] =
+                make_float4(r[4 * u] * post[f], r[4 * u + 1] * post[DIAG ? f + 1 : 0],
+                            r[4 * u + 2] * post[DIAG ? f + 2 : 0], r[4 * u + 3] * post[DIAG ? f + 3 : 0]);
+          }
         }
       }
+      fence_before();
     }
     tile = ntile;
     ch = nchk;

@@ -124,6 +124,8 @@ TF32_CASES = [
     (128, 112, "scalar", 3, 64, True),
     (64, 128, "diagonal", 2, 65, True),
     (128, 128, "scalar", 300, 130, True),
+    (64, 64, "scalar", 4, 1000, True),
+    (128, 64, "diagonal", 3, 300, True),
 ]
 
 
