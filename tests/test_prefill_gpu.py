@@ -181,3 +181,46 @@ def test_prefill_tf32_on_workload_laws(wname):
     torch.cuda.synchronize()
     _check_bound("state", S.cpu().numpy(), S_ref, S_mag)
     _check_bound("outputs", o.cpu().numpy(), o_ref, o_mag)
+
+
+@pytest.mark.parametrize("wname", ["mamba2", "gla"])
+def test_prompt_then_quantized_state(wname):
+    """The path a prompt takes into decode: the tensor-core prefill leaves S,
+    qstate_init quantizes it (dynamic rule, nearest) and qstate_readout reads
+    it, against the oracle's token-by-token FP32 state S_ref.  Bound, element
+    by element: |c s - S_ref| <= s/2 (rounding at the group's scale s, which
+    the dynamic rule keeps in range) + 2^-8 * S_mag (the prefill's bound), and
+    for the readout the same terms times |q_j| summed over j, plus the FP32
+    rounding of that sum."""
+    import torch
+    from ssm_decode_step_b200 import QState, qstate as Q
+    w = W.scaled_down(W.get(wname), 32)
+    T, L = w.tiles, 200
+    slots = [W.slot(w, t) for t in range(L)]
+    q, k, v, a, b = (np.ascontiguousarray(np.stack([s[i] for s in slots], axis=1)) for i in range(5))
+    S0 = np.zeros((T, w.dv, w.dk), np.float32)
+    S_ref, _ = _reference(T, w.dk, w.dv, w.decay, S0, q, k, v, a, b)
+    S_mag, _ = _reference(T, w.dk, w.dv, w.decay, S0, np.abs(q), np.abs(k), np.abs(v), a, b)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    S = dev(S0)
+    Q.prefill_tf32(Config(T, w.dk, w.dv, 8, 32, 0, w.decay), L, S, dev(q), dev(k), dev(v), dev(a), dev(b))
+    cfg = Config(T, w.dk, w.dv, 8, 32, 0, w.decay, "dynamic")
+    st = QState(cfg).init(S)
+    qr = np.random.default_rng(17).standard_normal((T, w.dk)).astype(np.float32)
+    o = torch.empty((T, w.dv), dtype=torch.float32, device="cuda")
+    st.readout(dev(qr), o)
+    torch.cuda.synchronize()
+    codes = st.codes.cpu().numpy().view(np.int8).astype(np.float32)   # INT8: one code per element
+    scales = st.scales.cpu().numpy()                                     # [T][dv][dk/32]
+    s_el = np.repeat(scales, 32, axis=2)
+    deq = codes * s_el
+    bound = 0.5 * s_el * (1 + 2.0 ** -20) + TOL_TF32 * S_mag + 1e-30
+    err = np.abs(deq.astype(np.float64) - S_ref)
+    assert (err <= bound).all(), f"dequantized state off by {float((err / bound).max()):.3g} x its bound"
+    o_ref = np.einsum("tij,tj->ti", S_ref.astype(np.float64), qr.astype(np.float64))
+    # plus the FP32 rounding of the readout's own sum (at most Dk * 2^-24 of
+    # the sum of magnitudes, taken as 2^-16)
+    o_bound = (np.einsum("tij,tj->ti", bound, np.abs(qr).astype(np.float64))
+               + 2.0 ** -16 * np.einsum("tij,tj->ti", np.abs(deq).astype(np.float64), np.abs(qr).astype(np.float64)))
+    o_err = np.abs(o.cpu().numpy().astype(np.float64) - o_ref)
+    assert (o_err <= o_bound).all(), f"readout off by {float((o_err / o_bound).max()):.3g} x its bound"
