@@ -8,6 +8,16 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def pytest_sessionstart(session):
+    """Build the CUDA library and the oracle if they are missing or stale
+    (both builders return at once when up to date), so that the suite runs
+    from a fresh checkout."""
+    from oracle import build as oracle_build
+    from ssm_decode_step_b200 import build as cuda_build
+    oracle_build.build()
+    cuda_build.build()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long CPU test")
