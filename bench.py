@@ -96,7 +96,7 @@ def source_sha() -> str:
         with open(os.path.join(pkg, "csrc", f), "rb") as fh:
             h.update(f.encode() + fh.read())
     from ssm_decode_step_b200 import build as B
-    h.update(" ".join(B.NVFLAGS).encode())
+    h.update(B.flags_key().encode())
     return h.hexdigest()[:16]
 
 

@@ -27,6 +27,20 @@ NVFLAGS = ARCH + ["-O3", "-std=c++17", "-lineinfo", "-fmad=false", "-Xcompiler",
 NVFLAGS += os.environ.get("QSTATE_NVCC_FLAGS", "").split()
 
 
+def flags_key() -> str:
+    """The nvcc flags without include directories (which name this checkout's
+    location): what the library's code depends on."""
+    out, skip = [], False
+    for f in NVFLAGS:
+        if skip:
+            skip = False
+        elif f == "-I":
+            skip = True
+        elif not f.startswith("-I"):
+            out.append(f)
+    return " ".join(out)
+
+
 def nvcc() -> str:
     for cand in (os.environ.get("NVCC"), shutil.which("nvcc"), "/usr/local/cuda/bin/nvcc"):
         if cand and os.path.exists(cand):
@@ -51,7 +65,7 @@ def _up_to_date() -> bool:
     if not (os.path.exists(LIB) and os.path.exists(STAMP)):
         return False
     with open(STAMP) as f:
-        if f.read() != " ".join(NVFLAGS):
+        if f.read() != flags_key():
             return False
     t = os.path.getmtime(LIB)
     return all(os.path.getmtime(d) <= t for d in _deps())
@@ -85,7 +99,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
         raise RuntimeError(f"link failed:\n{r.stderr}")
     os.replace(tmp, LIB)
     with open(STAMP, "w") as f:
-        f.write(" ".join(NVFLAGS))
+        f.write(flags_key())
     return LIB
 
 
