@@ -262,6 +262,16 @@ QS_API qs_status qstate_prefill_tf32(const qs_config* cfg, int length, float* S,
  * up since the library was loaded (current device; synchronous). */
 QS_API qs_status qstate_prefill_tf32_timeouts(unsigned int* count);
 
+/* Self-check of that bounded wait: launches one CTA of the tensor-core
+ * prefill kernel in a mode whose first wait for the tensor cores cannot
+ * complete (nothing has been committed to it), with a limit of `polls`
+ * polls; the CTA must give up, count the timeout, free its tensor memory
+ * and return, leaving the context usable.  Synchronous on the legacy
+ * default stream; *timed_out receives the number of CTAs that reported a
+ * timeout (1 when the mechanism works).  polls in [1, 2^20], else
+ * QS_ERR_INVALID_ARG before any launch. */
+QS_API qs_status qstate_prefill_tf32_wait_selfcheck(unsigned int polls, unsigned int* timed_out);
+
 /* Squared Frobenius norm of every tile of the stored state, for tracking
  * the state norm over a decode horizon (the norm inflation of per-token
  * dynamic scaling: "When Dynamic Scaling Fails", abstract and project page,

@@ -477,6 +477,7 @@ qs_status prefill_args(const qs_config* cfg, int length, float* S, const float* 
   p->o = o;
   p->L = length;
   p->dv = c.dv;
+  p->wait_probe = 0;
   *out = c;
   *work = true;
   return QS_OK;
@@ -525,6 +526,26 @@ qs_status qstate_prefill_tf32(const qs_config* cfg, int length, float* S, const 
     e = c.dv <= 64 ? QS_TC(128, 64) : QS_TC(128, 128);
 #undef QS_TC
   return from_cuda(e);
+}
+
+qs_status qstate_prefill_tf32_wait_selfcheck(unsigned int polls, unsigned int* timed_out) {
+  if (timed_out == nullptr || polls == 0 || polls > (1u << 20)) return QS_ERR_INVALID_ARG;
+  unsigned int* timeouts = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&timeouts), qs_tc_timeouts);
+  unsigned int before = 0, after = 0;
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&before, qs_tc_timeouts, sizeof(unsigned int));
+  if (e != cudaSuccess) return from_cuda(e);
+  qs::PrefillParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.L = 1;
+  p.dv = 64;
+  p.wait_probe = static_cast<int>(polls);
+  e = qs::launch_prefill_tc<64, 64, false>(p, 1, timeouts, nullptr);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(nullptr);
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&after, qs_tc_timeouts, sizeof(unsigned int));
+  if (e != cudaSuccess) return from_cuda(e);
+  *timed_out = after - before;
+  return QS_OK;
 }
 
 qs_status qstate_prefill_tf32_timeouts(unsigned int* count) {

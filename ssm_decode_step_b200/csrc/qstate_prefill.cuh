@@ -41,6 +41,7 @@ struct PrefillParams {
   float* o;            // [T][L][dv] or nullptr
   int L;
   int dv;
+  int wait_probe;      // tensor-core path only: > 0 runs the bounded-wait self-check instead
 };
 
 // Shared-memory layout (floats) of one CTA.

@@ -143,9 +143,9 @@ __device__ __forceinline__ void mbar_init(uint32_t mbar) {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 // Wait for the phase with the given parity to complete; false after
-// kTcSpinLimit polls.
-__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
-  for (long long i = 0; i < kTcSpinLimit; ++i) {
+// `limit` polls.
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, long long limit = kTcSpinLimit) {
+  for (long long i = 0; i < limit; ++i) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -306,12 +306,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     return *failed == 0;
   };
 
+  // Bounded-wait self-check: nothing has been committed, so this wait cannot
+  // complete; it must give up after p.wait_probe polls, and the CTA then
+  // skips all work, frees its tensor memory and returns.
+  int ntiles = tiles;
+  if (p.wait_probe > 0) {
+    if (warp == 0 && !mbar_wait(mbar, phase, p.wait_probe)) *failed = 1;
+    __syncthreads();
+    ntiles = 0;
+  }
+
   int tile = blockIdx.x, ch = 0;
   bool pending = false;   // the state write of the previous chunk is in flight
   TcInputs<DK> in;
-  if (tile < tiles) tc_load<DK>(in, p, static_cast<size_t>(tile) * p.L, min(C, p.L), warp, lane, irow, ivalid, DIAG);
+  if (tile < ntiles) tc_load<DK>(in, p, static_cast<size_t>(tile) * p.L, min(C, p.L), warp, lane, irow, ivalid, DIAG);
 
-  while (tile < tiles) {
+  while (tile < ntiles) {
     const int c0 = ch * C;
     const int Ce = min(C, p.L - c0);
     const size_t tok0 = static_cast<size_t>(tile) * p.L + c0;
@@ -508,7 +518,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ---- the next chunk's loads, in flight from here to the next chunk's staging
     int ntile = tile, nchk = ch + 1;
     if (nchk == nch) { nchk = 0; ntile += gridDim.x; }
-    if (ntile < tiles)
+    if (ntile < ntiles)
       tc_load<DK>(in, p, static_cast<size_t>(ntile) * p.L + nchk * C, min(C, p.L - nchk * C), warp, lane,
                   irow, ivalid, DIAG);
     if (!wait_mma()) break;

@@ -26,6 +26,7 @@ QS_OK, QS_ERR_INVALID_ARG, QS_ERR_UNSUPPORTED, QS_ERR_CUDA = 0, 1, 2, 3
 EXPORTS = ("qstate_query_sizes", "qstate_init", "qstate_decode_step", "qstate_readout",
            "qstate_fp32_decode_step", "qstate_lrb_query_sizes", "qstate_lrb_decode_step",
            "qstate_prefill", "qstate_prefill_tf32", "qstate_prefill_tf32_timeouts",
+           "qstate_prefill_tf32_wait_selfcheck",
            "qstate_state_sq_norms", "qstate_fp32_sq_norms",
            "qstate_selfcheck", "qstate_status_string", "qstate_version")
 
@@ -65,12 +66,14 @@ def lib() -> ctypes.CDLL:
         L.qstate_prefill.argtypes = [C, ctypes.c_int] + [P] * 8
         L.qstate_prefill_tf32.argtypes = [C, ctypes.c_int] + [P] * 8
         L.qstate_prefill_tf32_timeouts.argtypes = [P]
+        L.qstate_prefill_tf32_wait_selfcheck.argtypes = [ctypes.c_uint, P]
         L.qstate_state_sq_norms.argtypes = [C, P, P, P, P]
         L.qstate_fp32_sq_norms.argtypes = [C, P, P, P]
         for f in (L.qstate_query_sizes, L.qstate_init, L.qstate_decode_step, L.qstate_readout,
                   L.qstate_selfcheck, L.qstate_fp32_decode_step, L.qstate_state_sq_norms,
                   L.qstate_fp32_sq_norms, L.qstate_lrb_query_sizes, L.qstate_lrb_decode_step,
-                  L.qstate_prefill, L.qstate_prefill_tf32, L.qstate_prefill_tf32_timeouts):
+                  L.qstate_prefill, L.qstate_prefill_tf32, L.qstate_prefill_tf32_timeouts,
+                  L.qstate_prefill_tf32_wait_selfcheck):
             f.restype = ctypes.c_int
         L.qstate_status_string.argtypes = [ctypes.c_int]
         L.qstate_status_string.restype = ctypes.c_char_p
@@ -238,6 +241,15 @@ def prefill_tf32_timeouts() -> int:
     """CTAs of prefill_tf32 whose bounded wait for the tensor cores gave up."""
     n = ctypes.c_uint(0)
     _check(lib().qstate_prefill_tf32_timeouts(ctypes.byref(n)), "qstate_prefill_tf32_timeouts")
+    return n.value
+
+
+def prefill_tf32_wait_selfcheck(polls: int = 1000) -> int:
+    """Run the bounded-wait self-check of the tensor-core prefill; returns the
+    number of CTAs that reported a timeout (1 when the mechanism works)."""
+    n = ctypes.c_uint(0)
+    _check(lib().qstate_prefill_tf32_wait_selfcheck(polls, ctypes.byref(n)),
+           "qstate_prefill_tf32_wait_selfcheck")
     return n.value
 
 

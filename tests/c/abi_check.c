@@ -43,6 +43,10 @@ int main(void) {
   check(qstate_prefill_tf32(&pf, 8, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL) == QS_ERR_UNSUPPORTED,
         "tensor-core prefill rejects the delta rule");
 
+  unsigned int timed_out = 0;
+  check(qstate_prefill_tf32_wait_selfcheck(0, &timed_out) == QS_ERR_INVALID_ARG,
+        "wait self-check rejects a zero poll limit before any launch");
+
   const char* s = qstate_status_string(QS_OK);
   check(s != NULL && strlen(s) > 0, "status strings are defined");
   check(qstate_version() > 0, "version is positive");

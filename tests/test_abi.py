@@ -197,6 +197,10 @@ def test_prefill_tf32_validation():
     with pytest.raises(Q.QStateError):
         lib_call = lib.qstate_prefill_tf32_timeouts(None)
         Q._check(lib_call, "qstate_prefill_tf32_timeouts")
+    n = ctypes.c_uint(0)
+    assert lib.qstate_prefill_tf32_wait_selfcheck(0, ctypes.byref(n)) == Q.QS_ERR_INVALID_ARG
+    assert lib.qstate_prefill_tf32_wait_selfcheck(1 << 21, ctypes.byref(n)) == Q.QS_ERR_INVALID_ARG
+    assert lib.qstate_prefill_tf32_wait_selfcheck(1000, None) == Q.QS_ERR_INVALID_ARG
 
 
 def test_binding_raises():

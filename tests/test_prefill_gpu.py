@@ -224,3 +224,29 @@ def test_prompt_then_quantized_state(wname):
                + 2.0 ** -16 * np.einsum("tij,tj->ti", np.abs(deq).astype(np.float64), np.abs(qr).astype(np.float64)))
     o_err = np.abs(o.cpu().numpy().astype(np.float64) - o_ref)
     assert (o_err <= o_bound).all(), f"readout off by {float((o_err / o_bound).max()):.3g} x its bound"
+
+
+def test_bounded_wait_gives_up_and_leaves_the_context_usable():
+    """The tensor-core prefill's waits are bounded: a CTA launched so that its
+    first wait cannot complete (nothing committed) gives up after the poll
+    limit, counts one timeout, frees its tensor memory and returns; the next
+    prefill on the same context runs normally and counts none."""
+    import torch
+    from ssm_decode_step_b200 import qstate as Q
+    before = Q.prefill_tf32_timeouts()
+    assert Q.prefill_tf32_wait_selfcheck(1000) == 1
+    assert Q.prefill_tf32_timeouts() == before + 1
+    dk, dv, decay, T, L = 128, 64, "scalar", 3, 70
+    rng = np.random.default_rng(23)
+    S0 = (rng.standard_normal((T, dv, dk)) * 0.1).astype(np.float32)
+    q, k, v, a, b = _inputs(rng, T, L, dk, dv, decay)
+    S_ref, o_ref = _reference(T, dk, dv, decay, S0, q, k, v, a, b)
+    S_mag, o_mag = _reference(T, dk, dv, decay, np.abs(S0), np.abs(q), np.abs(k), np.abs(v), a, b)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    S = dev(S0)
+    o = torch.empty((T, L, dv), dtype=torch.float32, device="cuda")
+    Q.prefill_tf32(Config(T, dk, dv, 8, 32, 0, decay), L, S, dev(q), dev(k), dev(v), dev(a), dev(b), o)
+    torch.cuda.synchronize()
+    assert Q.prefill_tf32_timeouts() == before + 1
+    _check_bound("state", S.cpu().numpy(), S_ref, S_mag)
+    _check_bound("outputs", o.cpu().numpy(), o_ref, o_mag)
