@@ -70,6 +70,8 @@ __global__ void __launch_bounds__(kThreads, QS_MIN_BLOCKS) fp32_step_kernel(Step
   const int tid = threadIdx.x;
   const int c = tid % LPR, r0 = tid / LPR;
   const bool readout = p.o != nullptr;
+  grid_dep_wait();
+  grid_dep_launch();
 
   UnitCursor pre(blockIdx.x, p);
 #pragma unroll

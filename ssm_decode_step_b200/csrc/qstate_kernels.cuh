@@ -110,6 +110,17 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may be scheduled while the previous kernel of its stream is
+// still running; grid_dep_wait() returns once that kernel has completed and
+// its writes are visible, so every such kernel calls it before its first
+// global-memory access.  grid_dep_launch() lets the next kernel of the stream
+// be scheduled from here on (its CTAs take SM slots as ours retire and wait
+// in their own grid_dep_wait()).  Launched without the attribute, both do
+// nothing.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
 
 template <int N>

@@ -1,6 +1,7 @@
 // Definitions of the launchers declared in qstate_launch.h.
 #pragma once
 
+#include <cstdlib>
 #include <mutex>
 
 #include "qstate_launch.h"
@@ -25,6 +26,35 @@ static cudaError_t allow_smem(K kernel, std::once_flag& flag) {
   return err;
 }
 
+// Programmatic dependent launch for the streaming kernels (step, Low-Rank
+// Bypass step, readout, FP32-state step): each may be scheduled while the
+// kernel before it in the stream finishes, and waits for it in
+// grid_dep_wait() before touching global memory.  QSTATE_PDL=0 in the
+// environment launches them plainly.
+static bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("QSTATE_PDL");
+    return !(e && e[0] == '0' && e[1] == '\0');
+  }();
+  return on;
+}
+
+template <typename K, typename P>
+static cudaError_t launch_dependent(K kernel, long long grid, int threads, size_t smem,
+                                    cudaStream_t stream, const P& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 template <typename K>
 static cudaError_t launch_persistent(K kernel, size_t smem, const StepParams& p,
                                      cudaStream_t stream) {
@@ -38,8 +68,7 @@ static cudaError_t launch_persistent(K kernel, size_t smem, const StepParams& p,
   StepParams q = p;
   q.grid_tiles = static_cast<int>(grid / p.units_per_tile);
   q.grid_part = static_cast<int>(grid % p.units_per_tile);
-  kernel<<<static_cast<int>(grid), kThreads, smem, stream>>>(q);
-  return cudaGetLastError();
+  return launch_dependent(kernel, grid, kThreads, smem, stream, q);
 }
 
 // Launch a one-warp-per-range kernel (step, Low-Rank Bypass step, readout):
@@ -53,8 +82,7 @@ static cudaError_t launch_warps(K kernel, const P& p, size_t smem, cudaStream_t 
   long long grid = static_cast<long long>(per_sm) * device_sm_count();
   const long long need = (static_cast<long long>(p.nblocks) + kStepWarps - 1) / kStepWarps;
   if (grid > need) grid = need;
-  kernel<<<static_cast<int>(grid), kStepThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_dependent(kernel, grid, kStepThreads, smem, stream, p);
 }
 
 template <int BITS, int DK, int POLICY, bool BDR, bool DELTA, bool DIAG>

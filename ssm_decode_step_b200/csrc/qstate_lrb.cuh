@@ -208,6 +208,8 @@ __global__ void __launch_bounds__(kStepThreads, ((POLICY == 2 || BDR || MERGE) ?
   const unsigned b1 = static_cast<unsigned>((gw + 1) * p.nblocks / nw);
   if (b0 >= b1) return;
   const unsigned bpt = static_cast<unsigned>(p.bpt);
+  grid_dep_wait();
+  grid_dep_launch();
 
   uint8_t* codes_l = p.codes + CB * lane;
   const uint8_t* codes_blk = p.codes + 16 * lane;

@@ -271,6 +271,8 @@ __global__ void __launch_bounds__(kStepThreads, ((POLICY == 2 || BDR) ? QS_STEP_
   const unsigned b1 = static_cast<unsigned>((gw + 1) * p.nblocks / nw);
   if (b0 >= b1) return;  // warp-uniform; nothing in this kernel waits for other warps
   const unsigned bpt = static_cast<unsigned>(p.bpt);
+  grid_dep_wait();
+  grid_dep_launch();
 
   // per-lane bases; row block blk adds blk times a per-block stride
   uint8_t* codes_l = p.codes + CB * lane;
@@ -537,6 +539,8 @@ __global__ void __launch_bounds__(kStepThreads, QS_STEP_WARPS_PER_SM / kStepWarp
   const unsigned b1 = static_cast<unsigned>((gw + 1) * p.nblocks / nw);
   if (b0 >= b1) return;
   const unsigned bpt = static_cast<unsigned>(p.bpt);
+  grid_dep_wait();
+  grid_dep_launch();
   const uint8_t* codes_blk = p.codes + 16 * lane;
   const unsigned sstride = RW * ng;
   const float* scales_l = p.scales + rr * ng + g;
