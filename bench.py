@@ -643,14 +643,16 @@ def run_lrb(args, w, dev, stream, dist, pool, S0, l2, pool_bytes, plain_us):
 
 
 def run_e2e(args, w, arms, cfgs, states, dev, stream, dist, host, reinit):
-    """Same steps through the public API with host buffers: per step, copy
-    the inputs from pinned host memory, launch every arm, copy the readouts
-    back; all inside the timed region.  The copies are pipelined the way a
-    serving loop would run them: step t's inputs go up on a copy stream
-    while step t-1 computes, and step t-1's readouts come down on another
-    while step t computes (two device buffers of each, ordered by events;
-    the state updates stay in order on the compute stream)."""
+    """Same steps through the library's host-buffer pipeline
+    (qstate_pipeline_step, one C call per step): per step, the packed inputs
+    are copied up from pinned host memory, every arm's step runs, and the
+    readouts are copied back to pinned host memory; all inside the timed
+    region.  The copies run on the pipeline's own streams, three steps deep,
+    so step t's inputs go up and step t-1's readouts come down while the
+    state updates run in order on the compute stream."""
+    import math
     import torch
+    from ssm_decode_step_b200 import HostPipeline
 
     K = min(args.steps, args.e2e_steps)
     P = args.pool
@@ -662,63 +664,45 @@ def run_e2e(args, w, arms, cfgs, states, dev, stream, dist, host, reinit):
     for s in range(P):
         packed[s] = torch.from_numpy(np.concatenate([a[s].reshape(-1) for a in parts]))
     readout = w.readout
-    dbuf, views = [], []
-    for _ in range(2):
-        d = torch.empty(sum(sizes), dtype=torch.float32, device=dev)
-        vs, off = [], 0
-        for a, n in zip(parts, sizes):
-            vs.append(d[off:off + n].view(a.shape[1:]))
-            off += n
-        dbuf.append(d)
-        views.append(vs)
-    o_dev = [torch.empty((len(arms), T, w.dv), dtype=torch.float32, device=dev) for _ in range(2)]
     o_host = torch.empty((P, len(arms), T, w.dv), dtype=torch.float32).pin_memory()
-    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    up = [torch.cuda.Event() for _ in range(2)]     # inputs of buffer b on the device
-    done = [torch.cuda.Event() for _ in range(2)]   # buffer b's step computed
-    down = [torch.cuda.Event() for _ in range(2)]   # buffer b's readouts copied out
+    slots_in = [packed[s] for s in range(P)]
+    slots_out = [o_host[s] if readout else None for s in range(P)]
+    # the request group each arm steps at step t (the cycle repeats every `period` steps)
+    period = math.lcm(*[len(g) for g in states])
+    combos = [tuple(g[t % len(g)] for g in states) for t in range(period)]
+    pl = HostPipeline(combos[0], depth=3)
 
     def one(t):
-        b = t % 2
-        s_in.wait_event(done[b])                     # dbuf[b] no longer read
-        with torch.cuda.stream(s_in):
-            dbuf[b].copy_(packed[t % P], non_blocking=True)
-        up[b].record(s_in)
-        stream.wait_event(up[b])
-        stream.wait_event(down[b])                   # o_dev[b] copied out
-        v = views[b]
-        for ai in range(len(arms)):
-            states[ai][t % len(states[ai])].step(v[0] if readout else None, v[1], v[2], v[3], v[4],
-                                                 o_dev[b][ai] if readout else None, stream)
-        done[b].record(stream)
-        if readout:
-            s_out.wait_event(done[b])
-            with torch.cuda.stream(s_out):
-                o_host[t % P].copy_(o_dev[b], non_blocking=True)
-            down[b].record(s_out)
+        pl.step(slots_in[t % P], slots_out[t % P], stream, combos[t % period])
 
+    # warm-up: one full cycle of the pinned slots (the first transfer to or
+    # from a page-locked page costs more than later ones, as in any serving
+    # loop that reuses its staging buffers)
     reinit()
-    for t in range(max(3, args.warmup)):
+    for t in range(max(3, args.warmup, P)):
         one(t)
-    torch.cuda.synchronize()
+    pl.sync()
     reinit()
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s_in)
+    e0.record(stream)
+    pl.wait_stream(stream)
     for t in range(K):
         one(t)
-    s_in.wait_stream(stream)
-    s_in.wait_stream(s_out)
-    e1.record(s_in)
+    pl.join(stream)
+    e1.record(stream)
     torch.cuda.synchronize()
+    pl.close()
     ms = max_over_ranks(dist, [e0.elapsed_time(e1)], dev)[0]
     ws = dist.get_world_size() if dist is not None else 1
     return {"value": round(ws * K / (ms / 1e3), 2), "unit": "steps/s",
             "h2d_bytes_per_step": int(sum(sizes) * 4),
             "d2h_bytes_per_step": int(len(arms) * T * w.dv * 4) if readout else 0,
-            "steps": K, "pipelining": "inputs up / readouts down on their own streams, two buffers"}
+            "steps": K,
+            "pipelining": "qstate_pipeline_step: inputs up / readouts down on the pipeline's "
+                          "own streams, three buffers"}
 
 
 # ---------------------------------------------------------------------------

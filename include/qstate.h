@@ -152,6 +152,70 @@ QS_API qs_status qstate_decode_step(const qs_config* cfg, void* codes, float* sc
                              const float* v, const float* alpha,
                              const float* beta, float* o, cudaStream_t stream);
 
+/* Host-buffer decode pipeline: one decode step per call, as
+ * qstate_decode_step defines it, of n state families (at most 8) that
+ * consume the same token's inputs, with the inputs read from HOST memory
+ * and the readouts written back to HOST memory.  The pipeline owns `depth`
+ * (2..8) device copies of one step's inputs and readouts, a copy-in
+ * stream, a copy-out stream and their events: step t's inputs go up on the
+ * copy-in stream while earlier steps compute, its state updates run on the
+ * caller's stream (in call order), and its readouts come down on the
+ * copy-out stream while later steps compute.
+ *
+ * Host input of one step (packed, float): q [T][Dk] | k [T][Dk] | v [T][Dv]
+ * | alpha [T] (scalar decay) or [T][Dk] (diagonal) | beta [T].  Host output
+ * of one step: o [n][T][Dv] (family i's readout at offset i*T*Dv).  Page-
+ * locked host memory makes the copies asynchronous.  The copies of step t
+ * are in flight after the call returns: the caller keeps step t's input
+ * unchanged and does not read its output until qstate_pipeline_sync has
+ * returned, or until the call for step t + depth has returned (each call
+ * first waits, on the host, for the copies of the step that last used its
+ * device buffers).
+ *
+ * All families share num_tiles, dk, dv, delta and decay (each passes
+ * qstate_decode_step's checks); they differ in bits, group, policy and
+ * rounding.  The pipeline belongs to the device current at creation; calls
+ * from another current device return QS_ERR_INVALID_ARG.  One host thread
+ * at a time may use a pipeline.  After an error
+ * from qstate_pipeline_step the pipeline may hold a partial step: sync and
+ * destroy it. */
+typedef struct qs_pipeline qs_pipeline;
+
+/* Bytes of one step's host input and host output for n families of cfg.
+ * Host-only; launches nothing. */
+QS_API qs_status qstate_pipeline_query_sizes(const qs_config* cfg, int n, size_t* in_bytes,
+                                             size_t* out_bytes);
+
+/* Create a pipeline for families cfgs[0..n-1] with `depth` buffers on the
+ * current device (device memory, two streams, events).  Arguments are
+ * checked before any CUDA call. */
+QS_API qs_status qstate_pipeline_create(int n, const qs_config* cfgs, int depth,
+                                        qs_pipeline** out);
+
+/* Issue one step.  codes[i], scales[i], shadow[i]: family i's state (as for
+ * qstate_decode_step; shadow may be NULL, or shadow[i] NULL, for families
+ * that are not yoked).  host_out == NULL skips the readouts (no output
+ * copy).  `stream` runs the state updates. */
+QS_API qs_status qstate_pipeline_step(qs_pipeline* pl, void* const* codes, float* const* scales,
+                                      float* const* shadow, const void* host_in, void* host_out,
+                                      cudaStream_t stream);
+
+/* Make the pipeline's copy streams wait for the work submitted to `stream`
+ * so far (e.g. an event that opens a timed region), without blocking the
+ * host. */
+QS_API qs_status qstate_pipeline_wait_stream(qs_pipeline* pl, cudaStream_t stream);
+
+/* Make `stream` wait for every copy the pipeline has issued, without
+ * blocking the host. */
+QS_API qs_status qstate_pipeline_join(qs_pipeline* pl, cudaStream_t stream);
+
+/* Block the host until every step issued so far, with its copies, is done. */
+QS_API qs_status qstate_pipeline_sync(qs_pipeline* pl);
+
+/* Synchronize, then free the pipeline's device memory, streams and events.
+ * NULL is accepted and ignored. */
+QS_API qs_status qstate_pipeline_destroy(qs_pipeline* pl);
+
 /* Readout of the stored state without changing it: o_i = d_i . q with
  * d_ij = c_ij * s_ig (no decay; the fixed dot order above). */
 QS_API qs_status qstate_readout(const qs_config* cfg, const void* codes,

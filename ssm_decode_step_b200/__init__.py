@@ -5,8 +5,8 @@ this package holds its sources (csrc/), its build step (build.py), a thin
 ctypes binding (qstate.py) and the seeded synthetic workloads
 (workloads.py).
 """
-from .qstate import (Config, QState, QStateError, decode_step, init, query_sizes, readout,
-                     status_string)
+from .qstate import (Config, HostPipeline, QState, QStateError, decode_step, init, query_sizes,
+                     readout, status_string)
 
-__all__ = ["Config", "QState", "QStateError", "decode_step", "init", "query_sizes", "readout",
-           "status_string"]
+__all__ = ["Config", "HostPipeline", "QState", "QStateError", "decode_step", "init", "query_sizes",
+           "readout", "status_string"]

@@ -55,11 +55,47 @@ static cudaError_t launch_dependent(K kernel, long long grid, int threads, size_
   return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
+// Resident CTAs per SM of `kernel` at `threads` threads and `smem` bytes of
+// dynamic shared memory on the current device, cached per (kernel, device,
+// threads, smem): the occupancy query costs more host time than a launch.
+template <typename K>
+static cudaError_t resident_ctas(K kernel, int threads, size_t smem, int* per_sm) {
+  struct Entry {
+    const void* fn;
+    int dev, threads, n;
+    size_t smem;
+  };
+  static std::mutex mu;
+  static Entry cache[64];
+  static int used = 0;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  const void* fn = reinterpret_cast<const void*>(kernel);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i) {
+      const Entry& e = cache[i];
+      if (e.fn == fn && e.dev == dev && e.threads == threads && e.smem == smem) {
+        *per_sm = e.n;
+        return cudaSuccess;
+      }
+    }
+  }
+  int n = 0;
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem);
+  if (err != cudaSuccess) return err;
+  std::lock_guard<std::mutex> lock(mu);
+  if (used < 64) cache[used++] = Entry{fn, dev, threads, n, smem};
+  *per_sm = n;
+  return cudaSuccess;
+}
+
 template <typename K>
 static cudaError_t launch_persistent(K kernel, size_t smem, const StepParams& p,
                                      cudaStream_t stream) {
   int per_sm = 0;
-  cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, smem);
+  cudaError_t err = resident_ctas(kernel, kThreads, smem, &per_sm);
   if (err != cudaSuccess) return err;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
   const long long units = static_cast<long long>(p.tiles) * p.units_per_tile;
@@ -76,7 +112,7 @@ static cudaError_t launch_persistent(K kernel, size_t smem, const StepParams& p,
 template <typename K, typename P>
 static cudaError_t launch_warps(K kernel, const P& p, size_t smem, cudaStream_t stream) {
   int per_sm = 0;
-  cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kStepThreads, smem);
+  cudaError_t err = resident_ctas(kernel, kStepThreads, smem, &per_sm);
   if (err != cudaSuccess) return err;
   if (per_sm < 1) return cudaErrorInvalidConfiguration;
   long long grid = static_cast<long long>(per_sm) * device_sm_count();

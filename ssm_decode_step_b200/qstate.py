@@ -27,6 +27,9 @@ EXPORTS = ("qstate_query_sizes", "qstate_init", "qstate_decode_step", "qstate_re
            "qstate_fp32_decode_step", "qstate_lrb_query_sizes", "qstate_lrb_decode_step",
            "qstate_prefill", "qstate_prefill_tf32", "qstate_prefill_tf32_timeouts",
            "qstate_prefill_tf32_wait_selfcheck",
+           "qstate_pipeline_query_sizes", "qstate_pipeline_create", "qstate_pipeline_step",
+           "qstate_pipeline_wait_stream", "qstate_pipeline_join", "qstate_pipeline_sync",
+           "qstate_pipeline_destroy",
            "qstate_state_sq_norms", "qstate_fp32_sq_norms",
            "qstate_selfcheck", "qstate_status_string", "qstate_version")
 
@@ -67,13 +70,22 @@ def lib() -> ctypes.CDLL:
         L.qstate_prefill_tf32.argtypes = [C, ctypes.c_int] + [P] * 8
         L.qstate_prefill_tf32_timeouts.argtypes = [P]
         L.qstate_prefill_tf32_wait_selfcheck.argtypes = [ctypes.c_uint, P]
+        L.qstate_pipeline_query_sizes.argtypes = [C, ctypes.c_int, sz, sz]
+        L.qstate_pipeline_create.argtypes = [ctypes.c_int, C, ctypes.c_int, ctypes.POINTER(P)]
+        L.qstate_pipeline_step.argtypes = [P, P, P, P, P, P, P]
+        L.qstate_pipeline_wait_stream.argtypes = [P, P]
+        L.qstate_pipeline_join.argtypes = [P, P]
+        L.qstate_pipeline_sync.argtypes = [P]
+        L.qstate_pipeline_destroy.argtypes = [P]
         L.qstate_state_sq_norms.argtypes = [C, P, P, P, P]
         L.qstate_fp32_sq_norms.argtypes = [C, P, P, P]
         for f in (L.qstate_query_sizes, L.qstate_init, L.qstate_decode_step, L.qstate_readout,
                   L.qstate_selfcheck, L.qstate_fp32_decode_step, L.qstate_state_sq_norms,
                   L.qstate_fp32_sq_norms, L.qstate_lrb_query_sizes, L.qstate_lrb_decode_step,
                   L.qstate_prefill, L.qstate_prefill_tf32, L.qstate_prefill_tf32_timeouts,
-                  L.qstate_prefill_tf32_wait_selfcheck):
+                  L.qstate_prefill_tf32_wait_selfcheck, L.qstate_pipeline_query_sizes,
+                  L.qstate_pipeline_create, L.qstate_pipeline_step, L.qstate_pipeline_wait_stream,
+                  L.qstate_pipeline_join, L.qstate_pipeline_sync, L.qstate_pipeline_destroy):
             f.restype = ctypes.c_int
         L.qstate_status_string.argtypes = [ctypes.c_int]
         L.qstate_status_string.restype = ctypes.c_char_p
@@ -297,15 +309,97 @@ class QState:
         cb, sb, hb = query_sizes(cfg)
         assert cb == self.codes.numel() and sb == 4 * self.scales.numel()
         assert hb == (0 if self.shadow is None else 4 * self.shadow.numel())
+        # the C struct of cfg, built once: step() is called once per token
+        self._cc = cfg.c()
+        self._ccp = ctypes.byref(self._cc)
 
     def init(self, S0, stream=None) -> "QState":
         init(self.cfg, S0, self.codes, self.scales, self.shadow, stream)
         return self
 
     def step(self, q, k, v, alpha, beta, o=None, stream=None):
-        decode_step(self.cfg, self.codes, self.scales, self.shadow, q, k, v, alpha, beta, o, stream)
+        _check(lib().qstate_decode_step(self._ccp, _ptr(self.codes), _ptr(self.scales),
+                                        _ptr(self.shadow), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                        _ptr(beta), _ptr(o), _stream(stream)),
+               "qstate_decode_step")
         return o
 
     def readout(self, q, o, stream=None):
         readout(self.cfg, self.codes, self.scales, q, o, stream)
         return o
+
+
+def pipeline_query_sizes(cfg: Config, n: int):
+    """(input bytes, output bytes) of one step of a host-buffer pipeline over
+    n families of cfg's recurrence."""
+    a, b = ctypes.c_size_t(), ctypes.c_size_t()
+    cc = cfg.c()
+    _check(lib().qstate_pipeline_query_sizes(ctypes.byref(cc), n, ctypes.byref(a), ctypes.byref(b)),
+           "qstate_pipeline_query_sizes")
+    return a.value, b.value
+
+
+class HostPipeline:
+    """Host-buffer decode pipeline (qstate_pipeline_*): step() takes one
+    token's packed inputs from host memory (q | k | v | alpha | beta, float32,
+    page-locked for asynchronous copies), runs the decode step of every state
+    family on `stream`, and writes the readouts [n][T][dv] back to host
+    memory; the copies run on the pipeline's own streams, `depth` steps deep.
+    A step's host buffers may be reused, or its readouts read, once sync() has
+    returned or the step `depth` calls later has been issued."""
+
+    def __init__(self, states, depth: int = 3):
+        self.cfgs = [st.cfg for st in states]
+        n = len(self.cfgs)
+        arr = (qs_config * n)(*[c.c() for c in self.cfgs])
+        h = ctypes.c_void_p()
+        _check(lib().qstate_pipeline_create(n, arr, depth, ctypes.byref(h)), "qstate_pipeline_create")
+        self._h = h
+        self.depth = depth
+        self.in_bytes, self.out_bytes = pipeline_query_sizes(self.cfgs[0], n)
+        self._default = tuple(states)
+        self._arrays = {}
+
+    def _state_arrays(self, states):
+        key = tuple(id(st) for st in states)
+        got = self._arrays.get(key)
+        if got is None:
+            if [st.cfg for st in states] != self.cfgs:
+                raise ValueError("states do not match the pipeline's families")
+            n = len(states)
+            VP = ctypes.c_void_p
+            got = (tuple(states),  # keeps the states (and their ids) alive with the entry
+                   (VP * n)(*[_ptr(st.codes) for st in states]),
+                   (VP * n)(*[_ptr(st.scales) for st in states]),
+                   (VP * n)(*[_ptr(st.shadow) for st in states]))
+            self._arrays[key] = got
+        return got
+
+    def step(self, host_in, host_out=None, stream=None, states=None):
+        if host_in.numel() * host_in.element_size() < self.in_bytes:
+            raise ValueError("host input smaller than one step's packed inputs")
+        if host_out is not None and host_out.numel() * host_out.element_size() < self.out_bytes:
+            raise ValueError("host output smaller than one step's readouts")
+        _, codes, scales, shadow = self._state_arrays(self._default if states is None else states)
+        _check(lib().qstate_pipeline_step(self._h, codes, scales, shadow, _ptr(host_in),
+                                          _ptr(host_out), _stream(stream)), "qstate_pipeline_step")
+
+    def wait_stream(self, stream=None):
+        _check(lib().qstate_pipeline_wait_stream(self._h, _stream(stream)), "qstate_pipeline_wait_stream")
+
+    def join(self, stream=None):
+        _check(lib().qstate_pipeline_join(self._h, _stream(stream)), "qstate_pipeline_join")
+
+    def sync(self):
+        _check(lib().qstate_pipeline_sync(self._h), "qstate_pipeline_sync")
+
+    def close(self):
+        if self._h is not None:
+            h, self._h = self._h, None
+            _check(lib().qstate_pipeline_destroy(h), "qstate_pipeline_destroy")
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -47,6 +47,19 @@ int main(void) {
   check(qstate_prefill_tf32_wait_selfcheck(0, &timed_out) == QS_ERR_INVALID_ARG,
         "wait self-check rejects a zero poll limit before any launch");
 
+  size_t in_b = 0, out_b = 0;
+  check(qstate_pipeline_query_sizes(&c, 3, &in_b, &out_b) == QS_OK && out_b == (size_t)3 * 1024 * 128 * 4 &&
+            in_b == (size_t)1024 * (128 + 128 + 128 + 1 + 1) * 4,
+        "pipeline sizes");
+  qs_pipeline* pl = NULL;
+  check(qstate_pipeline_create(0, &c, 3, &pl) == QS_ERR_INVALID_ARG && pl == NULL,
+        "pipeline rejects zero families before any CUDA call");
+  check(qstate_pipeline_create(1, &c, 1, &pl) == QS_ERR_INVALID_ARG,
+        "pipeline rejects a depth below 2");
+  check(qstate_pipeline_step(NULL, NULL, NULL, NULL, NULL, NULL, 0) == QS_ERR_INVALID_ARG,
+        "pipeline step rejects a NULL pipeline");
+  check(qstate_pipeline_destroy(NULL) == QS_OK, "destroying NULL is a no-op");
+
   const char* s = qstate_status_string(QS_OK);
   check(s != NULL && strlen(s) > 0, "status strings are defined");
   check(qstate_version() > 0, "version is positive");

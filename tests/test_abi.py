@@ -206,3 +206,36 @@ def test_prefill_tf32_validation():
 def test_binding_raises():
     with pytest.raises(Q.QStateError):
         Q.query_sizes(_cfg(bits=5))
+
+
+def test_pipeline_sizes_and_validation_without_a_gpu():
+    """Host-buffer pipeline: sizes of one step's packed input and readouts,
+    and every argument check that runs before a CUDA call."""
+    L = Q.lib()
+    cfg = _cfg(num_tiles=5, dv=64, decay="diagonal")
+    inb, outb = Q.pipeline_query_sizes(cfg, 2)
+    assert inb == 4 * 5 * (128 + 128 + 64 + 128 + 1)       # q, k, v, diagonal alpha, beta
+    assert outb == 2 * 4 * 5 * 64
+    inb1, _ = Q.pipeline_query_sizes(_cfg(num_tiles=5, dv=64), 1)
+    assert inb1 == 4 * 5 * (128 + 128 + 64 + 1 + 1)         # scalar alpha
+    h = ctypes.c_void_p()
+    one = (Q.qs_config * 1)(_raw(cfg))
+    assert L.qstate_pipeline_create(0, one, 3, ctypes.byref(h)) == Q.QS_ERR_INVALID_ARG
+    assert L.qstate_pipeline_create(9, one, 3, ctypes.byref(h)) == Q.QS_ERR_INVALID_ARG
+    assert L.qstate_pipeline_create(1, one, 1, ctypes.byref(h)) == Q.QS_ERR_INVALID_ARG
+    assert L.qstate_pipeline_create(1, one, 9, ctypes.byref(h)) == Q.QS_ERR_INVALID_ARG
+    assert L.qstate_pipeline_create(1, one, 3, None) == Q.QS_ERR_INVALID_ARG
+    assert h.value is None
+    # families must share the recurrence (tiles, dk, dv, delta, decay)
+    for other in (_cfg(num_tiles=6, dv=64, decay="diagonal"), _cfg(num_tiles=5, dv=80, decay="diagonal"),
+                  _cfg(num_tiles=5, dv=64, decay="scalar"), _cfg(num_tiles=5, dv=64, decay="diagonal", delta=0)):
+        two = (Q.qs_config * 2)(_raw(cfg), _raw(other))
+        assert L.qstate_pipeline_create(2, two, 3, ctypes.byref(h)) == Q.QS_ERR_INVALID_ARG
+    # an unsupported family is reported as such
+    two = (Q.qs_config * 2)(_raw(cfg), _raw(_cfg(num_tiles=5, dv=64, decay="diagonal", group=16)))
+    assert L.qstate_pipeline_create(2, two, 3, ctypes.byref(h)) == Q.QS_ERR_UNSUPPORTED
+    assert L.qstate_pipeline_step(None, None, None, None, None, None, None) == Q.QS_ERR_INVALID_ARG
+    assert L.qstate_pipeline_sync(None) == Q.QS_ERR_INVALID_ARG
+    assert L.qstate_pipeline_join(None, None) == Q.QS_ERR_INVALID_ARG
+    assert L.qstate_pipeline_wait_stream(None, None) == Q.QS_ERR_INVALID_ARG
+    assert L.qstate_pipeline_destroy(None) == Q.QS_OK
