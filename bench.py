@@ -874,15 +874,19 @@ def run_recall(args):
     print(json.dumps(out))
 
 
-def prefill_flops(dk: int, dv: int, L: int, C: int = 32) -> int:
+def prefill_flops(dk: int, dv: int, L: int, C: int = 32, delta: int = 0) -> int:
     """Algorithmic FLOPs of the chunkwise prefill of one tile over L tokens:
     per chunk of c tokens, the state read 2 c dk dv, the local scores c^2 dk
     (the causal half of 2 c^2 dk), the intra-chunk outputs c^2 dv and the
-    state pass 2 c dk dv + dk dv."""
+    state pass 2 c dk dv + dk dv; the delta rule adds the projection of the
+    keys on the state 2 c dk dv, their scores c^2 dk and the forward
+    substitution c^2 dv."""
     f = 0
     for c0 in range(0, L, C):
         c = min(C, L - c0)
         f += 4 * c * dk * dv + c * c * (dk + dv) + dk * dv
+        if delta:
+            f += 2 * c * dk * dv + c * c * (dk + dv)
     return f
 
 
@@ -893,9 +897,9 @@ def prefill_bytes(dk: int, dv: int, L: int, diag: bool) -> int:
 
 
 def run_prefill(args):
-    """Time both prefill paths over `--prefill` tokens for every tile of the
+    """Time the prefill paths over `--prefill` tokens for every tile of the
     workload (inputs drawn from its laws, slot t mod P for token t), from a
-    zero state, with outputs: qstate_prefill (FP32 on the CUDA cores, against
+    zero state, with outputs (delta-rule workloads: the FP32 path only): qstate_prefill (FP32 on the CUDA cores, against
     the FP32 FMA peak of 148 SMs x 128 lanes x 2 FLOPs x the sampled SM
     clock) and qstate_prefill_tf32 (tensor cores, against the measured HBM
     copy bandwidth: its algorithmic bytes per launch / launch time, and its
@@ -906,8 +910,6 @@ def run_prefill(args):
     w = W.get(args.workload)
     if args.prefill_tiles > 0:
         w = W.scaled_down(w, args.prefill_tiles, layers=1)
-    if w.delta != 0:
-        raise SystemExit("the chunkwise prefill covers the linear write (delta = 0) workloads")
     L, P = args.prefill, max(1, min(args.pool, args.prefill))
     dev = torch.device("cuda")
     T = w.tiles
@@ -915,7 +917,7 @@ def run_prefill(args):
     idx = np.arange(L) % P
     arrs = [np.ascontiguousarray(np.stack([s[i] for s in slots], axis=1)[:, idx]) for i in range(5)]
     q, k, v, a, b = (torch.from_numpy(x).to(dev) for x in arrs)
-    cfg = Config(T, w.dk, w.dv, 8, 32, 0, w.decay)
+    cfg = Config(T, w.dk, w.dv, 8, 32, w.delta, w.decay)
     S = torch.zeros((T, w.dv, w.dk), dtype=torch.float32, device=dev)
     o = torch.empty((T, L, w.dv), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
@@ -929,7 +931,12 @@ def run_prefill(args):
            "tokens_per_tile": L, "launches": args.steps,
            "note": "the zeroing of S before every launch is inside the timed region (one memset)"}
     before = Q.prefill_tf32_timeouts()
-    for name, fn in (("fp32", Q.prefill), ("tf32", Q.prefill_tf32)):
+    paths = [("fp32", Q.prefill)]
+    if w.delta == 0:
+        paths.append(("tf32", Q.prefill_tf32))
+    else:
+        out["tf32"] = "not run: the tensor-core form covers the linear write (delta = 0) only"
+    for name, fn in paths:
         for _ in range(args.warmup):
             fn(cfg, L, S, q, k, v, a, b, o)
         torch.cuda.synchronize()
@@ -945,7 +952,7 @@ def run_prefill(args):
         sec = e0.elapsed_time(e1) / 1e3 / args.steps
         mhz = clocks.get("sm_mhz") or 1965
         if name == "fp32":
-            flops = T * prefill_flops(w.dk, w.dv, L)
+            flops = T * prefill_flops(w.dk, w.dv, L, delta=w.delta)
             peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
             out[name] = {"kernel": "prefill_kernel (CUDA cores, FP32)", "ms_per_prefill": round(sec * 1e3, 4),
                          "tokens_per_s": round(T * L / sec, 1), "tflops": round(flops / sec / 1e12, 3),
@@ -965,7 +972,8 @@ def run_prefill(args):
                          "frac_of_tf32_peak": round(flops / sec / 1e12 / tf32_peak, 4),
                          "flops": "prefill_flops (chunks of 64)", "clocks": clocks,
                          "speedup_vs_fp32": round(out["fp32"]["ms_per_prefill"] / (sec * 1e3), 2)}
-    out["tf32"]["timeouts"] = Q.prefill_tf32_timeouts() - before
+    if w.delta == 0:
+        out["tf32"]["timeouts"] = Q.prefill_tf32_timeouts() - before
     print(json.dumps(out))
 
 

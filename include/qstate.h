@@ -283,10 +283,16 @@ QS_API qs_status qstate_lrb_decode_step(const qs_config* cfg, int rank, int slot
  * write (delta = 0) with scalar decay (the Mamba-2 family whose chunkwise
  * realization LinQuant gives: Low-Precision Chunkwise Realization, state
  * write / state pass / state read / local score / intra-chunk output) or
- * diagonal decay (the GLA family, the same contractions per channel).  It
- * computes, for every tile, the token-by-token recurrence
- *   S_t = S_{t-1} Lambda_t + beta_t v_t k_t^T,   o_t = S_t q_t
- * regrouped in chunks of 32 tokens (exact in real arithmetic; in FP32 the
+ * diagonal decay (the GLA family, the same contractions per channel), and
+ * for the delta rule (delta = 1, the DeltaNet / Gated DeltaNet family, with
+ * either decay).  It computes, for every tile, the token-by-token recurrence
+ * of qstate_decode_step on an FP32 state,
+ *   S_t = S_{t-1} Lambda_t (I - delta beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *   o_t = S_t q_t,
+ * regrouped in chunks of 32 tokens (under the delta rule the corrected
+ * values w_t = beta_t (v_t - S_{t-1} Lambda_t k_t) of a chunk solve a unit
+ * lower-triangular system, by forward substitution; exact in real
+ * arithmetic; in FP32 the
  * summation order differs from the token-by-token order, so results agree
  * with qstate_fp32_decode_step applied token by token to within FP32
  * rounding, not bit for bit).  The state it leaves is the S0 that
@@ -297,9 +303,8 @@ QS_API qs_status qstate_lrb_decode_step(const qs_config* cfg, int rank, int slot
  *   alpha  [T][length] (QS_DECAY_SCALAR) or [T][length][Dk] (diagonal), in (0, 1]
  *   beta   [T][length] float
  *   o      [T][length][Dv] float, or NULL to skip the outputs
- * Only num_tiles, dk, dv, delta and decay of cfg are used; delta must be 0
- * (the delta rule's chunkwise form is not built), dv <= 128.  Under
- * diagonal decay a chunk may decay a channel by at most e^-170. */
+ * Only num_tiles, dk, dv, delta and decay of cfg are used; dv <= 128.
+ * Under diagonal decay a chunk may decay a channel by at most e^-170. */
 QS_API qs_status qstate_prefill(const qs_config* cfg, int length, float* S, const float* q,
                                 const float* k, const float* v, const float* alpha,
                                 const float* beta, float* o, cudaStream_t stream);
@@ -313,7 +318,8 @@ QS_API qs_status qstate_prefill(const qs_config* cfg, int length, float* S, cons
  * to about 2^-10 of the magnitudes summed, not to FP32 rounding: every
  * element of S and o is within 2^-8 of the same recurrence run on |S0|,
  * |q|, |k|, |v| (the sum of the magnitudes of its terms).  Arguments,
- * validation are those of qstate_prefill, with S, q and k 16-byte aligned;
+ * validation are those of qstate_prefill, with S, q and k 16-byte aligned
+ * and the linear write only (delta = 1 returns QS_ERR_UNSUPPORTED);
  * under either decay a chunk of 64 tokens may decay a channel by at most
  * e^-170 (the decay factors are split around the chunk's middle token).  A wait for the tensor
  * cores that does not end (a bounded poll) makes the CTA free its tensor

@@ -444,7 +444,7 @@ namespace {
 // there is work to launch.
 qs_status prefill_args(const qs_config* cfg, int length, float* S, const float* q, const float* k,
                        const float* v, const float* alpha, const float* beta, float* o, uintptr_t align,
-                       qs_config* out, qs::PrefillParams* p, bool* work) {
+                       bool allow_delta, qs_config* out, qs::PrefillParams* p, bool* work) {
   *work = false;
   if (cfg == nullptr) return QS_ERR_INVALID_ARG;
   qs_config c = *cfg;
@@ -454,7 +454,7 @@ qs_status prefill_args(const qs_config* cfg, int length, float* S, const float* 
   c.rounding = QS_ROUND_NEAREST;
   qs_status st = check_config(&c);
   if (st != QS_OK) return st;
-  if (c.delta != 0 || c.dv > 128) return QS_ERR_UNSUPPORTED;
+  if ((c.delta != 0 && !allow_delta) || c.dv > 128) return QS_ERR_UNSUPPORTED;
   if (length < 0) return QS_ERR_INVALID_ARG;
   if (c.num_tiles == 0 || length == 0) return QS_OK;
   const bool diag = c.decay == QS_DECAY_DIAGONAL;
@@ -491,14 +491,21 @@ qs_status qstate_prefill(const qs_config* cfg, int length, float* S, const float
   qs_config c;
   qs::PrefillParams p;
   bool work;
-  const qs_status st = prefill_args(cfg, length, S, q, k, v, alpha, beta, o, 4, &c, &p, &work);
+  const qs_status st = prefill_args(cfg, length, S, q, k, v, alpha, beta, o, 4, true, &c, &p, &work);
   if (st != QS_OK || !work) return st;
-  const bool diag = c.decay == QS_DECAY_DIAGONAL;
+  const int sel = (c.dk == 128 ? 4 : 0) + (c.decay == QS_DECAY_DIAGONAL ? 2 : 0) + (c.delta ? 1 : 0);
+  const int T = c.num_tiles;
   cudaError_t e;
-  if (c.dk == 64)
-    e = diag ? qs::launch_prefill<64, true>(p, c.num_tiles, stream) : qs::launch_prefill<64, false>(p, c.num_tiles, stream);
-  else
-    e = diag ? qs::launch_prefill<128, true>(p, c.num_tiles, stream) : qs::launch_prefill<128, false>(p, c.num_tiles, stream);
+  switch (sel) {
+    case 0: e = qs::launch_prefill<64, false, false>(p, T, stream); break;
+    case 1: e = qs::launch_prefill<64, false, true>(p, T, stream); break;
+    case 2: e = qs::launch_prefill<64, true, false>(p, T, stream); break;
+    case 3: e = qs::launch_prefill<64, true, true>(p, T, stream); break;
+    case 4: e = qs::launch_prefill<128, false, false>(p, T, stream); break;
+    case 5: e = qs::launch_prefill<128, false, true>(p, T, stream); break;
+    case 6: e = qs::launch_prefill<128, true, false>(p, T, stream); break;
+    default: e = qs::launch_prefill<128, true, true>(p, T, stream); break;
+  }
   return from_cuda(e);
 }
 
@@ -511,7 +518,8 @@ qs_status qstate_prefill_tf32(const qs_config* cfg, int length, float* S, const 
   qs_config c;
   qs::PrefillParams p;
   bool work;
-  const qs_status st = prefill_args(cfg, length, S, q, k, v, alpha, beta, o, 16, &c, &p, &work);
+  // the delta rule runs on the FP32 path only
+  const qs_status st = prefill_args(cfg, length, S, q, k, v, alpha, beta, o, 16, false, &c, &p, &work);
   if (st != QS_OK || !work) return st;
   unsigned int* timeouts = nullptr;
   cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&timeouts), qs_tc_timeouts);

@@ -28,8 +28,8 @@ template <int BITS, int DK>
 cudaError_t launch_init(const float* S0, uint8_t* codes, float* scales, float* shadow,
                         long long rows, int group, cudaStream_t stream);
 
-// Chunkwise prefill (delta = 0) of `tiles` tiles.
-template <int DK, bool DIAG>
+// Chunkwise prefill (linear write or delta rule) of `tiles` tiles.
+template <int DK, bool DIAG, bool DELTA>
 cudaError_t launch_prefill(const PrefillParams& p, int tiles, cudaStream_t stream);
 
 // Chunkwise prefill on the tensor cores (TF32 operands, FP32 accumulators);

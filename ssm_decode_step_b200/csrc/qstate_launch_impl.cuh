@@ -168,13 +168,13 @@ cudaError_t launch_lrb(const LrbParams& p0, int tiles, int dv, cudaStream_t stre
   return launch_warps(kernel, p, static_cast<size_t>(p.warp_bytes) * WARPS, stream);
 }
 
-template <int DK, bool DIAG>
+template <int DK, bool DIAG, bool DELTA>
 cudaError_t launch_prefill(const PrefillParams& p, int tiles, cudaStream_t stream) {
-  auto kernel = prefill_kernel<DK, DIAG>;
+  auto kernel = prefill_kernel<DK, DIAG, DELTA>;
   static std::once_flag flag;
   cudaError_t err = allow_smem(kernel, flag);
   if (err != cudaSuccess) return err;
-  const PrefillLayout L(DK, p.dv, DIAG);
+  const PrefillLayout L(DK, p.dv, DIAG, DELTA);
   kernel<<<tiles, kPrefillThreads, static_cast<size_t>(L.total) * sizeof(float), stream>>>(p);
   return cudaGetLastError();
 }
@@ -254,8 +254,10 @@ cudaError_t launch_init(const float* S0, uint8_t* codes, float* scales, float* s
   template cudaError_t launch_prefill_tc<D, M, DI>(const PrefillParams&, int, unsigned int*, cudaStream_t);
 
 #define QS_INSTANTIATE_PREFILL(D)                                                   \
-  template cudaError_t launch_prefill<D, false>(const PrefillParams&, int, cudaStream_t); \
-  template cudaError_t launch_prefill<D, true>(const PrefillParams&, int, cudaStream_t);  \
+  template cudaError_t launch_prefill<D, false, false>(const PrefillParams&, int, cudaStream_t); \
+  template cudaError_t launch_prefill<D, true, false>(const PrefillParams&, int, cudaStream_t);  \
+  template cudaError_t launch_prefill<D, false, true>(const PrefillParams&, int, cudaStream_t);  \
+  template cudaError_t launch_prefill<D, true, true>(const PrefillParams&, int, cudaStream_t);   \
   QS_INSTANTIATE_PREFILL_TC(D, 64, false) QS_INSTANTIATE_PREFILL_TC(D, 64, true)          \
   QS_INSTANTIATE_PREFILL_TC(D, 128, false) QS_INSTANTIATE_PREFILL_TC(D, 128, true)
 

@@ -1,9 +1,9 @@
-// Chunkwise prefill of the linear-write recurrence (delta = 0) on an FP32
-// state: qstate_prefill.  The state S_0 that the quantized decode path then
-// starts from (LinQuant, Low-Precision Chunkwise Realization, for the
-// Mamba-2 family: state write, state pass, state read, local score,
-// intra-chunk output; here in FP32, with the diagonal decay of the GLA
-// family as the per-channel extension).
+// Chunkwise prefill on an FP32 state: qstate_prefill.  The state S_0 that
+// the quantized decode path then starts from (LinQuant, Low-Precision
+// Chunkwise Realization, for the Mamba-2 family: state write, state pass,
+// state read, local score, intra-chunk output; here in FP32, with the
+// diagonal decay of the GLA family as the per-channel extension, and the
+// delta-rule write of the DeltaNet family, LinQuant's "delta-rule updates").
 //
 // Per tile, tokens are taken in chunks of C = 32.  With Lam_t the running
 // sum of log(alpha) over the chunk's tokens up to t (per channel for
@@ -17,6 +17,18 @@
 // factor is split around the chunk's middle token m as
 // (q_t e^{Lam_t - Lam_m}) . (k_s e^{Lam_m - Lam_s}), which stays in range
 // while a chunk decays any channel by less than e^{-170}.
+//
+// Delta rule (delta = 1).  The recurrence
+// S_t = S_{t-1} Lambda_t (I - beta_t k_t k_t^T) + beta_t v_t k_t^T is the
+// linear write S_t = S_{t-1} Lambda_t + w_t k_t^T with the corrected value
+//   w_t = beta_t (v_t - S_{t-1} Lambda_t k_t),
+// and unrolling S_{t-1} over the chunk gives
+//   w_t = beta_t (v_t - S (k_t * e^{Lam_t})) - sum_{s < t} B_ts w_s,
+//   B_ts = beta_t sum_j k_tj k_sj e^{Lam_tj - Lam_sj},
+// a unit lower-triangular system, solved by forward substitution (tokens in
+// order, s ascending); w then takes the place of beta_s v_s in the output
+// and the state pass (A without beta).  B is split around the middle token
+// like A.
 //
 // One CTA per tile, 256 threads; the state stays in shared memory (rows
 // padded to Dk + 1 floats) for the whole sequence.  Only the state pass is
@@ -46,8 +58,8 @@ struct PrefillParams {
 
 // Shared-memory layout (floats) of one CTA.
 struct PrefillLayout {
-  int S, qbar, kbar, qt, kh, v, lam, A, beta, elam, total;
-  __host__ __device__ PrefillLayout(int dk, int dv, bool diag) {
+  int S, qbar, kbar, qt, kh, kq, v, lam, A, B, beta, elam, total;
+  __host__ __device__ PrefillLayout(int dk, int dv, bool diag, bool delta = false) {
     constexpr int C = kPrefillChunk;
     int off = 0;
     S = off;    off += dv * (dk + 1);
@@ -55,30 +67,35 @@ struct PrefillLayout {
     kbar = off; off += C * dk;           // [s][j]: k_s * e^{Lam_C - Lam_s}
     qt = off;   off += C * (dk + 4);     // [t][j]: q_t (* e^{Lam_t - Lam_m} when diagonal)
     kh = off;   off += C * (dk + 4);     // [s][j]: k_s (* e^{Lam_m - Lam_s} when diagonal)
-    v = off;    off += C * dv;           // [s][i]
+    // delta rule, diagonal decay: [t][j] k_t * e^{Lam_t - Lam_m} (scalar decay uses kh)
+    kq = off;   off += (delta && diag) ? C * (dk + 4) : 0;
+    v = off;    off += C * dv;           // [s][i]: v, then w under the delta rule
     lam = off;  off += diag ? C * dk : C;  // [t][j] or [t]
-    A = off;    off += C * C;            // [t][s], beta_s folded in
+    A = off;    off += C * C;            // [t][s], beta_s folded in (linear write only)
+    B = off;    off += delta ? C * C : 0;  // [t][s], s < t: the delta rule's triangular system
     beta = off; off += C;
     elam = off; off += diag ? dk : 1;    // e^{Lam_C} per channel
     total = off;
   }
 };
 
-template <int DK, bool DIAG>
-__global__ void __launch_bounds__(kPrefillThreads, 2) prefill_kernel(PrefillParams p) {
+template <int DK, bool DIAG, bool DELTA>
+__global__ void __launch_bounds__(kPrefillThreads, DELTA ? 1 : 2) prefill_kernel(PrefillParams p) {
   constexpr int C = kPrefillChunk;
   constexpr int NT = kPrefillThreads;
   extern __shared__ __align__(16) float sm[];
   const int dv = p.dv;
-  const PrefillLayout Ly(DK, dv, DIAG);
+  const PrefillLayout Ly(DK, dv, DIAG, DELTA);
   float* S = sm + Ly.S;
   float* qbar = sm + Ly.qbar;
   float* kbar = sm + Ly.kbar;
   float* qt = sm + Ly.qt;
   float* kh = sm + Ly.kh;
+  float* kq = DIAG ? sm + Ly.kq : kh;
   float* V = sm + Ly.v;
   float* lam = sm + Ly.lam;
   float* A = sm + Ly.A;
+  float* Bm = sm + Ly.B;
   float* bt = sm + Ly.beta;
   float* elam = sm + Ly.elam;
   const int tid = threadIdx.x;
@@ -131,15 +148,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 2) prefill_kernel(PrefillPara
       const bool live = t < Ce;
       const float qv = live ? p.q[(tok0 + t) * DK + j] : 0.0f;
       const float kv = live ? p.k[(tok0 + t) * DK + j] : 0.0f;
+      // under the delta rule qbar first holds k_t * e^{Lam_t} (the projection
+      // S k of the corrected values); q_t * e^{Lam_t} replaces it after the solve
+      const float xv = DELTA ? kv : qv;
       if constexpr (DIAG) {
         const float lt = lam[t * DK + j], lC = lam[(C - 1) * DK + j], lm = lam[m * DK + j];
-        qbar[j * C + t] = qv * expf(lt);
+        qbar[j * C + t] = xv * expf(lt);
         kbar[t * DK + j] = kv * expf(lC - lt);
         qt[t * QP + j] = qv * expf(lt - lm);
         kh[t * QP + j] = kv * expf(lm - lt);
+        if constexpr (DELTA) kq[t * QP + j] = kv * expf(lt - lm);
       } else {
         const float lt = lam[t], lC = lam[C - 1];
-        qbar[j * C + t] = qv * expf(lt);
+        qbar[j * C + t] = xv * expf(lt);
         kbar[t * DK + j] = kv * expf(lC - lt);
         qt[t * QP + j] = qv;
         kh[t * QP + j] = kv;
@@ -152,6 +173,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 2) prefill_kernel(PrefillPara
       const int lane = tid & 31, w = tid >> 5;
       const int s = lane;
       float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      float bcc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
       const float4* kr = reinterpret_cast<const float4*>(kh + s * QP);
       for (int j4 = 0; j4 < DK / 4; ++j4) {
         const float4 kv = kr[j4];
@@ -162,21 +184,71 @@ __global__ void __launch_bounds__(kPrefillThreads, 2) prefill_kernel(PrefillPara
           acc[u] = fmaf(qv.y, kv.y, acc[u]);
           acc[u] = fmaf(qv.z, kv.z, acc[u]);
           acc[u] = fmaf(qv.w, kv.w, acc[u]);
+          if constexpr (DELTA) {
+            const float4 kt = reinterpret_cast<const float4*>(kq + (4 * w + u) * QP)[j4];
+            bcc[u] = fmaf(kt.x, kv.x, bcc[u]);
+            bcc[u] = fmaf(kt.y, kv.y, bcc[u]);
+            bcc[u] = fmaf(kt.z, kv.z, bcc[u]);
+            bcc[u] = fmaf(kt.w, kv.w, bcc[u]);
+          }
         }
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int t = 4 * w + u;
+        const float f = (!DIAG && s <= t && t < Ce) ? expf(lam[t] - lam[s]) : 1.0f;
         float a = 0.0f;
         if (s <= t && t < Ce) {
-          a = acc[u];
-          if constexpr (!DIAG) a *= expf(lam[t] - lam[s]);
-          a *= bt[s];
+          a = acc[u] * f;
+          if constexpr (!DELTA) a *= bt[s];
         }
         A[t * C + s] = a;
+        if constexpr (DELTA) Bm[t * C + s] = (s < t && t < Ce) ? bt[t] * (bcc[u] * f) : 0.0f;
       }
     }
     __syncthreads();
+    if constexpr (DELTA) {
+      // ---- r_t = beta_t (v_t - S (k_t e^{Lam_t})), in place of v (8 tokens per thread)
+      for (int e = tid; e < dv * (C / 8); e += NT) {
+        const int i = e % dv, tg = e / dv;
+        float acc[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc[u] = 0.0f;
+        const float* srow = S + i * SP;
+        for (int j = 0; j < DK; ++j) {
+          const float sv = srow[j];
+          const float4 a0 = *reinterpret_cast<const float4*>(qbar + j * C + 8 * tg);
+          const float4 a1 = *reinterpret_cast<const float4*>(qbar + j * C + 8 * tg + 4);
+          acc[0] = fmaf(sv, a0.x, acc[0]); acc[1] = fmaf(sv, a0.y, acc[1]);
+          acc[2] = fmaf(sv, a0.z, acc[2]); acc[3] = fmaf(sv, a0.w, acc[3]);
+          acc[4] = fmaf(sv, a1.x, acc[4]); acc[5] = fmaf(sv, a1.y, acc[5]);
+          acc[6] = fmaf(sv, a1.z, acc[6]); acc[7] = fmaf(sv, a1.w, acc[7]);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int t = 8 * tg + u;
+          V[t * dv + i] = bt[t] * (V[t * dv + i] - acc[u]);
+        }
+      }
+      __syncthreads();
+      // ---- forward substitution: w_t = r_t - sum_{s < t} B_ts w_s (s ascending)
+      for (int i = tid; i < dv; i += NT) {
+        for (int t = 1; t < Ce; ++t) {
+          float acc = V[t * dv + i];
+          for (int s2 = 0; s2 < t; ++s2) acc = fmaf(-Bm[t * C + s2], V[s2 * dv + i], acc);
+          V[t * dv + i] = acc;
+        }
+      }
+      // ---- qbar = q_t e^{Lam_t} for the state read of the outputs
+      if (p.o != nullptr) {
+        for (int e = tid; e < C * DK; e += NT) {
+          const int t = e / DK, j = e % DK;
+          const float qv = t < Ce ? p.q[(tok0 + t) * DK + j] : 0.0f;
+          qbar[j * C + t] = qv * expf(DIAG ? lam[t * DK + j] : lam[t]);
+        }
+      }
+      __syncthreads();
+    }
     // ---- outputs: state read + intra-chunk output
     if (p.o != nullptr) {
       for (int e = tid; e < dv * (C / 8); e += NT) {
@@ -217,7 +289,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 2) prefill_kernel(PrefillPara
 #pragma unroll
         for (int u = 0; u < JW; ++u) acc[u] = srow[u] * elam[DIAG ? jb + u : 0];
         for (int s = 0; s < Ce; ++s) {
-          const float w = bt[s] * V[s * dv + i];
+          const float w = DELTA ? V[s * dv + i] : bt[s] * V[s * dv + i];
           const float4* kr = reinterpret_cast<const float4*>(kbar + s * DK + jb);
 #pragma unroll
           for (int u4 = 0; u4 < JW / 4; ++u4) {

@@ -170,12 +170,14 @@ def test_prefill_validation():
     pre = lambda cfg, L, **kw: lib.qstate_prefill(ctypes.byref(cfg.c()), L, kw.get("S", A), kw.get("q", 2 * A),
                                                   kw.get("k", 3 * A), kw.get("v", 4 * A), kw.get("a", 5 * A),
                                                   kw.get("b", 6 * A), kw.get("o", 7 * A), None)
-    assert pre(_cfg(delta=1), 8) == Q.QS_ERR_UNSUPPORTED
     assert pre(_cfg(delta=0, dv=256), 8) == Q.QS_ERR_UNSUPPORTED
-    assert pre(_cfg(delta=0), -1) == Q.QS_ERR_INVALID_ARG
-    assert pre(_cfg(delta=0), 8, S=None) == Q.QS_ERR_INVALID_ARG
-    assert pre(_cfg(delta=0), 8, o=A + 64) == Q.QS_ERR_INVALID_ARG
-    assert pre(_cfg(delta=0), 0, S=None) == Q.QS_OK
+    assert pre(_cfg(delta=1, dv=256), 8) == Q.QS_ERR_UNSUPPORTED
+    for d in (0, 1):  # the FP32 path takes the linear write and the delta rule
+        assert pre(_cfg(delta=d), -1) == Q.QS_ERR_INVALID_ARG
+        assert pre(_cfg(delta=d), 8, S=None) == Q.QS_ERR_INVALID_ARG
+        assert pre(_cfg(delta=d), 8, o=A + 64) == Q.QS_ERR_INVALID_ARG
+        assert pre(_cfg(delta=d), 0, S=None) == Q.QS_OK
+    assert pre(_cfg(delta=2), 8) == Q.QS_ERR_INVALID_ARG
 
 
 def test_prefill_tf32_validation():
@@ -186,6 +188,7 @@ def test_prefill_tf32_validation():
         ctypes.byref(cfg.c()), L, kw.get("S", A), kw.get("q", 2 * A), kw.get("k", 3 * A),
         kw.get("v", 4 * A), kw.get("a", 5 * A), kw.get("b", 6 * A), kw.get("o", 7 * A), None)
     assert pre(_cfg(delta=1), 8) == Q.QS_ERR_UNSUPPORTED
+    assert pre(_cfg(delta=1), 0, S=None) == Q.QS_ERR_UNSUPPORTED
     assert pre(_cfg(delta=0, dv=256), 8) == Q.QS_ERR_UNSUPPORTED
     assert pre(_cfg(delta=0), -1) == Q.QS_ERR_INVALID_ARG
     assert pre(_cfg(delta=0), 8, S=None) == Q.QS_ERR_INVALID_ARG

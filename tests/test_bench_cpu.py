@@ -73,3 +73,15 @@ def test_reference_arm_contract():
     e2e = line["e2e"]
     assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_prefill_flops_of_the_delta_rule():
+    """The delta rule adds, per chunk of c tokens, the keys' projection on the
+    state (2 c dk dv), their scores (c^2 dk) and the forward substitution
+    (c^2 dv) to the linear write's count."""
+    for dk, dv, L in ((128, 128, 256), (64, 48, 33), (128, 64, 1)):
+        extra = sum(2 * c * dk * dv + c * c * (dk + dv)
+                    for c in (min(32, L - c0) for c0 in range(0, L, 32)))
+        assert bench.prefill_flops(dk, dv, L, delta=1) - bench.prefill_flops(dk, dv, L) == extra
+    # one full chunk of the linear write, term by term
+    assert bench.prefill_flops(128, 64, 32) == 4 * 32 * 128 * 64 + 32 * 32 * (128 + 64) + 128 * 64

@@ -1,11 +1,14 @@
-"""GPU checks of the chunkwise prefill (qstate_prefill and its tensor-core
-form qstate_prefill_tf32, delta = 0) against the oracle's token-by-token FP32
-recurrence (qo_fp32_step per token).
+"""GPU checks of the chunkwise prefill (qstate_prefill, linear write and
+delta rule, and its tensor-core form qstate_prefill_tf32, linear write)
+against the oracle's token-by-token FP32 recurrence (qo_fp32_step per token).
 
 The chunkwise form regroups the same sums, so the two agree to FP32 rounding
 rather than bit for bit.  Tolerance: every state element within 1e-4 of the
 tile's largest state magnitude and every output within 1e-4 of the token's
-largest output magnitude.  Derivation: a reordered FP32 sum of n terms is
+largest output magnitude (the delta rule too: its chunk solve is a forward
+substitution with unit diagonal and off-diagonal terms beta_t e^{...} k_t.k_s
+of magnitude at most one here, and the recurrence it reproduces contracts,
+so errors do not grow from chunk to chunk).  Derivation: a reordered FP32 sum of n terms is
 within about n * 2^-24 of the sum of their magnitudes; per chunk n is at most
 dk + 32 = 160 (1e-5), cancellation makes the error relative to the largest
 result a few times that, and the decay factors come from exp of running log
@@ -58,8 +61,8 @@ def _inputs(rng, T, L, dk, dv, decay):
     return q, k, v, a, b
 
 
-def _reference(T, dk, dv, decay, S0, q, k, v, a, b):
-    cfg = O.OracleConfig(T, dk, dv, 8, 32, 0, decay, "persistent")
+def _reference(T, dk, dv, decay, S0, q, k, v, a, b, delta=0):
+    cfg = O.OracleConfig(T, dk, dv, 8, 32, delta, decay, "persistent")
     S = S0.copy()
     o = np.empty((T, q.shape[1], dv), np.float32)
     for t in range(q.shape[1]):
@@ -107,6 +110,56 @@ def test_prefill_on_workload_laws(wname):
     S0 = np.zeros((T, w.dv, w.dk), np.float32)
     S_ref, o_ref = _reference(T, w.dk, w.dv, w.decay, S0, q, k, v, a, b)
     cfg = Config(T, w.dk, w.dv, 8, 32, 0, w.decay)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    S = dev(S0)
+    o = torch.empty((T, L, w.dv), dtype=torch.float32, device="cuda")
+    Q.prefill(cfg, L, S, dev(q), dev(k), dev(v), dev(a), dev(b), o)
+    _check(S.cpu().numpy(), S_ref, o.cpu().numpy(), o_ref)
+
+
+# (dk, dv, decay, tiles, length, with_o) for the delta rule
+DELTA_CASES = [
+    (128, 128, "scalar", 9, 100, True),
+    (128, 64, "diagonal", 5, 77, True),
+    (64, 48, "scalar", 4, 33, True),
+    (64, 16, "diagonal", 3, 1, True),
+    (128, 32, "scalar", 3, 64, False),
+    (64, 64, "diagonal", 2, 257, True),
+]
+
+
+@pytest.mark.parametrize("case", DELTA_CASES, ids=_id)
+def test_prefill_delta_rule_matches_token_by_token(case):
+    import torch
+    from ssm_decode_step_b200 import qstate as Q
+    dk, dv, decay, T, L, with_o = case
+    rng = np.random.default_rng(3 * dk + dv + T + L)
+    S0 = (rng.standard_normal((T, dv, dk)) * 0.1).astype(np.float32)
+    q, k, v, a, b = _inputs(rng, T, L, dk, dv, decay)
+    S_ref, o_ref = _reference(T, dk, dv, decay, S0, q, k, v, a, b, delta=1)
+    cfg = Config(T, dk, dv, 8, 32, 1, decay)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    S = dev(S0)
+    o = torch.empty((T, L, dv), dtype=torch.float32, device="cuda") if with_o else None
+    Q.prefill(cfg, L, S, dev(q), dev(k), dev(v), dev(a), dev(b), o)
+    _check(S.cpu().numpy(), S_ref, None if o is None else o.cpu().numpy(), o_ref)
+
+
+def test_prefill_delta_rule_on_gated_deltanet_laws():
+    """The Gated DeltaNet-shaped law (unit-norm keys, alpha = sigmoid(N(3,1)),
+    beta = sigmoid(N(0,1)); 64 tiles, 256 tokens from a zero state): the S_0
+    its quantized decode starts from, prefilled instead of warmed up token by
+    token."""
+    import torch
+    from ssm_decode_step_b200 import qstate as Q
+    w = W.scaled_down(W.get("gdn"), 64)
+    assert w.delta == 1
+    T, L = w.tiles, 256
+    slots = [W.slot(w, t) for t in range(L)]
+    q, k, v, a, b = (np.ascontiguousarray(np.stack([s[i] for s in slots], axis=1)) for i in range(5))
+    S0 = np.zeros((T, w.dv, w.dk), np.float32)
+    S_ref, o_ref = _reference(T, w.dk, w.dv, w.decay, S0, q, k, v, a, b, delta=1)
+    cfg = Config(T, w.dk, w.dv, 8, 32, 1, w.decay)
     dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
     S = dev(S0)
     o = torch.empty((T, L, w.dv), dtype=torch.float32, device="cuda")
