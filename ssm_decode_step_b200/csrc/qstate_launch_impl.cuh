@@ -168,14 +168,28 @@ cudaError_t launch_lrb(const LrbParams& p0, int tiles, int dv, cudaStream_t stre
   return launch_warps(kernel, p, static_cast<size_t>(p.warp_bytes) * WARPS, stream);
 }
 
+#ifndef QS_PREFILL_WIDE
+#define QS_PREFILL_WIDE 1
+#endif
+
 template <int DK, bool DIAG, bool DELTA>
 cudaError_t launch_prefill(const PrefillParams& p, int tiles, cudaStream_t stream) {
-  auto kernel = prefill_kernel<DK, DIAG, DELTA>;
-  static std::once_flag flag;
-  cudaError_t err = allow_smem(kernel, flag);
+  auto narrow = prefill_kernel<DK, DIAG, DELTA, kPrefillThreads>;
+  auto wide = prefill_kernel<DK, DIAG, DELTA, kPrefillThreadsWide>;
+  static std::once_flag f1, f2;
+  cudaError_t err = allow_smem(narrow, f1);
+  if (err == cudaSuccess) err = allow_smem(wide, f2);
   if (err != cudaSuccess) return err;
   const PrefillLayout L(DK, p.dv, DIAG, DELTA);
-  kernel<<<tiles, kPrefillThreads, static_cast<size_t>(L.total) * sizeof(float), stream>>>(p);
+  const size_t smem = static_cast<size_t>(L.total) * sizeof(float);
+  // 16 warps in one CTA where two CTAs of 8 warps do not fit on an SM
+  int per_sm = 0;
+  err = resident_ctas(narrow, kPrefillThreads, smem, &per_sm);
+  if (err != cudaSuccess) return err;
+  if (QS_PREFILL_WIDE && per_sm < 2)
+    wide<<<tiles, kPrefillThreadsWide, smem, stream>>>(p);
+  else
+    narrow<<<tiles, kPrefillThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -41,7 +41,10 @@
 namespace qs {
 
 constexpr int kPrefillChunk = 32;
+// Threads per CTA: 256 where two CTAs fit on an SM, 512 (one CTA) where the
+// state and the chunk buffers take more than half of the shared memory.
 constexpr int kPrefillThreads = 256;
+constexpr int kPrefillThreadsWide = 512;
 
 struct PrefillParams {
   float* S;            // [T][dv][dk], in: initial state, out: state after the L tokens
@@ -79,10 +82,10 @@ struct PrefillLayout {
   }
 };
 
-template <int DK, bool DIAG, bool DELTA>
-__global__ void __launch_bounds__(kPrefillThreads, DELTA ? 1 : 2) prefill_kernel(PrefillParams p) {
+template <int DK, bool DIAG, bool DELTA, int NT>
+__global__ void __launch_bounds__(NT, NT == kPrefillThreads ? 2 : 1) prefill_kernel(PrefillParams p) {
   constexpr int C = kPrefillChunk;
-  constexpr int NT = kPrefillThreads;
+  constexpr int TPW = C * 32 / NT;  // tokens per warp in the local scores
   extern __shared__ __align__(16) float sm[];
   const int dv = p.dv;
   const PrefillLayout Ly(DK, dv, DIAG, DELTA);
@@ -102,7 +105,7 @@ __global__ void __launch_bounds__(kPrefillThreads, DELTA ? 1 : 2) prefill_kernel
   const size_t tile = blockIdx.x;
   constexpr int SP = DK + 1;  // padded state row
   constexpr int QP = DK + 4;  // padded q / k row (16-byte aligned, no bank conflicts)
-  static_assert(kPrefillThreads == 8 * 32 && kPrefillChunk == 32, "8 warps x 4 tokens, 32 keys");
+  static_assert((NT == 256 || NT == 512) && C == 32, "8 or 16 warps, 32 keys");
 
   float* Sg = p.S + tile * dv * DK;
   for (int e = tid; e < dv * DK; e += NT) S[(e / DK) * SP + (e % DK)] = Sg[e];
@@ -168,7 +171,7 @@ __global__ void __launch_bounds__(kPrefillThreads, DELTA ? 1 : 2) prefill_kernel
     }
     __syncthreads();
     // ---- local scores A_ts (s <= t), beta_s folded in: warp w takes tokens
-    // t = 4w .. 4w+3, lane s one key; float4 steps along Dk
+    // t = TPW w .. TPW w + TPW - 1, lane s one key; float4 steps along Dk
     {
       const int lane = tid & 31, w = tid >> 5;
       const int s = lane;
@@ -178,14 +181,14 @@ __global__ void __launch_bounds__(kPrefillThreads, DELTA ? 1 : 2) prefill_kernel
       for (int j4 = 0; j4 < DK / 4; ++j4) {
         const float4 kv = kr[j4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float4 qv = reinterpret_cast<const float4*>(qt + (4 * w + u) * QP)[j4];
+        for (int u = 0; u < TPW; ++u) {
+          const float4 qv = reinterpret_cast<const float4*>(qt + (TPW * w + u) * QP)[j4];
           acc[u] = fmaf(qv.x, kv.x, acc[u]);
           acc[u] = fmaf(qv.y, kv.y, acc[u]);
           acc[u] = fmaf(qv.z, kv.z, acc[u]);
           acc[u] = fmaf(qv.w, kv.w, acc[u]);
           if constexpr (DELTA) {
-            const float4 kt = reinterpret_cast<const float4*>(kq + (4 * w + u) * QP)[j4];
+            const float4 kt = reinterpret_cast<const float4*>(kq + (TPW * w + u) * QP)[j4];
             bcc[u] = fmaf(kt.x, kv.x, bcc[u]);
             bcc[u] = fmaf(kt.y, kv.y, bcc[u]);
             bcc[u] = fmaf(kt.z, kv.z, bcc[u]);
@@ -194,8 +197,8 @@ __global__ void __launch_bounds__(kPrefillThreads, DELTA ? 1 : 2) prefill_kernel
         }
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int t = 4 * w + u;
+      for (int u = 0; u < TPW; ++u) {
+        const int t = TPW * w + u;
         const float f = (!DIAG && s <= t && t < Ce) ? expf(lam[t] - lam[s]) : 1.0f;
         float a = 0.0f;
         if (s <= t && t < Ce) {
