@@ -9,6 +9,7 @@
 #include "../../include/qstate.h"
 #include "qstate_fp32.cuh"
 #include "qstate_launch.h"
+#include "qstate_launch_prefill.h"
 #include "qstate_norms.cuh"
 
 namespace qs {

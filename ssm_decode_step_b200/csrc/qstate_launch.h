@@ -9,8 +9,6 @@
 #include "qstate_kernels.cuh"
 #include "qstate_step.cuh"
 #include "qstate_lrb.cuh"
-#include "qstate_prefill.cuh"
-#include "qstate_prefill_tc.cuh"
 
 namespace qs {
 
@@ -27,17 +25,6 @@ cudaError_t launch_lrb(const LrbParams& p, int tiles, int dv, cudaStream_t strea
 template <int BITS, int DK>
 cudaError_t launch_init(const float* S0, uint8_t* codes, float* scales, float* shadow,
                         long long rows, int group, cudaStream_t stream);
-
-// Chunkwise prefill (linear write or delta rule) of `tiles` tiles.
-template <int DK, bool DIAG, bool DELTA>
-cudaError_t launch_prefill(const PrefillParams& p, int tiles, cudaStream_t stream);
-
-// Chunkwise prefill on the tensor cores (TF32 operands, FP32 accumulators);
-// MDV = 64 or 128 accumulator rows (dv <= MDV); timeouts counts CTAs whose
-// bounded wait for the tensor cores gave up.
-template <int DK, int MDV, bool DIAG>
-cudaError_t launch_prefill_tc(const PrefillParams& p, int tiles, unsigned int* timeouts,
-                              cudaStream_t stream);
 
 // Streaming multiprocessors of the current device (queried once per device).
 int device_sm_count();

@@ -253,3 +253,39 @@ def test_many_tiles_sampled():
     tiles[-1] = T - 1
     rep = P.lockstep(cfg, S0, steps, tiles=tiles, label="300k tiles")
     assert rep.code_flips == 0
+
+
+@pytest.mark.parametrize("policy,bits,dv", [("dynamic", 4, 128), ("yoked", 4, 64), ("persistent", 8, 96)])
+def test_back_to_back_steps_on_one_state(policy, bits, dv):
+    """Steps on the same state launched one right after the other, with every
+    input already on the device and nothing else in the stream between them:
+    each launch may be scheduled while the previous one finishes
+    (programmatic dependent launch) and must still read the state that
+    launch wrote.  Free run against the oracle, every step's readout and the
+    final state."""
+    import torch
+    from ssm_decode_step_b200 import QState
+    rng = np.random.default_rng(23 + dv)
+    T, dk, n = 300, 128, 24
+    cfg = Config(T, dk, dv, bits, 32, 1, "scalar", policy, "nearest")
+    S0 = (rng.standard_normal((T, dv, dk)) / np.sqrt(dk)).astype(np.float32)
+    steps = P.random_steps(rng, T, dk, dv, "scalar", n)
+    dev = torch.device("cuda")
+    stack = [torch.from_numpy(np.ascontiguousarray(np.stack([s[i] for s in steps]))).to(dev)
+             for i in range(5)]
+    st = QState(cfg, dev).init(torch.from_numpy(S0).to(dev))
+    o = torch.empty((n, T, dv), dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+    for t in range(n):
+        st.step(stack[0][t], stack[1][t], stack[2][t], stack[3][t], stack[4][t], o[t])
+    torch.cuda.synchronize()
+    ora = O.init(P.oracle_cfg(cfg), S0)
+    o_gpu = o.cpu().numpy()
+    for t, (q, k, v, a, b) in enumerate(steps):
+        o_ref = O.step(ora, q, k, v, a, b)
+        P.compare_readout(o_gpu[t], o_ref, f"back-to-back {policy} step {t}")
+    rep = P.compare_state(cfg, st.codes.cpu().numpy(), st.scales.cpu().numpy(), ora, None,
+                          f"back-to-back {policy} final state")
+    assert rep.code_flips == 0
+    if st.shadow is not None:
+        assert np.array_equal(st.shadow.cpu().numpy(), ora.shadow)
