@@ -63,11 +63,19 @@
  *
  * Conventions for every entry point:
  *   - All array pointers are DEVICE pointers owned by the caller; the
- *     library allocates no memory and keeps no state between calls.
+ *     library allocates no memory and keeps no state between calls (the
+ *     host-buffer pipeline below is the one exception: it owns its staging
+ *     buffers, streams and events).
  *   - codes, scales, shadow are updated in place; other inputs are read.
  *   - Work is enqueued on `stream` and returns immediately; QS_OK means
  *     "validated and launched".  Execution errors surface at the caller's
  *     next synchronization on that stream.
+ *   - Stream order holds as for any launch.  The decode-step, readout and
+ *     FP32-step kernels are launched with programmatic dependent launch:
+ *     they may be scheduled while the kernel before them in the stream
+ *     finishes, and wait for it to complete (its writes visible) before
+ *     touching any memory.  The environment variable QSTATE_PDL=0 launches
+ *     them plainly.
  *   - Arguments are validated before anything is launched.  A NULL
  *     required pointer, a misaligned pointer (codes, shadow: 32 bytes;
  *     S0, scales, q, k, v, alpha when diagonal: 16 bytes; alpha when
