@@ -66,7 +66,7 @@ struct PrefillLayout {
     constexpr int C = kPrefillChunk;
     int off = 0;
     S = off;    off += dv * (dk + 1);
-    qbar = off; off += dk * C;           // [j][t]: q_t * e^{Lam_t}
+    qbar = off; off += dk * (C + 4);     // [j][t]: q_t * e^{Lam_t} (rows padded to C + 4)
     kbar = off; off += C * dk;           // [s][j]: k_s * e^{Lam_C - Lam_s}
     qt = off;   off += C * (dk + 4);     // [t][j]: q_t (* e^{Lam_t - Lam_m} when diagonal)
     kh = off;   off += C * (dk + 4);     // [s][j]: k_s (* e^{Lam_m - Lam_s} when diagonal)
@@ -81,6 +81,28 @@ struct PrefillLayout {
     total = off;
   }
 };
+
+// State read of two rows for 8 tokens: a[u] = sum_j r0[j] x[j][u], b[u] =
+// sum_j r1[j] x[j][u], j ascending (x rows xs floats apart, 16-byte aligned).
+template <int DK>
+__device__ __forceinline__ void state_read2(const float* r0, const float* r1, const float* x, int xs,
+                                            float (&a)[8], float (&b)[8]) {
+#pragma unroll
+  for (int u = 0; u < 8; ++u) a[u] = b[u] = 0.0f;
+  for (int j = 0; j < DK; ++j) {
+    const float s0 = r0[j], s1 = r1[j];
+    const float4 x0 = *reinterpret_cast<const float4*>(x + j * xs);
+    const float4 x1 = *reinterpret_cast<const float4*>(x + j * xs + 4);
+    a[0] = fmaf(s0, x0.x, a[0]); a[1] = fmaf(s0, x0.y, a[1]);
+    a[2] = fmaf(s0, x0.z, a[2]); a[3] = fmaf(s0, x0.w, a[3]);
+    a[4] = fmaf(s0, x1.x, a[4]); a[5] = fmaf(s0, x1.y, a[5]);
+    a[6] = fmaf(s0, x1.z, a[6]); a[7] = fmaf(s0, x1.w, a[7]);
+    b[0] = fmaf(s1, x0.x, b[0]); b[1] = fmaf(s1, x0.y, b[1]);
+    b[2] = fmaf(s1, x0.z, b[2]); b[3] = fmaf(s1, x0.w, b[3]);
+    b[4] = fmaf(s1, x1.x, b[4]); b[5] = fmaf(s1, x1.y, b[5]);
+    b[6] = fmaf(s1, x1.z, b[6]); b[7] = fmaf(s1, x1.w, b[7]);
+  }
+}
 
 template <int DK, bool DIAG, bool DELTA, int NT>
 __global__ void __launch_bounds__(NT, NT == kPrefillThreads ? 2 : 1) prefill_kernel(PrefillParams p) {
@@ -105,6 +127,9 @@ __global__ void __launch_bounds__(NT, NT == kPrefillThreads ? 2 : 1) prefill_ker
   const size_t tile = blockIdx.x;
   constexpr int SP = DK + 1;  // padded state row
   constexpr int QP = DK + 4;  // padded q / k row (16-byte aligned, no bank conflicts)
+  const int hv = dv / 2;      // rows i and i + hv go to one thread (dv is a multiple of 16)
+  constexpr int QB = C + 4;   // padded qbar row: float4 stores of 4 tokens by consecutive j
+                              // land in 8 different bank groups
   static_assert((NT == 256 || NT == 512) && C == 32, "8 or 16 warps, 32 keys");
 
   float* Sg = p.S + tile * dv * DK;
@@ -146,28 +171,35 @@ __global__ void __launch_bounds__(NT, NT == kPrefillThreads ? 2 : 1) prefill_ker
     __syncthreads();
     // ---- decayed copies of q and k
     const int m = (Ce - 1) / 2;
-    for (int e = tid; e < C * DK; e += NT) {
-      const int t = e / DK, j = e % DK;
-      const bool live = t < Ce;
-      const float qv = live ? p.q[(tok0 + t) * DK + j] : 0.0f;
-      const float kv = live ? p.k[(tok0 + t) * DK + j] : 0.0f;
-      // under the delta rule qbar first holds k_t * e^{Lam_t} (the projection
-      // S k of the corrected values); q_t * e^{Lam_t} replaces it after the solve
-      const float xv = DELTA ? kv : qv;
-      if constexpr (DIAG) {
-        const float lt = lam[t * DK + j], lC = lam[(C - 1) * DK + j], lm = lam[m * DK + j];
-        qbar[j * C + t] = xv * expf(lt);
-        kbar[t * DK + j] = kv * expf(lC - lt);
-        qt[t * QP + j] = qv * expf(lt - lm);
-        kh[t * QP + j] = kv * expf(lm - lt);
-        if constexpr (DELTA) kq[t * QP + j] = kv * expf(lt - lm);
-      } else {
-        const float lt = lam[t], lC = lam[C - 1];
-        qbar[j * C + t] = xv * expf(lt);
-        kbar[t * DK + j] = kv * expf(lC - lt);
-        qt[t * QP + j] = qv;
-        kh[t * QP + j] = kv;
+    // thread (j, 4 tokens): global reads coalesced along j, one float4 of qbar
+    for (int e = tid; e < DK * (C / 4); e += NT) {
+      const int j = e % DK, t0 = 4 * (e / DK);
+      float xb[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int t = t0 + u;
+        const bool live = t < Ce;
+        const float qv = live ? p.q[(tok0 + t) * DK + j] : 0.0f;
+        const float kv = live ? p.k[(tok0 + t) * DK + j] : 0.0f;
+        // under the delta rule qbar first holds k_t * e^{Lam_t} (the projection
+        // S k of the corrected values); q_t * e^{Lam_t} replaces it after the solve
+        const float xv = DELTA ? kv : qv;
+        if constexpr (DIAG) {
+          const float lt = lam[t * DK + j], lC = lam[(C - 1) * DK + j], lm = lam[m * DK + j];
+          xb[u] = xv * expf(lt);
+          kbar[t * DK + j] = kv * expf(lC - lt);
+          qt[t * QP + j] = qv * expf(lt - lm);
+          kh[t * QP + j] = kv * expf(lm - lt);
+          if constexpr (DELTA) kq[t * QP + j] = kv * expf(lt - lm);
+        } else {
+          const float lt = lam[t], lC = lam[C - 1];
+          xb[u] = xv * expf(lt);
+          kbar[t * DK + j] = kv * expf(lC - lt);
+          qt[t * QP + j] = qv;
+          kh[t * QP + j] = kv;
+        }
       }
+      *reinterpret_cast<float4*>(qbar + j * QB + t0) = make_float4(xb[0], xb[1], xb[2], xb[3]);
     }
     __syncthreads();
     // ---- local scores A_ts (s <= t), beta_s folded in: warp w takes tokens
@@ -211,26 +243,17 @@ __global__ void __launch_bounds__(NT, NT == kPrefillThreads ? 2 : 1) prefill_ker
     }
     __syncthreads();
     if constexpr (DELTA) {
-      // ---- r_t = beta_t (v_t - S (k_t e^{Lam_t})), in place of v (8 tokens per thread)
-      for (int e = tid; e < dv * (C / 8); e += NT) {
-        const int i = e % dv, tg = e / dv;
-        float acc[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) acc[u] = 0.0f;
-        const float* srow = S + i * SP;
-        for (int j = 0; j < DK; ++j) {
-          const float sv = srow[j];
-          const float4 a0 = *reinterpret_cast<const float4*>(qbar + j * C + 8 * tg);
-          const float4 a1 = *reinterpret_cast<const float4*>(qbar + j * C + 8 * tg + 4);
-          acc[0] = fmaf(sv, a0.x, acc[0]); acc[1] = fmaf(sv, a0.y, acc[1]);
-          acc[2] = fmaf(sv, a0.z, acc[2]); acc[3] = fmaf(sv, a0.w, acc[3]);
-          acc[4] = fmaf(sv, a1.x, acc[4]); acc[5] = fmaf(sv, a1.y, acc[5]);
-          acc[6] = fmaf(sv, a1.z, acc[6]); acc[7] = fmaf(sv, a1.w, acc[7]);
-        }
+      // ---- r_t = beta_t (v_t - S (k_t e^{Lam_t})), in place of v (rows i, i + dv/2;
+      // 8 tokens per thread)
+      for (int e = tid; e < hv * (C / 8); e += NT) {
+        const int i0 = e % hv, i1 = i0 + hv, tg = e / hv;
+        float a0[8], a1[8];
+        state_read2<DK>(S + i0 * SP, S + i1 * SP, qbar + 8 * tg, QB, a0, a1);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const int t = 8 * tg + u;
-          V[t * dv + i] = bt[t] * (V[t * dv + i] - acc[u]);
+          V[t * dv + i0] = bt[t] * (V[t * dv + i0] - a0[u]);
+          V[t * dv + i1] = bt[t] * (V[t * dv + i1] - a1[u]);
         }
       }
       __syncthreads();
@@ -244,67 +267,82 @@ __global__ void __launch_bounds__(NT, NT == kPrefillThreads ? 2 : 1) prefill_ker
       }
       // ---- qbar = q_t e^{Lam_t} for the state read of the outputs
       if (p.o != nullptr) {
-        for (int e = tid; e < C * DK; e += NT) {
-          const int t = e / DK, j = e % DK;
-          const float qv = t < Ce ? p.q[(tok0 + t) * DK + j] : 0.0f;
-          qbar[j * C + t] = qv * expf(DIAG ? lam[t * DK + j] : lam[t]);
+        for (int e = tid; e < DK * (C / 4); e += NT) {
+          const int j = e % DK, t0 = 4 * (e / DK);
+          float xb[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int t = t0 + u;
+            const float qv = t < Ce ? p.q[(tok0 + t) * DK + j] : 0.0f;
+            xb[u] = qv * expf(DIAG ? lam[t * DK + j] : lam[t]);
+          }
+          *reinterpret_cast<float4*>(qbar + j * QB + t0) = make_float4(xb[0], xb[1], xb[2], xb[3]);
         }
       }
       __syncthreads();
     }
     // ---- outputs: state read + intra-chunk output
     if (p.o != nullptr) {
-      for (int e = tid; e < dv * (C / 8); e += NT) {
-        const int i = e % dv, tg = e / dv;  // 8 tokens per thread
-        float acc[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) acc[u] = 0.0f;
-        const float* srow = S + i * SP;
-        for (int j = 0; j < DK; ++j) {
-          const float sv = srow[j];
-          const float4 a0 = *reinterpret_cast<const float4*>(qbar + j * C + 8 * tg);
-          const float4 a1 = *reinterpret_cast<const float4*>(qbar + j * C + 8 * tg + 4);
-          acc[0] = fmaf(sv, a0.x, acc[0]); acc[1] = fmaf(sv, a0.y, acc[1]);
-          acc[2] = fmaf(sv, a0.z, acc[2]); acc[3] = fmaf(sv, a0.w, acc[3]);
-          acc[4] = fmaf(sv, a1.x, acc[4]); acc[5] = fmaf(sv, a1.y, acc[5]);
-          acc[6] = fmaf(sv, a1.z, acc[6]); acc[7] = fmaf(sv, a1.w, acc[7]);
-        }
+      for (int e = tid; e < hv * (C / 8); e += NT) {
+        const int i0 = e % hv, i1 = i0 + hv, tg = e / hv;  // rows i, i + dv/2; 8 tokens
+        float a0[8], a1[8];
+        state_read2<DK>(S + i0 * SP, S + i1 * SP, qbar + 8 * tg, QB, a0, a1);
         for (int s = 0; s < C; ++s) {
-          const float vs = V[s * dv + i];
+          const float v0 = V[s * dv + i0], v1 = V[s * dv + i1];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) acc[u] = fmaf(A[(8 * tg + u) * C + s], vs, acc[u]);
+          for (int u = 0; u < 8; ++u) {
+            const float a = A[(8 * tg + u) * C + s];
+            a0[u] = fmaf(a, v0, a0[u]);
+            a1[u] = fmaf(a, v1, a1[u]);
+          }
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const int t = 8 * tg + u;
-          if (t < Ce) p.o[(tok0 + t) * dv + i] = acc[u];
+          if (t < Ce) {
+            p.o[(tok0 + t) * dv + i0] = a0[u];
+            p.o[(tok0 + t) * dv + i1] = a1[u];
+          }
         }
       }
       __syncthreads();
     }
     // ---- state pass: S = S e^{Lam_C} + sum_s beta_s v_s kbar_s^T
     {
-      constexpr int JW = 16;  // columns per thread
-      for (int e = tid; e < dv * (DK / JW); e += NT) {
-        const int i = e % dv, jb = (e / dv) * JW;
-        float acc[JW];
-        float* srow = S + i * SP + jb;
+      constexpr int JW = 16;  // columns per thread, rows i and i + dv/2
+      for (int e = tid; e < hv * (DK / JW); e += NT) {
+        const int i0 = e % hv, i1 = i0 + hv, jb = (e / hv) * JW;
+        float a0[JW], a1[JW];
+        float* s0 = S + i0 * SP + jb;
+        float* s1 = S + i1 * SP + jb;
 #pragma unroll
-        for (int u = 0; u < JW; ++u) acc[u] = srow[u] * elam[DIAG ? jb + u : 0];
+        for (int u = 0; u < JW; ++u) {
+          const float f = elam[DIAG ? jb + u : 0];
+          a0[u] = s0[u] * f;
+          a1[u] = s1[u] * f;
+        }
         for (int s = 0; s < Ce; ++s) {
-          const float w = DELTA ? V[s * dv + i] : bt[s] * V[s * dv + i];
+          const float w0 = DELTA ? V[s * dv + i0] : bt[s] * V[s * dv + i0];
+          const float w1 = DELTA ? V[s * dv + i1] : bt[s] * V[s * dv + i1];
           const float4* kr = reinterpret_cast<const float4*>(kbar + s * DK + jb);
 #pragma unroll
           for (int u4 = 0; u4 < JW / 4; ++u4) {
             const float4 kv = kr[u4];
-            acc[4 * u4 + 0] = fmaf(w, kv.x, acc[4 * u4 + 0]);
-            acc[4 * u4 + 1] = fmaf(w, kv.y, acc[4 * u4 + 1]);
-            acc[4 * u4 + 2] = fmaf(w, kv.z, acc[4 * u4 + 2]);
-            acc[4 * u4 + 3] = fmaf(w, kv.w, acc[4 * u4 + 3]);
+            a0[4 * u4 + 0] = fmaf(w0, kv.x, a0[4 * u4 + 0]);
+            a0[4 * u4 + 1] = fmaf(w0, kv.y, a0[4 * u4 + 1]);
+            a0[4 * u4 + 2] = fmaf(w0, kv.z, a0[4 * u4 + 2]);
+            a0[4 * u4 + 3] = fmaf(w0, kv.w, a0[4 * u4 + 3]);
+            a1[4 * u4 + 0] = fmaf(w1, kv.x, a1[4 * u4 + 0]);
+            a1[4 * u4 + 1] = fmaf(w1, kv.y, a1[4 * u4 + 1]);
+            a1[4 * u4 + 2] = fmaf(w1, kv.z, a1[4 * u4 + 2]);
+            a1[4 * u4 + 3] = fmaf(w1, kv.w, a1[4 * u4 + 3]);
           }
         }
 #pragma unroll
-        for (int u = 0; u < JW; ++u) srow[u] = acc[u];
+        for (int u = 0; u < JW; ++u) {
+          s0[u] = a0[u];
+          s1[u] = a1[u];
+        }
       }
     }
   }
