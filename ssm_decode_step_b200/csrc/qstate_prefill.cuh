@@ -36,6 +36,7 @@
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 #include <cuda_runtime.h>
 
 namespace qs {
@@ -61,18 +62,19 @@ struct PrefillParams {
 
 // Shared-memory layout (floats) of one CTA.
 struct PrefillLayout {
-  int S, qbar, kbar, qt, kh, kq, v, lam, A, B, beta, elam, total;
+  int S, qbar, kg, kbar, qt, kh, kq, v, lam, A, B, beta, elam, total;
   __host__ __device__ PrefillLayout(int dk, int dv, bool diag, bool delta = false) {
     constexpr int C = kPrefillChunk;
     int off = 0;
     S = off;    off += dv * (dk + 1);
     qbar = off; off += dk * (C + 4);     // [j][t]: q_t * e^{Lam_t} (rows padded to C + 4)
+    kg = off;   off += delta ? dk * (C + 4) : 0;  // delta rule: [j][t] k_t * e^{Lam_t}, same padding
     kbar = off; off += C * dk;           // [s][j]: k_s * e^{Lam_C - Lam_s}
     qt = off;   off += C * (dk + 4);     // [t][j]: q_t (* e^{Lam_t - Lam_m} when diagonal)
     kh = off;   off += C * (dk + 4);     // [s][j]: k_s (* e^{Lam_m - Lam_s} when diagonal)
     // delta rule, diagonal decay: [t][j] k_t * e^{Lam_t - Lam_m} (scalar decay uses kh)
     kq = off;   off += (delta && diag) ? C * (dk + 4) : 0;
-    v = off;    off += C * dv;           // [s][i]: v, then w under the delta rule
+    v = off;    off += C * (dv + 1);     // [s][i] (rows padded to dv + 1): v, then w (delta rule)
     lam = off;  off += diag ? C * dk : C;  // [t][j] or [t]
     A = off;    off += C * C;            // [t][s], beta_s folded in (linear write only)
     B = off;    off += delta ? C * C : 0;  // [t][s], s < t: the delta rule's triangular system
@@ -82,25 +84,24 @@ struct PrefillLayout {
   }
 };
 
-// State read of two rows for 8 tokens: a[u] = sum_j r0[j] x[j][u], b[u] =
-// sum_j r1[j] x[j][u], j ascending (x rows xs floats apart, 16-byte aligned).
-template <int DK>
+// State read of two rows for TT (4 or 8) tokens: a[u] = sum_j r0[j] x[j][u],
+// b[u] = sum_j r1[j] x[j][u], j ascending (x rows xs floats apart, 16-byte
+// aligned).
+template <int DK, int TT>
 __device__ __forceinline__ void state_read2(const float* r0, const float* r1, const float* x, int xs,
-                                            float (&a)[8], float (&b)[8]) {
+                                            float (&a)[TT], float (&b)[TT]) {
 #pragma unroll
-  for (int u = 0; u < 8; ++u) a[u] = b[u] = 0.0f;
+  for (int u = 0; u < TT; ++u) a[u] = b[u] = 0.0f;
   for (int j = 0; j < DK; ++j) {
     const float s0 = r0[j], s1 = r1[j];
-    const float4 x0 = *reinterpret_cast<const float4*>(x + j * xs);
-    const float4 x1 = *reinterpret_cast<const float4*>(x + j * xs + 4);
-    a[0] = fmaf(s0, x0.x, a[0]); a[1] = fmaf(s0, x0.y, a[1]);
-    a[2] = fmaf(s0, x0.z, a[2]); a[3] = fmaf(s0, x0.w, a[3]);
-    a[4] = fmaf(s0, x1.x, a[4]); a[5] = fmaf(s0, x1.y, a[5]);
-    a[6] = fmaf(s0, x1.z, a[6]); a[7] = fmaf(s0, x1.w, a[7]);
-    b[0] = fmaf(s1, x0.x, b[0]); b[1] = fmaf(s1, x0.y, b[1]);
-    b[2] = fmaf(s1, x0.z, b[2]); b[3] = fmaf(s1, x0.w, b[3]);
-    b[4] = fmaf(s1, x1.x, b[4]); b[5] = fmaf(s1, x1.y, b[5]);
-    b[6] = fmaf(s1, x1.z, b[6]); b[7] = fmaf(s1, x1.w, b[7]);
+#pragma unroll
+    for (int h = 0; h < TT / 4; ++h) {
+      const float4 xv = *reinterpret_cast<const float4*>(x + j * xs + 4 * h);
+      a[4 * h + 0] = fmaf(s0, xv.x, a[4 * h + 0]); a[4 * h + 1] = fmaf(s0, xv.y, a[4 * h + 1]);
+      a[4 * h + 2] = fmaf(s0, xv.z, a[4 * h + 2]); a[4 * h + 3] = fmaf(s0, xv.w, a[4 * h + 3]);
+      b[4 * h + 0] = fmaf(s1, xv.x, b[4 * h + 0]); b[4 * h + 1] = fmaf(s1, xv.y, b[4 * h + 1]);
+      b[4 * h + 2] = fmaf(s1, xv.z, b[4 * h + 2]); b[4 * h + 3] = fmaf(s1, xv.w, b[4 * h + 3]);
+    }
   }
 }
 
@@ -113,6 +114,7 @@ __global__ void __launch_bounds__(NT, NT == kPrefillThreads ? 2 : 1) prefill_ker
   const PrefillLayout Ly(DK, dv, DIAG, DELTA);
   float* S = sm + Ly.S;
   float* qbar = sm + Ly.qbar;
+  float* kg = sm + Ly.kg;
   float* kbar = sm + Ly.kbar;
   float* qt = sm + Ly.qt;
   float* kh = sm + Ly.kh;
@@ -128,6 +130,7 @@ __global__ void __launch_bounds__(NT, NT == kPrefillThreads ? 2 : 1) prefill_ker
   constexpr int SP = DK + 1;  // padded state row
   constexpr int QP = DK + 4;  // padded q / k row (16-byte aligned, no bank conflicts)
   const int hv = dv / 2;      // rows i and i + hv go to one thread (dv is a multiple of 16)
+  const int VS = dv + 1;      // padded row of V
   constexpr int QB = C + 4;   // padded qbar row: float4 stores of 4 tokens by consecutive j
                               // land in 8 different bank groups
   static_assert((NT == 256 || NT == 512) && C == 32, "8 or 16 warps, 32 keys");
@@ -142,7 +145,7 @@ __global__ void __launch_bounds__(NT, NT == kPrefillThreads ? 2 : 1) prefill_ker
     // ---- chunk inputs
     for (int e = tid; e < C * dv; e += NT) {
       const int s = e / dv, i = e % dv;
-      V[e] = s < Ce ? p.v[(tok0 + s) * dv + i] : 0.0f;
+      V[s * VS + i] = s < Ce ? p.v[(tok0 + s) * dv + i] : 0.0f;
     }
     if (tid < C) bt[tid] = tid < Ce ? p.beta[tok0 + tid] : 0.0f;
     // ---- running log-decay over the chunk
@@ -174,32 +177,35 @@ __global__ void __launch_bounds__(NT, NT == kPrefillThreads ? 2 : 1) prefill_ker
     // thread (j, 4 tokens): global reads coalesced along j, one float4 of qbar
     for (int e = tid; e < DK * (C / 4); e += NT) {
       const int j = e % DK, t0 = 4 * (e / DK);
-      float xb[4];
+      float xb[4], gb[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int t = t0 + u;
         const bool live = t < Ce;
         const float qv = live ? p.q[(tok0 + t) * DK + j] : 0.0f;
         const float kv = live ? p.k[(tok0 + t) * DK + j] : 0.0f;
-        // under the delta rule qbar first holds k_t * e^{Lam_t} (the projection
-        // S k of the corrected values); q_t * e^{Lam_t} replaces it after the solve
-        const float xv = DELTA ? kv : qv;
         if constexpr (DIAG) {
           const float lt = lam[t * DK + j], lC = lam[(C - 1) * DK + j], lm = lam[m * DK + j];
-          xb[u] = xv * expf(lt);
+          const float el = expf(lt);
+          xb[u] = qv * el;
+          gb[u] = kv * el;  // delta rule: the keys' projection on the state
           kbar[t * DK + j] = kv * expf(lC - lt);
           qt[t * QP + j] = qv * expf(lt - lm);
           kh[t * QP + j] = kv * expf(lm - lt);
           if constexpr (DELTA) kq[t * QP + j] = kv * expf(lt - lm);
         } else {
           const float lt = lam[t], lC = lam[C - 1];
-          xb[u] = xv * expf(lt);
+          const float el = expf(lt);
+          xb[u] = qv * el;
+          gb[u] = kv * el;
           kbar[t * DK + j] = kv * expf(lC - lt);
           qt[t * QP + j] = qv;
           kh[t * QP + j] = kv;
         }
       }
       *reinterpret_cast<float4*>(qbar + j * QB + t0) = make_float4(xb[0], xb[1], xb[2], xb[3]);
+      if constexpr (DELTA)
+        *reinterpret_cast<float4*>(kg + j * QB + t0) = make_float4(gb[0], gb[1], gb[2], gb[3]);
     }
     __syncthreads();
     // ---- local scores A_ts (s <= t), beta_s folded in: warp w takes tokens
@@ -244,67 +250,76 @@ __global__ void __launch_bounds__(NT, NT == kPrefillThreads ? 2 : 1) prefill_ker
     __syncthreads();
     if constexpr (DELTA) {
       // ---- r_t = beta_t (v_t - S (k_t e^{Lam_t})), in place of v (rows i, i + dv/2;
-      // 8 tokens per thread)
-      for (int e = tid; e < hv * (C / 8); e += NT) {
-        const int i0 = e % hv, i1 = i0 + hv, tg = e / hv;
-        float a0[8], a1[8];
-        state_read2<DK>(S + i0 * SP, S + i1 * SP, qbar + 8 * tg, QB, a0, a1);
+      // TT tokens per thread)
+      auto project = [&](auto tt) {
+        constexpr int TT = decltype(tt)::value;
+        for (int e = tid; e < hv * (C / TT); e += NT) {
+          const int i0 = e % hv, i1 = i0 + hv, tg = e / hv;
+          float a0[TT], a1[TT];
+          state_read2<DK, TT>(S + i0 * SP, S + i1 * SP, kg + TT * tg, QB, a0, a1);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int t = 8 * tg + u;
-          V[t * dv + i0] = bt[t] * (V[t * dv + i0] - a0[u]);
-          V[t * dv + i1] = bt[t] * (V[t * dv + i1] - a1[u]);
-        }
-      }
-      __syncthreads();
-      // ---- forward substitution: w_t = r_t - sum_{s < t} B_ts w_s (s ascending)
-      for (int i = tid; i < dv; i += NT) {
-        for (int t = 1; t < Ce; ++t) {
-          float acc = V[t * dv + i];
-          for (int s2 = 0; s2 < t; ++s2) acc = fmaf(-Bm[t * C + s2], V[s2 * dv + i], acc);
-          V[t * dv + i] = acc;
-        }
-      }
-      // ---- qbar = q_t e^{Lam_t} for the state read of the outputs
-      if (p.o != nullptr) {
-        for (int e = tid; e < DK * (C / 4); e += NT) {
-          const int j = e % DK, t0 = 4 * (e / DK);
-          float xb[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int t = t0 + u;
-            const float qv = t < Ce ? p.q[(tok0 + t) * DK + j] : 0.0f;
-            xb[u] = qv * expf(DIAG ? lam[t * DK + j] : lam[t]);
+          for (int u = 0; u < TT; ++u) {
+            const int t = TT * tg + u;
+            V[t * VS + i0] = bt[t] * (V[t * VS + i0] - a0[u]);
+            V[t * VS + i1] = bt[t] * (V[t * VS + i1] - a1[u]);
           }
-          *reinterpret_cast<float4*>(qbar + j * QB + t0) = make_float4(xb[0], xb[1], xb[2], xb[3]);
         }
-      }
+      };
+      if (hv * (C / 8) >= NT) project(std::integral_constant<int, 8>{});
+      else project(std::integral_constant<int, 4>{});
+      __syncthreads();
+      // ---- forward substitution: w_t = r_t - sum_{s < t} B_ts w_s, P lanes of one
+      // warp per row (partial sums over s = sub, sub + P, ..., then added by shuffles)
+      auto solve = [&](auto pp) {
+        constexpr int PL = decltype(pp)::value;
+        const int sub = tid % PL;
+        for (int base = tid - sub; base < PL * dv; base += NT) {
+          const int i = base / PL;
+          for (int t = 1; t < Ce; ++t) {
+            float part = 0.0f;
+            for (int s2 = sub; s2 < t; s2 += PL) part = fmaf(Bm[t * C + s2], V[s2 * VS + i], part);
+#pragma unroll
+            for (int d = 1; d < PL; d <<= 1) part += __shfl_xor_sync(0xffffffffu, part, d);
+            if (sub == 0) V[t * VS + i] -= part;
+            __syncwarp();
+          }
+        }
+      };
+      // 2 dv and 4 dv are multiples of 32, so every warp is wholly inside or
+      // outside the rows of each pass (the shuffles and __syncwarp need all lanes)
+      if (NT >= 4 * dv) solve(std::integral_constant<int, 4>{});
+      else solve(std::integral_constant<int, 2>{});
       __syncthreads();
     }
     // ---- outputs: state read + intra-chunk output
     if (p.o != nullptr) {
-      for (int e = tid; e < hv * (C / 8); e += NT) {
-        const int i0 = e % hv, i1 = i0 + hv, tg = e / hv;  // rows i, i + dv/2; 8 tokens
-        float a0[8], a1[8];
-        state_read2<DK>(S + i0 * SP, S + i1 * SP, qbar + 8 * tg, QB, a0, a1);
-        for (int s = 0; s < C; ++s) {
-          const float v0 = V[s * dv + i0], v1 = V[s * dv + i1];
+      auto outputs = [&](auto tt) {
+        constexpr int TT = decltype(tt)::value;
+        for (int e = tid; e < hv * (C / TT); e += NT) {
+          const int i0 = e % hv, i1 = i0 + hv, tg = e / hv;  // rows i, i + dv/2; TT tokens
+          float a0[TT], a1[TT];
+          state_read2<DK, TT>(S + i0 * SP, S + i1 * SP, qbar + TT * tg, QB, a0, a1);
+          for (int s = 0; s < C; ++s) {
+            const float v0 = V[s * VS + i0], v1 = V[s * VS + i1];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const float a = A[(8 * tg + u) * C + s];
-            a0[u] = fmaf(a, v0, a0[u]);
-            a1[u] = fmaf(a, v1, a1[u]);
+            for (int u = 0; u < TT; ++u) {
+              const float a = A[(TT * tg + u) * C + s];
+              a0[u] = fmaf(a, v0, a0[u]);
+              a1[u] = fmaf(a, v1, a1[u]);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < TT; ++u) {
+            const int t = TT * tg + u;
+            if (t < Ce) {
+              p.o[(tok0 + t) * dv + i0] = a0[u];
+              p.o[(tok0 + t) * dv + i1] = a1[u];
+            }
           }
         }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int t = 8 * tg + u;
-          if (t < Ce) {
-            p.o[(tok0 + t) * dv + i0] = a0[u];
-            p.o[(tok0 + t) * dv + i1] = a1[u];
-          }
-        }
-      }
+      };
+      if (hv * (C / 8) >= NT) outputs(std::integral_constant<int, 8>{});
+      else outputs(std::integral_constant<int, 4>{});
       __syncthreads();
     }
     // ---- state pass: S = S e^{Lam_C} + sum_s beta_s v_s kbar_s^T
@@ -322,8 +337,8 @@ __global__ void __launch_bounds__(NT, NT == kPrefillThreads ? 2 : 1) prefill_ker
           a1[u] = s1[u] * f;
         }
         for (int s = 0; s < Ce; ++s) {
-          const float w0 = DELTA ? V[s * dv + i0] : bt[s] * V[s * dv + i0];
-          const float w1 = DELTA ? V[s * dv + i1] : bt[s] * V[s * dv + i1];
+          const float w0 = DELTA ? V[s * VS + i0] : bt[s] * V[s * VS + i0];
+          const float w1 = DELTA ? V[s * VS + i1] : bt[s] * V[s * VS + i1];
           const float4* kr = reinterpret_cast<const float4*>(kbar + s * DK + jb);
 #pragma unroll
           for (int u4 = 0; u4 < JW / 4; ++u4) {
