@@ -647,7 +647,7 @@ def run_e2e(args, w, arms, cfgs, states, dev, stream, dist, host, reinit):
     (qstate_pipeline_step, one C call per step): per step, the packed inputs
     are copied up from pinned host memory, every arm's step runs, and the
     readouts are copied back to pinned host memory; all inside the timed
-    region.  The copies run on the pipeline's own streams, three steps deep,
+    region.  The copies run on the pipeline's own streams, four steps deep,
     so step t's inputs go up and step t-1's readouts come down while the
     state updates run in order on the compute stream."""
     import math
@@ -670,7 +670,7 @@ def run_e2e(args, w, arms, cfgs, states, dev, stream, dist, host, reinit):
     # the request group each arm steps at step t (the cycle repeats every `period` steps)
     period = math.lcm(*[len(g) for g in states])
     combos = [tuple(g[t % len(g)] for g in states) for t in range(period)]
-    pl = HostPipeline(combos[0], depth=3)
+    pl = HostPipeline(combos[0], depth=4)
 
     def one(t):
         pl.step(slots_in[t % P], slots_out[t % P], stream, combos[t % period])
@@ -702,7 +702,7 @@ def run_e2e(args, w, arms, cfgs, states, dev, stream, dist, host, reinit):
             "d2h_bytes_per_step": int(len(arms) * T * w.dv * 4) if readout else 0,
             "steps": K,
             "pipelining": "qstate_pipeline_step: inputs up / readouts down on the pipeline's "
-                          "own streams, three buffers"}
+                          "own streams, four buffers"}
 
 
 # ---------------------------------------------------------------------------
