@@ -60,6 +60,13 @@ struct PrefillParams {
   int wait_probe;      // tensor-core path only: > 0 runs the bounded-wait self-check instead
 };
 
+// Row stride of V in shared memory: a multiple of 32 plus 8 floats.  Lanes
+// on consecutive rows i read consecutive banks; in the delta rule's split
+// substitution the 4 lanes of a row read tokens s = sub + 4k, whose rows
+// then start 8 banks apart, so the 8 rows x 4 lanes of a warp hit 32
+// different banks.
+__host__ __device__ constexpr int prefill_vs(int dv) { return (dv + 31) / 32 * 32 + 8; }
+
 // Shared-memory layout (floats) of one CTA.
 struct PrefillLayout {
   int S, qbar, kg, kbar, qt, kh, kq, v, lam, A, B, beta, elam, total;
@@ -74,7 +81,8 @@ struct PrefillLayout {
     kh = off;   off += C * (dk + 4);     // [s][j]: k_s (* e^{Lam_m - Lam_s} when diagonal)
     // delta rule, diagonal decay: [t][j] k_t * e^{Lam_t - Lam_m} (scalar decay uses kh)
     kq = off;   off += (delta && diag) ? C * (dk + 4) : 0;
-    v = off;    off += C * (dv + 1);     // [s][i] (rows padded to dv + 1): v, then w (delta rule)
+    // [s][i]: v, then w (delta rule); row stride = 8 mod 32 floats (prefill_vs)
+    v = off;    off += C * prefill_vs(dv);
     lam = off;  off += diag ? C * dk : C;  // [t][j] or [t]
     A = off;    off += C * C;            // [t][s], beta_s folded in (linear write only)
     B = off;    off += delta ? C * C : 0;  // [t][s], s < t: the delta rule's triangular system
@@ -130,7 +138,7 @@ __global__ void __launch_bounds__(NT, NT == kPrefillThreads ? 2 : 1) prefill_ker
   constexpr int SP = DK + 1;  // padded state row
   constexpr int QP = DK + 4;  // padded q / k row (16-byte aligned, no bank conflicts)
   const int hv = dv / 2;      // rows i and i + hv go to one thread (dv is a multiple of 16)
-  const int VS = dv + 1;      // padded row of V
+  const int VS = prefill_vs(dv);  // padded row of V
   constexpr int QB = C + 4;   // padded qbar row: float4 stores of 4 tokens by consecutive j
                               // land in 8 different bank groups
   static_assert((NT == 256 || NT == 512) && C == 32, "8 or 16 warps, 32 keys");
@@ -269,7 +277,8 @@ __global__ void __launch_bounds__(NT, NT == kPrefillThreads ? 2 : 1) prefill_ker
       else project(std::integral_constant<int, 4>{});
       __syncthreads();
       // ---- forward substitution: w_t = r_t - sum_{s < t} B_ts w_s, P lanes of one
-      // warp per row (partial sums over s = sub, sub + P, ..., then added by shuffles)
+      // warp per row (partial sums over s = sub, sub + P, ..., then added by shuffles;
+      // V's row stride keeps the lanes of a warp on different banks)
       auto solve = [&](auto pp) {
         constexpr int PL = decltype(pp)::value;
         const int sub = tid % PL;
