@@ -57,6 +57,8 @@ def _deps():
 
 
 STAMP = LIB + ".flags"
+# ptxas's resource report (registers, spills, shared memory per kernel) of the last build
+PTXAS_LOG = os.path.join(BUILD, "ptxas.log")
 
 
 def _up_to_date() -> bool:
@@ -76,7 +78,8 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
         return LIB
     os.makedirs(BUILD, exist_ok=True)
     cc = nvcc()
-    extra = ["-Xptxas", "-v"] if ptxas_info else []
+    # the resource report changes no code; it is kept in PTXAS_LOG
+    extra = ["-Xptxas", "-v"]
 
     def compile_one(src):
         obj = os.path.join(BUILD, os.path.basename(src) + ".o")
@@ -88,6 +91,9 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
 
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
         results = list(ex.map(compile_one, _sources()))
+    with open(PTXAS_LOG, "w") as f:
+        for _, log in results:
+            f.write(log)
     if verbose or ptxas_info:
         for _, log in results:
             if log:
@@ -101,6 +107,31 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     with open(STAMP, "w") as f:
         f.write(flags_key())
     return LIB
+
+
+def ptxas_report() -> dict:
+    """{kernel (mangled name): {"registers": n, "spill_stores": bytes,
+    "spill_loads": bytes}} from the last build's ptxas report (rebuilt when
+    the report is missing)."""
+    import re
+    if not os.path.exists(PTXAS_LOG):
+        build(force=True)
+    out, cur = {}, None
+    with open(PTXAS_LOG) as f:
+        for line in f:
+            m = re.search(r"Compiling entry function '(\S+)'", line)
+            if m:
+                cur = m.group(1)
+                out[cur] = {}
+                continue
+            m = re.search(r"(\d+) bytes spill stores, (\d+) bytes spill loads", line)
+            if m and cur:
+                out[cur]["spill_stores"] = int(m.group(1))
+                out[cur]["spill_loads"] = int(m.group(2))
+            m = re.search(r"Used (\d+) registers", line)
+            if m and cur:
+                out[cur]["registers"] = int(m.group(1))
+    return out
 
 
 if __name__ == "__main__":
