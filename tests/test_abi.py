@@ -242,3 +242,22 @@ def test_pipeline_sizes_and_validation_without_a_gpu():
     assert L.qstate_pipeline_join(None, None) == Q.QS_ERR_INVALID_ARG
     assert L.qstate_pipeline_wait_stream(None, None) == Q.QS_ERR_INVALID_ARG
     assert L.qstate_pipeline_destroy(None) == Q.QS_OK
+
+
+def test_host_pipeline_fails_loudly_without_a_device():
+    """Creating a pipeline needs the device (memory, streams, events): with
+    none, the binding raises the library's CUDA error; there is no fallback."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a CUDA device is present")
+
+    class Fake:
+        def __init__(self, cfg):
+            self.cfg = cfg
+
+    with pytest.raises(Q.QStateError) as e:
+        Q.HostPipeline([Fake(_cfg()), Fake(_cfg(policy="yoked"))], depth=3)
+    assert e.value.status == Q.QS_ERR_CUDA
+    with pytest.raises(Q.QStateError) as e:
+        Q.HostPipeline([Fake(_cfg()), Fake(_cfg(num_tiles=5))], depth=3)
+    assert e.value.status == Q.QS_ERR_INVALID_ARG    # checked before any CUDA call
