@@ -125,6 +125,7 @@ DELTA_CASES = [
     (64, 16, "diagonal", 3, 1, True),
     (128, 32, "scalar", 3, 64, False),
     (64, 64, "diagonal", 2, 257, True),
+    (128, 128, "diagonal", 3, 70, True),   # the largest shared-memory configuration (212.6 KB)
 ]
 
 
