@@ -39,11 +39,12 @@
  *        Quantization", abstract: a stored element whose value moves
  *        against its update is rounded one step toward it.)
  * qmax = 2^(bits-1) - 1.  Dot products "." are evaluated in one fixed
- * order: each 32-column chunk is summed as two fused multiply-add chains
- * from +0 in column order, one over its even and one over its odd columns,
- * the chunk sum is even + odd, and the chunk sums are combined by a balanced
- * pairwise tree in column order.  Codes, scales and the shadow are therefore
- * reproducible bit for bit on any conforming implementation.
+ * order: each 32-column chunk is summed as eight fused multiply-add chains
+ * from +0, chain r over the chunk's columns r, r+8, r+16, r+24 in that
+ * order; the chunk sum is ((p0 + p4) + (p2 + p6)) + ((p1 + p5) + (p3 + p7));
+ * and the chunk sums are combined by a balanced pairwise tree in column
+ * order.  Codes, scales and the shadow are therefore reproducible bit for
+ * bit on any conforming implementation.
  *
  * Scale policies ("When Dynamic Scaling Fails", project page): per-token
  * dynamic reads its scale from the state it is about to quantize;

@@ -25,7 +25,7 @@ FAULTS = {
     "none": 0, "drop_delta": 1, "write_sign": 2, "decay_skipped": 3,
     "read_k_for_q": 4, "group_index": 5, "bdr_reference": 6,
     "round_trunc": 7, "beta_on_v_only": 8, "diag_decay_row": 9,
-    "persist_update": 10, "yoked_from_x": 11,
+    "persist_update": 10, "yoked_from_x": 11, "lrb_sign_last": 12,
 }
 
 
@@ -61,38 +61,76 @@ class OracleConfig:
                     ROUNDING[self.rounding])
 
 
-_lib = None
+_libs = {}
+_active = None      # the mutation build while a mistake is planted, else None
+_planted = "none"
+
+
+def _load(path: str, mutations: bool) -> ctypes.CDLL:
+    L = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    C = ctypes.POINTER(_Cfg)
+    for name, args in {
+        "qo_check": [C],
+        "qo_num_threads": [],
+        "qo_pack": [ctypes.c_int, ctypes.c_int64, P, P],
+        "qo_unpack": [ctypes.c_int, ctypes.c_int64, P, P],
+        "qo_init": [C, P, P, P, P],
+        "qo_step": [C, P, P, P, P, P, P, P, P, P, P],
+        "qo_readout": [C, P, P, P, P],
+        "qo_fp32_step": [C, P, P, P, P, P, P, P],
+        "qo_sq_norms": [C, P, P, P],
+        "qo_lrb_step": [C, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P],
+        "qo_fp32_sq_norms": [C, P, P],
+    }.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = ctypes.c_int
+    L.qo_dot.argtypes = [P, P, ctypes.c_int]
+    L.qo_dot.restype = ctypes.c_float
+    if mutations:
+        L.qo_set_fault.argtypes = [ctypes.c_int]
+        L.qo_set_fault.restype = None
+    return L
 
 
 def lib() -> ctypes.CDLL:
-    global _lib
-    if _lib is None:
-        path = _build.build()
-        L = ctypes.CDLL(path)
-        P = ctypes.c_void_p
-        C = ctypes.POINTER(_Cfg)
-        for name, args in {
-            "qo_check": [C],
-            "qo_num_threads": [],
-            "qo_pack": [ctypes.c_int, ctypes.c_int64, P, P],
-            "qo_unpack": [ctypes.c_int, ctypes.c_int64, P, P],
-            "qo_init": [C, P, P, P, P],
-            "qo_step": [C, P, P, P, P, P, P, P, P, P, P],
-            "qo_readout": [C, P, P, P, P],
-            "qo_fp32_step": [C, P, P, P, P, P, P, P],
-            "qo_sq_norms": [C, P, P, P],
-            "qo_lrb_step": [C, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P],
-            "qo_fp32_sq_norms": [C, P, P],
-        }.items():
-            f = getattr(L, name)
-            f.argtypes = args
-            f.restype = ctypes.c_int
-        L.qo_dot.argtypes = [P, P, ctypes.c_int]
-        L.qo_dot.restype = ctypes.c_float
-        L.qo_set_fault.argtypes = [ctypes.c_int]
-        L.qo_set_fault.restype = None
-        _lib = L
-    return _lib
+    """The oracle library every call goes to: the oracle proper, or its
+    mutation build while planted() is active."""
+    if _active is not None:
+        return _active
+    if "plain" not in _libs:
+        _libs["plain"] = _load(_build.build(), False)
+    return _libs["plain"]
+
+
+class planted:
+    """Context manager that routes every oracle call to the mutation build
+    with one mistake planted, and back to the oracle proper on exit (also on
+    an exception)."""
+
+    def __init__(self, fault: str):
+        self.fault = fault
+
+    def __enter__(self):
+        global _active, _planted
+        if "mut" not in _libs:
+            _build.build()
+            _libs["mut"] = _load(_build.MUT_LIB, True)
+        _libs["mut"].qo_set_fault(FAULTS[self.fault])
+        _active, _planted = _libs["mut"], self.fault
+        return self
+
+    def __exit__(self, *exc):
+        global _active, _planted
+        _libs["mut"].qo_set_fault(0)
+        _active, _planted = None, "none"
+        return False
+
+
+def planted_fault() -> str:
+    """The mistake planted right now ("none" outside planted())."""
+    return _planted
 
 
 def _p(a):
@@ -112,10 +150,6 @@ def _ok(rc, what):
 
 def num_threads() -> int:
     return lib().qo_num_threads()
-
-
-def set_fault(name: str) -> None:
-    lib().qo_set_fault(FAULTS[name])
 
 
 def dot(a, b) -> np.float32:

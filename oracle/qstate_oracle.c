@@ -29,8 +29,8 @@
  *                             sigma > 0 and n*s' < d_j then n += 1; if
  *                             sigma < 0 and n*s' > d_j then n -= 1; clamp
  *   9. store                  codes, and s' for dynamic / yoked
- * Dot products "." use qo_dot's fixed order (even / odd chains per 32
- * entries, pairwise tree over the chunks).
+ * Dot products "." use qo_dot's fixed order (eight interleaved chains per
+ * 32 entries, pairwise tree over the chunks).
  */
 #include "qstate_oracle.h"
 
@@ -44,9 +44,18 @@
 #define QO_MAX_DK 1024
 #define QO_MAX_RANK 32
 
+/* Planted mistakes (test build only).  The oracle proper is compiled
+ * without QO_MUTATIONS, where every FAULT(...) below is the constant 0 and
+ * the branches it guards are gone; oracle/build.py compiles the same file a
+ * second time with QO_MUTATIONS into a separate library that the mutation
+ * test alone loads. */
+#ifdef QO_MUTATIONS
 static int g_fault = QO_FAULT_NONE;
-
 void qo_set_fault(int fault) { g_fault = fault; }
+#define FAULT(x) (g_fault == (x))
+#else
+#define FAULT(x) 0
+#endif
 
 int qo_num_threads(void) {
 #ifdef _OPENMP
@@ -71,21 +80,20 @@ int qo_check(const qo_cfg* c) {
   return 0;
 }
 
-/* Fixed-order dot product over n = 32 * 2^m entries: each 32-entry chunk is
- * summed as two fused multiply-add chains from +0 in index order, one over
- * its even entries and one over its odd entries; chunk sum = even + odd; the
- * chunk sums are combined by a balanced pairwise tree in order:
- * ((c0 + c1) + (c2 + c3)) + ... */
+/* Fixed-order dot product over n = 32 * 2^m entries.  Each 32-entry chunk
+ * is summed as eight fused multiply-add chains from +0, chain r over the
+ * entries j = r, r + 8, r + 16, r + 24 of the chunk in that order; the chunk
+ * sum is ((p0 + p4) + (p2 + p6)) + ((p1 + p5) + (p3 + p7)); the chunk sums
+ * are combined by a balanced pairwise tree in order: ((c0 + c1) + (c2 + c3))
+ * + ... */
 float qo_dot(const float* a, const float* b, int n) {
   float part[QO_MAX_DK / 32];
   int chunks = n / 32;
   for (int c = 0; c < chunks; ++c) {
-    float even = 0.0f, odd = 0.0f;
-    for (int i = 0; i < 16; ++i) {
-      even = fmaf(a[32 * c + 2 * i], b[32 * c + 2 * i], even);
-      odd = fmaf(a[32 * c + 2 * i + 1], b[32 * c + 2 * i + 1], odd);
-    }
-    part[c] = even + odd;
+    float p[8];
+    for (int r = 0; r < 8; ++r) p[r] = 0.0f;
+    for (int j = 0; j < 32; ++j) p[j % 8] = fmaf(a[32 * c + j], b[32 * c + j], p[j % 8]);
+    part[c] = ((p[0] + p[4]) + (p[2] + p[6])) + ((p[1] + p[5]) + (p[3] + p[7]));
   }
   for (int width = chunks; width > 1; width /= 2)
     for (int m = 0; m < width / 2; ++m) part[m] = part[2 * m] + part[2 * m + 1];
@@ -96,9 +104,9 @@ static float sign_of(float x) { return x > 0.0f ? 1.0f : (x < 0.0f ? -1.0f : 0.0
 
 /* Decay factor applied to column j of row i of tile t. */
 static float decay_at(const qo_cfg* c, const float* alpha, int t, int i, int j) {
-  if (g_fault == QO_FAULT_DECAY_SKIPPED) return 1.0f;
+  if (FAULT(QO_FAULT_DECAY_SKIPPED)) return 1.0f;
   if (c->decay == QO_DECAY_SCALAR) return alpha[t];
-  if (g_fault == QO_FAULT_DIAG_DECAY_ROW) return alpha[(size_t)t * c->dk + (i % c->dk)];
+  if (FAULT(QO_FAULT_DIAG_DECAY_ROW)) return alpha[(size_t)t * c->dk + (i % c->dk)];
   return alpha[(size_t)t * c->dk + j];
 }
 
@@ -109,9 +117,9 @@ static float row_write(const qo_cfg* c, const float* Sp, const float* k, float v
                        float beta, float* x) {
   const int dk = c->dk;
   float w;
-  if (c->delta && g_fault != QO_FAULT_DROP_DELTA) {
+  if (c->delta && !FAULT(QO_FAULT_DROP_DELTA)) {
     float u = qo_dot(Sp, k, dk);
-    if (g_fault == QO_FAULT_BETA_ON_V_ONLY)
+    if (FAULT(QO_FAULT_BETA_ON_V_ONLY))
       w = beta * v_i - u;
     else
       w = beta * (v_i - u);
@@ -119,7 +127,7 @@ static float row_write(const qo_cfg* c, const float* Sp, const float* k, float v
     w = beta * v_i;
   }
   for (int j = 0; j < dk; ++j) {
-    if (g_fault == QO_FAULT_WRITE_SIGN)
+    if (FAULT(QO_FAULT_WRITE_SIGN))
       x[j] = fmaf(-w, k[j], Sp[j]);
     else
       x[j] = fmaf(w, k[j], Sp[j]);
@@ -134,7 +142,7 @@ static float row_write(const qo_cfg* c, const float* Sp, const float* k, float v
 static int32_t nearest_code(float x, float inv, int qmax, double* pre) {
   double p = (double)x * (double)inv;
   if (pre) *pre = p;
-  double r = (g_fault == QO_FAULT_ROUND_TRUNC) ? trunc(p) : rint(p);
+  double r = (FAULT(QO_FAULT_ROUND_TRUNC)) ? trunc(p) : rint(p);
   r = fmax(r, -(double)qmax);
   r = fmin(r, (double)qmax);
   return (int32_t)r;
@@ -156,9 +164,9 @@ static void requantize_row(const qo_cfg* c, const float* x, const float* Sp,
   for (int g = 0; g < ng; ++g) {
     float s_new;
     int policy = c->policy;
-    if (g_fault == QO_FAULT_PERSIST_UPDATE && policy == QO_SCALE_PERSISTENT)
+    if (FAULT(QO_FAULT_PERSIST_UPDATE) && policy == QO_SCALE_PERSISTENT)
       policy = QO_SCALE_DYNAMIC;
-    if (g_fault == QO_FAULT_YOKED_FROM_X && policy == QO_SCALE_YOKED)
+    if (FAULT(QO_FAULT_YOKED_FROM_X) && policy == QO_SCALE_YOKED)
       policy = QO_SCALE_DYNAMIC;
     if (policy == QO_SCALE_PERSISTENT) {
       s_new = srow[g];
@@ -178,7 +186,7 @@ static void requantize_row(const qo_cfg* c, const float* x, const float* Sp,
       for (int j = g * G; j < (g + 1) * G; ++j) {
         int32_t n = nearest_code(x[j], inv, qmax, pre ? &pre[j] : NULL);
         if (c->rounding == QO_ROUND_BDR) {
-          float ref = (g_fault == QO_FAULT_BDR_REFERENCE) ? Sp[j] : d[j];
+          float ref = (FAULT(QO_FAULT_BDR_REFERENCE)) ? Sp[j] : d[j];
           float dq = (float)n * s_new;
           if (sigma[j] > 0.0f && dq < ref)
             n += 1;
@@ -244,14 +252,14 @@ int qo_step(const qo_cfg* c, int32_t* codes, float* scales, float* shadow,
       /* 1. dequantize with the decayed scale: S' = c * (s * a) */
       for (int j = 0; j < dk; ++j) {
         int g = j / G;
-        if (g_fault == QO_FAULT_GROUP_INDEX) g = (g + 1) % ng;
+        if (FAULT(QO_FAULT_GROUP_INDEX)) g = (g + 1) % ng;
         d[j] = (float)crow[j] * srow[g];
         Sp[j] = (float)crow[j] * (srow[g] * decay_at(c, alpha, t, i, j));
       }
       /* 2-3. write */
       float w = row_write(c, Sp, kt, v[(size_t)t * dv + i], beta[t], x);
       /* 4. readout from the updated, not yet requantized row */
-      if (o) o[row] = qo_dot(x, g_fault == QO_FAULT_READ_K_FOR_Q ? kt : qt, dk);
+      if (o) o[row] = qo_dot(x, FAULT(QO_FAULT_READ_K_FOR_Q) ? kt : qt, dk);
       /* 5. yoked shadow */
       const float* R = NULL;
       if (c->policy == QO_SCALE_YOKED) {
@@ -308,21 +316,21 @@ int qo_lrb_step(const qo_cfg* c, int rank, int slot, int32_t* codes, float* scal
       /* c. dequantize with the accumulated decay: S'_j = c * (s * A_j) */
       for (int j = 0; j < dk; ++j) {
         int g = j / G;
-        if (g_fault == QO_FAULT_GROUP_INDEX) g = (g + 1) % ng;
+        if (FAULT(QO_FAULT_GROUP_INDEX)) g = (g + 1) % ng;
         d[j] = (float)crow[j] * srow[g];
         Sp[j] = (float)crow[j] * (srow[g] * A[j]);
       }
       /* d. write coefficient against the effective state S' + sum_r U_r K_r^T */
       float w;
       const float vi = v[row];
-      if (c->delta && g_fault != QO_FAULT_DROP_DELTA) {
+      if (c->delta && !FAULT(QO_FAULT_DROP_DELTA)) {
         float u = qo_dot(Sp, kt, dk);
         for (int r = 0; r < slot; ++r) u = fmaf(Ut[(size_t)i * rank + r], kk[r], u);
-        w = (g_fault == QO_FAULT_BETA_ON_V_ONLY) ? beta[t] * vi - u : beta[t] * (vi - u);
+        w = (FAULT(QO_FAULT_BETA_ON_V_ONLY)) ? beta[t] * vi - u : beta[t] * (vi - u);
       } else {
         w = beta[t] * vi;
       }
-      if (g_fault == QO_FAULT_WRITE_SIGN) w = -w;
+      if (FAULT(QO_FAULT_WRITE_SIGN)) w = -w;
       /* yoked shadow: the FP32 reference advances every step */
       const float* R = NULL;
       if (c->policy == QO_SCALE_YOKED) {
@@ -335,7 +343,7 @@ int qo_lrb_step(const qo_cfg* c, int rank, int slot, int32_t* codes, float* scal
       if (!merge) {
         /* e. bypass: the write joins the buffer; the stored state is untouched */
         if (o) {
-          float oi = qo_dot(Sp, g_fault == QO_FAULT_READ_K_FOR_Q ? kt : qt, dk);
+          float oi = qo_dot(Sp, FAULT(QO_FAULT_READ_K_FOR_Q) ? kt : qt, dk);
           for (int r = 0; r < slot; ++r) oi = fmaf(Ut[(size_t)i * rank + r], kq[r], oi);
           o[row] = fmaf(w, kqn, oi);
         }
@@ -351,9 +359,9 @@ int qo_lrb_step(const qo_cfg* c, int rank, int slot, int32_t* codes, float* scal
           }
           x[j] = fmaf(w, kt[j], xj);
           M[j] = fmaf(w, kt[j], mj);
-          sg[j] = sign_of(M[j]);
+          sg[j] = FAULT(QO_FAULT_LRB_SIGN_LAST) ? sign_of(w) * sign_of(kt[j]) : sign_of(M[j]);
         }
-        if (o) o[row] = qo_dot(x, g_fault == QO_FAULT_READ_K_FOR_Q ? kt : qt, dk);
+        if (o) o[row] = qo_dot(x, FAULT(QO_FAULT_READ_K_FOR_Q) ? kt : qt, dk);
         requantize_row(c, x, Sp, d, R, sg, crow, srow, prequant ? prequant + row * dk : NULL);
       }
     }
@@ -378,7 +386,7 @@ int qo_readout(const qo_cfg* c, const int32_t* codes, const float* scales,
       size_t row = (size_t)t * dv + i;
       for (int j = 0; j < dk; ++j) {
         int g = j / G;
-        if (g_fault == QO_FAULT_GROUP_INDEX) g = (g + 1) % ng;
+        if (FAULT(QO_FAULT_GROUP_INDEX)) g = (g + 1) % ng;
         d[j] = (float)codes[row * dk + j] * scales[row * ng + g];
       }
       o[row] = qo_dot(d, q + (size_t)t * dk, dk);
@@ -436,7 +444,7 @@ int qo_fp32_step(const qo_cfg* c, float* S, const float* q, const float* k,
       row_write(c, Sp, kt, v[row], beta[t], x);
       memcpy(Srow, x, sizeof(float) * dk);
       if (o)
-        o[row] = qo_dot(x, g_fault == QO_FAULT_READ_K_FOR_Q ? kt : q + (size_t)t * dk, dk);
+        o[row] = qo_dot(x, FAULT(QO_FAULT_READ_K_FOR_Q) ? kt : q + (size_t)t * dk, dk);
     }
   }
   return 0;

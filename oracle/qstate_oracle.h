@@ -24,10 +24,11 @@
  * Arithmetic is IEEE FP32 in a fixed operation order (compiled with
  * -ffp-contract=off; fmaf only where written).  The dequantized, decayed
  * state is c * (s * a) (the decay folded into the group scale first).  Dot
- * products are fixed as: per 32-column chunk, one fused multiply-add chain
- * over the even columns and one over the odd columns, each from +0 in column
- * order, chunk sum = even + odd; chunk sums combined by a balanced pairwise
- * tree in column order.
+ * products are fixed as: per 32-column chunk, eight fused multiply-add
+ * chains from +0, chain r over the columns r, r + 8, r + 16, r + 24 of the
+ * chunk in that order, chunk sum ((p0 + p4) + (p2 + p6)) + ((p1 + p5) +
+ * (p3 + p7)); chunk sums combined by a balanced pairwise tree in column
+ * order.
  *
  * Parity status: every function here is pinned by the CPU tests in
  * tests/test_oracle_pins.py (closed forms, invariants, brute force); the
@@ -137,8 +138,9 @@ int qo_fp32_sq_norms(const qo_cfg* c, const float* S, double* out);
 float qo_dot(const float* a, const float* b, int n);
 
 /* Mistakes that a mutation test plants on purpose, to show that the pins
- * catch them.  0 = none (the default, and the only value outside that
- * test). */
+ * catch them.  Only the mutation build of this file (compiled with
+ * QO_MUTATIONS into liboracle_mut.so) has them and exports qo_set_fault;
+ * the oracle proper (liboracle.so) is compiled without them. */
 enum {
   QO_FAULT_NONE = 0,
   QO_FAULT_DROP_DELTA = 1,      /* delta-rule correction term left out       */
@@ -152,9 +154,12 @@ enum {
   QO_FAULT_DIAG_DECAY_ROW = 9,  /* diagonal decay indexed by row, not column  */
   QO_FAULT_PERSIST_UPDATE = 10, /* persistent scale recomputed every step    */
   QO_FAULT_YOKED_FROM_X = 11,   /* yoked scale taken from the quantized path */
-  QO_FAULT_COUNT = 12
+  QO_FAULT_LRB_SIGN_LAST = 12,  /* merge BDR sign from the last write only   */
+  QO_FAULT_COUNT = 13
 };
+#ifdef QO_MUTATIONS
 void qo_set_fault(int fault);
+#endif
 
 #ifdef __cplusplus
 }

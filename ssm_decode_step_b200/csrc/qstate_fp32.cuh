@@ -118,10 +118,7 @@ __global__ void __launch_bounds__(kThreads, QS_MIN_BLOCKS) fp32_step_kernel(Step
       const float v_i = reinterpret_cast<const float*>(st + L.v)[r];
       float wcoef;
       if constexpr (DELTA) {
-        float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-        for (int m = 0; m < 16; ++m) acc = __ffma2_rn(x[m], kk[m], acc);
-        wcoef = __fmul_rn(beta, __fsub_rn(v_i, row_tree<LPR>(acc)));
+        wcoef = __fmul_rn(beta, __fsub_rn(v_i, row_tree<LPR>(chunk_sum(x, kk))));
       } else {
         wcoef = __fmul_rn(beta, v_i);
       }
@@ -130,10 +127,7 @@ __global__ void __launch_bounds__(kThreads, QS_MIN_BLOCKS) fp32_step_kernel(Step
       if (readout) {
         float2 qv[16];
         load_pairs(st + L.q, c, qv);
-        float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-        for (int m = 0; m < 16; ++m) acc = __ffma2_rn(x[m], qv[m], acc);
-        const float o = row_tree<LPR>(acc);
+        const float o = row_tree<LPR>(chunk_sum(x, qv));
         if (c == 0) p.o[grow0 + r] = o;
       }
       float* dst = p.shadow + (grow0 + r) * DK + 32 * c;

@@ -14,10 +14,10 @@
 //
 // Arithmetic.  Each thread holds its chunk as 16 register pairs of adjacent
 // columns (2m, 2m+1) and works with the packed FP32 instructions of sm_100
-// (__ffma2_rn, __fmul2_rn, __fadd2_rn).  The two lanes of the packed dot
-// product chains are exactly the even-column and odd-column chains of the
-// fixed order; the lanes of a row then add their chunk sums with xor
-// shuffles 1, 2, which is the pairwise tree of the definition.  Every other
+// (__ffma2_rn, __fmul2_rn, __fadd2_rn).  The four packed accumulators of a
+// chunk's dot product carry the eight chains of the fixed order (ChunkDot
+// below); the lanes of a row then add their chunk sums with xor shuffles 1,
+// 2, which is the pairwise tree of the definition.  Every other
 // FP32 operation is element-wise, so packed and scalar forms give the same
 // bits; explicit rounding intrinsics keep the compiler from contracting or
 // reordering (and the library is built -fmad=false).  Codes are unpacked by
@@ -256,11 +256,39 @@ __device__ __forceinline__ void pack_chunk(const float2 (&y)[16], uint32_t (&w)[
   }
 }
 
-// even + odd chains of the chunk, then the pairwise tree across the LPR
-// lanes of the row (xor 1, then xor 2)
+// The fixed dot-product order within a 32-column chunk held as 16 register
+// pairs (2m, 2m+1): eight fused multiply-add chains from +0, chain r over
+// the columns r, r + 8, r + 16, r + 24 in that order.  Pair m carries the
+// columns 2m and 2m + 1, so packed accumulator p[m & 3] holds the chains
+// (2(m & 3), 2(m & 3) + 1), and feeding the pairs in ascending m keeps every
+// chain in column order.  The chunk sum is ((c0 + c4) + (c2 + c6)) +
+// ((c1 + c5) + (c3 + c7)).
+struct ChunkDot {
+  float2 p[4];
+  __device__ __forceinline__ ChunkDot() {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) p[i] = make_float2(0.0f, 0.0f);
+  }
+  __device__ __forceinline__ void add(int m, float2 a, float2 b) { p[m & 3] = __ffma2_rn(a, b, p[m & 3]); }
+  __device__ __forceinline__ float sum() const {
+    const float2 q = __fadd2_rn(__fadd2_rn(p[0], p[2]), __fadd2_rn(p[1], p[3]));
+    return __fadd_rn(q.x, q.y);
+  }
+};
+
+// The whole chunk a . b in the fixed order.
+__device__ __forceinline__ float chunk_sum(const float2 (&a)[16], const float2 (&b)[16]) {
+  ChunkDot d;
+#pragma unroll
+  for (int m = 0; m < 16; ++m) d.add(m, a[m], b[m]);
+  return d.sum();
+}
+
+// The chunk sums of a row's LPR lanes combined by the pairwise tree (xor 1,
+// then xor 2): ((c0 + c1) + (c2 + c3)); every lane of the row gets the same
+// bits because each addition is commutative.
 template <int LPR>
-__device__ __forceinline__ float row_tree(float2 acc) {
-  float t = __fadd_rn(acc.x, acc.y);
+__device__ __forceinline__ float row_tree(float t) {
 #pragma unroll
   for (int m = 1; m < LPR; m <<= 1) t = __fadd_rn(t, __shfl_xor_sync(0xffffffffu, t, m));
   return t;

@@ -150,14 +150,11 @@ __device__ __forceinline__ void lrb_issue_block(const BlockCursor<SLOT, DEPTH>& 
   }
 }
 
-// Even/odd chains of a 32-column chunk against another, then the pairwise
-// tree across the LPR lanes of the row: the fixed dot order.
+// The chunk's eight chains against another chunk, then the pairwise tree
+// across the LPR lanes of the row: the fixed dot order.
 template <int LPR>
 __device__ __forceinline__ float chunk_dot(const float2 (&a)[16], const float2 (&b)[16]) {
-  float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-  for (int m = 0; m < 16; ++m) acc = __ffma2_rn(a[m], b[m], acc);
-  return row_tree<LPR>(acc);
+  return row_tree<LPR>(chunk_sum(a, b));
 }
 
 // POLICY: 0 dynamic, 1 persistent, 2 yoked.  MERGE: last step of the period.

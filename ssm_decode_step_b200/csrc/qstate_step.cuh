@@ -378,10 +378,7 @@ __global__ void __launch_bounds__(kStepThreads, ((POLICY == 2 || BDR) ? QS_STEP_
     // ---- a3/a4: key projection and rank-1 write
     float wcoef;
     if constexpr (DELTA) {
-      float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-      for (int m = 0; m < 16; ++m) acc = __ffma2_rn(Sp[m], kk[m], acc);
-      wcoef = __fmul_rn(beta, __fsub_rn(v_i, row_tree<LPR>(acc)));
+      wcoef = __fmul_rn(beta, __fsub_rn(v_i, row_tree<LPR>(chunk_sum(Sp, kk))));
     } else {
       wcoef = __fmul_rn(beta, v_i);
     }
@@ -391,15 +388,15 @@ __global__ void __launch_bounds__(kStepThreads, ((POLICY == 2 || BDR) ? QS_STEP_
 
     // ---- a5: readout from the updated state
     if (readout) {
-      float2 acc = make_float2(0.0f, 0.0f);
+      ChunkDot acc;
       const float4* qp4 = reinterpret_cast<const float4*>(tv + L.q) + c * (kChunkStride / 4);
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
         const float4 t = qp4[m];
-        acc = __ffma2_rn(x[2 * m], make_float2(t.x, t.y), acc);
-        acc = __ffma2_rn(x[2 * m + 1], make_float2(t.z, t.w), acc);
+        acc.add(2 * m, x[2 * m], make_float2(t.x, t.y));
+        acc.add(2 * m + 1, x[2 * m + 1], make_float2(t.z, t.w));
       }
-      const float o = row_tree<LPR>(acc);
+      const float o = row_tree<LPR>(acc.sum());
       if (c == 0) o_l[blk * RW] = o;
     }
 
@@ -427,10 +424,7 @@ __global__ void __launch_bounds__(kStepThreads, ((POLICY == 2 || BDR) ? QS_STEP_
       }
       float wr;
       if constexpr (DELTA) {
-        float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll
-        for (int mm = 0; mm < 16; ++mm) acc = __ffma2_rn(rs[mm], kk[mm], acc);
-        wr = __fmul_rn(beta, __fsub_rn(v_i, row_tree<LPR>(acc)));
+        wr = __fmul_rn(beta, __fsub_rn(v_i, row_tree<LPR>(chunk_sum(rs, kk))));
       } else {
         wr = wcoef;
       }
@@ -590,10 +584,10 @@ __global__ void __launch_bounds__(kStepThreads, QS_STEP_WARPS_PER_SM / kStepWarp
     const float sc = reinterpret_cast<const float*>(s + O_SCALES)[lane];
     float2 d[16];
     decode_chunk<BITS>(w, d);
-    float2 acc = make_float2(0.0f, 0.0f);
+    ChunkDot acc;
 #pragma unroll
-    for (int m = 0; m < 16; ++m) acc = __ffma2_rn(__fmul2_rn(d[m], f2(sc)), qq[m], acc);
-    const float o = row_tree<LPR>(acc);
+    for (int m = 0; m < 16; ++m) acc.add(m, __fmul2_rn(d[m], f2(sc)), qq[m]);
+    const float o = row_tree<LPR>(acc.sum());
     if (c == 0) o_l[static_cast<size_t>(cur.blk) * RW] = o;
   }
   cp_async_wait<0>();

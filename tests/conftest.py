@@ -18,6 +18,21 @@ def pytest_sessionstart(session):
     cuda_build.build()
 
 
+@pytest.fixture(autouse=True)
+def _oracle_unplanted():
+    """Every test starts and ends with the oracle proper: a planted mistake
+    (tests/test_oracle_mutations.py) never outlives its own test."""
+    import sys as _sys
+    O = _sys.modules.get("oracle.oracle")
+    if O is not None:
+        assert O.planted_fault() == "none", "a planted oracle mistake leaked into this test"
+    yield
+    O = _sys.modules.get("oracle.oracle")
+    if O is not None and O.planted_fault() != "none":
+        O._active, O._planted = None, "none"
+        raise AssertionError("this test left a planted oracle mistake active")
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long CPU test")

@@ -3,8 +3,8 @@ fix, each independent of the oracle's own code path.
 
 Every pin is a plain function that raises AssertionError on failure, so that
 test_oracle_pins.py runs them one by one and test_oracle_mutations.py can
-run them all against an oracle with a mistake planted in it (see
-qo_set_fault) and require that some pin catches each mistake.
+run them all against the oracle's mutation build with a mistake planted in
+it (oracle.planted) and require that some pin catches each mistake.
 
 Sources:
 * eq. (1) and its decay / delta / write-gate choices: "LinQuant: Functional
@@ -379,6 +379,56 @@ def pin_bdr_bruteforce():
     assert moved > 0
 
 
+def pin_bdr_reversal_explained():
+    """North_star invariant (5), clause 1 ("BDR never moves an element against
+    its update"), as it holds under the stored-value reading of the move.
+    The move is measured from d = c * s, the element as stored before the
+    step.  Without decay (Lambda = I) no element ends the step against its
+    update, under a fixed or a changing scale.  With decay, an element can:
+    the decay shrinks it before the write, and when the shrinkage exceeds
+    what one code step can restore it stays on the wrong side of d.  The
+    pin checks both directions and the bound: an element that ends against
+    sigma after BDR has sigma (d - S') > s'/2 (S' the decayed element before
+    the write) when its code is not at the clamp, and sigma (d - S') > 0
+    when it is.  Derivation: x lies on the update's side of S', nearest puts
+    n s' within s'/2 of x, and BDR's step adds s' when n s' was against d."""
+    rng = _rng(28)
+    T, dk, dv, G = 8, 32, 4, 16
+    seen_against = 0
+    for bits in (4, 8):
+        qmax = (1 << (bits - 1)) - 1
+        for policy in ("persistent", "dynamic"):
+            for decay_lo in (1.0, 0.8):
+                cfg = O.OracleConfig(T, dk, dv, bits, G, 0, "diagonal", policy, "bdr")
+                st = O.init(cfg, (rng.standard_normal((T, dv, dk)) * 0.5).astype(F32))
+                for _ in range(10):
+                    q, k, v, a, b = _inputs(rng, T, dk, dv, "diagonal")
+                    if decay_lo == 1.0:
+                        a = np.ones_like(a)
+                    v = (v * 0.05).astype(F32)
+                    prev = st.copy()
+                    O.step(st, q, k, v, a, b, want_o=False)
+                    s_old = np.repeat(prev.scales, G, axis=-1)
+                    d = (prev.codes.astype(F32) * s_old).astype(F32)
+                    Sp = (prev.codes.astype(F32) * (s_old * a[:, None, :]).astype(F32)).astype(F32)
+                    w = (b[:, None] * v).astype(F32)
+                    sigma = np.sign(w)[:, :, None] * np.sign(k)[:, None, :]
+                    s_new = np.repeat(st.scales, G, axis=-1)
+                    val = (st.codes.astype(F32) * s_new).astype(F32)
+                    against = (((sigma > 0) & (val < d)) | ((sigma < 0) & (val > d))) & (s_new > 0)
+                    if decay_lo == 1.0:
+                        assert not np.any(against), (bits, policy)
+                        continue
+                    seen_against += int(against.sum())
+                    shrink = sigma * (d.astype(np.float64) - Sp)
+                    slack = 1e-6 * (np.abs(d) + np.abs(Sp) + s_new)
+                    clamped = np.abs(st.codes) == qmax
+                    assert np.all(shrink[against & ~clamped] > 0.5 * s_new[against & ~clamped]
+                                  - slack[against & ~clamped]), (bits, policy)
+                    assert np.all(shrink[against & clamped] > -slack[against & clamped]), (bits, policy)
+    assert seen_against > 0
+
+
 def pin_yoked_shadow_is_fp32_run():
     """The yoked shadow follows the unquantized FP32 recurrence bit for bit
     (the full-precision reference run alongside)."""
@@ -516,12 +566,12 @@ def pin_pack_layout():
 
 
 def pin_dot_order():
-    """The fixed dot-product order: even / odd chains within each 32-column
-    chunk, pairwise tree over the chunks (worked examples in
-    tests/golden/layout_and_order.json)."""
+    """The fixed dot-product order: eight interleaved chains within each
+    32-column chunk, a fixed combine of the chains, pairwise tree over the
+    chunks (worked examples in tests/golden/layout_and_order.json)."""
     with open(os.path.join(GOLDEN, "layout_and_order.json")) as f:
         data = json.load(f)
-    for key in ("dot_order_chunks", "dot_order_even_odd"):
+    for key in ("dot_order_chunks", "dot_order_combine", "dot_order_chain_sequence"):
         d = data[key]
         a = np.zeros(d["n"], F32)
         b = np.zeros(d["n"], F32)
@@ -529,19 +579,21 @@ def pin_dot_order():
             a[int(idx)] = val
             b[int(idx)] = 1.0
         assert O.dot(a, b) == F32(d["expected"]), key
-        # the order matters: a left-to-right sum gives another value
+        # a left-to-right sum, where the fixture says so, gives another value
         acc = F32(0.0)
         for j in range(d["n"]):
             acc = F32(acc + F32(a[j] * b[j]))
         assert acc == F32(d["left_to_right"]), key
-    # and within the error bound of the exact value on random data
+    # and within the error bound of the exact value on random data: every
+    # product passes through at most 4 chain steps, 3 combine additions and
+    # log2(n / 32) tree additions
     rng = _rng(27)
     for n in (32, 64, 128, 256):
         for _ in range(20):
             a = rng.standard_normal(n).astype(F32)
             b = rng.standard_normal(n).astype(F32)
             exact = float(np.dot(a.astype(np.float64), b.astype(np.float64)))
-            bound = (16 + np.log2(n // 32) + 3) * 2.0 ** -24 * float(np.abs(a.astype(np.float64) * b).sum())
+            bound = (4 + 3 + np.log2(n // 32) + 1) * 2.0 ** -24 * float(np.abs(a.astype(np.float64) * b).sum())
             assert abs(float(O.dot(a, b)) - exact) <= bound
 
 
@@ -671,6 +723,53 @@ def pin_lrb_merge_closed_form():
     assert np.count_nonzero(st.codes != want) <= np.count_nonzero(near_tie)
 
 
+def pin_lrb_merge_bdr_follows_accumulated_update():
+    """At a Low-Rank Bypass merge with rank > 1, BDR's direction is the sign
+    of the period's accumulated update M = sum_r U_r K'_r^T + w k^T, not of the
+    last write alone ("Preserving Updates...", abstract: the buffer merges
+    before rounding, BDR acts at the rounding).  Checked element by element
+    against the nearest-rounding merge of the same buffers, with M formed in
+    float64 from the buffers; elements whose M is too close to 0 for its
+    sign to be certain are skipped.  The case is built so that many
+    reversed elements have sign(M) != sign(w k_j)."""
+    rng = _rng(44)
+    T, dk, dv, R, G = 16, 64, 16, 3, 32
+    qmax = 7
+    checked = differing = 0
+    for period in range(3):
+        cN = O.OracleConfig(T, dk, dv, 4, G, 0, "diagonal", "persistent", "nearest")
+        cB = O.OracleConfig(T, dk, dv, 4, G, 0, "diagonal", "persistent", "bdr")
+        stB = O.init(cB, (rng.standard_normal((T, dv, dk)) * 0.5).astype(F32))
+        stN = O.State(cN, stB.codes.copy(), stB.scales.copy())
+        bB, bN = O.LrbBuffers(cB, R), O.LrbBuffers(cN, R)
+        for slot in range(R):
+            q, k, v, a, b = _inputs(rng, T, dk, dv, "diagonal")
+            v = (v * 0.05).astype(F32)
+            if slot == R - 1:
+                prev_codes, prev_scales = stB.codes.copy(), stB.scales.copy()
+                a64 = a.astype(np.float64)
+                M = np.einsum("tir,trj->tij", bB.U[:, :, :slot].astype(np.float64),
+                              bB.K[:, :slot].astype(np.float64) * a64[:, None, :])
+                w = (b[:, None] * v).astype(F32).astype(np.float64)
+                M += w[:, :, None] * k.astype(np.float64)[:, None, :]
+                lastsign = np.sign(w)[:, :, None] * np.sign(k)[:, None, :]
+            O.lrb_step(stB, bB, q, k, v, a, b, want_o=False)
+            O.lrb_step(stN, bN, q, k, v, a, b, want_o=False)
+        s_el = np.repeat(prev_scales, G, axis=-1)
+        d = (prev_codes.astype(F32) * s_el).astype(F32)
+        n_near = stN.codes
+        dq = (n_near.astype(F32) * s_el).astype(F32)
+        mag = np.abs(M).max(axis=-1, keepdims=True)
+        sure = np.abs(M) > 1e-5 * mag
+        sigma = np.sign(M)
+        rev = ((sigma > 0) & (dq < d)) | ((sigma < 0) & (dq > d))
+        want = np.where(rev, np.clip(n_near + sigma.astype(np.int64), -qmax, qmax), n_near)
+        assert np.array_equal(stB.codes[sure], want[sure])
+        checked += int(sure.sum())
+        differing += int((sure & rev & (sigma != lastsign)).sum())
+    assert checked > 0 and differing > 0
+
+
 def pin_lrb_preserves_small_writes():
     """The point of the bypass: a write of 0.3 code steps per step is rounded
     away by every per-step requantization (persistent scale, no decay), but
@@ -708,6 +807,7 @@ ALL_PINS = [
     pin_persistent_scales_fixed,
     pin_zero_scale_group,
     pin_bdr_bruteforce,
+    pin_bdr_reversal_explained,
     pin_yoked_shadow_is_fp32_run,
     pin_yoked_scale_from_shadow_only,
     pin_high_bit_tracks_fp32,
@@ -719,5 +819,6 @@ ALL_PINS = [
     pin_lrb_rank1_is_step,
     pin_lrb_bypass_tracks_fp32,
     pin_lrb_merge_closed_form,
+    pin_lrb_merge_bdr_follows_accumulated_update,
     pin_lrb_preserves_small_writes,
 ]

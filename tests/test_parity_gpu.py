@@ -146,7 +146,9 @@ def test_zero_update_keeps_persistent_codes():
 
 def test_clipping_and_huge_updates():
     """Persistent and yoked scales clip; updates of millions of grid steps
-    and overflowing values go through the clamping path."""
+    and overflowing values go through the clamping path.  The last step
+    writes v = 3e38, so readouts overflow: the GPU must give NaN and
+    infinities of the same sign exactly where the oracle does."""
     rng = np.random.default_rng(5)
     T, dk, dv = 6, 128, 64
     S0 = (rng.standard_normal((T, dv, dk)) * 1e-3).astype(np.float32)
@@ -159,6 +161,16 @@ def test_clipping_and_huge_updates():
         for rnd in ("nearest", "bdr"):
             cfg = Config(T, dk, dv, 8, 64, 0, "scalar", pol, rnd)
             P.lockstep(cfg, S0, steps, label=f"clip-{pol}-{rnd}")
+            # the overflow step, free-run, with its readouts compared by pattern
+            gpu = P.GpuRun(cfg, S0)
+            ora = O.init(P.oracle_cfg(cfg), S0)
+            for t, (q, k, v, a, b) in enumerate(steps):
+                o = gpu.step(q, k, v, a, b)
+                o_ref = O.step(ora, q, k, v, a, b)
+                P.compare_readout(o, o_ref, f"clip-{pol}-{rnd} free step {t}")
+            assert not np.all(np.isfinite(o_ref)), "the overflow step overflowed no readout"
+            c, s_, sh = gpu.state()
+            P.compare_state(cfg, c, s_, ora, None, f"clip-{pol}-{rnd} after the overflow step")
 
 
 # Full-size workloads at the benchmark's launch configuration, on sampled
