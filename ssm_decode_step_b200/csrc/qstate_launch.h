@@ -8,6 +8,7 @@
 
 #include "qstate_kernels.cuh"
 #include "qstate_step.cuh"
+#include "qstate_stream.cuh"
 #include "qstate_lrb.cuh"
 
 namespace qs {

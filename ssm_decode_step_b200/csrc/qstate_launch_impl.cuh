@@ -121,33 +121,64 @@ static cudaError_t launch_warps(K kernel, const P& p, size_t smem, cudaStream_t 
   return launch_dependent(kernel, grid, kStepThreads, smem, stream, p);
 }
 
+// The decode step: the streamed kernel for the dynamic and persistent
+// policies, the shared-memory ring kernel for the yoked policy (whose FP32
+// shadow is too large to stream through registers).
 template <int BITS, int DK, int POLICY, bool BDR, bool DELTA, bool DIAG>
 cudaError_t launch_step(const StepParams& p0, cudaStream_t stream) {
-  constexpr int D = step_depth<POLICY>();
   constexpr int RW = 32 / (DK / 32);  // rows per row block
-  constexpr int WARPS = kStepWarps;
-  auto kernel = step_kernel<BITS, DK, POLICY, BDR, DELTA, DIAG, D>;
-  static std::once_flag flag;
-  cudaError_t err = allow_smem(kernel, flag);
-  if (err != cudaSuccess) return err;
-  WarpStepParams p;
-  p.codes = p0.codes;
-  p.scales = p0.scales;
-  p.shadow = p0.shadow;
-  p.q = p0.q;
-  p.k = p0.k;
-  p.v = p0.v;
-  p.alpha = p0.alpha;
-  p.beta = p0.beta;
-  p.o = p0.o;
-  p.bpt = p0.dv / RW;
-  p.nblocks = p0.tiles * p.bpt;  // < 2^31 (checked by the caller)
-  p.group = p0.group;
-  // tile-vector slots: every tile that D consecutive row blocks can touch
-  p.ntv = (D - 1 + p.bpt - 1) / p.bpt + 1;
-  const WarpLayout L(BITS, DK, DIAG, BDR, POLICY == 2);
-  p.warp_bytes = L.bytes(D, p.ntv);
-  return launch_warps(kernel, p, static_cast<size_t>(p.warp_bytes) * WARPS, stream);
+  if constexpr (POLICY != 2) {
+    auto kernel = stream_step_kernel<BITS, DK, POLICY, BDR, DELTA, DIAG>;
+    static std::once_flag flag;
+    cudaError_t err = allow_smem(kernel, flag);
+    if (err != cudaSuccess) return err;
+    StreamParams p;
+    p.codes = p0.codes;
+    p.scales = p0.scales;
+    p.q = p0.q;
+    p.k = p0.k;
+    p.v = p0.v;
+    p.alpha = p0.alpha;
+    p.beta = p0.beta;
+    p.o = p0.o;
+    p.bpt = p0.dv / RW;
+    p.nblocks = p0.tiles * p.bpt;  // < 2^31 (checked by the caller)
+    p.group = p0.group;
+    p.two23 = 0x4B000000u;
+    const StreamLayout L(DK, DIAG, BDR && POLICY == 0);
+    int per_sm = 0;
+    err = resident_ctas(kernel, 32, static_cast<size_t>(L.bytes()), &per_sm);
+    if (err != cudaSuccess) return err;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    long long grid = static_cast<long long>(per_sm) * device_sm_count();
+    if (grid > p.nblocks) grid = p.nblocks;
+    return launch_dependent(kernel, grid, 32, static_cast<size_t>(L.bytes()), stream, p);
+  } else {
+    constexpr int D = step_depth<POLICY>();
+    constexpr int WARPS = kStepWarps;
+    auto kernel = step_kernel<BITS, DK, POLICY, BDR, DELTA, DIAG, D>;
+    static std::once_flag flag;
+    cudaError_t err = allow_smem(kernel, flag);
+    if (err != cudaSuccess) return err;
+    WarpStepParams p;
+    p.codes = p0.codes;
+    p.scales = p0.scales;
+    p.shadow = p0.shadow;
+    p.q = p0.q;
+    p.k = p0.k;
+    p.v = p0.v;
+    p.alpha = p0.alpha;
+    p.beta = p0.beta;
+    p.o = p0.o;
+    p.bpt = p0.dv / RW;
+    p.nblocks = p0.tiles * p.bpt;  // < 2^31 (checked by the caller)
+    p.group = p0.group;
+    // tile-vector slots: every tile that D consecutive row blocks can touch
+    p.ntv = (D - 1 + p.bpt - 1) / p.bpt + 1;
+    const WarpLayout L(BITS, DK, DIAG, BDR, true);
+    p.warp_bytes = L.bytes(D, p.ntv);
+    return launch_warps(kernel, p, static_cast<size_t>(p.warp_bytes) * WARPS, stream);
+  }
 }
 
 template <int BITS, int DK, int POLICY, bool BDR, bool DELTA, bool DIAG, bool MERGE>

@@ -1,16 +1,18 @@
 """Register use of the built kernels, from ptxas's resource report of the
 last build (no GPU needed).
 
-The kernels the benchmark times for its workloads must not spill; a few
-rarely used combinations at the register cap (yoked or Low-Rank Bypass
-merges with Bounded Directional Rounding at 168 registers, four tensor-core
-prefill instances at 128) spill a few bytes to local memory, and no kernel
-may spill more than 64 bytes."""
+The decode-step kernels the benchmark times for its workloads (the
+streamed kernel for dynamic and persistent scales, the ring kernel for the
+yoked one) must not spill; a few rarely used combinations at the register
+cap (yoked or Low-Rank Bypass merges with Bounded Directional Rounding at
+168 registers, four tensor-core prefill instances at 128) spill a few bytes
+to local memory, and no kernel may spill more than 64 bytes."""
 import re
 
 from ssm_decode_step_b200 import build as B
 
-STEP = re.compile(r"_ZN2qs11step_kernelILi(\d)ELi(\d+)ELi(\d)ELb(\d)ELb(\d)ELb(\d)ELi\dE")
+# the ring kernel (yoked policy) and the streamed kernel (dynamic, persistent)
+STEP = re.compile(r"_ZN2qs(?:11step_kernel|18stream_step_kernel)ILi(\d)ELi(\d+)ELi(\d)ELb(\d)ELb(\d)ELb(\d)E")
 
 
 def _step_key(name):
