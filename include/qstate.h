@@ -225,6 +225,46 @@ QS_API qs_status qstate_pipeline_sync(qs_pipeline* pl);
  * NULL is accepted and ignored. */
 QS_API qs_status qstate_pipeline_destroy(qs_pipeline* pl);
 
+/* Bytes of device memory that qstate_decode_step_host_static stages one
+ * step through (32 MiB): a static array of the library that every GPU which
+ * loads the library holds until the process exits. */
+#define QS_STATIC_STAGE_BYTES ((size_t)32 << 20)
+
+/* One decode step of one state family, as qstate_decode_step defines it,
+ * with its inputs read from HOST memory and its readouts written back to
+ * HOST memory, that allocates nothing.  It has no counterpart in the pages
+ * the method comes from: it exists for callers that may not allocate device
+ * memory themselves, such as an engine whose own memory manager owns the
+ * whole device budget (a cudaMalloc outside it can fail or fragment that
+ * budget) or a serving loop that cannot afford cudaMalloc's implicit
+ * device-wide synchronization.  The host-buffer pipeline above stages
+ * through device buffers it allocates at creation; this call stages through
+ * a fixed static device array of QS_STATIC_STAGE_BYTES bytes instead, and
+ * calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * host_in: the packed host input of one step in the pipeline's layout
+ * (q | k | v | alpha | beta, qstate_pipeline_query_sizes with n = 1);
+ * host_out: o [T][Dv] floats, or NULL for no readout.  codes, scales and
+ * shadow are DEVICE pointers, as for qstate_decode_step.  Everything is
+ * enqueued on `stream` in order: the input copy, the step, the output copy;
+ * the caller keeps host_in unchanged and reads host_out only after
+ * synchronizing with `stream`.  Page-locked host memory makes the copies
+ * asynchronous.
+ *
+ * Limits and sharing: a step whose input bytes plus (when host_out is not
+ * NULL) output bytes exceed QS_STATIC_STAGE_BYTES returns
+ * QS_ERR_UNSUPPORTED before any CUDA call.  The first call on a device looks
+ * up the array's device address on that device (with it current) and keeps
+ * it; make that first call before any stream capture.  Every call on a
+ * device shares the one array, which keeps the last call's contents: each
+ * call writes every byte it reads from it, so nothing needs to start at
+ * zero, but calls that overlap on the GPU (on different streams, or from
+ * several host threads) overwrite each other's staging and race.  The other
+ * argument checks and errors are qstate_decode_step's. */
+QS_API qs_status qstate_decode_step_host_static(const qs_config* cfg, void* codes, float* scales,
+                                                float* shadow, const void* host_in, float* host_out,
+                                                cudaStream_t stream);
+
 /* Readout of the stored state without changing it: o_i = d_i . q with
  * d_ij = c_ij * s_ig (no decay; the fixed dot order above). */
 QS_API qs_status qstate_readout(const qs_config* cfg, const void* codes,

@@ -29,7 +29,7 @@ EXPORTS = ("qstate_query_sizes", "qstate_init", "qstate_decode_step", "qstate_re
            "qstate_prefill_tf32_wait_selfcheck",
            "qstate_pipeline_query_sizes", "qstate_pipeline_create", "qstate_pipeline_step",
            "qstate_pipeline_wait_stream", "qstate_pipeline_join", "qstate_pipeline_sync",
-           "qstate_pipeline_destroy",
+           "qstate_pipeline_destroy", "qstate_decode_step_host_static",
            "qstate_state_sq_norms", "qstate_fp32_sq_norms",
            "qstate_selfcheck", "qstate_status_string", "qstate_version")
 
@@ -77,6 +77,7 @@ def lib() -> ctypes.CDLL:
         L.qstate_pipeline_join.argtypes = [P, P]
         L.qstate_pipeline_sync.argtypes = [P]
         L.qstate_pipeline_destroy.argtypes = [P]
+        L.qstate_decode_step_host_static.argtypes = [C, P, P, P, P, P, P]
         L.qstate_state_sq_norms.argtypes = [C, P, P, P, P]
         L.qstate_fp32_sq_norms.argtypes = [C, P, P, P]
         for f in (L.qstate_query_sizes, L.qstate_init, L.qstate_decode_step, L.qstate_readout,
@@ -85,7 +86,8 @@ def lib() -> ctypes.CDLL:
                   L.qstate_prefill, L.qstate_prefill_tf32, L.qstate_prefill_tf32_timeouts,
                   L.qstate_prefill_tf32_wait_selfcheck, L.qstate_pipeline_query_sizes,
                   L.qstate_pipeline_create, L.qstate_pipeline_step, L.qstate_pipeline_wait_stream,
-                  L.qstate_pipeline_join, L.qstate_pipeline_sync, L.qstate_pipeline_destroy):
+                  L.qstate_pipeline_join, L.qstate_pipeline_sync, L.qstate_pipeline_destroy,
+                  L.qstate_decode_step_host_static):
             f.restype = ctypes.c_int
         L.qstate_status_string.argtypes = [ctypes.c_int]
         L.qstate_status_string.restype = ctypes.c_char_p
@@ -327,6 +329,21 @@ class QState:
     def readout(self, q, o, stream=None):
         readout(self.cfg, self.codes, self.scales, q, o, stream)
         return o
+
+
+def decode_step_host_static(cfg: Config, codes, scales, shadow, host_in, host_out=None,
+                            stream=None) -> None:
+    """qstate_decode_step_host_static: one decode step with inputs from host
+    memory (the packed layout of pipeline_query_sizes with n = 1) and
+    readouts back to host memory, staged through the library's static device
+    array instead of any allocation.  host_in / host_out are host tensors
+    (page-locked for asynchronous copies); read host_out after synchronizing
+    with `stream`."""
+    cc = cfg.c()
+    _check(lib().qstate_decode_step_host_static(ctypes.byref(cc), _ptr(codes), _ptr(scales),
+                                                _ptr(shadow), _ptr(host_in), _ptr(host_out),
+                                                _stream(stream)),
+           "qstate_decode_step_host_static")
 
 
 def pipeline_query_sizes(cfg: Config, n: int):
