@@ -5,11 +5,13 @@
                     [--workload gdn|mamba2|gla|stack24|tiny-gdn]
 
 One "step" advances the workload's batch by one token under each of its
-arms (for the default Gated DeltaNet-shaped workload: INT4 G32 with dynamic,
-persistent and yoked scales, one kernel launch each, readout on).  The
+arms.  The default workload is the largest, the 24-layer gated delta-rule
+stack (12288 tiles of Dk = Dv = 128, readout every step) under its two arms,
+INT4 G32 persistent + BDR and INT8 G32 dynamic: one kernel launch each.  The
 metric is decode steps/s (whole job; N GPUs run independent shards, so
 scaling is weak) and the algorithmic state traffic in GB/s as a fraction of
-the measured HBM peak.
+the measured HBM peak; the roofline line reports the quantized-state arm
+furthest from that peak.
 
 L2 residency: an arm's state can be smaller than B200's L2, so each arm's
 steps rotate over G independent request groups whose states together exceed
@@ -17,11 +19,15 @@ steps rotate over G independent request groups whose states together exceed
 other); step t uses group t mod G and pool slot t mod P of the inputs.  No
 state or input is therefore warm in L2 when its step runs.
 
-Timing: W untimed warm-up steps per arm (eager and graph), then the states
-are re-initialized and each arm's K steps are replayed from CUDA graphs,
-bracketed by CUDA events on the launching stream, with a barrier and a
-device synchronize on both sides; the max over ranks is reported.  SM clocks
-and throttle reasons are sampled through NVML during the timed region.
+Timing: W untimed warm-up steps per arm (eager), then every CUDA graph the
+timed region replays (a full cycle of P steps and the K mod P tail) is
+replayed once, the states are re-initialized, and each arm's K steps are
+replayed from those graphs, bracketed by CUDA events on the launching
+stream, with a barrier and a device synchronize on both sides; the max over
+ranks is reported.  Between the synchronize and the first timed event the
+stream writes a buffer twice the L2 size (clearing L2 and keeping the GPU
+busy up to the timed region).  SM clocks and throttle reasons are sampled
+through NVML during the timed region.
 
 The `e2e` figure runs the same steps through the public API with host
 buffers: each step copies its inputs from pinned host memory, launches the
@@ -85,8 +91,9 @@ def state_bytes(w: W.Workload, arm: W.Arm) -> int:
 
 # The sources the decode-step kernel is compiled from: a committed traffic
 # figure stays valid while none of them, nor the nvcc flags, changes.
-STEP_SOURCES = ("qstate_step.cuh", "qstate_kernels.cuh", "qstate_launch.h", "qstate_launch_impl.cuh",
-                "inst_b4_d128.cu", "inst_b4_d64.cu", "inst_b8_d128.cu", "inst_b8_d64.cu")
+STEP_SOURCES = ("qstate_step.cuh", "qstate_stream.cuh", "qstate_kernels.cuh", "qstate_launch.h",
+                "qstate_launch_impl.cuh", "inst_b4_d128.cu", "inst_b4_d64.cu", "inst_b8_d128.cu",
+                "inst_b8_d64.cu")
 
 
 def source_sha() -> str:
@@ -203,6 +210,23 @@ class ClockSampler:
 # distributed plumbing (barrier and max over ranks only; no data-path collective)
 # ---------------------------------------------------------------------------
 
+def pool_slots(w: W.Workload, l2: int) -> int:
+    """Input slots: enough that the pool exceeds twice the L2 size (so no
+    step finds its inputs in L2), a power of two from 16 to 64."""
+    per_slot = w.tiles * (2 * w.dk + w.dv + (w.dk if w.decay == "diagonal" else 1) + 1) * 4
+    P = 16
+    while P < 64 and P * per_slot < 2 * l2:
+        P *= 2
+    return P
+
+
+def l2_flush(dev, l2: int):
+    """A device buffer of twice the L2 size, written (on the current stream)
+    between the last synchronize and the first timed event."""
+    import torch
+    return torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -296,18 +320,22 @@ def run_ours(args):
 
     from ssm_decode_step_b200 import Config, QState, qstate as Q
     Q.lib()
-    w = W.get(args.workload)
+    # N GPUs split one workload: rank r owns the contiguous tile range
+    # [r T / N, (r + 1) T / N) (tiles are independent; no exchange)
+    w_all = W.get(args.workload)
+    w = W.shard(w_all, rank, ws) if ws > 1 else w_all
     arms = list(w.arms)
     K, Wm = args.steps, args.warmup
     readout = w.readout
 
     # input pool on the device: P slots of (q, k, v, alpha, beta)
-    P = args.pool
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    P = args.pool or pool_slots(w, l2)
+    args.pool = P
     host = W.pool(w, P)
     pool = [torch.from_numpy(a).to(dev) for a in host]
 
     # request groups so that all groups' states exceed 2x L2
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     pool_bytes = P * sum(a[0].nbytes for a in host)
 
     def groups_for(arm):
@@ -359,13 +387,17 @@ def run_ours(args):
 
     graphs = [capture(ai, P) for ai in range(len(arms))]
     tails = [capture(ai, tail) if tail else None for ai in range(len(arms))]
-    # warm the graph path, then restart every state from S0
+    # warm every graph the timed region replays (the first replay of a graph
+    # uploads it), then restart every state from S0
     with torch.cuda.stream(stream):
         for ai in range(len(arms)):
             graphs[ai].replay()
+            if tails[ai] is not None:
+                tails[ai].replay()
     stream.synchronize()
     reinit()
     torch.cuda.synchronize()
+    flush = l2_flush(dev, l2)
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in arms]
     sampler = ClockSampler(local)
@@ -374,6 +406,8 @@ def run_ours(args):
     torch.cuda.synchronize()
     with sampler:
         with torch.cuda.stream(stream):
+            flush.fill_(1.0)
+            flush.fill_(2.0)
             for ai in range(len(arms)):
                 ev[ai][0].record(stream)
                 for _ in range(n_main):
@@ -385,6 +419,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
+    del flush
     arm_ms = [a.elapsed_time(b) for a, b in ev]
     arm_ms = max_over_ranks(dist, arm_ms, dev)
     total_ms = sum(arm_ms)
@@ -399,11 +434,17 @@ def run_ours(args):
     e2e = run_e2e(args, w, arms, cfgs, states, dev, stream, dist, host, reinit)
 
     peak, peak_src = load_peak()
-    bytes_step = sum(arm_bytes(w, a, readout) for a in arms)
-    value = ws * K / (total_ms / 1e3)
+    # whole-job rates: every step advances all ranks' shards, i.e. the whole
+    # workload, and the slowest rank's time is the step time
+    bytes_step = sum(arm_bytes(w_all, a, readout) for a in arms)
+    value = K / (total_ms / 1e3)
     gbs = bytes_step * K / (total_ms / 1e3) / 1e9
-    dom = int(np.argmax(arm_ms))
-    dom_bytes = arm_bytes(w, arms[dom], readout)
+    # the roofline line: the quantized-state arm furthest from the HBM peak
+    # (the yoked arm moves mostly its FP32 shadow and is reported per arm)
+    quant = [i for i, a in enumerate(arms) if a.policy != "yoked"] or list(range(len(arms)))
+    fracs = {i: arm_bytes(w, arms[i], readout) / (arm_ms[i] / 1e3 / K) / 1e9 / peak for i in quant}
+    dom = min(fracs, key=fracs.get)
+    dom_bytes = arm_bytes(w, arms[dom], readout)      # per GPU (this rank's shard)
     dom_s = arm_ms[dom] / 1e3 / K
     achieved = dom_bytes / dom_s / 1e9
     kernel_key = f"{w.name}:{arms[dom].name}"
@@ -425,13 +466,14 @@ def run_ours(args):
         "warmup": Wm,
         "ms_per_step": round(total_ms / K, 6),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong",
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic (seeded; shapes and value laws of the workload)",
         "config": {
-            "workload": w.description,
-            "tiles": w.tiles,
+            "workload": f"{w_all.name}: {w_all.description}",
+            "tiles": w_all.tiles,
+            "tiles_per_gpu": w.tiles,
             "step": f"one token for all {w.tiles} tiles under each arm ({len(arms)} launches)",
             "arms": [a.name for a in arms],
             "readout": readout,
@@ -442,14 +484,17 @@ def run_ours(args):
                  f"{state_bytes(w, a) / 1e6:.1f} MB state + {pool_bytes / 1e6:.0f} MB of input "
                  f"slots rotated; L2 {l2 / 1e6:.0f} MB)")
                 for a, g, res in zip(arms, groups, l2_resident)),
-            "parallelism": f"independent tile shards, {ws} GPU(s), no collective on the step",
+            "parallelism": (f"tile shards on {ws} GPU(s): rank r owns tiles [r*T/N, (r+1)*T/N) of the "
+                            f"one workload; no collective on the step"),
         },
         "state_gbs": round(gbs, 1),
         "state_frac": round(gbs / peak, 4),
         "arms": per_arm,
         "roofline": {
             "bound": "hbm",
-            "kernel": f"step_kernel ({kernel_key})",
+            "kernel": f"{'stream_step_kernel' if arms[dom].policy != 'yoked' else 'step_kernel'} "
+                      f"({kernel_key}; the quantized-state arm furthest from the peak)",
+            "quantized_arms_frac": {arms[i].name: round(f, 4) for i, f in fracs.items()},
             "achieved": round(achieved, 1),
             "peak": peak,
             "peak_source": peak_src,
@@ -465,7 +510,7 @@ def run_ours(args):
             "state_memory_ratio": {a.name: round(w.tiles * w.dv * w.dk * 4 / state_bytes(w, a), 3)
                                    for a in arms}}),
         "lrb": lrb,
-        "gpu_launches": K * len(arms),
+        "gpu_launches": ws * K * len(arms),
         "clocks": clocks,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -696,8 +741,8 @@ def run_e2e(args, w, arms, cfgs, states, dev, stream, dist, host, reinit):
     torch.cuda.synchronize()
     pl.close()
     ms = max_over_ranks(dist, [e0.elapsed_time(e1)], dev)[0]
-    ws = dist.get_world_size() if dist is not None else 1
-    return {"value": round(ws * K / (ms / 1e3), 2), "unit": "steps/s",
+    # each rank pipelines its shard: a step of every rank is one whole-workload step
+    return {"value": round(K / (ms / 1e3), 2), "unit": "steps/s",
             "h2d_bytes_per_step": int(sum(sizes) * 4),
             "d2h_bytes_per_step": int(len(arms) * T * w.dv * 4) if readout else 0,
             "steps": K,
@@ -780,7 +825,7 @@ def run_recall(args):
     torch.cuda.set_device(0)
     kstar, vstar = W.probe(w)
     S0 = plant(W.initial_state(w), kstar, vstar)
-    P = max(1, min(args.pool, H))
+    P = max(1, min(args.pool or 64, H))
     pool = [torch.from_numpy(a).to(dev) for a in W.pool(w, P)]
     kst = torch.from_numpy(kstar).to(dev)
     zk = torch.zeros((T, dk), dtype=torch.float32, device=dev)
@@ -910,7 +955,7 @@ def run_prefill(args):
     w = W.get(args.workload)
     if args.prefill_tiles > 0:
         w = W.scaled_down(w, args.prefill_tiles, layers=1)
-    L, P = args.prefill, max(1, min(args.pool, args.prefill))
+    L, P = args.prefill, max(1, min(args.pool or 64, args.prefill))
     dev = torch.device("cuda")
     T = w.tiles
     slots = [W.slot(w, t) for t in range(P)]
@@ -980,12 +1025,13 @@ def run_prefill(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=8192,
-                    help="timed steps (default: 4 request groups x the 2048-token horizon)")
+    ap.add_argument("--steps", type=int, default=2048,
+                    help="timed steps per arm")
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="gdn", choices=list(W.WORKLOADS))
-    ap.add_argument("--pool", type=int, default=64, help="input slots on the device")
+    ap.add_argument("--workload", default="stack24", choices=list(W.WORKLOADS))
+    ap.add_argument("--pool", type=int, default=0,
+                    help="input slots on the device (0: enough to exceed 2x L2, 16 to 64)")
     ap.add_argument("--groups", type=int, default=0, help="request groups (0: enough to exceed 2x L2)")
     ap.add_argument("--e2e-steps", type=int, default=1024)
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")

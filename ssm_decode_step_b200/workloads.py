@@ -18,7 +18,7 @@ Randomness layout (fixed, so that every consumer sees the same bytes):
 """
 from __future__ import annotations
 
-from dataclasses import dataclass, field
+from dataclasses import dataclass, field, replace
 from typing import Callable, Dict, List, Optional, Tuple
 
 import numpy as np
@@ -56,10 +56,15 @@ class Workload:
     s0_std: float = 0.1
     draw: str = "gdn"               # which input law to use (see _draw_slot)
     readout: bool = True
+    tile_ids: Optional[Tuple[int, ...]] = None   # a shard: these tiles of the whole draw
+
+    @property
+    def all_tiles(self) -> int:
+        return self.layers * self.batch * self.heads
 
     @property
     def tiles(self) -> int:
-        return self.layers * self.batch * self.heads
+        return self.all_tiles if self.tile_ids is None else len(self.tile_ids)
 
     @property
     def tiles_per_layer(self) -> int:
@@ -191,6 +196,27 @@ def get(name_or_index) -> Workload:
     return WORKLOADS[name_or_index]
 
 
+def shard(w: Workload, rank: int, world: int) -> Workload:
+    """Rank `rank`'s part of the workload on `world` GPUs: the contiguous
+    tile range [rank T / world, (rank + 1) T / world) of the whole draw.
+    Tiles are independent recurrences, so the shards need no exchange; a
+    shard draws exactly the inputs and initial state that the whole
+    workload gives those tiles (per-layer seeds included)."""
+    if not 0 <= rank < world:
+        raise ValueError("rank out of range")
+    T = w.all_tiles
+    ids = tuple(range(rank * T // world, (rank + 1) * T // world))
+    return replace(w, name=f"{w.name}[{rank}/{world}]", tile_ids=ids)
+
+
+def _select(w: Workload, tiles: Optional[np.ndarray]) -> Optional[np.ndarray]:
+    """Indices into the whole draw: the shard's tiles, then `tiles` within them."""
+    if w.tile_ids is None:
+        return tiles
+    ids = np.asarray(w.tile_ids)
+    return ids if tiles is None else ids[np.asarray(tiles)]
+
+
 def _seeds(w: Workload) -> List[Tuple[int, int]]:
     """(seed, tiles) per layer block."""
     if w.layer_seeds is None:
@@ -207,7 +233,8 @@ def initial_state(w: Workload, tiles: Optional[np.ndarray] = None) -> np.ndarray
         rng = np.random.default_rng([seed, 1])
         blocks.append(rng.standard_normal((T, w.dv, w.dk)) * w.s0_std)
     S0 = np.ascontiguousarray(np.concatenate(blocks, axis=0), dtype=np.float32)
-    return S0 if tiles is None else np.ascontiguousarray(S0[tiles])
+    sel = _select(w, tiles)
+    return S0 if sel is None else np.ascontiguousarray(S0[sel])
 
 
 def slot(w: Workload, t: int, tiles: Optional[np.ndarray] = None):
@@ -219,8 +246,9 @@ def slot(w: Workload, t: int, tiles: Optional[np.ndarray] = None):
         for p, a in zip(parts, _draw_slot(w.draw, rng, T, w.dk, w.dv, w.decay)):
             p.append(a)
     out = tuple(np.ascontiguousarray(np.concatenate(p, axis=0)) for p in parts)
-    if tiles is not None:
-        out = tuple(np.ascontiguousarray(a[tiles]) for a in out)
+    sel = _select(w, tiles)
+    if sel is not None:
+        out = tuple(np.ascontiguousarray(a[sel]) for a in out)
     return out
 
 
@@ -233,7 +261,6 @@ def pool(w: Workload, n_slots: int, tiles: Optional[np.ndarray] = None):
 def scaled_down(w: Workload, tiles_per_layer: int, layers: Optional[int] = None,
                 steps: Optional[int] = None) -> Workload:
     """Same laws and arms with fewer tiles (for tests that must finish fast)."""
-    from dataclasses import replace
     L = w.layers if layers is None else layers
     seeds = None if w.layer_seeds is None else w.layer_seeds[:L]
     return replace(w, name=w.name + "-small", layers=L, batch=1, heads=tiles_per_layer,
@@ -244,7 +271,8 @@ def probe(w: Workload, tiles: Optional[np.ndarray] = None):
     """(k*, v*) of the recall measurement: per tile a unit-norm key and a
     N(0, 1) value, from default_rng([seed, 3]) (float32 [T][dk], [T][dv])."""
     rng = np.random.default_rng([w.seed, 3])
-    k = _unit_rows(rng.standard_normal((w.tiles, w.dk)))
-    v = rng.standard_normal((w.tiles, w.dv))
-    f = lambda a: np.ascontiguousarray(a if tiles is None else a[tiles], dtype=np.float32)
+    k = _unit_rows(rng.standard_normal((w.all_tiles, w.dk)))
+    v = rng.standard_normal((w.all_tiles, w.dv))
+    sel = _select(w, tiles)
+    f = lambda a: np.ascontiguousarray(a if sel is None else a[sel], dtype=np.float32)
     return f(k), f(v)
