@@ -17,8 +17,8 @@
 // as its codes are unpacked.  No shared memory, copy or barrier sits on the
 // state's path.  The per-tile vectors (k, q, diagonal alpha, alpha, beta)
 // go by cp.async into one of two per-warp shared-memory slots a tile ahead;
-// k lives in registers for the tile, q and diagonal alpha are read from the
-// slot.  New codes, scales and o leave straight from registers.
+// k lives in registers for the tile (or, for the BDR instances, is re-read
+// from the slot at each use), q and diagonal alpha are read from the slot.  New codes, scales and o leave straight from registers.
 //
 // Element arithmetic (the definition of include/qstate.h, fixed order):
 //   unpack     INT4: one LOP3 per element builds the float 2^23 + 16^p (c+8)
@@ -44,12 +44,23 @@ namespace qs {
 
 // Registers per thread of the streamed step: 128 leaves room for 16 resident
 // warps per SM; BDR instances hold the stored codes and the update-sign
-// masks as well and get 200 (10 warps per SM).
+// masks as well and get 160 (12 warps per SM), INT8 ones (twice the words)
+// 200.
 #ifndef QS_STREAM_REGS
 #define QS_STREAM_REGS 128
 #endif
 #ifndef QS_STREAM_REGS_BDR
-#define QS_STREAM_REGS_BDR 200
+#define QS_STREAM_REGS_BDR 160
+#endif
+#ifndef QS_STREAM_REGS_BDR8
+#define QS_STREAM_REGS_BDR8 200
+#endif
+// Where the tile's key vector lives: 1 reads it from its shared-memory slot
+// at each use, 0 holds it in registers for the tile, -1 (default) does the
+// former for the BDR instances (whose packed-word masks and stored codes
+// take registers of their own) and the latter for the others.
+#ifndef QS_STREAM_K_SMEM
+#define QS_STREAM_K_SMEM -1
 #endif
 
 struct StreamParams {
@@ -87,6 +98,21 @@ struct StreamLayout {
   }
   __host__ __device__ int bytes() const { return 2 * slot; }
 };
+
+// A staged Dk vector's chunk c as 16 pairs, re-read from shared memory at
+// every call (volatile: the compiler may not keep an earlier read instead).
+__device__ __forceinline__ void load_pairs_v(const unsigned char* base, int c, float2 (&v)[16]) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(base)) + c * (kChunkStride * 4);
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    float4 t;
+    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];\n"
+                 : "=f"(t.x), "=f"(t.y), "=f"(t.z), "=f"(t.w)
+                 : "r"(a + 16 * m));
+    v[2 * m] = make_float2(t.x, t.y);
+    v[2 * m + 1] = make_float2(t.z, t.w);
+  }
+}
 
 // Streamed loads: codes and scales through L2 only (each byte is read once
 // per launch), v through the read-only path (the lanes of a row share it).
@@ -260,7 +286,8 @@ __device__ __forceinline__ void key_sign_masks(const float2 (&kk)[16], uint32_t 
 
 // POLICY: 0 dynamic, 1 persistent.
 template <int BITS, int DK, int POLICY, bool BDR, bool DELTA, bool DIAG>
-__global__ void __maxnreg__(BDR ? QS_STREAM_REGS_BDR : QS_STREAM_REGS) stream_step_kernel(StreamParams p) {
+__global__ void __maxnreg__(BDR ? (BITS == 8 ? QS_STREAM_REGS_BDR8 : QS_STREAM_REGS_BDR) : QS_STREAM_REGS)
+    stream_step_kernel(StreamParams p) {
   static_assert(POLICY == 0 || POLICY == 1, "the yoked policy has its own kernel");
   constexpr int LPR = DK / 32;
   constexpr int RW = 32 / LPR;
@@ -276,6 +303,7 @@ __global__ void __maxnreg__(BDR ? QS_STREAM_REGS_BDR : QS_STREAM_REGS) stream_st
   constexpr bool BDR_FLOAT = BDR && POLICY == 0;
   // fixed scales the packed-word BDR and the fast reciprocal take directly
   constexpr float kScaleHi = POLICY == 1 ? 0x1p100f : 0x1p126f;
+  constexpr bool KS = QS_STREAM_K_SMEM < 0 ? BDR : QS_STREAM_K_SMEM != 0;
 
   extern __shared__ __align__(128) unsigned char smem[];
   const int lane = threadIdx.x & 31;
@@ -347,7 +375,11 @@ __global__ void __maxnreg__(BDR ? QS_STREAM_REGS_BDR : QS_STREAM_REGS) stream_st
   const unsigned char* tv = smem;
   auto enter_tile = [&]() {
     tv = smem + slot * L.slot;
-    load_pairs(tv + L.k, c, kk);
+    if constexpr (KS) {
+      if constexpr (BDR) load_pairs(tv + L.k, c, kk);   // for the sign masks only
+    } else {
+      load_pairs(tv + L.k, c, kk);
+    }
     const float* misc = reinterpret_cast<const float*>(tv + L.misc);
     beta = misc[1];
     a_scalar = DIAG ? 1.0f : misc[0];
@@ -404,13 +436,21 @@ __global__ void __maxnreg__(BDR ? QS_STREAM_REGS_BDR : QS_STREAM_REGS) stream_st
     // ---- a3/a4: key projection and rank-1 write
     float wcoef;
     if constexpr (DELTA) {
-      wcoef = __fmul_rn(beta, __fsub_rn(v_i, row_tree<LPR>(chunk_sum(Sp, kk))));
+      float2 ku[16];
+      if constexpr (KS) load_pairs_v(tv + L.k, c, ku);
+      const float2(&k1)[16] = KS ? ku : kk;
+      wcoef = __fmul_rn(beta, __fsub_rn(v_i, row_tree<LPR>(chunk_sum(Sp, k1))));
     } else {
       wcoef = __fmul_rn(beta, v_i);
     }
     float2 x[16];
+    {
+      float2 kx[16];
+      if constexpr (KS) load_pairs_v(tv + L.k, c, kx);
+      const float2(&k2)[16] = KS ? kx : kk;
 #pragma unroll
-    for (int m = 0; m < 16; ++m) x[m] = __ffma2_rn(f2(wcoef), kk[m], Sp[m]);
+      for (int m = 0; m < 16; ++m) x[m] = __ffma2_rn(f2(wcoef), k2[m], Sp[m]);
+    }
 
     // ---- a5: readout from the updated state
     if (readout) {
@@ -476,13 +516,14 @@ __global__ void __maxnreg__(BDR ? QS_STREAM_REGS_BDR : QS_STREAM_REGS) stream_st
             uint32_t wold[CW];
 #pragma unroll
             for (int q = 0; q < CW; ++q) wold[q] = cold[q] ^ TOPS;
-            float2 cv[16], dd[16], sk[16];
+            float2 cv[16], dd[16], sk[16], kr[16];
+            load_pairs_v(tv + L.k, c, kr);
             unpack_codes<BITS>(wold, cv, e23);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               dd[i] = __fmul2_rn(cv[i], f2(s_old));
-              sk[i] = make_float2(kk[i].x > 0.0f ? 1.0f : (kk[i].x < 0.0f ? -1.0f : 0.0f),
-                                  kk[i].y > 0.0f ? 1.0f : (kk[i].y < 0.0f ? -1.0f : 0.0f));
+              sk[i] = make_float2(kr[i].x > 0.0f ? 1.0f : (kr[i].x < 0.0f ? -1.0f : 0.0f),
+                                  kr[i].y > 0.0f ? 1.0f : (kr[i].y < 0.0f ? -1.0f : 0.0f));
             }
             bdr_chunk<BITS>(y, dd, sk, swf, sp);
           }
