@@ -18,7 +18,8 @@
 // state's path.  The per-tile vectors (k, q, diagonal alpha, alpha, beta)
 // go by cp.async into one of two per-warp shared-memory slots a tile ahead;
 // k lives in registers for the tile (or, for the BDR instances, is re-read
-// from the slot at each use), q and diagonal alpha are read from the slot.  New codes, scales and o leave straight from registers.
+// from the slot at each use), q and diagonal alpha are read from the slot.
+// New codes, scales and o leave straight from registers.
 //
 // Element arithmetic (the definition of include/qstate.h, fixed order):
 //   unpack     INT4: one LOP3 per element builds the float 2^23 + 16^p (c+8)
