@@ -362,17 +362,21 @@ QS_API qs_status qstate_prefill(const qs_config* cfg, int length, float* S, cons
  * (tcgen05.mma, kind::tf32, FP32 accumulators in tensor memory; chunks of
  * 64 tokens; the state stays in tensor memory for the whole sequence).
  * The operands of every contraction are rounded to TF32 (10 explicit
- * mantissa bits, round to nearest) and the state is read at TF32
- * precision by the state read, so results agree with the FP32 recurrence
+ * mantissa bits, round to nearest with ties away from zero, as cvt.rna
+ * does) and the state is read at TF32 precision (low mantissa bits
+ * dropped) by the state read, so results agree with the FP32 recurrence
  * to about 2^-10 of the magnitudes summed, not to FP32 rounding: every
  * element of S and o is within 2^-8 of the same recurrence run on |S0|,
  * |q|, |k|, |v| (the sum of the magnitudes of its terms).  Arguments,
  * validation are those of qstate_prefill, with S, q and k 16-byte aligned
  * and the linear write only (delta = 1 returns QS_ERR_UNSUPPORTED);
  * under either decay a chunk of 64 tokens may decay a channel by at most
- * e^-170 (the decay factors are split around the chunk's middle token).  A wait for the tensor
- * cores that does not end (a bounded poll) makes the CTA free its tensor
- * memory and return; qstate_prefill_tf32_timeouts reports the count. */
+ * e^-170 (the decay factors are split around the chunk's middle token).
+ * A wait for the tensor cores that does not end (a bounded poll) makes the
+ * CTA free its tensor memory and return; qstate_prefill_tf32_timeouts
+ * reports the count.  After a launch that counted a timeout, S and o of
+ * that launch are undefined: compare the count before and after the call
+ * (after synchronizing) and discard the results when it rose. */
 QS_API qs_status qstate_prefill_tf32(const qs_config* cfg, int length, float* S, const float* q,
                                      const float* k, const float* v, const float* alpha,
                                      const float* beta, float* o, cudaStream_t stream);

@@ -577,6 +577,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   if (tid == 0 && *failed) atomicAdd(timeouts, 1u);
   fence_after();
+  // On the timeout path a committed tcgen05.mma may still be writing these
+  // tensor-memory columns when they are freed here (that is what the wait
+  // gave up on), so the launch's S and o are undefined once a timeout is
+  // counted; the caller checks the count.
   if (warp == 0)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(kTcCols) : "memory");
 }

@@ -242,13 +242,25 @@ def prefill(cfg: Config, length: int, S, q, k, v, alpha, beta, o=None, stream=No
            "qstate_prefill")
 
 
-def prefill_tf32(cfg: Config, length: int, S, q, k, v, alpha, beta, o=None, stream=None) -> None:
+def prefill_tf32(cfg: Config, length: int, S, q, k, v, alpha, beta, o=None, stream=None,
+                 check_timeouts: bool = True) -> None:
     """The same prefill on the tensor cores (TF32 operands, FP32 accumulators);
-    S, q and k 16-byte aligned."""
+    S, q and k 16-byte aligned.  With check_timeouts (the default) the call
+    synchronizes and raises if a CTA's bounded wait for the tensor cores gave
+    up during it (S and o are then undefined); without it the call stays
+    asynchronous and the caller compares prefill_tf32_timeouts() itself."""
     cc = cfg.c()
+    before = prefill_tf32_timeouts() if check_timeouts else 0
     _check(lib().qstate_prefill_tf32(ctypes.byref(cc), length, _ptr(S), _ptr(q), _ptr(k), _ptr(v),
                                      _ptr(alpha), _ptr(beta), _ptr(o), _stream(stream)),
            "qstate_prefill_tf32")
+    if check_timeouts:
+        import torch
+        torch.cuda.synchronize()
+        gave_up = prefill_tf32_timeouts() - before
+        if gave_up:
+            raise RuntimeError(f"qstate_prefill_tf32: {gave_up} CTA(s) gave up waiting for the "
+                               "tensor cores; S and o of this call are undefined")
 
 
 def prefill_tf32_timeouts() -> int:
