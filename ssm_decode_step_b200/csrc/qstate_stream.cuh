@@ -34,9 +34,12 @@
 //   round      fused(x * (1/s') + 1.5 * 2^23 + 2^(bits-1)): the exact product
 //              rounded to an integer, held in the low mantissa bits as the
 //              offset-binary code; persistent scales clamp every element
+//              (the lower side by a min/max, the upper by the saturating
+//              pack)
 //   BDR        persistent: on the packed words (below); dynamic: the
 //              dequantized comparison of qstate_kernels.cuh
-//   pack       offset-binary fields to two's complement words
+//   pack       dynamic: offset-binary fields to two's complement words;
+//              persistent: saturating integer packs
 #pragma once
 
 #include "qstate_kernels.cuh"
@@ -230,6 +233,48 @@ __device__ __forceinline__ void pack_offset(const float2 (&y)[16], uint32_t (&w)
       const uint32_t t1 =
           __byte_perm(__float_as_uint(y[2 * q + 1].x), __float_as_uint(y[2 * q + 1].y), 0x0040u);
       w[q] = __byte_perm(t0, t1, 0x5410u);
+    }
+  }
+}
+
+// Pack 32 rounded values (floats kMagic + 2^(BITS-1) + n, as pairs
+// (2m, 2m+1)) whose lower side is already clamped to -qmax into BITS words
+// of two's complement codes, clamping the upper side on the way:
+// cvt.pack.sat converts two 32-bit integers with saturation to the field's
+// range (at most 2^(BITS-1) - 1 = qmax on the upper side) and shifts them
+// in below the word built so far (d = c << 2 BITS | sat(a) << BITS |
+// sat(b)).  The integer n is the float's bits less those of kMagic +
+// 2^(BITS-1): exact while the float lies in [2^23, 2^24), and every larger
+// float (huge or infinite products) gives a larger integer, which
+// saturates to qmax as the definition's clamp does.
+template <int BITS>
+__device__ __forceinline__ void pack_sat(const float2 (&y)[16], uint32_t (&w)[BITS]) {
+  constexpr float kOff = kMagic + (BITS == 4 ? 8.0f : 128.0f);
+  const int off = static_cast<int>(__float_as_uint(kOff));
+  auto n = [&](float v) { return static_cast<int>(__float_as_uint(v)) - off; };
+  if constexpr (BITS == 4) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      // columns 8q .. 8q+7 = pairs 4q .. 4q+3; the last pair goes in first
+      uint32_t d = 0;
+#pragma unroll
+      for (int m = 3; m >= 0; --m)
+        asm("cvt.pack.sat.s4.s32.b32 %0, %1, %2, %3;"
+            : "=r"(d)
+            : "r"(n(y[4 * q + m].y)), "r"(n(y[4 * q + m].x)), "r"(d));
+      w[q] = d;
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      // columns 4q .. 4q+3 = pairs 2q, 2q+1
+      uint32_t d = 0;
+#pragma unroll
+      for (int m = 1; m >= 0; --m)
+        asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;"
+            : "=r"(d)
+            : "r"(n(y[2 * q + m].y)), "r"(n(y[2 * q + m].x)), "r"(d));
+      w[q] = d;
     }
   }
 }
@@ -484,10 +529,11 @@ __global__ void __maxnreg__(BDR ? (BITS == 8 ? QS_STREAM_REGS_BDR8 : QS_STREAM_R
 #pragma unroll
     for (int i = 0; i < 16; ++i) y[i] = __ffma2_rn(x[i], f2(inv), f2(kOff));
     if constexpr (POLICY == 1) {
+      // the lower side of the clamp; pack_sat clamps the upper side
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        y[i].x = fminf(fmaxf(y[i].x, kOff - kQf), kOff + kQf);
-        y[i].y = fminf(fmaxf(y[i].y, kOff - kQf), kOff + kQf);
+        y[i].x = fmaxf(y[i].x, kOff - kQf);
+        y[i].y = fmaxf(y[i].y, kOff - kQf);
       }
     }
     // The fast forms above are exact for a finite group max and a scale in
@@ -540,19 +586,26 @@ __global__ void __maxnreg__(BDR ? (BITS == 8 ? QS_STREAM_REGS_BDR8 : QS_STREAM_R
 
     // ---- a9: pack (and BDR on the packed words), store
     uint32_t out[CW];
-    pack_offset<BITS>(y, out);
-    if constexpr (BDR_WORDS) {
-      const bool pos = wcoef > 0.0f;
-      const uint32_t on = (wcoef != 0.0f) ? words_on : 0u;
+    if constexpr (POLICY == 1) {
+      // two's complement words straight from the saturating pack; the
+      // packed-word BDR steps fields in offset binary (no carry can cross
+      // a field there), so it flips the fields' top bits around its step
+      pack_sat<BITS>(y, out);
+      if constexpr (BDR_WORDS) {
+        const bool pos = wcoef > 0.0f;
+        const uint32_t on = (wcoef != 0.0f) ? words_on : 0u;
 #pragma unroll
-      for (int q = 0; q < CW; ++q) {
-        const uint32_t P = pos ? kp[q] : kn[q];
-        const uint32_t M = pos ? kn[q] : kp[q];
-        out[q] = bdr_fixed_scale<BITS>(out[q], cold[q], P, M, on);
+        for (int q = 0; q < CW; ++q) {
+          const uint32_t P = pos ? kp[q] : kn[q];
+          const uint32_t M = pos ? kn[q] : kp[q];
+          out[q] = bdr_fixed_scale<BITS>(out[q] ^ TOPS, cold[q], P, M, on) ^ TOPS;
+        }
       }
-    }
+    } else {
+      pack_offset<BITS>(y, out);
 #pragma unroll
-    for (int q = 0; q < CW; ++q) out[q] ^= TOPS;
+      for (int q = 0; q < CW; ++q) out[q] ^= TOPS;
+    }
     if constexpr (CW == 4) {
       st_global_v4(codes_at(b), out);
     } else {
