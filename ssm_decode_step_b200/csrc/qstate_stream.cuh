@@ -287,33 +287,39 @@ __host__ __device__ constexpr uint32_t field_tops() { return BITS == 4 ? 0x88888
 // Bounded Directional Rounding under a fixed scale, on packed words.  With
 // s' = s (persistent) and s a normal float, n s' < c s exactly when n < c,
 // so the rule of include/qstate.h becomes an integer comparison of the new
-// and the stored code, field by field.  N, C: offset-binary fields (new and
-// stored codes) in [1, 2^BITS - 1]; P, M: the top bit of every field whose
-// update sign sigma is > 0, < 0.  x >= y per field: the borrow-free
-// difference (x | top) - (y & ~top) compares the low bits, and its top bit
-// combined with the fields' own top bits gives the full comparison.  A
-// field steps up (sigma > 0, n < c) or down (sigma < 0, n > c); the result
-// lies between n and c, so it stays in range and no carry crosses fields.
-// `on` (all ones or zero) switches the rule on or off for the whole word.
+// and the stored code, field by field.  N, C: two's complement fields (new
+// and stored codes, each in [-qmax, qmax]); PF: every bit of the fields
+// whose update sign sigma is > 0; AM: the top bit of the fields whose
+// sigma is not 0; `on` (all ones or zero) switches the rule on or off for
+// the whole word.  One comparison serves both directions: a field compares
+// A = n, B = c where sigma > 0 and A = c, B = n where sigma < 0, and acts
+// where A < B.  Signed x >= y per field: the borrow-free difference
+// (x | top) - (y & ~top) compares the low bits, and its top bit combined
+// with the fields' own sign bits gives the full comparison.  The step of
+// +-1 runs in offset binary (top bits flipped), where no carry can cross a
+// field: the result lies between n and c.
 template <int BITS>
-__device__ __forceinline__ uint32_t bdr_fixed_scale(uint32_t N, uint32_t C, uint32_t P, uint32_t M,
+__device__ __forceinline__ uint32_t bdr_fixed_scale(uint32_t N, uint32_t C, uint32_t PF, uint32_t AM,
                                                     uint32_t on) {
   constexpr uint32_t H = field_tops<BITS>();
-  const uint32_t zNC = (N | H) - (C & ~H);
-  const uint32_t zCN = (C | H) - (N & ~H);
-  const uint32_t geNC = (N & ~C) | (~(N ^ C) & zNC);
-  const uint32_t geCN = (C & ~N) | (~(N ^ C) & zCN);
-  const uint32_t up = ~geNC & P & on;
-  const uint32_t down = ~geCN & M & on;
-  return N + (up >> (BITS - 1)) - (down >> (BITS - 1));
+  const uint32_t A = (N & PF) | (C & ~PF);
+  const uint32_t B = (C & PF) | (N & ~PF);
+  const uint32_t z = (A | H) - (B & ~H);
+  const uint32_t ge = (~A & B) | (~(A ^ B) & z);  // top bits: A >= B
+  const uint32_t act = ~ge & AM & on;
+  const uint32_t up = act & PF;
+  const uint32_t down = act ^ up;
+  return (((N ^ H) + (up >> (BITS - 1))) - (down >> (BITS - 1))) ^ H;
 }
 
-// Update-sign masks of a tile for the packed-word BDR: the top bit of every
-// field whose key entry is > 0 (kp) or < 0 (kn), for this lane's 32 columns.
+// Update-sign masks of a tile for the packed-word BDR, for this lane's 32
+// columns: kpf / knf hold every bit of the fields whose key entry is > 0 /
+// < 0, am the top bit of the fields whose key entry is not 0.
 template <int BITS>
-__device__ __forceinline__ void key_sign_masks(const float2 (&kk)[16], uint32_t (&kp)[BITS],
-                                               uint32_t (&kn)[BITS]) {
+__device__ __forceinline__ void key_sign_masks(const float2 (&kk)[16], uint32_t (&kpf)[BITS],
+                                               uint32_t (&knf)[BITS], uint32_t (&am)[BITS]) {
   constexpr int PER = 32 / BITS;  // fields per word
+  constexpr uint32_t FIELD = (1u << BITS) - 1u;
 #pragma unroll
   for (int q = 0; q < BITS; ++q) {
     uint32_t p = 0, n = 0;
@@ -321,12 +327,13 @@ __device__ __forceinline__ void key_sign_masks(const float2 (&kk)[16], uint32_t 
     for (int i = 0; i < PER; ++i) {
       const int j = q * PER + i;
       const float kv = (j & 1) ? kk[j >> 1].y : kk[j >> 1].x;
-      const uint32_t top = 1u << (BITS * i + BITS - 1);
-      p |= kv > 0.0f ? top : 0u;
-      n |= kv < 0.0f ? top : 0u;
+      const uint32_t f = FIELD << (BITS * i);
+      p |= kv > 0.0f ? f : 0u;
+      n |= kv < 0.0f ? f : 0u;
     }
-    kp[q] = p;
-    kn[q] = n;
+    kpf[q] = p;
+    knf[q] = n;
+    am[q] = (p | n) & field_tops<BITS>();
   }
 }
 
@@ -417,7 +424,7 @@ __global__ void __maxnreg__(BDR ? (BITS == 8 ? QS_STREAM_REGS_BDR8 : QS_STREAM_R
 
   float2 kk[16];
   float beta = 0.0f, a_scalar = 1.0f;
-  uint32_t kp[BDR_WORDS ? CW : 1], kn[BDR_WORDS ? CW : 1];
+  uint32_t kp[BDR_WORDS ? CW : 1], kn[BDR_WORDS ? CW : 1], am[BDR_WORDS ? CW : 1];
   const unsigned char* tv = smem;
   auto enter_tile = [&]() {
     tv = smem + slot * L.slot;
@@ -429,7 +436,7 @@ __global__ void __maxnreg__(BDR ? (BITS == 8 ? QS_STREAM_REGS_BDR8 : QS_STREAM_R
     const float* misc = reinterpret_cast<const float*>(tv + L.misc);
     beta = misc[1];
     a_scalar = DIAG ? 1.0f : misc[0];
-    if constexpr (BDR_WORDS) key_sign_masks<BITS>(kk, kp, kn);
+    if constexpr (BDR_WORDS) key_sign_masks<BITS>(kk, kp, kn, am);
     if constexpr (BDR_FLOAT) {
       // sign(k_j) per column, in the layout of k, written once per tile
       if (rr == 0) {
@@ -456,7 +463,7 @@ __global__ void __maxnreg__(BDR ? (BITS == 8 ? QS_STREAM_REGS_BDR8 : QS_STREAM_R
     uint32_t cold[BDR_WORDS ? CW : 1];
     if constexpr (BDR_WORDS) {
 #pragma unroll
-      for (int q = 0; q < CW; ++q) cold[q] = in.w[q] ^ TOPS;
+      for (int q = 0; q < CW; ++q) cold[q] = in.w[q];
     }
     const float s_old = in.s, v_i = in.v;
     // BDR's reference under a changing scale: d = c * s
@@ -562,7 +569,7 @@ __global__ void __maxnreg__(BDR ? (BITS == 8 ? QS_STREAM_REGS_BDR8 : QS_STREAM_R
           if (!zero && !(sp < kScaleHi)) {
             uint32_t wold[CW];
 #pragma unroll
-            for (int q = 0; q < CW; ++q) wold[q] = cold[q] ^ TOPS;
+            for (int q = 0; q < CW; ++q) wold[q] = cold[q];
             float2 cv[16], dd[16], sk[16], kr[16];
             load_pairs_v(tv + L.k, c, kr);
             unpack_codes<BITS>(wold, cv, e23);
@@ -587,18 +594,15 @@ __global__ void __maxnreg__(BDR ? (BITS == 8 ? QS_STREAM_REGS_BDR8 : QS_STREAM_R
     // ---- a9: pack (and BDR on the packed words), store
     uint32_t out[CW];
     if constexpr (POLICY == 1) {
-      // two's complement words straight from the saturating pack; the
-      // packed-word BDR steps fields in offset binary (no carry can cross
-      // a field there), so it flips the fields' top bits around its step
+      // two's complement words straight from the saturating pack, compared
+      // with the stored words as they are
       pack_sat<BITS>(y, out);
       if constexpr (BDR_WORDS) {
         const bool pos = wcoef > 0.0f;
         const uint32_t on = (wcoef != 0.0f) ? words_on : 0u;
 #pragma unroll
         for (int q = 0; q < CW; ++q) {
-          const uint32_t P = pos ? kp[q] : kn[q];
-          const uint32_t M = pos ? kn[q] : kp[q];
-          out[q] = bdr_fixed_scale<BITS>(out[q] ^ TOPS, cold[q], P, M, on) ^ TOPS;
+          out[q] = bdr_fixed_scale<BITS>(out[q], cold[q], pos ? kp[q] : kn[q], am[q], on);
         }
       }
     } else {
