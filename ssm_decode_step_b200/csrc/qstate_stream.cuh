@@ -238,15 +238,18 @@ __device__ __forceinline__ void pack_offset(const float2 (&y)[16], uint32_t (&w)
 }
 
 // Pack 32 rounded values (floats kMagic + 2^(BITS-1) + n, as pairs
-// (2m, 2m+1)) whose lower side is already clamped to -qmax into BITS words
-// of two's complement codes, clamping the upper side on the way:
+// (2m, 2m+1)) into BITS words of two's complement codes, saturating them to
+// the field's range [-2^(BITS-1), 2^(BITS-1) - 1] on the way (the upper
+// bound is qmax; the lower one, one below -qmax, the caller handles):
 // cvt.pack.sat converts two 32-bit integers with saturation to the field's
 // range (at most 2^(BITS-1) - 1 = qmax on the upper side) and shifts them
 // in below the word built so far (d = c << 2 BITS | sat(a) << BITS |
 // sat(b)).  The integer n is the float's bits less those of kMagic +
-// 2^(BITS-1): exact while the float lies in [2^23, 2^24), and every larger
-// float (huge or infinite products) gives a larger integer, which
-// saturates to qmax as the definition's clamp does.
+// 2^(BITS-1): exact while the float lies in [2^23, 2^24); every larger
+// float (huge or +infinite products) gives a larger integer, which
+// saturates to qmax, and every smaller one (huge negative, -infinite) a
+// smaller integer, which saturates to the field's minimum, as the
+// definition's clamp does once that minimum is raised to -qmax.
 template <int BITS>
 __device__ __forceinline__ void pack_sat(const float2 (&y)[16], uint32_t (&w)[BITS]) {
   constexpr float kOff = kMagic + (BITS == 4 ? 8.0f : 128.0f);
@@ -277,6 +280,17 @@ __device__ __forceinline__ void pack_sat(const float2 (&y)[16], uint32_t (&w)[BI
       w[q] = d;
     }
   }
+}
+
+// INT4 words from pack_sat hold fields in [-8, 7]; the codes' range is
+// [-7, 7], so every field equal to -8 (binary 1000) steps up by one.  A
+// field is 1000 when its top bit is set and its three low bits are zero:
+// adding 7 to the low bits carries into the field's top bit exactly when
+// they are not all zero (no carry leaves the field).
+__device__ __forceinline__ uint32_t int4_raise_min(uint32_t w) {
+  const uint32_t low_nonzero = (w & 0x77777777u) + 0x77777777u;
+  const uint32_t is_min = w & ~low_nonzero & 0x88888888u;
+  return w + (is_min >> 3);
 }
 
 // The top bit of every field of a packed word (4-bit fields for INT4, 8-bit
@@ -535,8 +549,9 @@ __global__ void __maxnreg__(BDR ? (BITS == 8 ? QS_STREAM_REGS_BDR8 : QS_STREAM_R
     float2 y[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) y[i] = __ffma2_rn(x[i], f2(inv), f2(kOff));
-    if constexpr (POLICY == 1) {
-      // the lower side of the clamp; pack_sat clamps the upper side
+    if constexpr (POLICY == 1 && BITS == 8) {
+      // the lower side of the clamp; pack_sat clamps the upper side (INT4
+      // raises -8 to -7 on the packed words instead)
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         y[i].x = fmaxf(y[i].x, kOff - kQf);
@@ -597,6 +612,10 @@ __global__ void __maxnreg__(BDR ? (BITS == 8 ? QS_STREAM_REGS_BDR8 : QS_STREAM_R
       // two's complement words straight from the saturating pack, compared
       // with the stored words as they are
       pack_sat<BITS>(y, out);
+      if constexpr (BITS == 4) {
+#pragma unroll
+        for (int q = 0; q < CW; ++q) out[q] = int4_raise_min(out[q]);
+      }
       if constexpr (BDR_WORDS) {
         const bool pos = wcoef > 0.0f;
         const uint32_t on = (wcoef != 0.0f) ? words_on : 0u;
