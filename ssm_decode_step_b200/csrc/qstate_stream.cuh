@@ -48,13 +48,13 @@ namespace qs {
 
 // Registers per thread of the streamed step: 128 leaves room for 16 resident
 // warps per SM; BDR instances hold the stored codes and the update-sign
-// masks as well and get 160 (12 warps per SM), INT8 ones (twice the words)
-// 200.
+// masks as well and get 168, the most that still leaves 12 warps per SM
+// (65536 / (168 x 32) = 12.2), INT8 ones (twice the words) 200.
 #ifndef QS_STREAM_REGS
 #define QS_STREAM_REGS 128
 #endif
 #ifndef QS_STREAM_REGS_BDR
-#define QS_STREAM_REGS_BDR 160
+#define QS_STREAM_REGS_BDR 168
 #endif
 #ifndef QS_STREAM_REGS_BDR8
 #define QS_STREAM_REGS_BDR8 200
@@ -237,60 +237,66 @@ __device__ __forceinline__ void pack_offset(const float2 (&y)[16], uint32_t (&w)
   }
 }
 
-// Pack 32 rounded values (floats kMagic + 2^(BITS-1) + n, as pairs
-// (2m, 2m+1)) into BITS words of two's complement codes, saturating them to
-// the field's range [-2^(BITS-1), 2^(BITS-1) - 1] on the way (the upper
-// bound is qmax; the lower one, one below -qmax, the caller handles):
-// cvt.pack.sat converts two 32-bit integers with saturation to the field's
-// range (at most 2^(BITS-1) - 1 = qmax on the upper side) and shifts them
-// in below the word built so far (d = c << 2 BITS | sat(a) << BITS |
-// sat(b)).  The integer n is the float's bits less those of kMagic +
-// 2^(BITS-1): exact while the float lies in [2^23, 2^24); every larger
-// float (huge or +infinite products) gives a larger integer, which
-// saturates to qmax, and every smaller one (huge negative, -infinite) a
-// smaller integer, which saturates to the field's minimum, as the
-// definition's clamp does once that minimum is raised to -qmax.
-template <int BITS>
-__device__ __forceinline__ void pack_sat(const float2 (&y)[16], uint32_t (&w)[BITS]) {
-  constexpr float kOff = kMagic + (BITS == 4 ? 8.0f : 128.0f);
+// Pack 32 rounded INT8 values (floats kMagic + 128 + n, as pairs
+// (2m, 2m+1)) into 8 words of two's complement codes, saturating them to
+// [-128, 127] on the way (the upper bound is qmax; the caller clamps the
+// lower side to -qmax beforehand): cvt.pack.sat converts two 32-bit
+// integers with saturation to the field's range and shifts them in below
+// the word built so far (d = c << 16 | sat(a) << 8 | sat(b)).  The integer
+// n is the float's bits less those of kMagic + 128: exact while the float
+// lies in [2^23, 2^24); every larger float (huge or +infinite products)
+// gives a larger integer, which saturates to qmax as the definition's clamp
+// does.
+__device__ __forceinline__ void pack_sat8(const float2 (&y)[16], uint32_t (&w)[8]) {
+  constexpr float kOff = kMagic + 128.0f;
   const int off = static_cast<int>(__float_as_uint(kOff));
   auto n = [&](float v) { return static_cast<int>(__float_as_uint(v)) - off; };
-  if constexpr (BITS == 4) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      // columns 8q .. 8q+7 = pairs 4q .. 4q+3; the last pair goes in first
-      uint32_t d = 0;
+  for (int q = 0; q < 8; ++q) {
+    // columns 4q .. 4q+3 = pairs 2q, 2q+1; the last pair goes in first
+    uint32_t d = 0;
 #pragma unroll
-      for (int m = 3; m >= 0; --m)
-        asm("cvt.pack.sat.s4.s32.b32 %0, %1, %2, %3;"
-            : "=r"(d)
-            : "r"(n(y[4 * q + m].y)), "r"(n(y[4 * q + m].x)), "r"(d));
-      w[q] = d;
-    }
-  } else {
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      // columns 4q .. 4q+3 = pairs 2q, 2q+1
-      uint32_t d = 0;
-#pragma unroll
-      for (int m = 1; m >= 0; --m)
-        asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;"
-            : "=r"(d)
-            : "r"(n(y[2 * q + m].y)), "r"(n(y[2 * q + m].x)), "r"(d));
-      w[q] = d;
-    }
+    for (int m = 1; m >= 0; --m)
+      asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;"
+          : "=r"(d)
+          : "r"(n(y[2 * q + m].y)), "r"(n(y[2 * q + m].x)), "r"(d));
+    w[q] = d;
   }
 }
 
-// INT4 words from pack_sat hold fields in [-8, 7]; the codes' range is
-// [-7, 7], so every field equal to -8 (binary 1000) steps up by one.  A
-// field is 1000 when its top bit is set and its three low bits are zero:
-// adding 7 to the low bits carries into the field's top bit exactly when
-// they are not all zero (no carry leaves the field).
-__device__ __forceinline__ uint32_t int4_raise_min(uint32_t w) {
-  const uint32_t low_nonzero = (w & 0x77777777u) + 0x77777777u;
-  const uint32_t is_min = w & ~low_nonzero & 0x88888888u;
-  return w + (is_min >> 3);
+// Offset-binary INT4 words whose fields lie in [0, 15]; the codes' range
+// is [1, 15] (code -7 .. 7), so every field equal to 0 steps up by one.  A
+// field is nonzero when its top bit is set or adding 7 to its three low
+// bits carries into the top bit.
+__device__ __forceinline__ uint32_t int4_raise_zero(uint32_t w) {
+  const uint32_t nonzero = ((w & 0x77777777u) + 0x77777777u) | w;
+  return w + ((~nonzero & 0x88888888u) >> 3);
+}
+
+// Pack 32 rounded INT4 values (floats y = kMagic + 8 + n, as pairs
+// (2m, 2m+1)) into 4 offset-binary words, fields m = n + 8 saturated to
+// [0, 15].  One packed fused multiply-add takes y to (y - kMagic) 2^-149:
+// y 2^-149 lies in [2^-126, 2^-125), where the float grid is 2^-149, so
+// product and difference are exact and the result is m 2^-149, whose bits
+// read as an integer are m itself (a subnormal for 0 <= m < 2^23).
+// Smaller y (huge negative or -infinite products) give negative floats,
+// whose bits read as a negative integer; larger y (huge or +infinite) give
+// positive floats whose bits exceed 15.  cvt.pack.sat then saturates each
+// to [0, 15] as the definition's clamp does (the caller raises 0 to 1) and
+// shifts it in below the word built so far.
+__device__ __forceinline__ void pack4_subnormal(const float2 (&y)[16], uint32_t (&w)[4]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t d = 0;
+#pragma unroll
+    for (int m = 3; m >= 0; --m) {
+      const float2 z = __ffma2_rn(y[4 * q + m], f2(0x1p-149f), f2(-0x1.8p-126f));
+      asm("cvt.pack.sat.u4.s32.b32 %0, %1, %2, %3;"
+          : "=r"(d)
+          : "r"(__float_as_uint(z.y)), "r"(__float_as_uint(z.x)), "r"(d));
+    }
+    w[q] = d;
+  }
 }
 
 // The top bit of every field of a packed word (4-bit fields for INT4, 8-bit
@@ -301,34 +307,31 @@ __host__ __device__ constexpr uint32_t field_tops() { return BITS == 4 ? 0x88888
 // Bounded Directional Rounding under a fixed scale, on packed words.  With
 // s' = s (persistent) and s a normal float, n s' < c s exactly when n < c,
 // so the rule of include/qstate.h becomes an integer comparison of the new
-// and the stored code, field by field.  N, C: two's complement fields (new
-// and stored codes, each in [-qmax, qmax]); PF: every bit of the fields
-// whose update sign sigma is > 0; AM: the top bit of the fields whose
-// sigma is not 0; `on` (all ones or zero) switches the rule on or off for
-// the whole word.  One comparison serves both directions: a field compares
-// A = n, B = c where sigma > 0 and A = c, B = n where sigma < 0, and acts
-// where A < B.  Signed x >= y per field: the borrow-free difference
+// and the stored code, field by field.  N, C: offset-binary fields (code +
+// 2^(BITS-1), new and stored, each in [1, 2^BITS - 1]); PF: every bit of
+// the fields whose update sign sigma is > 0; AM: the lowest bit of the
+// fields whose sigma is not 0, and of none where the rule is off for the
+// word.  One comparison serves both directions: a field compares A = n,
+// B = c where sigma > 0 and A = c, B = n where sigma < 0, and acts where
+// A < B.  Unsigned x >= y per field: the borrow-free difference
 // (x | top) - (y & ~top) compares the low bits, and its top bit combined
-// with the fields' own sign bits gives the full comparison.  The step of
-// +-1 runs in offset binary (top bits flipped), where no carry can cross a
-// field: the result lies between n and c.
+// with the fields' own top bits gives the full comparison.  The step of +-1
+// moves a field toward c, so no carry or borrow crosses a field.
 template <int BITS>
-__device__ __forceinline__ uint32_t bdr_fixed_scale(uint32_t N, uint32_t C, uint32_t PF, uint32_t AM,
-                                                    uint32_t on) {
+__device__ __forceinline__ uint32_t bdr_fixed_scale(uint32_t N, uint32_t C, uint32_t PF, uint32_t AM) {
   constexpr uint32_t H = field_tops<BITS>();
   const uint32_t A = (N & PF) | (C & ~PF);
   const uint32_t B = (C & PF) | (N & ~PF);
   const uint32_t z = (A | H) - (B & ~H);
-  const uint32_t ge = (~A & B) | (~(A ^ B) & z);  // top bits: A >= B
-  const uint32_t act = ~ge & AM & on;
+  const uint32_t ge = (A & ~B) | (~(A ^ B) & z);  // top bits: A >= B
+  const uint32_t act = ~(ge >> (BITS - 1)) & AM;  // lowest bits: A < B
   const uint32_t up = act & PF;
-  const uint32_t down = act ^ up;
-  return (((N ^ H) + (up >> (BITS - 1))) - (down >> (BITS - 1))) ^ H;
+  return N + up - (act ^ up);
 }
 
 // Update-sign masks of a tile for the packed-word BDR, for this lane's 32
 // columns: kpf / knf hold every bit of the fields whose key entry is > 0 /
-// < 0, am the top bit of the fields whose key entry is not 0.
+// < 0, am the lowest bit of the fields whose key entry is not 0.
 template <int BITS>
 __device__ __forceinline__ void key_sign_masks(const float2 (&kk)[16], uint32_t (&kpf)[BITS],
                                                uint32_t (&knf)[BITS], uint32_t (&am)[BITS]) {
@@ -347,7 +350,7 @@ __device__ __forceinline__ void key_sign_masks(const float2 (&kk)[16], uint32_t 
     }
     kpf[q] = p;
     knf[q] = n;
-    am[q] = (p | n) & field_tops<BITS>();
+    am[q] = (p | n) & (field_tops<BITS>() >> (BITS - 1));
   }
 }
 
@@ -477,7 +480,7 @@ __global__ void __maxnreg__(BDR ? (BITS == 8 ? QS_STREAM_REGS_BDR8 : QS_STREAM_R
     uint32_t cold[BDR_WORDS ? CW : 1];
     if constexpr (BDR_WORDS) {
 #pragma unroll
-      for (int q = 0; q < CW; ++q) cold[q] = in.w[q];
+      for (int q = 0; q < CW; ++q) cold[q] = in.w[q] ^ TOPS;  // offset binary
     }
     const float s_old = in.s, v_i = in.v;
     // BDR's reference under a changing scale: d = c * s
@@ -550,7 +553,7 @@ __global__ void __maxnreg__(BDR ? (BITS == 8 ? QS_STREAM_REGS_BDR8 : QS_STREAM_R
 #pragma unroll
     for (int i = 0; i < 16; ++i) y[i] = __ffma2_rn(x[i], f2(inv), f2(kOff));
     if constexpr (POLICY == 1 && BITS == 8) {
-      // the lower side of the clamp; pack_sat clamps the upper side (INT4
+      // the lower side of the clamp; pack_sat8 clamps the upper side (INT4
       // raises -8 to -7 on the packed words instead)
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -584,7 +587,7 @@ __global__ void __maxnreg__(BDR ? (BITS == 8 ? QS_STREAM_REGS_BDR8 : QS_STREAM_R
           if (!zero && !(sp < kScaleHi)) {
             uint32_t wold[CW];
 #pragma unroll
-            for (int q = 0; q < CW; ++q) wold[q] = cold[q];
+            for (int q = 0; q < CW; ++q) wold[q] = cold[q] ^ TOPS;
             float2 cv[16], dd[16], sk[16], kr[16];
             load_pairs_v(tv + L.k, c, kr);
             unpack_codes<BITS>(wold, cv, e23);
@@ -609,21 +612,27 @@ __global__ void __maxnreg__(BDR ? (BITS == 8 ? QS_STREAM_REGS_BDR8 : QS_STREAM_R
     // ---- a9: pack (and BDR on the packed words), store
     uint32_t out[CW];
     if constexpr (POLICY == 1) {
-      // two's complement words straight from the saturating pack, compared
-      // with the stored words as they are
-      pack_sat<BITS>(y, out);
+      // offset-binary words from a saturating pack, compared with the stored
+      // words in offset binary, then flipped back to two's complement
       if constexpr (BITS == 4) {
+        pack4_subnormal(y, out);
 #pragma unroll
-        for (int q = 0; q < CW; ++q) out[q] = int4_raise_min(out[q]);
+        for (int q = 0; q < CW; ++q) out[q] = int4_raise_zero(out[q]);
+      } else {
+        pack_sat8(y, out);
+#pragma unroll
+        for (int q = 0; q < CW; ++q) out[q] ^= TOPS;
       }
       if constexpr (BDR_WORDS) {
         const bool pos = wcoef > 0.0f;
         const uint32_t on = (wcoef != 0.0f) ? words_on : 0u;
 #pragma unroll
         for (int q = 0; q < CW; ++q) {
-          out[q] = bdr_fixed_scale<BITS>(out[q], cold[q], pos ? kp[q] : kn[q], am[q], on);
+          out[q] = bdr_fixed_scale<BITS>(out[q], cold[q], pos ? kp[q] : kn[q], am[q] & on);
         }
       }
+#pragma unroll
+      for (int q = 0; q < CW; ++q) out[q] ^= TOPS;
     } else {
       pack_offset<BITS>(y, out);
 #pragma unroll
