@@ -10,6 +10,7 @@
 #include "qstate_step.cuh"
 #include "qstate_stream.cuh"
 #include "qstate_lrb.cuh"
+#include "qstate_lrb_stream.cuh"
 
 namespace qs {
 

@@ -181,11 +181,34 @@ cudaError_t launch_step(const StepParams& p0, cudaStream_t stream) {
   }
 }
 
+// The Low-Rank Bypass step: the streamed bypass kernel for the steps that
+// keep the stored state under the dynamic and persistent policies, the ring
+// kernel for the merge and for the yoked policy.
 template <int BITS, int DK, int POLICY, bool BDR, bool DELTA, bool DIAG, bool MERGE>
 cudaError_t launch_lrb(const LrbParams& p0, int tiles, int dv, cudaStream_t stream) {
   constexpr int D = 2;
   constexpr int RW = 32 / (DK / 32);
   constexpr int WARPS = kStepWarps;
+  if constexpr (POLICY != 2 && !MERGE) {
+    // coefficient registers for ranks up to 8, or up to 16
+    const bool small = p0.rpad <= 8;
+    auto kernel = small ? lrb_bypass_kernel<BITS, DK, DELTA, DIAG, 2> : lrb_bypass_kernel<BITS, DK, DELTA, DIAG, 4>;
+    static std::once_flag flag_small, flag_large;
+    cudaError_t err = allow_smem(kernel, small ? flag_small : flag_large);
+    if (err != cudaSuccess) return err;
+    LrbParams p = p0;
+    p.bpt = dv / RW;
+    p.nblocks = tiles * p.bpt;  // < 2^31 (checked by the caller)
+    p.two23 = 0x4B000000u;
+    const BypassLayout L(DK, DIAG, p.rank);
+    int per_sm = 0;
+    err = resident_ctas(kernel, 32, static_cast<size_t>(L.bytes()), &per_sm);
+    if (err != cudaSuccess) return err;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    long long grid = static_cast<long long>(per_sm) * device_sm_count();
+    if (grid > p.nblocks) grid = p.nblocks;
+    return launch_dependent(kernel, grid, 32, static_cast<size_t>(L.bytes()), stream, p);
+  }
   auto kernel = lrb_step_kernel<BITS, DK, POLICY, BDR, DELTA, DIAG, MERGE, D>;
   static std::once_flag flag;
   cudaError_t err = allow_smem(kernel, flag);

@@ -46,6 +46,7 @@ struct LrbParams {
   int rank;
   int rpad;        // rank rounded up to a multiple of 4
   int slot;        // position of this step in the period
+  uint32_t two23;  // the bits of 2^23 for the streamed INT4 unpack
 };
 
 // One warp's shared memory: DEPTH ring slots, then ntv tile-vector slots.

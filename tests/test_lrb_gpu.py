@@ -89,3 +89,32 @@ def test_lrb_rank1_is_the_plain_step():
         ca, sa, _ = a.state()
         cb, sb, _ = b.state()
         assert np.array_equal(ca, cb) and np.array_equal(sa, sb)
+
+
+def test_lrb_without_readout():
+    """Bypass and merge steps with the readout off (o = NULL: q is neither
+    read nor staged) leave the same state and buffers as the oracle's steps."""
+    import torch
+    from ssm_decode_step_b200 import qstate as Q
+    rng = np.random.default_rng(17)
+    T, dk, dv, R = 23, 128, 64, 5
+    for bits, dc in ((4, "scalar"), (8, "diagonal")):
+        cfg = Config(T, dk, dv, bits, 32, 1, dc, "persistent", "bdr")
+        S0 = (rng.standard_normal((T, dv, dk)) * 0.3).astype(np.float32)
+        gpu = P.GpuRun(cfg, S0)
+        buf = Q.LrbBuffers(cfg, R)
+        ocfg = P.oracle_cfg(cfg)
+        ora = O.init(ocfg, S0)
+        obuf = O.LrbBuffers(ocfg, R)
+        for t, (q, k, v, a, bb) in enumerate(P.random_steps(rng, T, dk, dv, dc, 2 * R + 1, scale=0.3)):
+            O.lrb_step(ora, obuf, q, k, v, a, bb)
+            buf.step(gpu.st, gpu.t(q), gpu.t(k), gpu.t(v), gpu.t(a), gpu.t(bb), None)
+            torch.cuda.synchronize()
+            c, s, _ = gpu.state()
+            rep = P.compare_state(cfg, c, s, ora, None, f"no readout int{bits} {dc} step {t}")
+            assert rep.code_flips == 0, rep
+            if buf.slot > 0:
+                n = buf.slot
+                assert np.array_equal(buf.A[buf.cur].cpu().numpy(), obuf.A), f"step {t}: A"
+                assert np.array_equal(buf.K[buf.cur][:, :n].cpu().numpy(), obuf.K[:, :n]), f"step {t}: K"
+                assert np.array_equal(buf.U[:, :, :n].cpu().numpy(), obuf.U[:, :, :n]), f"step {t}: U"
