@@ -119,6 +119,11 @@ __device__ __forceinline__ void cp_async_wait() {
 // in their own grid_dep_wait()).  Launched without the attribute, both do
 // nothing.
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+// A hint that brings the line holding p into L2 and nothing into registers.
+// It may precede grid_dep_wait(): the loads that use the data come after
+// the wait and read L2, where the previous kernel's writes land, so an
+// early prefetch can only save their trip to DRAM, never return stale data.
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];\n" ::"l"(p)); }
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 
 __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }

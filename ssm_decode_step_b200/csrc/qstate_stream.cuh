@@ -391,8 +391,6 @@ __global__ void __maxnreg__(BDR ? (BITS == 8 ? QS_STREAM_REGS_BDR8 : QS_STREAM_R
   const unsigned b1 = static_cast<unsigned>((blockIdx.x + 1) * static_cast<long long>(p.nblocks) / nw);
   if (b0 >= b1) return;
   const unsigned bpt = static_cast<unsigned>(p.bpt);
-  grid_dep_wait();
-  grid_dep_launch();
 
   // per-lane bases; row block b adds b times a per-block stride (one wide
   // multiply-add of the 32-bit block index per address)
@@ -404,6 +402,20 @@ __global__ void __maxnreg__(BDR ? (BITS == 8 ? QS_STREAM_REGS_BDR8 : QS_STREAM_R
   auto codes_at = [&](unsigned b) { return codes_l + static_cast<unsigned long long>(b) * CSTRIDE; };
   auto scale_at = [&](unsigned b) { return scales_l + static_cast<unsigned long long>(b) * sstride; };
   auto v_at = [&](unsigned b) { return v_l + static_cast<unsigned long long>(b) * RW; };
+
+  // INT4: the first two row blocks' codes and scales toward L2 while the
+  // previous kernel of the stream finishes (the INT8 instances, at their
+  // register cap, would spill for it)
+  if constexpr (BITS == 4) {
+    prefetch_l2(codes_at(b0));
+    prefetch_l2(scale_at(b0));
+    if (b0 + 1 < b1) {
+      prefetch_l2(codes_at(b0 + 1));
+      prefetch_l2(scale_at(b0 + 1));
+    }
+  }
+  grid_dep_wait();
+  grid_dep_launch();
 
   // ---- per-tile vectors: cp.async into the warp's two slots
   const uint32_t slots = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
