@@ -13,16 +13,17 @@
 // with K'_r = K_in_r a the buffered keys decayed by this step, in the fixed
 // operation order of include/qstate.h.  The work decomposition is the plain
 // streamed step's (qstate_stream.cuh): one warp per CTA, a contiguous range of
-// row blocks per warp, each lane's codes, scale and v loaded into registers
-// two row blocks ahead (its row's buffered coefficients U at the start of the
-// row block), and each tile's vectors (k, q,
-// the step's decay, A_in and the buffered keys) staged by cp.async into one of
-// two shared-memory slots a tile ahead.  On entering a tile a warp forms A, the
-// decayed keys and their products with k and q; the warp whose range holds the
-// tile's first row block also writes A_out and K_out (the caller swaps the two
-// copies between steps, so no warp reads what another writes in the launch).
-// The last slot of a period (the merge) and every slot of the yoked policy run
-// the ring kernel of qstate_lrb.cuh.
+// row blocks per warp, each lane's codes, scale, v and its row's buffered
+// coefficients U loaded into registers two row blocks ahead, and each tile's
+// vectors (k, q, the step's decay, A_in and the buffered keys) staged by
+// cp.async into one of two shared-memory slots a tile ahead.  On entering a
+// tile a warp forms A, the decayed keys and their products with k and q; the
+// warp whose range holds the tile's first row block also writes A_out and
+// K_out (the caller swaps the two copies between steps, so no warp reads what
+// another writes in the launch).  Per row block each code word is unpacked,
+// dequantized and fed to both dot products' chains at once.  The last slot of
+// a period (the merge) and every slot of the yoked policy run the ring kernel
+// of qstate_lrb.cuh.
 #pragma once
 
 #include "qstate_lrb.cuh"
