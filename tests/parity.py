@@ -60,9 +60,17 @@ def compare_state(cfg, gpu_codes_packed: np.ndarray, gpu_scales: np.ndarray,
             f"{what}: {rep.code_flips} code flips away from a half-step boundary"
         assert rep.code_flips <= CODE_FLIP_FRACTION * rep.elements, \
             f"{what}: {rep.code_flips} code flips of {rep.elements}"
+    # scales: non-finite ones (a group maximum that overflowed) by pattern,
+    # NaN where the oracle has NaN and infinities of the same sign; the
+    # relative bound on the finite ones
     s_ref = ora.scales.astype(np.float64)
-    rel = np.abs(gpu_scales.astype(np.float64) - s_ref) / np.maximum(np.abs(s_ref), 1e-38)
-    rel[(s_ref == 0) & (gpu_scales == 0)] = 0.0
+    s_gpu = np.asarray(gpu_scales).astype(np.float64)
+    assert np.array_equal(np.isnan(s_gpu), np.isnan(s_ref)), f"{what}: NaN scales differ"
+    assert np.array_equal(np.isposinf(s_gpu), np.isposinf(s_ref)) and \
+        np.array_equal(np.isneginf(s_gpu), np.isneginf(s_ref)), f"{what}: infinite scales differ"
+    fin = np.isfinite(s_ref)
+    rel = np.abs(s_gpu[fin] - s_ref[fin]) / np.maximum(np.abs(s_ref[fin]), 1e-38)
+    rel[(s_ref[fin] == 0) & (s_gpu[fin] == 0)] = 0.0
     rep.worst_scale_rel = float(rel.max()) if rel.size else 0.0
     assert rep.worst_scale_rel <= SCALE_REL, f"{what}: scale rel err {rep.worst_scale_rel}"
     return rep

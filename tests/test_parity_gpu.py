@@ -173,6 +173,57 @@ def test_clipping_and_huge_updates():
             P.compare_state(cfg, c, s_, ora, None, f"clip-{pol}-{rnd} after the overflow step")
 
 
+def _boundary_case(bits, T=4, dk=128, dv=64, group=32):
+    """A state whose groups have power-of-two scales (one code of each group
+    at qmax) and updates that put x / s' on half-integers (ties), on the
+    range's edges and beyond it, under both update signs, with and without
+    decay, then overflowing values."""
+    qmax = 7 if bits == 4 else 127
+    rng = np.random.default_rng(bits)
+    e = 2.0 ** -3
+    codes = rng.integers(-qmax, qmax + 1, size=(T, dv, dk))
+    codes[:, :, ::group] = qmax                        # each group's maximum: s = 2^-3 exactly
+    S0 = (codes * e).astype(np.float32)
+    kpat = np.array([1.0, -1.0, 0.5, 0.0, -0.5, 2.0, -2.0, 0.25], np.float32)
+    k = np.tile(kpat, (T, dk // 8))
+    halves = np.arange(-(qmax + 3), qmax + 3) + 0.5    # ..., -q-2.5, ..., q+2.5
+    far = np.array([-1e4, -3 * qmax, 3 * qmax, 1e4])
+    h = np.concatenate([halves, far, -halves[::-1] * 2.0])
+    v = np.resize(h, (T, dv)).astype(np.float64) * e
+    q = rng.standard_normal((T, dk)).astype(np.float32)
+    one, half = np.ones(T, np.float32), np.full(T, 0.5, np.float32)
+    steps = [(q, k, v.astype(np.float32), one, one),
+             (q, -k, (v[:, ::-1] * 0.75).astype(np.float32), half, one),
+             (q, k, np.where(np.arange(dv) % 2 == 0, 3e38, -3e38)[None, :].repeat(T, 0).astype(np.float32),
+              one, one)]
+    return S0, steps
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_rounding_boundaries_and_saturation(bits):
+    """Ties (x / s' on half-integers) round to even, values on and beyond
+    the range's edges clamp to +-qmax (the INT4 saturating pack through the
+    subnormal grid, the INT8 saturating pack), BDR steps toward the update
+    on both sides, and overflowing updates: codes, scales and readouts
+    against the oracle, in lock-step and free run."""
+    S0, steps = _boundary_case(bits)
+    T, dv, dk = S0.shape
+    for pol in ("persistent", "dynamic"):
+        for rnd in ("nearest", "bdr"):
+            cfg = Config(T, dk, dv, bits, 32, 0, "scalar", pol, rnd)
+            rep = P.lockstep(cfg, S0, steps, label=f"edges-int{bits}-{pol}-{rnd}")
+            assert rep.code_flips == 0, rep
+            gpu = P.GpuRun(cfg, S0)
+            ora = O.init(P.oracle_cfg(cfg), S0)
+            for t, (q, k, v, a, b) in enumerate(steps):
+                o = gpu.step(q, k, v, a, b)
+                o_ref = O.step(ora, q, k, v, a, b)
+                P.compare_readout(o, o_ref, f"edges-int{bits}-{pol}-{rnd} free step {t}")
+                c, s_, _ = gpu.state()
+                rep = P.compare_state(cfg, c, s_, ora, None, f"edges-int{bits}-{pol}-{rnd} free step {t}")
+                assert rep.code_flips == 0, rep
+
+
 # Full-size workloads at the benchmark's launch configuration, on sampled
 # tiles (tiles are independent, so a sampled tile is an exact check of that
 # tile).
