@@ -380,8 +380,10 @@ def pin_bdr_bruteforce():
 
 
 def pin_bdr_reversal_explained():
-    """North_star invariant (5), clause 1 ("BDR never moves an element against
-    its update"), as it holds under the stored-value reading of the move.
+    """The specification's BDR invariant, its first clause (BDR never moves
+    an element against its update), as it holds under the stored-value
+    reading of the move ("Preserving Updates", abstract: BDR rounds the
+    elements that moved opposite to their updates toward them).
     The move is measured from d = c * s, the element as stored before the
     step.  Without decay (Lambda = I) no element ends the step against its
     update, under a fixed or a changing scale.  With decay, an element can:
